@@ -1,0 +1,187 @@
+"""ctypes wrapper of the C oracle (orc.c).  Test infrastructure only."""
+import ctypes
+import os
+
+import numpy as np
+
+from .build import LIB, build_oracle
+
+FP8_PER_TOKEN = 0
+FP8_PER_GROUP128 = 1
+MXFP4 = 2
+
+_lib = None
+
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def load(path: str = LIB):
+    """Load (building first if needed) the oracle shared library."""
+    global _lib
+    if _lib is not None and path == LIB:
+        return _lib
+    build_oracle() if path == LIB else None
+    lib = ctypes.CDLL(os.path.abspath(path))
+    lib.orc_bf16_to_double.argtypes = [ctypes.c_uint16]
+    lib.orc_bf16_to_double.restype = ctypes.c_double
+    lib.orc_bf16_from_double.argtypes = [ctypes.c_double]
+    lib.orc_bf16_from_double.restype = ctypes.c_uint16
+    lib.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+    lib.orc_e4m3_decode.restype = ctypes.c_double
+    lib.orc_e4m3_encode.argtypes = [ctypes.c_double]
+    lib.orc_e4m3_encode.restype = ctypes.c_uint8
+    lib.orc_e2m1_decode.argtypes = [ctypes.c_uint8]
+    lib.orc_e2m1_decode.restype = ctypes.c_double
+    lib.orc_e2m1_encode.argtypes = [ctypes.c_double]
+    lib.orc_e2m1_encode.restype = ctypes.c_uint8
+    lib.orc_mx_scale_code.argtypes = [ctypes.c_double]
+    lib.orc_mx_scale_code.restype = ctypes.c_uint8
+    lib.orc_rstd.argtypes = [_u16p, ctypes.c_int64, ctypes.c_float]
+    lib.orc_rstd.restype = ctypes.c_double
+    lib.orc_quant_rows.argtypes = [_u16p, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
+                                   _u8p, ctypes.c_void_p]
+    lib.orc_quant_rows.restype = ctypes.c_int
+    lib.orc_rmsnorm_quant.argtypes = [ctypes.POINTER(_u16p), ctypes.c_int, _u16p, _u16p,
+                                      ctypes.c_float, ctypes.c_int, ctypes.c_int64,
+                                      ctypes.c_int64, _u8p, ctypes.c_void_p, _u16p, _u16p]
+    lib.orc_rmsnorm_quant.restype = ctypes.c_int
+    lib.orc_qk_norm_gate.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                     ctypes.c_int, ctypes.c_int, _u16p, _u16p,
+                                     ctypes.c_float, _u16p, _u16p, _u16p]
+    lib.orc_qk_norm_gate.restype = ctypes.c_int
+    if path == LIB:
+        _lib = lib
+    return lib
+
+
+def _p16(a):
+    return None if a is None else a.ctypes.data_as(_u16p)
+
+
+def _p8(a):
+    return a.ctypes.data_as(_u8p)
+
+
+def _u16(a):
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("bf16 arrays travel as uint16 bit patterns")
+    return a
+
+
+def scale_shape(mode: int, M: int, H: int):
+    return {FP8_PER_TOKEN: (M,), FP8_PER_GROUP128: (M, H // 128), MXFP4: (M, H // 32)}[mode]
+
+
+def code_shape(mode: int, M: int, H: int):
+    return (M, H // 2) if mode == MXFP4 else (M, H)
+
+
+def _scale_dtype(mode):
+    return np.uint8 if mode == MXFP4 else np.float32
+
+
+# ---- scalar format helpers (vectorised over numpy inputs) -------------------
+
+def bf16_to_double(bits, lib=None):
+    lib = lib or load()
+    return np.array([lib.orc_bf16_to_double(int(b)) for b in np.ravel(bits)]).reshape(np.shape(bits))
+
+
+def bf16_from_double(v, lib=None):
+    lib = lib or load()
+    return np.array([lib.orc_bf16_from_double(float(x)) for x in np.ravel(v)],
+                    dtype=np.uint16).reshape(np.shape(v))
+
+
+def e4m3_encode(v, lib=None):
+    lib = lib or load()
+    return np.array([lib.orc_e4m3_encode(float(x)) for x in np.ravel(v)],
+                    dtype=np.uint8).reshape(np.shape(v))
+
+
+def e4m3_decode(c, lib=None):
+    lib = lib or load()
+    return np.array([lib.orc_e4m3_decode(int(x)) for x in np.ravel(c)]).reshape(np.shape(c))
+
+
+def e2m1_encode(v, lib=None):
+    lib = lib or load()
+    return np.array([lib.orc_e2m1_encode(float(x)) for x in np.ravel(v)],
+                    dtype=np.uint8).reshape(np.shape(v))
+
+
+def e2m1_decode(c, lib=None):
+    lib = lib or load()
+    return np.array([lib.orc_e2m1_decode(int(x)) for x in np.ravel(c)]).reshape(np.shape(c))
+
+
+def mx_scale_code(amax, lib=None):
+    lib = lib or load()
+    return np.array([lib.orc_mx_scale_code(float(x)) for x in np.ravel(amax)],
+                    dtype=np.uint8).reshape(np.shape(amax))
+
+
+# ---- row operations ---------------------------------------------------------
+
+def rstd(h_bits, eps: float, lib=None) -> float:
+    lib = lib or load()
+    h = _u16(h_bits)
+    return lib.orc_rstd(_p16(h), h.size, eps)
+
+
+def quant_rows(y_bits, mode: int, lib=None):
+    """Quantize bf16 rows [M, H]; returns (codes, scales)."""
+    lib = lib or load()
+    y = _u16(y_bits)
+    M, H = y.shape
+    q = np.zeros(code_shape(mode, M, H), dtype=np.uint8)
+    s = np.zeros(scale_shape(mode, M, H), dtype=_scale_dtype(mode))
+    rc = lib.orc_quant_rows(_p16(y), mode, M, H, _p8(q), s.ctypes.data_as(ctypes.c_void_p))
+    if rc != 0:
+        raise OracleError(f"orc_quant_rows rejected mode={mode} H={H}")
+    return q, s
+
+
+def rmsnorm_quant(parts, residual, weight, eps: float, mode: int, lib=None):
+    """Unfused reference sequence over [M, H] rows.
+
+    parts: list of P uint16 [M, H] arrays; residual: uint16 [M, H] or None;
+    weight: uint16 [H].  Returns dict(q, scale, residual_out, y).
+    """
+    lib = lib or load()
+    parts = [_u16(p) for p in parts]
+    M, H = parts[0].shape
+    arr = (_u16p * len(parts))(*[_p16(p) for p in parts])
+    res = None if residual is None else _u16(residual)
+    w = _u16(weight)
+    q = np.zeros(code_shape(mode, M, H), dtype=np.uint8)
+    s = np.zeros(scale_shape(mode, M, H), dtype=_scale_dtype(mode))
+    r_out = np.zeros((M, H), dtype=np.uint16)
+    y = np.zeros((M, H), dtype=np.uint16)
+    rc = lib.orc_rmsnorm_quant(arr, len(parts), _p16(res), _p16(w), eps, mode, M, H, _p8(q),
+                               s.ctypes.data_as(ctypes.c_void_p), _p16(r_out), _p16(y))
+    if rc != 0:
+        raise OracleError(f"orc_rmsnorm_quant rejected P={len(parts)} mode={mode} H={H}")
+    return {"q": q, "scale": s, "residual_out": r_out, "y": y}
+
+
+def qk_norm_gate(qkv, row_stride: int, Hq: int, Hk: int, D: int, q_weight, k_weight,
+                 eps: float, lib=None):
+    """qkv: uint16 [M, row_stride]; returns dict(q [M,Hq,D], k [M,Hk,D], gate [M,Hq,D])."""
+    lib = lib or load()
+    x = _u16(qkv)
+    M = x.shape[0]
+    q = np.zeros((M, Hq, D), dtype=np.uint16)
+    k = np.zeros((M, Hk, D), dtype=np.uint16)
+    g = np.zeros((M, Hq, D), dtype=np.uint16)
+    rc = lib.orc_qk_norm_gate(_p16(x), M, row_stride, Hq, Hk, D, _p16(_u16(q_weight)),
+                              _p16(_u16(k_weight)), eps, _p16(q), _p16(k), _p16(g))
+    if rc != 0:
+        raise OracleError("orc_qk_norm_gate rejected the shape")
+    return {"q": q, "k": k, "gate": g}

@@ -1,0 +1,413 @@
+/*
+ * Plain CPU oracle for the fused residual-add + RMSNorm + activation
+ * quantization path and for the QK Gemma-RMSNorm + gate prologue.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file; only the tests, the smoke check and the CPU baseline of the
+ * benchmark do.  It shares no code, header, table or constant generator with
+ * the CUDA library: every format rule below is written out here from its
+ * definition, single-threaded, in fp64 wherever the definition does not fix
+ * the precision.
+ *
+ * Sources (page title, then section):
+ *  [AR]   sglang PR #29723, "Fused AllReduce + RMSNorm + per-token FP8 /
+ *         MXFP4 quant on AMD (AITER)": "Modifications" (the tuple
+ *         (fp8_output, residual_out, per_token_scale), scale shaped (M,1)) and
+ *         "Accuracy Tests" (the fused kernel equals the unfused
+ *         AllReduce -> RMSNorm -> quantize sequence).
+ *  [MONO] sgl-amd-mono PR #26, "Whole-layer monokernels for Muse Spark",
+ *         commit notes: online MXFP4 quantization of activations; the xn task
+ *         quantizes the bf16 normed row and is bit-exact against the
+ *         stand-alone quantization of that row.
+ *  [QK]   sglang PR #27656, "Fuse QK RMSNorm + gate extraction Triton kernel
+ *         for Qwen3.5 on HIP": "Motivation" (interleaved
+ *         [q_h0, gate_h0, q_h1, gate_h1, ...] layout, GemmaRMSNorm on q and k,
+ *         contiguous q, k, gate outputs).
+ *  [OCP]  OCP Microscaling (MX) v1.0: shared scale X = 2^(floor(log2 amax) -
+ *         emax_elem), emax_elem = 2 for E2M1; E8M0 scale; E4M3 "fn" element
+ *         format (max 448, no infinities).
+ *
+ * Readings where the pages are silent (each one is listed in the design
+ * notes under the same tag):
+ *  A1  RMSNorm is h * 1/sqrt(mean(h^2) + eps) * w, mean over the row.
+ *  A2  Gemma weight is (1 + w) formed in fp64, not rounded to bf16.
+ *  A3  partials are summed in fp32 in order p = 0..P-1, then the residual is
+ *      added in fp32, then ONE rounding to bf16 gives h (= residual_out);
+ *      the norm reads the bf16 h.
+ *  A4  y = bf16_rn(h * rstd * w): one rounding of the fp64 product.
+ *  A5  FP8 is OCP E4M3 "fn" (max 448), round-to-nearest-even, saturating.
+ *  A6  FP8 scale = fl32(amax / 448); code = e4m3(fl32(y / scale)) with a true
+ *      fp32 division.
+ *  A7  all-zero FP8 row/group: scale 1.0, codes 0.
+ *  A8  all-zero MX block: scale code 0 (2^-127), codes 0.
+ *  A9  element 2i in the low nibble of byte i; scales row-major.
+ *  A11 a NaN or infinite MX block amax gives scale code 0xFF.
+ *
+ * Build: plain C99, -O2 -ffp-contract=off, no fast-math, x86-64 SSE float
+ * arithmetic (FLT_EVAL_METHOD == 0), so `float` operations are IEEE binary32
+ * with round-to-nearest-even.
+ */
+#include <float.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#if !defined(FLT_EVAL_METHOD) || FLT_EVAL_METHOD != 0
+#error "the oracle needs float arithmetic evaluated in binary32"
+#endif
+
+/* Mode numbers of the quantization step (the interface's values). */
+#define ORC_FP8_PER_TOKEN 0
+#define ORC_FP8_PER_GROUP128 1
+#define ORC_MXFP4 2
+
+#define ORC_OK 0
+#define ORC_BAD -1
+
+/* ------------------------------------------------------------------ */
+/* Number formats                                                       */
+/* ------------------------------------------------------------------ */
+
+/* bf16 bit pattern -> its exact value (bf16 is the top half of binary32). */
+double orc_bf16_to_double(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static float bf16_to_float(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/*
+ * Round a finite double to the nearest point of a binary floating-point grid
+ * with `mbits` stored mantissa bits and minimum normal exponent `emin`
+ * (subnormals below it, spacing 2^(emin - mbits)); ties go to the even
+ * multiple of the spacing, i.e. the even mantissa.  The exponent range is
+ * unbounded above: overflow is handled by the caller.
+ */
+static double round_to_grid(double v, int mbits, int emin)
+{
+    if (v == 0.0 || !isfinite(v))
+        return v;
+    int e2;
+    (void)frexp(fabs(v), &e2);    /* |v| = m 2^e2, m in [0.5, 1) */
+    int ex = e2 - 1;              /* floor(log2 |v|) */
+    if (ex < emin)
+        ex = emin;
+    double quantum = ldexp(1.0, ex - mbits);
+    double n = nearbyint(fabs(v) / quantum); /* exact quotient; ties-to-even */
+    return copysign(n * quantum, v);
+}
+
+/* IEEE round-to-nearest-even of a double to bf16 (8 significant bits,
+ * emin -126, overflow to infinity), returned as a bit pattern. */
+uint16_t orc_bf16_from_double(double v)
+{
+    if (isnan(v))
+        return (uint16_t)(signbit(v) ? 0xFFC0u : 0x7FC0u);
+    double r = round_to_grid(v, 7, -126);
+    float f;
+    if (fabs(r) >= 0x1p128)
+        f = signbit(r) ? -INFINITY : INFINITY;
+    else
+        f = (float)r; /* exact: r has <= 8 significant bits within binary32 range */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+/* OCP E4M3 "fn": 1 sign, 4 exponent (bias 7), 3 mantissa bits; no infinity;
+ * S.1111.111 is NaN; largest finite 1.75 * 2^8 = 448; smallest subnormal 2^-9. */
+double orc_e4m3_decode(uint8_t c)
+{
+    int s = c >> 7, e = (c >> 3) & 0xF, m = c & 7;
+    double mag;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        mag = ldexp((double)m, -9);
+    else
+        mag = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+/* Round to E4M3 with round-to-nearest-even and saturation to +-448
+ * ("satfinite"); NaN gives 0x7F. */
+uint8_t orc_e4m3_encode(double v)
+{
+    if (isnan(v))
+        return 0x7F;
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double r = fabs(round_to_grid(v, 3, -6));
+    if (r > 448.0)
+        r = 448.0;
+    if (r == 0.0)
+        return sign;
+    int e2;
+    (void)frexp(r, &e2);
+    int ex = e2 - 1;
+    if (ex < -6) /* subnormal: r = m * 2^-9 */
+        return (uint8_t)(sign | (uint8_t)(r / 0x1p-9));
+    int m = (int)((r / ldexp(1.0, ex) - 1.0) * 8.0);
+    return (uint8_t)(sign | ((ex + 7) << 3) | m);
+}
+
+/* OCP E2M1: 1 sign, 2 exponent (bias 1), 1 mantissa bit; magnitudes
+ * {0, 0.5, 1, 1.5, 2, 3, 4, 6}; no NaN, no infinity. */
+double orc_e2m1_decode(uint8_t c)
+{
+    int s = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+    double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -mag : mag;
+}
+
+/* Round to E2M1, nearest-even, saturating to +-6; the sign is kept, so a
+ * negative value that rounds to zero gives -0 (code 0x8). */
+uint8_t orc_e2m1_encode(double v)
+{
+    uint8_t sign = signbit(v) ? 0x8 : 0x0;
+    double r = fabs(round_to_grid(v, 1, 0));
+    if (r > 6.0)
+        r = 6.0;
+    if (r == 0.0)
+        return sign;
+    int e2;
+    (void)frexp(r, &e2);
+    int ex = e2 - 1;
+    if (ex < 0) /* subnormal: only 0.5 */
+        return (uint8_t)(sign | 0x1);
+    int m = (int)((r / ldexp(1.0, ex) - 1.0) * 2.0);
+    return (uint8_t)(sign | ((ex + 1) << 1) | m);
+}
+
+/* [OCP] shared exponent of an MX block: e = floor(log2(amax)) - 2 (2 is the
+ * largest exponent of E2M1), clamped to the E8M0 range [-127, 127].
+ * Returns the E8M0 code e + 127; amax == 0 gives code 0 (A8); a NaN or
+ * infinite amax gives 0xFF (A11). */
+uint8_t orc_mx_scale_code(double amax)
+{
+    if (!isfinite(amax))
+        return 0xFF;
+    if (amax == 0.0)
+        return 0x00;
+    int e2;
+    (void)frexp(amax, &e2);
+    int e = (e2 - 1) - 2;
+    if (e < -127)
+        e = -127;
+    if (e > 127)
+        e = 127;
+    return (uint8_t)(e + 127);
+}
+
+/* ------------------------------------------------------------------ */
+/* Quantization of bf16 rows ([AR] "Modifications", [MONO] bit-exact    */
+/* quantization of the bf16 row, [OCP])                                 */
+/* ------------------------------------------------------------------ */
+
+/* FP8 E4M3 of one group of n bf16 values with one fp32 scale (A5-A7). */
+static void quant_fp8_group(const uint16_t* y, int64_t n, uint8_t* q, float* scale_out)
+{
+    float amax = 0.0f;
+    for (int64_t j = 0; j < n; ++j) {
+        float a = fabsf(bf16_to_float(y[j]));
+        if (a > amax)
+            amax = a;
+    }
+    float scale = (amax == 0.0f) ? 1.0f : amax / 448.0f; /* one binary32 division */
+    for (int64_t j = 0; j < n; ++j) {
+        float t = bf16_to_float(y[j]) / scale;            /* one binary32 division */
+        q[j] = orc_e4m3_encode((double)t);
+    }
+    *scale_out = scale;
+}
+
+/* MXFP4 of one 32-element block: E8M0 scale code, then E2M1 codes of
+ * y_j * 2^-e, packed two per byte, element 2i in the low nibble (A9). */
+static void quant_mx_block(const uint16_t* y, uint8_t* packed, uint8_t* scale_code)
+{
+    double amax = 0.0;
+    int any_nan = 0;
+    for (int j = 0; j < 32; ++j) {
+        double a = fabs(orc_bf16_to_double(y[j]));
+        if (isnan(a))
+            any_nan = 1;
+        else if (a > amax)
+            amax = a;
+    }
+    if (any_nan)
+        amax = NAN;
+    uint8_t sc = orc_mx_scale_code(amax);
+    int e = (int)sc - 127;
+    for (int i = 0; i < 16; ++i) {
+        double v0 = ldexp(orc_bf16_to_double(y[2 * i]), -e);     /* exact */
+        double v1 = ldexp(orc_bf16_to_double(y[2 * i + 1]), -e); /* exact */
+        uint8_t c0 = orc_e2m1_encode(v0), c1 = orc_e2m1_encode(v1);
+        packed[i] = (uint8_t)(c0 | (c1 << 4));
+    }
+    *scale_code = sc;
+}
+
+/*
+ * Quantize M bf16 rows of length H.
+ *   mode 0: out_q [M,H] E4M3, out_scale fp32 [M]
+ *   mode 1: out_q [M,H] E4M3, out_scale fp32 [M, H/128] row-major
+ *   mode 2: out_q [M,H/2] packed E2M1, out_scale u8 E8M0 [M, H/32] row-major
+ */
+int orc_quant_rows(const uint16_t* y, int mode, int64_t M, int64_t H,
+                   uint8_t* out_q, void* out_scale)
+{
+    if (M < 0 || H <= 0)
+        return ORC_BAD;
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t* yr = y + m * H;
+        if (mode == ORC_FP8_PER_TOKEN) {
+            quant_fp8_group(yr, H, out_q + m * H, (float*)out_scale + m);
+        } else if (mode == ORC_FP8_PER_GROUP128) {
+            if (H % 128)
+                return ORC_BAD;
+            for (int64_t g = 0; g < H / 128; ++g)
+                quant_fp8_group(yr + g * 128, 128, out_q + m * H + g * 128,
+                                (float*)out_scale + m * (H / 128) + g);
+        } else if (mode == ORC_MXFP4) {
+            if (H % 32)
+                return ORC_BAD;
+            for (int64_t b = 0; b < H / 32; ++b)
+                quant_mx_block(yr + b * 32, out_q + m * (H / 2) + b * 16,
+                               (uint8_t*)out_scale + m * (H / 32) + b);
+        } else {
+            return ORC_BAD;
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* RMSNorm ([AR] "Accuracy Tests": the unfused sequence)                */
+/* ------------------------------------------------------------------ */
+
+/* rstd = 1/sqrt(mean(h^2) + eps) in fp64 over n bf16 values (A1). */
+double orc_rstd(const uint16_t* h, int64_t n, float eps)
+{
+    double ss = 0.0;
+    for (int64_t j = 0; j < n; ++j) {
+        double v = orc_bf16_to_double(h[j]);
+        ss += v * v;
+    }
+    return 1.0 / sqrt(ss / (double)n + (double)eps);
+}
+
+/*
+ * The unfused reference sequence, row by row:
+ *   h  = bf16( (((part_0 + part_1) + ...) + part_{P-1}) + residual )   fp32 adds (A3)
+ *   residual_out = h
+ *   y  = bf16( h * rstd * w )                                           fp64 (A1, A4)
+ *   (q, scale) = quantize(y)                                            (A5-A9)
+ * residual may be NULL (no residual add); out_residual and out_y may be NULL.
+ */
+int orc_rmsnorm_quant(const uint16_t* const* parts, int P, const uint16_t* residual,
+                      const uint16_t* weight, float eps, int mode, int64_t M, int64_t H,
+                      uint8_t* out_q, void* out_scale, uint16_t* out_residual,
+                      uint16_t* out_y)
+{
+    if (P < 1 || P > 8 || M < 0 || H <= 0 || !parts || !weight)
+        return ORC_BAD;
+    if (mode == ORC_FP8_PER_GROUP128 && H % 128)
+        return ORC_BAD;
+    if (mode == ORC_MXFP4 && H % 32)
+        return ORC_BAD;
+    if (mode < 0 || mode > 2)
+        return ORC_BAD;
+    uint16_t* hbuf = (uint16_t*)malloc((size_t)H * sizeof(uint16_t));
+    uint16_t* ybuf = (uint16_t*)malloc((size_t)H * sizeof(uint16_t));
+    if (!hbuf || !ybuf) {
+        free(hbuf);
+        free(ybuf);
+        return ORC_BAD;
+    }
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t j = 0; j < H; ++j) {
+            float s = bf16_to_float(parts[0][m * H + j]);
+            for (int p = 1; p < P; ++p)
+                s = s + bf16_to_float(parts[p][m * H + j]);
+            if (residual)
+                s = s + bf16_to_float(residual[m * H + j]);
+            hbuf[j] = orc_bf16_from_double((double)s);
+        }
+        double rstd = orc_rstd(hbuf, H, eps);
+        for (int64_t j = 0; j < H; ++j)
+            ybuf[j] = orc_bf16_from_double(orc_bf16_to_double(hbuf[j]) * rstd *
+                                           orc_bf16_to_double(weight[j]));
+        if (out_residual)
+            memcpy(out_residual + m * H, hbuf, (size_t)H * sizeof(uint16_t));
+        if (out_y)
+            memcpy(out_y + m * H, ybuf, (size_t)H * sizeof(uint16_t));
+        int rc;
+        if (mode == ORC_FP8_PER_TOKEN)
+            rc = orc_quant_rows(ybuf, mode, 1, H, out_q + m * H, (float*)out_scale + m);
+        else if (mode == ORC_FP8_PER_GROUP128)
+            rc = orc_quant_rows(ybuf, mode, 1, H, out_q + m * H,
+                                (float*)out_scale + m * (H / 128));
+        else
+            rc = orc_quant_rows(ybuf, mode, 1, H, out_q + m * (H / 2),
+                                (uint8_t*)out_scale + m * (H / 32));
+        if (rc != ORC_OK) {
+            free(hbuf);
+            free(ybuf);
+            return rc;
+        }
+    }
+    free(hbuf);
+    free(ybuf);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* QK Gemma-RMSNorm + gate ([QK] "Motivation", "Modifications")         */
+/* ------------------------------------------------------------------ */
+
+/* One head: y = bf16(x * rstd * (1 + w)) over D values (A1, A2, A4). */
+static void gemma_norm_head(const uint16_t* x, const uint16_t* w, int D, float eps,
+                            uint16_t* y)
+{
+    double rstd = orc_rstd(x, D, eps);
+    for (int d = 0; d < D; ++d)
+        y[d] = orc_bf16_from_double(orc_bf16_to_double(x[d]) * rstd *
+                                    (1.0 + orc_bf16_to_double(w[d])));
+}
+
+/*
+ * Token m's row starts at qkv + m*row_stride (elements).  Head h < Hq of q
+ * sits at [2hD, 2hD + D), its gate at [(2h+1)D, (2h+2)D); head h < Hk of k
+ * sits at [2 Hq D + hD, 2 Hq D + (h+1)D).  Outputs are contiguous
+ * q [M,Hq,D], k [M,Hk,D], gate [M,Hq,D]; the gate is a bit copy.
+ */
+int orc_qk_norm_gate(const uint16_t* qkv, int64_t M, int64_t row_stride, int Hq, int Hk,
+                     int D, const uint16_t* q_weight, const uint16_t* k_weight, float eps,
+                     uint16_t* out_q, uint16_t* out_k, uint16_t* out_gate)
+{
+    if (M < 0 || Hq < 0 || Hk < 0 || D <= 0 ||
+        row_stride < (int64_t)(2 * Hq + Hk) * D)
+        return ORC_BAD;
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t* row = qkv + m * row_stride;
+        for (int h = 0; h < Hq; ++h) {
+            gemma_norm_head(row + (int64_t)2 * h * D, q_weight, D, eps,
+                            out_q + (m * Hq + h) * D);
+            memcpy(out_gate + (m * Hq + h) * D, row + (int64_t)(2 * h + 1) * D,
+                   (size_t)D * sizeof(uint16_t));
+        }
+        for (int h = 0; h < Hk; ++h)
+            gemma_norm_head(row + (int64_t)2 * Hq * D + (int64_t)h * D, k_weight, D, eps,
+                            out_k + (m * Hk + h) * D);
+    }
+    return ORC_OK;
+}

@@ -1,0 +1,480 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each pin takes a loaded oracle library (`lib`) and raises AssertionError when
+the oracle disagrees with: values printed by the format specifications
+(tests/golden/), an independent brute-force or library computation (torch's
+float8 conversion, exhaustive nearest-point search over a format's grid,
+Python `decimal` at 60 digits), closed forms, or invariants.  The same pins
+run against deliberately broken copies of the oracle in
+test_oracle_mutations.py, where at least one of them must fail.
+"""
+import json
+import math
+import os
+from decimal import Decimal, getcontext
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+# ----------------------------------------------------------------------------
+# helpers that do not use the oracle
+# ----------------------------------------------------------------------------
+
+
+def all_finite_bf16():
+    """All finite bf16 bit patterns and their values (float64)."""
+    bits = np.arange(65536, dtype=np.uint32)
+    f = (bits << 16).astype(np.uint32).view(np.float32)
+    keep = np.isfinite(f)
+    return bits[keep].astype(np.uint16), f[keep].astype(np.float64)
+
+
+def bf16_bits_to_f64(bits):
+    return (np.asarray(bits, dtype=np.uint32) << 16).astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def f32_to_bf16_bits_torch(a):
+    """binary32 -> bf16 round-to-nearest-even, by torch's own conversion."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def read_table(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                c, v = line.split()
+                rows.append((int(c, 16), float(v)))
+    return rows
+
+
+def brute_encode(v, grid_vals, grid_codes, sign_bit):
+    """Nearest point of a sign-magnitude grid by exhaustive search; ties go to
+    the even code; beyond the largest point, the largest point (saturation)."""
+    v = np.asarray(v, dtype=np.float64)
+    # Any magnitude above the largest point has that point as its nearest;
+    # clipping keeps the differences below exact in binary64.
+    mag = np.minimum(np.abs(v), 2.0 * grid_vals.max())
+    d = np.abs(mag[:, None] - grid_vals[None, :])
+    dmin = d.min(axis=1, keepdims=True)
+    cand = d == dmin
+    even = (grid_codes[None, :] & 1) == 0
+    pick_even = cand & even
+    has_even = pick_even.any(axis=1)
+    idx = np.where(has_even, pick_even.argmax(axis=1), cand.argmax(axis=1))
+    codes = grid_codes[idx].astype(np.int64)
+    codes = np.where(np.signbit(v), codes | sign_bit, codes)
+    return codes.astype(np.uint8)
+
+
+def e4m3_grid_torch():
+    codes = np.arange(0x7F, dtype=np.uint8)  # 0x00..0x7E: the positive finite points
+    vals = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return vals, codes
+
+
+def e2m1_grid_golden():
+    t = read_table("ocp_e2m1.txt")
+    codes = np.array([c for c, v in t if c < 8], dtype=np.uint8)
+    vals = np.array([v for c, v in t if c < 8], dtype=np.float64)
+    return vals, codes
+
+
+def brute_mx_scale_code(amax):
+    """The E8M0 code c with 4 * 2^(c-127) <= amax < 8 * 2^(c-127), found by
+    comparing against exact powers of two; c = 0 when amax is below 2^-125."""
+    if amax == 0:
+        return 0
+    for c in range(0, 255):
+        lo, hi = 4.0 * 2.0 ** (c - 127), 8.0 * 2.0 ** (c - 127)
+        if amax < hi and (amax >= lo or c == 0):
+            return c
+    raise AssertionError("no E8M0 code")
+
+
+def nearest_bf16_decimal(x: Decimal) -> int:
+    """bf16 bit pattern nearest to a high-precision value (ties to even)."""
+    if x == 0:
+        return 0x8000 if x.is_signed() else 0
+    neg = x < 0
+    ax = -x if neg else x
+    f = np.float32(float(ax))
+    base = int(np.array([f]).view(np.uint32)[0] >> 16)
+    best = None
+    for b in range(max(base - 2, 0), min(base + 3, 0x7F80)):
+        val = Decimal(float(bf16_bits_to_f64([b])[0]))
+        d = abs(val - ax)
+        key = (d, b & 1)
+        if best is None or key < best[0]:
+            best = (key, b)
+    b = best[1]
+    return b | 0x8000 if neg else b
+
+
+def decimal_rstd(h_vals, eps32):
+    getcontext().prec = 60
+    ss = sum(Decimal(float(v)) ** 2 for v in h_vals)
+    ms = ss / Decimal(len(h_vals))
+    return Decimal(1) / (ms + Decimal(float(eps32))).sqrt()
+
+
+def ref_y_bits(h_vals, w_vals, eps, gemma=False):
+    getcontext().prec = 60
+    r = decimal_rstd(h_vals, np.float32(eps))
+    out = []
+    for h, w in zip(h_vals, w_vals):
+        wd = Decimal(float(w))
+        if gemma:
+            wd = Decimal(1) + wd
+        out.append(nearest_bf16_decimal(Decimal(float(h)) * r * wd))
+    return np.array(out, dtype=np.uint16)
+
+
+def ref_quant_fp8(y_bits, group):
+    """Library formulation: fp32 amax, fp32 amax/448, fp32 y/scale, torch's
+    float8_e4m3fn conversion (nearest-even; never reached above 464 here)."""
+    y = bf16_bits_to_f64(y_bits).astype(np.float32)
+    M, H = y.shape
+    codes = np.zeros((M, H), dtype=np.uint8)
+    scales = np.zeros((M, H // group), dtype=np.float32)
+    for m in range(M):
+        for g in range(H // group):
+            seg = y[m, g * group:(g + 1) * group]
+            amax = np.float32(np.max(np.abs(seg)))
+            scale = np.float32(1.0) if amax == 0 else np.float32(amax / np.float32(448.0))
+            t = (seg / scale).astype(np.float32)
+            c = torch.from_numpy(t).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            codes[m, g * group:(g + 1) * group] = c
+            scales[m, g] = scale
+    return codes, scales
+
+
+def ref_quant_mx(y_bits):
+    y = bf16_bits_to_f64(y_bits)
+    M, H = y.shape
+    gv, gc = e2m1_grid_golden()
+    packed = np.zeros((M, H // 2), dtype=np.uint8)
+    sc = np.zeros((M, H // 32), dtype=np.uint8)
+    for m in range(M):
+        for b in range(H // 32):
+            blk = y[m, b * 32:(b + 1) * 32]
+            c = brute_mx_scale_code(float(np.max(np.abs(blk))))
+            v = blk * 2.0 ** (-(c - 127))
+            codes = brute_encode(v, gv, gc, 0x8)
+            packed[m, b * 16:(b + 1) * 16] = codes[0::2] | (codes[1::2] << 4)
+            sc[m, b] = c
+    return packed, sc
+
+
+def ref_residual_bits(parts_bits, res_bits):
+    s = bf16_bits_to_f64(parts_bits[0]).astype(np.float32)
+    for p in parts_bits[1:]:
+        s = (s + bf16_bits_to_f64(p).astype(np.float32)).astype(np.float32)
+    if res_bits is not None:
+        s = (s + bf16_bits_to_f64(res_bits).astype(np.float32)).astype(np.float32)
+    return f32_to_bf16_bits_torch(s)
+
+
+def bf16_bits_from_torch(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+# ----------------------------------------------------------------------------
+# pins
+# ----------------------------------------------------------------------------
+
+
+def pin_e4m3_decode(lib):
+    codes = np.arange(256, dtype=np.uint8)
+    mine = oracle.e4m3_decode(codes, lib)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(ref)), "E4M3 NaN codes"
+    ok = ~np.isnan(ref)
+    assert np.array_equal(mine[ok], ref[ok]), "E4M3 decode vs torch"
+    assert np.array_equal(np.signbit(mine[ok]), np.signbit(ref[ok])), "E4M3 signed zero"
+    for c, v in read_table("ocp_e4m3_points.txt"):
+        got = lib.orc_e4m3_decode(c)
+        if math.isnan(v):
+            assert math.isnan(got), f"code {c:#x} must be NaN"
+        else:
+            assert got == v and math.copysign(1, got) == math.copysign(1, v), f"code {c:#x}"
+
+
+def pin_e4m3_encode(lib):
+    bits, vals = all_finite_bf16()
+    mine = oracle.e4m3_encode(vals, lib)
+    gv, gc = e4m3_grid_torch()
+    brute = brute_encode(vals, gv, gc, 0x80)
+    assert np.array_equal(mine, brute), "E4M3 encode vs exhaustive nearest-even search"
+    inr = np.abs(vals) <= 464.0
+    tq = torch.from_numpy(vals[inr].astype(np.float32)).to(torch.float8_e4m3fn)
+    assert np.array_equal(mine[inr], tq.view(torch.uint8).numpy()), "E4M3 encode vs torch"
+    assert lib.orc_e4m3_encode(1e30) == 0x7E and lib.orc_e4m3_encode(-1e30) == 0xFE
+    assert lib.orc_e4m3_encode(float("nan")) == 0x7F
+    # every finite code survives decode -> encode
+    for c in range(256):
+        if (c & 0x7F) == 0x7F:
+            continue
+        assert lib.orc_e4m3_encode(lib.orc_e4m3_decode(c)) == c, f"round trip {c:#x}"
+
+
+def pin_e2m1(lib):
+    for c, v in read_table("ocp_e2m1.txt"):
+        got = lib.orc_e2m1_decode(c)
+        assert got == v and math.copysign(1, got) == math.copysign(1, v), f"E2M1 decode {c:#x}"
+        assert lib.orc_e2m1_encode(v) == c, f"E2M1 round trip {c:#x}"
+    bits, vals = all_finite_bf16()
+    gv, gc = e2m1_grid_golden()
+    assert np.array_equal(oracle.e2m1_encode(vals, lib), brute_encode(vals, gv, gc, 0x8)), \
+        "E2M1 encode vs exhaustive nearest-even search"
+    # the tie points of the grid go to the even code
+    ties = {0.25: 0x0, 0.75: 0x2, 1.25: 0x2, 1.75: 0x4, 2.5: 0x4, 3.5: 0x6, 5.0: 0x6}
+    for v, c in ties.items():
+        assert lib.orc_e2m1_encode(v) == c and lib.orc_e2m1_encode(-v) == c | 0x8, f"tie {v}"
+
+
+def pin_bf16_rounding(lib):
+    rng = np.random.default_rng(7)
+    # binary32 inputs: torch's float -> bfloat16 conversion is nearest-even
+    f = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32) * np.float32(3.0),
+        (rng.integers(0, 2 ** 32, 20000, dtype=np.uint64).astype(np.uint32)).view(np.float32),
+    ])
+    f = f[np.isfinite(f)]
+    mine = oracle.bf16_from_double(f.astype(np.float64), lib)
+    assert np.array_equal(mine, f32_to_bf16_bits_torch(f)), "bf16 rounding of binary32"
+    # binary64 inputs near bf16 midpoints: exact comparison with Fractions
+    b = rng.integers(1, 0x7F7F, 400).astype(np.uint16)
+    lo = bf16_bits_to_f64(b)
+    hi = bf16_bits_to_f64(b + 1)
+    cases = []
+    for a, c in zip(lo, hi):
+        mid = (a + c) / 2
+        cases += [mid, np.nextafter(mid, 0), np.nextafter(mid, np.inf), a, c]
+    for v in cases + [-x for x in cases]:
+        got = int(lib.orc_bf16_from_double(float(v)))
+        fv = Fraction(float(v))
+        base = int(np.array([np.float32(abs(float(v)))]).view(np.uint32)[0] >> 16)
+        best = None
+        for cand in range(max(base - 2, 0), base + 3):
+            d = abs(Fraction(float(bf16_bits_to_f64([cand])[0])) - abs(fv))
+            key = (d, cand & 1)
+            if best is None or key < best[0]:
+                best = (key, cand)
+        want = best[1] | (0x8000 if v < 0 else 0)
+        assert got == want, f"bf16 rounding of {v!r}: {got:#x} vs {want:#x}"
+    # ties go to even, and one bf16 step in [8, 16) is the page's 6.25e-2
+    pv = json.load(open(os.path.join(GOLDEN, "page_values.json")))["cases"][0]
+    step, low = pv["value"], pv["binade_low"]
+    assert lib.orc_bf16_to_double(lib.orc_bf16_from_double(low + step)) == low + step
+    assert lib.orc_bf16_to_double(lib.orc_bf16_from_double(low + step / 2)) == low
+    assert lib.orc_bf16_to_double(lib.orc_bf16_from_double(low + 1.5 * step)) == low + 2 * step
+    assert lib.orc_bf16_from_double(3.5e38) == 0x7F80
+
+
+def pin_mx_scale(lib):
+    bits, vals = all_finite_bf16()
+    pos = vals[vals > 0]
+    mine = oracle.mx_scale_code(pos, lib)
+    sample = np.concatenate([pos[::7], pos[:300], pos[-300:]])
+    want = np.array([brute_mx_scale_code(float(a)) for a in sample], dtype=np.uint8)
+    got = oracle.mx_scale_code(sample, lib)
+    assert np.array_equal(got, want), "E8M0 code vs exact power-of-two brackets"
+    # power-of-two boundaries: 2^k -> k - 2; the bf16 just below 2^k -> k - 3
+    for k in range(-120, 127):
+        assert lib.orc_mx_scale_code(2.0 ** k) == k - 2 + 127, f"2^{k}"
+        below = 2.0 ** k * (1 - 2 ** -8)
+        assert lib.orc_mx_scale_code(below) == max(k - 3 + 127, 0), f"below 2^{k}"
+    assert lib.orc_mx_scale_code(0.0) == 0
+    assert lib.orc_mx_scale_code(2.0 ** -133) == 0  # smallest bf16 subnormal
+    assert lib.orc_mx_scale_code(float("inf")) == 0xFF
+    assert np.all(mine <= 252)
+
+
+def pin_worked_rows(lib):
+    cases = {c["id"]: c for c in json.load(open(os.path.join(GOLDEN, "worked_rows.json")))["cases"]}
+    w1 = cases["W1"]
+    H = w1["H"]
+    x = bf16_bits_from_torch(torch.full((1, H), w1["x_value"], dtype=torch.bfloat16))
+    w = bf16_bits_from_torch(torch.full((H,), w1["w_value"], dtype=torch.bfloat16))
+    r = oracle.rmsnorm_quant([x], None, w, w1["eps"], oracle.FP8_PER_TOKEN, lib)
+    assert np.all(bf16_bits_to_f64(r["y"]) == w1["y_value"]), "W1 y"
+    assert r["scale"][0] == np.float32(w1["fp8_per_token"]["scale"]), "W1 scale"
+    assert np.all(r["q"] == int(w1["fp8_per_token"]["code"], 16)), "W1 codes"
+    r = oracle.rmsnorm_quant([x], None, w, w1["eps"], oracle.MXFP4, lib)
+    assert np.all(r["scale"] == w1["mxfp4"]["scale_code"]), "W1 MX scale"
+    assert np.all(r["q"] == int(w1["mxfp4"]["byte"], 16)), "W1 MX bytes"
+
+    w2 = cases["W2"]
+    y = np.zeros((1, w2["pad_to"]), dtype=np.float32)
+    y[0, :len(w2["y"])] = w2["y"]
+    q, s = oracle.quant_rows(f32_to_bf16_bits_torch(y), w2["mode"], lib)
+    assert s[0, 0] == np.float32(w2["scale"]), "W2 scale"
+    want = [int(c, 16) for c in w2["codes"]]
+    assert list(q[0, :len(want)]) == want, f"W2 codes {q[0, :3]}"
+    assert np.all(q[0, len(want):] == int(w2["pad_code"], 16))
+
+    w3 = cases["W3"]
+    y = np.zeros((1, w3["pad_to"]), dtype=np.float32)
+    y[0, :len(w3["y"])] = w3["y"]
+    q, s = oracle.quant_rows(f32_to_bf16_bits_torch(y), w3["mode"], lib)
+    assert s[0, 0] == w3["scale_code"], "W3 scale"
+    want = [int(c, 16) for c in w3["bytes"]]
+    assert list(q[0, :len(want)]) == want, f"W3 bytes {[hex(v) for v in q[0, :3]]}"
+    assert np.all(q[0, len(want):] == int(w3["pad_byte"], 16))
+
+    w4 = cases["W4"]
+    z = np.zeros((1, w4["H"]), dtype=np.uint16)
+    q, s = oracle.quant_rows(z, oracle.MXFP4, lib)
+    assert np.all(s == w4["mx_scale_code"]) and np.all(q == int(w4["mx_byte"], 16)), "W4 MX"
+    for mode in (oracle.FP8_PER_TOKEN, oracle.FP8_PER_GROUP128):
+        q, s = oracle.quant_rows(z, mode, lib)
+        assert np.all(s == w4["fp8_scale"]) and np.all(q == int(w4["fp8_code"], 16)), "W4 FP8"
+
+
+def pin_rstd_closed_form(lib):
+    for c in (0.5, 2.0, 3.0, -7.25, 1e-3, 100.0):
+        for H in (32, 96, 7168):
+            for eps in (1e-6, 1e-5, 0.0):
+                h = bf16_bits_from_torch(torch.full((H,), c, dtype=torch.bfloat16))
+                cb = float(bf16_bits_to_f64(h[:1])[0])
+                want = 1.0 / math.sqrt(cb * cb + float(np.float32(eps)))
+                got = oracle.rstd(h, eps, lib)
+                assert got == want, f"rstd c={c} H={H} eps={eps}: {got} vs {want}"
+                w = bf16_bits_from_torch(torch.full((H,), 1.25, dtype=torch.bfloat16))
+                r = oracle.rmsnorm_quant([h.reshape(1, H)], None, w, eps, oracle.MXFP4, lib)
+                yb = ref_y_bits([cb], [1.25], eps)[0]
+                assert np.all(r["y"] == yb), f"constant-row y c={c} H={H}"
+
+
+def pin_quant_stage_random(lib):
+    """Quantization stage on random bf16 rows vs the library/brute formulations."""
+    g = torch.Generator().manual_seed(11)
+    y = torch.randn((6, 512), generator=g) * torch.pow(10.0, torch.rand((6, 1), generator=g) * 4 - 2)
+    y[1, 5] *= 50.0
+    y[2, :128] = 0.0
+    y[3, 32:64] = 0.0
+    y[4, 64:96] = 2.0 ** -130  # subnormal block
+    yb = bf16_bits_from_torch(y.to(torch.bfloat16))
+    for mode, group in ((oracle.FP8_PER_TOKEN, 512), (oracle.FP8_PER_GROUP128, 128)):
+        q, s = oracle.quant_rows(yb, mode, lib)
+        rq, rs = ref_quant_fp8(yb, group)
+        assert np.array_equal(q, rq), f"FP8 codes mode {mode}"
+        assert np.array_equal(s.reshape(rs.shape), rs), f"FP8 scales mode {mode}"
+        # invariant: the largest element of a non-zero group encodes as +-448
+        for m in range(yb.shape[0]):
+            for gi in range(512 // group):
+                seg = bf16_bits_to_f64(yb[m, gi * group:(gi + 1) * group])
+                if np.any(seg != 0):
+                    j = int(np.argmax(np.abs(seg)))
+                    assert q[m, gi * group + j] & 0x7F == 0x7E, "amax element is 448"
+    q, s = oracle.quant_rows(yb, oracle.MXFP4, lib)
+    rq, rs = ref_quant_mx(yb)
+    assert np.array_equal(q, rq), "MXFP4 codes"
+    assert np.array_equal(s, rs), "MXFP4 scales"
+
+
+def _small_case(seed, M, H, P, residual):
+    g = torch.Generator().manual_seed(seed)
+    parts = []
+    for _ in range(P):
+        t = torch.randn((M, H), generator=g) * (torch.rand((M, 1), generator=g) * 8 + 0.1)
+        parts.append(bf16_bits_from_torch(t.to(torch.bfloat16)))
+    res = bf16_bits_from_torch(torch.randn((M, H), generator=g).to(torch.bfloat16)) if residual else None
+    w = bf16_bits_from_torch((1 + 0.3 * torch.randn((H,), generator=g)).to(torch.bfloat16))
+    return parts, res, w
+
+
+def pin_full_path_bruteforce(lib):
+    """Tiny rows: the whole unfused sequence recomputed independently."""
+    cases = [(1, 2, 32, 1, True, oracle.FP8_PER_TOKEN), (2, 3, 32, 2, True, oracle.MXFP4),
+             (3, 2, 64, 3, False, oracle.MXFP4), (4, 2, 128, 4, True, oracle.FP8_PER_GROUP128),
+             (5, 2, 256, 1, True, oracle.FP8_PER_GROUP128), (6, 1, 96, 4, True, oracle.FP8_PER_TOKEN)]
+    for seed, M, H, P, has_res, mode in cases:
+        parts, res, w = _small_case(seed, M, H, P, has_res)
+        eps = 1e-6 if seed % 2 else 1e-5
+        r = oracle.rmsnorm_quant(parts, res, w, eps, mode, lib)
+        h = ref_residual_bits(parts, res)
+        assert np.array_equal(r["residual_out"], h), f"residual case {seed}"
+        wv = bf16_bits_to_f64(w)
+        y = np.stack([ref_y_bits(bf16_bits_to_f64(h[m]), wv, eps) for m in range(M)])
+        assert np.array_equal(r["y"], y), f"y case {seed}"
+        if mode == oracle.MXFP4:
+            rq, rs = ref_quant_mx(y)
+        else:
+            rq, rs = ref_quant_fp8(y, H if mode == oracle.FP8_PER_TOKEN else 128)
+        assert np.array_equal(r["q"], rq), f"codes case {seed}"
+        assert np.array_equal(r["scale"].reshape(rs.shape), rs), f"scales case {seed}"
+
+
+def pin_partial_sum_order(lib):
+    """A3: fp32 sums in order p = 0..P-1, then the residual, one bf16 rounding."""
+    g = torch.Generator().manual_seed(21)
+    M, H, P = 16, 2048, 4
+    c = torch.pow(10.0, torch.rand((H,), generator=g) * 2 - 1)
+    parts = [bf16_bits_from_torch((torch.randn((M, H), generator=g) * c).to(torch.bfloat16))
+             for _ in range(P)]
+    res = bf16_bits_from_torch(torch.randn((M, H), generator=g).to(torch.bfloat16))
+    w = bf16_bits_from_torch(torch.ones((H,), dtype=torch.bfloat16))
+    # Rows where binary32 rounding of the running sum decides the bf16 result:
+    # p0 = s(1 + 2^-7), p1 = s 2^-30, r = -s 2^-8.  Exactly, h is just above
+    # the bf16 midpoint s(1 + 2^-8) and rounds up; in binary32, p0 + p1 drops
+    # the 2^-30 term, the sum lands on the midpoint and rounds to even (down).
+    k = np.arange(-20, 20)
+    s = 2.0 ** k
+    vals = [np.concatenate([s * (1 + 2 ** -7), -s * (1 + 2 ** -7)]),
+            np.concatenate([s * 2.0 ** -30, -s * 2.0 ** -30]),
+            np.concatenate([-s * 2.0 ** -8, s * 2.0 ** -8])]
+    cons = [f32_to_bf16_bits_torch(v.astype(np.float32)) for v in vals]
+    n = cons[0].size
+    for i in range(3):
+        tgt = parts[i] if i < 2 else res
+        tgt[0, :n] = cons[i]
+    for i in range(2, P):
+        parts[i][0, :n] = 0
+    r = oracle.rmsnorm_quant(parts, res, w, 1e-6, oracle.MXFP4, lib)
+    want = ref_residual_bits(parts, res)
+    assert np.array_equal(r["residual_out"], want), "fp32 partial sum order"
+    # the construction really separates the two orders of rounding
+    exact = [nearest_bf16_decimal(sum(Decimal(float(bf16_bits_to_f64([c[i]])[0])) for c in cons))
+             for i in range(n)]
+    assert not np.any(np.array(exact, dtype=np.uint16) == want[0, :n])
+
+
+def pin_qk_layout(lib):
+    """Interleaved q/gate heads, k after them, v never read; each head checked
+    against the decimal Gemma norm, each gate against its own source slice."""
+    M, Hq, Hk, D = 2, 3, 2, 32
+    stride = (2 * Hq + 2 * Hk) * D + 16  # v heads, then padding
+    g = torch.Generator().manual_seed(5)
+    qkv = torch.randn((M, stride), generator=g).to(torch.bfloat16)
+    # per head a distinct offset, so a misplaced slice cannot pass
+    for h in range(2 * Hq + Hk):
+        qkv[:, h * D:(h + 1) * D] += float(h + 1)
+    x = bf16_bits_from_torch(qkv)
+    x[:, (2 * Hq + Hk) * D:] = 0x7FC0  # v heads and padding: NaN, must not leak
+    qw = bf16_bits_from_torch((0.1 * torch.randn((D,), generator=g)).to(torch.bfloat16))
+    kw = bf16_bits_from_torch((0.1 * torch.randn((D,), generator=g)).to(torch.bfloat16))
+    r = oracle.qk_norm_gate(x, stride, Hq, Hk, D, qw, kw, 1e-6, lib)
+    qwv, kwv = bf16_bits_to_f64(qw), bf16_bits_to_f64(kw)
+    for m in range(M):
+        for h in range(Hq):
+            src = bf16_bits_to_f64(x[m, 2 * h * D:(2 * h + 1) * D])
+            assert np.array_equal(r["q"][m, h], ref_y_bits(src, qwv, 1e-6, gemma=True)), f"q {m},{h}"
+            assert np.array_equal(r["gate"][m, h], x[m, (2 * h + 1) * D:(2 * h + 2) * D]), f"gate {m},{h}"
+        for h in range(Hk):
+            off = 2 * Hq * D + h * D
+            src = bf16_bits_to_f64(x[m, off:off + D])
+            assert np.array_equal(r["k"][m, h], ref_y_bits(src, kwv, 1e-6, gemma=True)), f"k {m},{h}"
+
+
+ALL_PINS = [pin_e4m3_decode, pin_e4m3_encode, pin_e2m1, pin_bf16_rounding, pin_mx_scale,
+            pin_worked_rows, pin_rstd_closed_form, pin_quant_stage_random,
+            pin_full_path_bruteforce, pin_partial_sum_order, pin_qk_layout]
