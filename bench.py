@@ -1,0 +1,580 @@
+"""Benchmark of the fused residual-add + RMSNorm + quantization path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+A step is one fused call over the prefill MXFP4 workload (M=8192 rows of
+H=7168, P=4 same-device partial buffers summed in the kernel, residual add,
+RMSNorm, MXFP4 quantization): every step of the hot path on one batch.
+`value` is rows/s over all ranks (weak scaling: each rank owns its own 8192
+rows, no collective on the data path).  Inputs are larger than L2 (587 MB),
+so no flush is needed between steps.
+
+Rank 0 prints one JSON line.  It also carries, for N=1, the secondary
+workloads (large prefill group-128 in place, per-token decode at M=16, the
+decode sweep per mode, the QK prologue), each timed with CUDA events, and the
+CPU oracle timed on a bounded sample of the same workload.
+
+`--impl reference` times the CPU oracle instead (the method's plain
+definition; there is no runnable GPU reference for this path) on the same
+metric, one bounded sample of rows per step.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "rows/s and achieved HBM GB/s (% of B200 peak); µs/call at M≤16"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------
+# ranks
+# ---------------------------------------------------------------------------
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def dist_max(value: float, device) -> float:
+    """Max of a scalar over ranks (1 rank: the value itself)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own rows (independent problems)."""
+    return base + 1000 * rank
+
+
+def aggregate(rows_per_rank: int, world: int, ms_per_step_max: float) -> float:
+    """Whole-job rows/s: all ranks' rows over the slowest rank's step time."""
+    return rows_per_rank * world / (ms_per_step_max * 1e-3)
+
+
+# ---------------------------------------------------------------------------
+# clocks (read-only sampling of the GPU's clocks and throttle reasons)
+# ---------------------------------------------------------------------------
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, period_ms: int = 50):
+        self.proc = None
+        self.out = None
+        self.dev = device_index
+        self.period = period_ms
+
+    def _uuid(self):
+        import torch
+        try:
+            return "GPU-" + str(torch.cuda.get_device_properties(self.dev).uuid)
+        except Exception:
+            return None
+
+    def start(self):
+        uid = self._uuid()
+        if uid is None:
+            return
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", str(self.period)],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(self.period / 1000.0)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.seek(0)
+        rows = [ln.strip().split(", ") for ln in self.out.read().splitlines() if ln.strip()]
+        os.unlink(self.out.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[0]))
+                mx.append(float(r[1]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[4:8]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# GPU timing helpers
+# ---------------------------------------------------------------------------
+
+
+def time_steps(fn_step, steps: int, warmup: int, device, stream):
+    """Untimed warm-up, then `steps` calls bracketed by a barrier and a
+    synchronize, timed with CUDA events on the launching stream.
+    Returns ms per step on this rank."""
+    import torch
+    for _ in range(warmup):
+        fn_step()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    return e0.elapsed_time(e1) / steps
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mxfp4_quantization_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(f.encode())
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel_key: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; None otherwise."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        d = json.load(open(p))
+    except (OSError, ValueError):
+        return None
+    e = d.get(kernel_key)
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def hbm_peak():
+    try:
+        d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+
+
+def make_row_call(fn, wl, device, seed):
+    import torch
+    from mxfp4_quantization_b200 import synth
+    wl = synth.RowWorkload(**{**wl.__dict__, "seed": seed})
+    inp = wl.inputs(device=device)
+    parts, res, w = inp["parts"], inp["residual"], inp["weight"]
+    q, s = fn.alloc_outputs(wl.mode, wl.M, wl.H, device)
+    r_out = res if wl.in_place else torch.empty_like(res)
+    ptrs = [p.data_ptr() for p in parts]
+    stream = torch.cuda.current_stream(device)
+    sp = stream.cuda_stream
+
+    def step():
+        st = fn.fn_rmsnorm_quant(ptrs, len(ptrs), res.data_ptr(), w.data_ptr(), wl.eps, wl.mode,
+                                 wl.M, wl.H, q.data_ptr(), s.data_ptr(), r_out.data_ptr(), None,
+                                 sp)
+        if st != fn.FN_OK:
+            raise fn.FusedNormError("fn_rmsnorm_quant", st)
+
+    return step, stream, {"parts": parts, "residual": res, "weight": w, "q": q, "scale": s,
+                          "r_out": r_out}
+
+
+def e2e_row(fn, wl, device, steps, warmup, seed):
+    """Rows/s through the public tensor API from pinned host memory: each step
+    copies the step's inputs host->device, runs the fused call and reads the
+    quantized tuple (codes, scales, residual_out) back to pinned host memory."""
+    import torch
+    from mxfp4_quantization_b200 import synth
+    wl = synth.RowWorkload(**{**wl.__dict__, "seed": seed})
+    src = wl.inputs(device=device)
+    h_parts = [p.to("cpu").pin_memory() for p in src["parts"]]
+    h_res = src["residual"].to("cpu").pin_memory()
+    w = src["weight"]
+    d_parts = [torch.empty_like(p) for p in src["parts"]]
+    d_res = torch.empty_like(src["residual"])
+    q, s = fn.alloc_outputs(wl.mode, wl.M, wl.H, device)
+    d_rout = torch.empty_like(d_res)
+    h_q = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    h_s = torch.empty(s.shape, dtype=s.dtype, pin_memory=True)
+    h_rout = torch.empty(d_rout.shape, dtype=d_rout.dtype, pin_memory=True)
+    del src
+    h2d = sum(p.numel() * p.element_size() for p in h_parts) + h_res.numel() * 2
+    d2h = q.numel() * q.element_size() + s.numel() * s.element_size() + d_rout.numel() * 2
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        for hp, dp in zip(h_parts, d_parts):
+            dp.copy_(hp, non_blocking=True)
+        d_res.copy_(h_res, non_blocking=True)
+        fn.rmsnorm_quant(d_parts, w, wl.eps, wl.mode, residual=d_res, out_residual=d_rout,
+                         out_q=q, out_scale=s)
+        h_q.copy_(q, non_blocking=True)
+        h_s.copy_(s, non_blocking=True)
+        h_rout.copy_(d_rout, non_blocking=True)
+
+    ms = time_steps(step, steps, warmup, device, stream)
+    return ms, h2d, d2h
+
+
+def time_graph_calls(make_calls, n_sets, replays, device):
+    """µs per call of `n_sets` calls captured in one CUDA graph (median of
+    replays), plus one eager call's device time."""
+    import torch
+    calls = make_calls(n_sets)
+    s = torch.cuda.Stream(device)
+    s.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(s):
+        for c in calls[:3]:
+            c()
+        torch.cuda.synchronize(device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for c in calls:
+                c()
+    torch.cuda.synchronize(device)
+    g.replay()
+    torch.cuda.synchronize(device)
+    times = []
+    with torch.cuda.stream(s):
+        for _ in range(replays):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            g.replay()
+            e1.record(s)
+            torch.cuda.synchronize(device)
+            times.append(e0.elapsed_time(e1) * 1e3 / len(calls))
+        eager = []
+        for _ in range(20):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            calls[0]()
+            e1.record(s)
+            torch.cuda.synchronize(device)
+            eager.append(e0.elapsed_time(e1) * 1e3)
+    del g
+    return statistics.median(times), statistics.median(eager)
+
+
+def decode_calls(fn, wl, device):
+    """Factory of rotating-buffer calls for a small-M workload: enough input
+    sets that their total exceeds L2, so every call reads cold inputs."""
+    import torch
+
+    def make(n):
+        inp = wl.inputs(device=device)
+        parts0, res0, w = inp["parts"], inp["residual"], inp["weight"]
+        calls = []
+        for i in range(n):
+            parts = [p.roll(i, 0).clone() for p in parts0]
+            res = res0.roll(i, 0).clone()
+            q, s = fn.alloc_outputs(wl.mode, wl.M, wl.H, device)
+            r_out = torch.empty_like(res)
+            ptrs = [p.data_ptr() for p in parts]
+            keep = (parts, res, q, s, r_out)
+
+            def call(ptrs=ptrs, res=res, q=q, s=s, r_out=r_out, keep=keep):
+                sp = torch.cuda.current_stream(device).cuda_stream
+                st = fn.fn_rmsnorm_quant(ptrs, len(ptrs), res.data_ptr(), w.data_ptr(), wl.eps,
+                                         wl.mode, wl.M, wl.H, q.data_ptr(), s.data_ptr(),
+                                         r_out.data_ptr(), None, sp)
+                assert st == fn.FN_OK
+            calls.append(call)
+        return calls
+    return make
+
+
+def qk_calls(fn, wl, device):
+    import torch
+
+    def make(n):
+        inp = wl.inputs(device=device)
+        calls = []
+        for i in range(n):
+            qkv = inp["qkv"].roll(i, 0).clone()
+            out = fn.QKOutput(torch.empty((wl.M, wl.Hq, wl.D), dtype=torch.bfloat16, device=device),
+                              torch.empty((wl.M, wl.Hk, wl.D), dtype=torch.bfloat16, device=device),
+                              torch.empty((wl.M, wl.Hq, wl.D), dtype=torch.bfloat16, device=device))
+
+            def call(qkv=qkv, out=out):
+                fn.qk_norm_gate(qkv, wl.Hq, wl.Hk, wl.D, inp["q_weight"], inp["k_weight"],
+                                wl.eps, out=out)
+            calls.append(call)
+        return calls
+    return make
+
+
+def secondary_workloads(fn, device, peak):
+    """Every other workload, each on its own timed region (N=1 only)."""
+    import torch
+    from mxfp4_quantization_b200 import synth
+    res = {}
+    # large prefill, per-group-128, residual in place (inputs 1.07 GB > L2)
+    wl = synth.PREFILL_GROUP128
+    step, stream, keep = make_row_call(fn, wl, device, wl.seed)
+    ms = time_steps(step, 200, 5, device, stream)
+    b = wl.bytes_per_call()
+    res["prefill_group128"] = {"M": wl.M, "H": wl.H, "us_per_call": ms * 1e3,
+                               "rows_per_s": wl.M / (ms * 1e-3), "GB_s": b / (ms * 1e-3) / 1e9,
+                               "frac_of_peak": b / (ms * 1e-3) / 1e9 / peak,
+                               "bytes_per_call": b, "variant": fn.fn_last_variant()}
+    del keep
+    torch.cuda.empty_cache()
+
+    def small(wl, per_call_bytes, make):
+        n_sets = max(64, int(2 * L2_BYTES / per_call_bytes) + 1)
+        n_sets = min(n_sets, 8192)
+        us, eager = time_graph_calls(make, n_sets, 7, device)
+        return {"us_per_call_graph": us, "us_eager_device": eager, "calls_per_graph": n_sets,
+                "GB_s": per_call_bytes / (us * 1e-6) / 1e9}
+
+    wl = synth.PER_TOKEN_SMALL
+    r = small(wl, wl.bytes_per_call(), decode_calls(fn, wl, device))
+    r["variant"] = fn.fn_last_variant()
+    res["per_token_small"] = r
+    names = {synth.FP8_PER_TOKEN: "fp8_per_token", synth.FP8_PER_GROUP128: "fp8_per_group128",
+             synth.MXFP4: "mxfp4"}
+    dec = {}
+    for mode in (synth.FP8_PER_TOKEN, synth.FP8_PER_GROUP128, synth.MXFP4):
+        for M in synth.DECODE_M:
+            wl = synth.decode(M, mode)
+            r = small(wl, wl.bytes_per_call(), decode_calls(fn, wl, device))
+            r["variant"] = fn.fn_last_variant()
+            dec[f"{names[mode]}_m{M}"] = r
+        torch.cuda.empty_cache()
+    res["decode"] = dec
+    qk = {}
+    for M in synth.QK_M:
+        wl = synth.qk_prologue(M)
+        qk[f"m{M}"] = small(wl, wl.bytes_per_call(), qk_calls(fn, wl, device))
+    res["qk_prologue"] = qk
+    return res
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reported baseline; the reference arm)
+# ---------------------------------------------------------------------------
+
+
+def oracle_rows_per_s(rows: int, min_seconds: float, max_seconds: float, seed: int = 3):
+    """The oracle, as it stands, single-threaded, on `rows` rows of the prefill
+    MXFP4 recipe, repeated until `min_seconds` have passed."""
+    import oracle
+    from mxfp4_quantization_b200 import synth
+    wl = synth.RowWorkload(**{**synth.PREFILL_MXFP4.__dict__, "seed": seed})
+    inp = wl.inputs(device="cpu", M=rows)
+    parts = [synth.to_bits(p) for p in inp["parts"]]
+    res, w = synth.to_bits(inp["residual"]), synth.to_bits(inp["weight"])
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle.rmsnorm_quant(parts, res, w, wl.eps, wl.mode)
+        done += rows
+        el = time.perf_counter() - t0
+        if el >= min_seconds or el >= max_seconds:
+            break
+    return done / el, done, el
+
+
+def reference_arm(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    from mxfp4_quantization_b200 import synth
+    oracle.load()
+    wl = synth.PREFILL_MXFP4
+    rate, _, _ = oracle_rows_per_s(8, 0.5, 5.0)
+    budget_s = 90.0
+    rows_per_step = int(max(1, min(wl.M, rate * budget_s / max(1, args.steps + args.warmup))))
+    inp = synth.RowWorkload(**{**wl.__dict__}).inputs(device="cpu", M=rows_per_step)
+    parts = [synth.to_bits(p) for p in inp["parts"]]
+    res, w = synth.to_bits(inp["residual"]), synth.to_bits(inp["weight"])
+    for _ in range(args.warmup):
+        oracle.rmsnorm_quant(parts, res, w, wl.eps, wl.mode)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.rmsnorm_quant(parts, res, w, wl.eps, wl.mode)
+    el = time.perf_counter() - t0
+    value = rows_per_step * args.steps / el
+    sample = (f"{rows_per_step} rows of the prefill MXFP4 workload (H=7168, P=4) per step, "
+              f"single-threaded oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "prefill_mxfp4", "M": wl.M, "H": wl.H, "P": wl.P,
+                       "mode": "mxfp4", "rows_per_step": rows_per_step},
+            "cpu_baseline": {"value": value, "unit": "rows/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# main arm
+# ---------------------------------------------------------------------------
+
+
+def main_arm(args):
+    import torch
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        world = max(world, 1)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    init_dist(world, "nccl")
+    if rank == 0:
+        from mxfp4_quantization_b200.build import build_library
+        build_library()
+    barrier(device)
+    from mxfp4_quantization_b200 import fusednorm as fn
+    from mxfp4_quantization_b200 import synth
+
+    wl = synth.PREFILL_MXFP4
+    seed = rank_seed(wl.seed, rank)
+    step, stream, keep = make_row_call(fn, wl, device, seed)
+    clocks = ClockSampler(local)
+    # warm-up outside the sampled region, then sample clocks over the timed steps
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    clocks.start()
+    ms = time_steps(step, args.steps, 0, device, stream)
+    clk = clocks.stop()
+    variant, launch = fn.fn_last_variant(), fn.fn_last_launch()
+    ms_max = dist_max(ms, device)
+    value = aggregate(wl.M, world, ms_max)
+    bytes_call = wl.bytes_per_call()
+    peak, peak_kind = hbm_peak()
+    achieved = bytes_call / (ms * 1e-3) / 1e9
+    del keep
+    torch.cuda.empty_cache()
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_ms, h2d, d2h = e2e_row(fn, wl, device, e2e_steps, 2, seed)
+    e2e_ms_max = dist_max(e2e_ms, device)
+
+    extra = None
+    cpu = None
+    if world == 1 and not args.no_extras:
+        extra = secondary_workloads(fn, device, peak)
+    if world == 1 and not args.no_cpu_baseline:
+        rate, rows, el = oracle_rows_per_s(256, args.cpu_seconds, 3 * args.cpu_seconds)
+        cpu = {"value": rate, "unit": "rows/s", "cores": 1, "kind": "oracle",
+               "sample": f"{rows} rows (256 rows of the prefill MXFP4 recipe, H=7168, P=4, "
+                         f"repeated) in {el:.1f} s, single-threaded; "
+                         f"host has {os.cpu_count()} cores"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "prefill_mxfp4", "M": wl.M, "H": wl.H, "P": wl.P,
+                       "mode": "mxfp4", "eps": wl.eps, "rows_per_gpu": wl.M,
+                       "io": "bf16 in; E2M1 codes + E8M0 scales + bf16 residual out",
+                       "l2": "inputs larger than L2 (587 MB per step), no flush",
+                       "parallelism": f"dp{world} (independent rows, no collective)"},
+            "hbm_GB_s": achieved, "frac_of_peak": achieved / peak,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": peak_kind,
+                         "traffic": measured_traffic("rq_mxfp4_p4_h7168"),
+                         "algorithmic_bytes_per_launch": bytes_call,
+                         "kernel": "rq_kernel<MXFP4, P<=4, V=4>",
+                         "launch": list(launch), "variant": variant},
+            "e2e": {"value": aggregate(wl.M, world, e2e_ms_max), "unit": "rows/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps},
+            "gpu_launches": args.steps,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+            "workloads": extra,
+        }
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        barrier(device)
+        dist.destroy_process_group()
+    return 0
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    a = ap.parse_args(argv)
+    a.warmup = max(a.warmup, 3)  # timing rule: at least 3 untimed warm-up steps
+    return a
+
+
+if __name__ == "__main__":
+    args = parse()
+    sys.exit(reference_arm(args) if args.impl == "reference" else main_arm(args))

@@ -1,0 +1,171 @@
+/*
+ * fusednorm.h — C ABI of the B200 (sm_100a) fused residual-add + RMSNorm +
+ * activation-quantization library, libfusednorm.so.
+ *
+ * Sources (page title, then section):
+ *  - sglang PR #29723, "Fused AllReduce + RMSNorm + per-token FP8 / MXFP4 quant
+ *    on AMD (AITER)", "Modifications": the fused call returns the tuple
+ *    (fp8_output, residual_out, per_token_scale) with the scale shaped (M, 1),
+ *    or signals "cannot fuse" before any work; "Accuracy Tests": the fused
+ *    kernel equals the unfused AllReduce -> RMSNorm -> quantize sequence.
+ *    Review comments: a failure after collective entry must not turn into a
+ *    silent per-rank fallback; the carried output dtype must not be lost.
+ *  - sgl-amd-mono PR #26, "Whole-layer monokernels for Muse Spark", commit
+ *    notes: online MXFP4 quantization of the bf16 normed row, bit-exact
+ *    against the stand-alone quantization of that row.
+ *  - sglang PR #27656, "Fuse QK RMSNorm + gate extraction Triton kernel for
+ *    Qwen3.5 on HIP", "Motivation"/"Modifications": one kernel reads q and gate
+ *    from the interleaved [q_h0, gate_h0, q_h1, gate_h1, ...] projection output
+ *    with strides, applies GemmaRMSNorm to q and k, and writes contiguous q, k
+ *    and gate.
+ *  - OCP Microscaling (MX) v1.0: MXFP4 = E2M1 elements, one E8M0 scale per
+ *    32-element block, X = 2^(floor(log2 amax) - 2).
+ *
+ * The cross-GPU all-reduce in front of the norm is replaced by an in-kernel
+ * sum of up to 8 partial buffers that live on the same device.
+ *
+ * Conventions for every entry point:
+ *  - bf16 tensors are IEEE bfloat16 bit patterns, row-major, contiguous rows
+ *    (row stride H elements unless a stride argument says otherwise).
+ *  - Every data pointer is a DEVICE pointer owned by the caller.  The library
+ *    allocates nothing, keeps no state besides a thread-local record of the
+ *    last dispatch, and never synchronizes: work is queued on `stream`
+ *    (a cudaStream_t passed as void*; NULL means the legacy default stream).
+ *  - All argument checks run on the host before anything is launched; on any
+ *    error nothing is launched and no output is touched.  M == 0 returns
+ *    FN_OK and launches nothing.
+ *  - A launch that the CUDA runtime rejects returns FN_ERR_CUDA.
+ *  - Calls are thread-safe.  The kernels contain no spin-waits and no flags
+ *    shared between thread blocks.
+ */
+#ifndef FUSEDNORM_H
+#define FUSEDNORM_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FN_API __attribute__((visibility("default")))
+#else
+#define FN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Quantization of the normed row y (sglang PR #29723, "Modifications"). */
+typedef enum {
+    FN_FP8_PER_TOKEN = 0,    /* E4M3, one fp32 scale per row: scale [M]          */
+    FN_FP8_PER_GROUP128 = 1, /* E4M3, one fp32 scale per 128 elements [M, H/128] */
+    FN_MXFP4 = 2             /* E2M1 codes, one E8M0 byte per 32 elements [M, H/32] */
+} fn_mode;
+
+typedef enum {
+    FN_OK = 0,
+    FN_ERR_INVALID = -1,     /* null pointer, bad size, bad mode, forbidden overlap */
+    FN_ERR_ALIGN = -2,       /* a pointer or stride breaks the alignment rule      */
+    FN_ERR_UNSUPPORTED = -3, /* valid request outside the built shapes (e.g. H)    */
+    FN_ERR_CUDA = -4,        /* the CUDA runtime rejected the launch               */
+    FN_ERR_TIMEOUT = -5      /* reserved: no kernel here waits on another          */
+} fn_status;
+
+/* Which kernel the calling thread's last successful call launched. */
+typedef enum {
+    FN_VARIANT_NONE = 0,        /* nothing launched (M == 0 or an error)          */
+    FN_VARIANT_ROW_CTA = 1,     /* one thread block per row                        */
+    FN_VARIANT_ROW_CLUSTER = 2, /* a cluster of 2..8 blocks per row (small M)      */
+    FN_VARIANT_QUANT_ONLY = 3,  /* fn_quant                                        */
+    FN_VARIANT_QK_WARP = 4      /* fn_qk_norm_gate: one warp per (token, head)     */
+} fn_variant;
+
+#define FN_MAX_PARTS 8
+#define FN_MAX_H 32768
+#define FN_MAX_HEAD_DIM 1024
+
+/*
+ * Fused (partial sum) + residual add + RMSNorm + quantization over M rows of
+ * H elements.  Per row, with every add in fp32:
+ *     h  = bf16_rn( ((x_0 + x_1) + ... + x_{P-1}) + residual )
+ *     residual_out = h
+ *     y  = bf16_rn( h * rsqrt(mean(h^2) + eps) * weight )
+ *     (out_q, out_scale) = quantize(y, mode)
+ *   FP8 modes:  scale = amax / 448 (fp32 division; 1.0 when amax == 0),
+ *               code  = E4M3 round-to-nearest-even, saturating, of y / scale.
+ *   MXFP4:      per 32-element block e = floor(log2 amax) - 2 clamped to
+ *               [-127, 127], scale byte = e + 127 (0 for an all-zero block),
+ *               code = E2M1 round-to-nearest-even, saturating to 6, of
+ *               y * 2^-e; element 2i in the low nibble of byte i.
+ *
+ * x_parts      HOST array of num_parts DEVICE pointers, each bf16 [M, H].
+ * num_parts    P, 1..FN_MAX_PARTS.
+ * residual     bf16 [M, H], or NULL (no residual add).
+ * weight       bf16 [H].
+ * eps          finite, >= 0.
+ * mode         fn_mode.
+ * M, H         M >= 0; H % 8 == 0, 8 <= H <= FN_MAX_H; H % 128 == 0 for
+ *              FN_FP8_PER_GROUP128, H % 32 == 0 for FN_MXFP4.
+ * out_q        FP8: u8 [M, H]; MXFP4: u8 [M, H/2].
+ * out_scale    FN_FP8_PER_TOKEN: fp32 [M]; FN_FP8_PER_GROUP128: fp32 [M, H/128];
+ *              FN_MXFP4: u8 E8M0 [M, H/32].  All row-major.
+ * out_residual bf16 [M, H].  Required when residual != NULL and may then be
+ *              the residual pointer itself (in-place update).  With residual
+ *              == NULL it is optional and receives the partial sum h.
+ * out_y        bf16 [M, H] normed row (the "emit bf16" side output), or NULL.
+ * Alignment    every bf16 pointer 16 bytes; out_q 8 bytes; out_scale 4 bytes
+ *              for fp32 scales.  Otherwise FN_ERR_ALIGN.
+ * Overlap      outputs must not overlap each other or any input, except
+ *              out_residual == residual exactly.  Otherwise FN_ERR_INVALID.
+ */
+FN_API int fn_rmsnorm_quant(const void* const* x_parts, int num_parts, const void* residual,
+                     const void* weight, float eps, int mode, int64_t M, int64_t H,
+                     void* out_q, void* out_scale, void* out_residual, void* out_y,
+                     void* stream);
+
+/*
+ * The quantization step alone on existing bf16 rows y [M, H] (the third
+ * launch of the unfused AllReduce -> RMSNorm -> quantize sequence in sglang
+ * PR #29723; the stand-alone row quantization the monokernel notes compare
+ * against).  Same modes, layouts, alignment and overlap rules as
+ * fn_rmsnorm_quant; runs the same device code as its quantization stage.
+ */
+FN_API int fn_quant(const void* y, int mode, int64_t M, int64_t H, void* out_q, void* out_scale,
+             void* stream);
+
+/*
+ * QK Gemma-RMSNorm + gate extraction (sglang PR #27656, "Motivation").
+ * Token m's row starts at qkv + m * row_stride (elements).  Within it, q head
+ * h (h < Hq) is at [2hD, 2hD + D), its gate at [(2h+1)D, (2h+2)D), and k head
+ * h (h < Hk) at [2 Hq D + hD, 2 Hq D + (h+1)D); what follows (v) is not read.
+ *     out_q[m,h,:]    = bf16_rn( q * rsqrt(mean(q^2) + eps) * (1 + q_weight) )
+ *     out_k[m,h,:]    = bf16_rn( k * rsqrt(mean(k^2) + eps) * (1 + k_weight) )
+ *     out_gate[m,h,:] = gate (bit copy)
+ * qkv          bf16, M rows of row_stride elements; 16-byte aligned.
+ * row_stride   elements, multiple of 8, >= (2 Hq + Hk) D.
+ * Hq, Hk       >= 0 (Hq + Hk >= 1).   D: multiple of 8, 8..FN_MAX_HEAD_DIM.
+ * q_weight, k_weight   bf16 [D] (k_weight may be NULL when Hk == 0).
+ * out_q [M,Hq,D], out_k [M,Hk,D], out_gate [M,Hq,D]: bf16, contiguous,
+ *              16-byte aligned, no overlap with each other or with qkv.
+ */
+FN_API int fn_qk_norm_gate(const void* qkv, int64_t M, int64_t row_stride, int Hq, int Hk, int D,
+                    const void* q_weight, const void* k_weight, float eps, void* out_q,
+                    void* out_k, void* out_gate, void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+FN_API const char* fn_status_string(int status);
+
+/* fn_variant of the calling thread's last call (FN_VARIANT_NONE after an error). */
+FN_API int fn_last_variant(void);
+
+/* Launch shape of the calling thread's last launch: out[0] grid blocks,
+ * out[1] threads per block, out[2] blocks per cluster (1 = none),
+ * out[3] elements per thread-vector group (vectors of 8 bf16 per thread). */
+FN_API void fn_last_launch(int32_t out[4]);
+
+/* Library ABI version (major * 100 + minor). */
+FN_API int fn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FUSEDNORM_H */

@@ -1,0 +1,136 @@
+// Device helpers for the sm_100a kernels: 128-bit streaming loads/stores,
+// bf16 packing, and the packed E4M3 / E2M1 conversions (PTX `cvt` with
+// round-to-nearest-even and saturation to the largest finite value).
+#pragma once
+#include <cstdint>
+
+namespace fn {
+
+// ---- memory -----------------------------------------------------------------
+
+// Read-only input that no output aliases: non-coherent path, no L1 allocation
+// (each byte is read once).
+__device__ __forceinline__ uint4 ld_stream_nc(const uint4* p) {
+  uint4 r;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
+}
+
+// Input that an output may alias in place (the residual): coherent load.
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// Small, reused operand (the norm weight): normal cached read-only load.
+__device__ __forceinline__ uint4 ld_keep(const uint4* p) { return __ldg(p); }
+
+__device__ __forceinline__ void st_stream(uint4* p, uint4 v) {
+  asm volatile("st.global.L1::no_allocate.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_stream(uint2* p, uint2 v) {
+  asm volatile("st.global.L1::no_allocate.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x), "r"(v.y)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_stream(uint32_t* p, uint32_t v) {
+  asm volatile("st.global.L1::no_allocate.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// ---- bf16 -------------------------------------------------------------------
+
+// Element 2i of a packed pair lives in the low half (little-endian memory).
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Two fp32 -> packed bf16 pair, each rounded to nearest even (subnormals kept).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t word(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+__device__ __forceinline__ void set_word(uint4& v, int i, uint32_t w) {
+  if (i == 0) v.x = w;
+  else if (i == 1) v.y = w;
+  else if (i == 2) v.z = w;
+  else v.w = w;
+}
+
+// ---- FP8 E4M3 -----------------------------------------------------------------
+
+// Two fp32 -> two E4M3 codes (nearest even, saturating to +-448); `lo` lands in
+// the low byte.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// ---- FP4 E2M1 -----------------------------------------------------------------
+
+// Eight fp32 -> eight E2M1 codes (nearest even, saturating to +-6) packed in a
+// 32-bit word: element 2i in the low nibble of byte i.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
+  uint32_t d;
+  asm("{\n\t"
+      ".reg .b8 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+      "mov.b32 %0, {q0, q1, q2, q3};\n\t"
+      "}"
+      : "=r"(d)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+        "f"(v[7]));
+  return d;
+}
+
+// ---- reductions ------------------------------------------------------------------
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Max over aligned groups of `G` lanes (G a power of two, <= 32).
+template <int G>
+__device__ __forceinline__ float group_max(float v) {
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// MX block exponent from the block amax (a non-negative value of a bf16):
+// e = floor(log2 amax) - 2, clamped to [-127, 127]; zero and bf16 subnormals
+// (binary32 exponent field 0) give -127.  Returns the E8M0 code e + 127, and
+// 2^-e (always a normal binary32, since e <= 125) in `inv`.  A NaN or
+// infinite amax gives code 0xFF.
+__device__ __forceinline__ uint32_t mx_scale(float amax, float& inv) {
+  uint32_t ef = __float_as_uint(amax) >> 23;  // sign is 0
+  int e = (ef == 0) ? -127 : max((int)ef - 129, -127);
+  inv = __uint_as_float((uint32_t)(127 - e) << 23);
+  return ef == 0xFF ? 0xFFu : (uint32_t)(e + 127);
+}
+
+}  // namespace fn

@@ -1,0 +1,339 @@
+// Host side of libfusednorm.so: argument checks, dispatch, launches.
+// The C ABI and its contract are declared in include/fusednorm.h.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "fusednorm.h"
+#include "qk_kernel.cuh"
+#include "rq_params.h"
+
+namespace {
+
+thread_local int tl_variant = FN_VARIANT_NONE;
+thread_local int32_t tl_launch[4] = {0, 0, 0, 0};
+
+struct Range {
+  uintptr_t lo, hi;  // [lo, hi)
+};
+
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+Range range_of(const void* p, int64_t bytes) {
+  const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+  return Range{lo, lo + static_cast<uintptr_t>(bytes)};
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return n;
+}
+
+int round32(int x) { return (x + 31) / 32 * 32; }
+
+// ---- rmsnorm_quant / quant dispatch -----------------------------------------
+
+using fn::RQKernel;
+
+// Kernel instance for (mode, P, V, cluster, norm).
+RQKernel pick_kernel(int mode, int P, int V, bool cluster, bool norm) {
+  const int maxp = (!norm || P == 1) ? 1 : P == 2 ? 2 : P <= 4 ? 4 : 8;
+#define FN_CASE(MODE, MAXP) \
+  if (mode == MODE && maxp == MAXP) return fn::rq_pick_##MODE##_##MAXP(V, cluster, norm);
+  FN_CASE(0, 1) FN_CASE(0, 2) FN_CASE(0, 4) FN_CASE(0, 8)
+  FN_CASE(1, 1) FN_CASE(1, 2) FN_CASE(1, 4) FN_CASE(1, 8)
+  FN_CASE(2, 1) FN_CASE(2, 2) FN_CASE(2, 4) FN_CASE(2, 8)
+#undef FN_CASE
+  return nullptr;
+}
+
+// Smallest power-of-two V in {1..16} with ceil(nvec / V) <= 256 threads.
+int row_vectors_per_thread(int nvec) {
+  int V = 1;
+  while (V < 16 && (nvec + V - 1) / V > 256) V *= 2;
+  return V;
+}
+
+// Cluster size for a small-M launch: the largest C in 2..8 that splits the
+// row into equal segments aligned to the quantization group, each at most 512
+// vectors, with M * C blocks fitting on the GPU at once.  0 when none fits.
+int pick_cluster(int64_t M, int nvec, int mode, int sms) {
+  const int align = mode == FN_FP8_PER_GROUP128 ? 16 : mode == FN_MXFP4 ? 4 : 1;
+  for (int C = 8; C >= 2; --C) {
+    if (nvec % C) continue;
+    const int seg = nvec / C;
+    if (seg % align || seg > 512 || seg < 32) continue;
+    if (M * C > sms) continue;
+    return C;
+  }
+  return 0;
+}
+
+int check_mode_shape(int mode, int64_t M, int64_t H) {
+  if (mode < FN_FP8_PER_TOKEN || mode > FN_MXFP4) return FN_ERR_INVALID;
+  if (M < 0 || H <= 0 || H % 8) return FN_ERR_INVALID;
+  if (mode == FN_FP8_PER_GROUP128 && H % 128) return FN_ERR_INVALID;
+  if (mode == FN_MXFP4 && H % 32) return FN_ERR_INVALID;
+  if (H > FN_MAX_H) return FN_ERR_UNSUPPORTED;
+  if (M > (int64_t)INT32_MAX / 8) return FN_ERR_UNSUPPORTED;  // grid size
+  return FN_OK;
+}
+
+int64_t code_bytes(int mode, int64_t M, int64_t H) { return mode == FN_MXFP4 ? M * H / 2 : M * H; }
+
+int64_t scale_bytes(int mode, int64_t M, int64_t H) {
+  if (mode == FN_FP8_PER_TOKEN) return M * 4;
+  if (mode == FN_FP8_PER_GROUP128) return M * (H / 128) * 4;
+  return M * (H / 32);
+}
+
+int check_outputs_align(int mode, const void* out_q, const void* out_scale) {
+  if (!aligned(out_q, mode == FN_MXFP4 ? 4 : 8)) return FN_ERR_ALIGN;
+  if (mode != FN_MXFP4 && !aligned(out_scale, 4)) return FN_ERR_ALIGN;
+  return FN_OK;
+}
+
+int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, void* stream,
+              int variant_if_norm) {
+  const int nvec = prm.nvec;
+  const int sms = sm_count();
+  if (sms <= 0) return FN_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  fn::RQParams p = prm;
+
+  const int C = norm ? pick_cluster(M, nvec, mode, sms) : 0;
+  if (C >= 2) {
+    p.seg = nvec / C;
+    const int threads = round32(p.seg);
+    RQKernel k = pick_kernel(mode, P, 1, true, true);
+    if (!k) return FN_ERR_UNSUPPORTED;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(M * C));
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k, p) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return FN_ERR_CUDA;
+    }
+    tl_variant = FN_VARIANT_ROW_CLUSTER;
+    tl_launch[0] = (int32_t)(M * C);
+    tl_launch[1] = threads;
+    tl_launch[2] = C;
+    tl_launch[3] = 1;
+  } else {
+    const int V = row_vectors_per_thread(nvec);
+    p.seg = nvec;
+    const int threads = round32((nvec + V - 1) / V);
+    RQKernel k = pick_kernel(mode, P, V, false, norm);
+    if (!k) return FN_ERR_UNSUPPORTED;
+    k<<<(unsigned)M, threads, 0, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return FN_ERR_CUDA;
+    tl_variant = norm ? variant_if_norm : FN_VARIANT_QUANT_ONLY;
+    tl_launch[0] = (int32_t)M;
+    tl_launch[1] = threads;
+    tl_launch[2] = 1;
+    tl_launch[3] = V;
+  }
+  return FN_OK;
+}
+
+template <int VPL>
+int launch_qk_v(const fn::QKParams& p, int64_t items, int sms, cudaStream_t st) {
+  const int wpb = items <= (int64_t)8 * sms ? 1 : 8;
+  const int64_t blocks = (items + wpb - 1) / wpb;
+  fn::qk_kernel<VPL><<<(unsigned)blocks, wpb * 32, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return FN_ERR_CUDA;
+  tl_launch[0] = (int32_t)blocks;
+  tl_launch[1] = wpb * 32;
+  tl_launch[2] = 1;
+  tl_launch[3] = VPL;
+  return FN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fn_version(void) { return 100; }
+
+int fn_last_variant(void) { return tl_variant; }
+
+void fn_last_launch(int32_t out[4]) {
+  if (out) std::memcpy(out, tl_launch, sizeof tl_launch);
+}
+
+const char* fn_status_string(int status) {
+  switch (status) {
+    case FN_OK: return "ok";
+    case FN_ERR_INVALID: return "invalid argument (null pointer, size, mode or overlap)";
+    case FN_ERR_ALIGN: return "misaligned pointer or stride";
+    case FN_ERR_UNSUPPORTED: return "shape outside the built kernels";
+    case FN_ERR_CUDA: return "CUDA launch failed";
+    case FN_ERR_TIMEOUT: return "timed out";
+    default: return "unknown status";
+  }
+}
+
+int fn_rmsnorm_quant(const void* const* x_parts, int num_parts, const void* residual,
+                     const void* weight, float eps, int mode, int64_t M, int64_t H,
+                     void* out_q, void* out_scale, void* out_residual, void* out_y,
+                     void* stream) {
+  tl_variant = FN_VARIANT_NONE;
+  if (!x_parts || num_parts < 1 || num_parts > FN_MAX_PARTS) return FN_ERR_INVALID;
+  int rc = check_mode_shape(mode, M, H);
+  if (rc != FN_OK) return rc;
+  if (!std::isfinite(eps) || eps < 0.f) return FN_ERR_INVALID;
+  if (!weight || !out_q || !out_scale) return FN_ERR_INVALID;
+  if (residual && !out_residual) return FN_ERR_INVALID;
+  for (int p = 0; p < num_parts; ++p) {
+    if (!x_parts[p]) return FN_ERR_INVALID;
+    if (!aligned(x_parts[p], 16)) return FN_ERR_ALIGN;
+  }
+  if (!aligned(weight, 16) || (residual && !aligned(residual, 16)) ||
+      (out_residual && !aligned(out_residual, 16)) || (out_y && !aligned(out_y, 16)))
+    return FN_ERR_ALIGN;
+  if ((rc = check_outputs_align(mode, out_q, out_scale)) != FN_OK) return rc;
+
+  const int64_t row_bytes = M * H * 2;
+  Range outs[4];
+  int no = 0;
+  outs[no++] = range_of(out_q, code_bytes(mode, M, H));
+  outs[no++] = range_of(out_scale, scale_bytes(mode, M, H));
+  if (out_residual) outs[no++] = range_of(out_residual, row_bytes);
+  if (out_y) outs[no++] = range_of(out_y, row_bytes);
+  if (M > 0) {
+    for (int i = 0; i < no; ++i)
+      for (int j = i + 1; j < no; ++j)
+        if (overlap(outs[i], outs[j])) return FN_ERR_INVALID;
+    Range ins[FN_MAX_PARTS + 2];
+    int ni = 0;
+    for (int p = 0; p < num_parts; ++p) ins[ni++] = range_of(x_parts[p], row_bytes);
+    ins[ni++] = range_of(weight, H * 2);
+    const Range res_in = residual ? range_of(residual, row_bytes) : Range{0, 0};
+    for (int i = 0; i < no; ++i) {
+      for (int j = 0; j < ni; ++j)
+        if (overlap(outs[i], ins[j])) return FN_ERR_INVALID;
+      if (residual && overlap(outs[i], res_in) &&
+          !(out_residual == residual && i == 2))
+        return FN_ERR_INVALID;
+    }
+  }
+  if (M == 0) return FN_OK;
+
+  fn::RQParams prm;
+  std::memset(&prm, 0, sizeof prm);
+  for (int p = 0; p < num_parts; ++p) prm.parts[p] = static_cast<const uint4*>(x_parts[p]);
+  prm.residual = static_cast<const uint4*>(residual);
+  prm.weight = static_cast<const uint4*>(weight);
+  prm.out_residual = static_cast<uint4*>(out_residual);
+  prm.out_y = static_cast<uint4*>(out_y);
+  prm.out_q = static_cast<uint8_t*>(out_q);
+  prm.out_scale = out_scale;
+  prm.M = M;
+  prm.nvec = (int)(H / 8);
+  prm.P = num_parts;
+  prm.eps = eps;
+  return launch_rq(prm, mode, num_parts, M, true, stream, FN_VARIANT_ROW_CTA);
+}
+
+int fn_quant(const void* y, int mode, int64_t M, int64_t H, void* out_q, void* out_scale,
+             void* stream) {
+  tl_variant = FN_VARIANT_NONE;
+  int rc = check_mode_shape(mode, M, H);
+  if (rc != FN_OK) return rc;
+  if (!y || !out_q || !out_scale) return FN_ERR_INVALID;
+  if (!aligned(y, 16)) return FN_ERR_ALIGN;
+  if ((rc = check_outputs_align(mode, out_q, out_scale)) != FN_OK) return rc;
+  if (M > 0) {
+    const Range in = range_of(y, M * H * 2);
+    const Range q = range_of(out_q, code_bytes(mode, M, H));
+    const Range s = range_of(out_scale, scale_bytes(mode, M, H));
+    if (overlap(in, q) || overlap(in, s) || overlap(q, s)) return FN_ERR_INVALID;
+  }
+  if (M == 0) return FN_OK;
+  fn::RQParams prm;
+  std::memset(&prm, 0, sizeof prm);
+  prm.parts[0] = static_cast<const uint4*>(y);
+  prm.out_q = static_cast<uint8_t*>(out_q);
+  prm.out_scale = out_scale;
+  prm.M = M;
+  prm.nvec = (int)(H / 8);
+  prm.P = 1;
+  return launch_rq(prm, mode, 1, M, false, stream, FN_VARIANT_QUANT_ONLY);
+}
+
+int fn_qk_norm_gate(const void* qkv, int64_t M, int64_t row_stride, int Hq, int Hk, int D,
+                    const void* q_weight, const void* k_weight, float eps, void* out_q,
+                    void* out_k, void* out_gate, void* stream) {
+  tl_variant = FN_VARIANT_NONE;
+  if (M < 0 || Hq < 0 || Hk < 0 || Hq + Hk < 1 || D <= 0 || D % 8) return FN_ERR_INVALID;
+  if (D > FN_MAX_HEAD_DIM) return FN_ERR_UNSUPPORTED;
+  if (row_stride % 8 || row_stride < (int64_t)(2 * Hq + Hk) * D) return FN_ERR_INVALID;
+  if (!std::isfinite(eps) || eps < 0.f) return FN_ERR_INVALID;
+  if (!qkv || (Hq > 0 && (!q_weight || !out_q || !out_gate)) || (Hk > 0 && (!k_weight || !out_k)))
+    return FN_ERR_INVALID;
+  if (!aligned(qkv, 16) || (q_weight && !aligned(q_weight, 16)) ||
+      (k_weight && !aligned(k_weight, 16)) || (out_q && !aligned(out_q, 16)) ||
+      (out_k && !aligned(out_k, 16)) || (out_gate && !aligned(out_gate, 16)))
+    return FN_ERR_ALIGN;
+  if (M > (int64_t)INT32_MAX / 8 || (int64_t)M * (Hq + Hk) > (int64_t)INT32_MAX)
+    return FN_ERR_UNSUPPORTED;
+  if (M > 0) {
+    const Range in = range_of(qkv, ((M - 1) * row_stride + (int64_t)(2 * Hq + Hk) * D) * 2);
+    Range outs[3];
+    int no = 0;
+    if (Hq > 0) {
+      outs[no++] = range_of(out_q, M * Hq * D * 2);
+      outs[no++] = range_of(out_gate, M * Hq * D * 2);
+    }
+    if (Hk > 0) outs[no++] = range_of(out_k, M * Hk * D * 2);
+    for (int i = 0; i < no; ++i) {
+      if (overlap(outs[i], in)) return FN_ERR_INVALID;
+      if (q_weight && overlap(outs[i], range_of(q_weight, D * 2))) return FN_ERR_INVALID;
+      if (k_weight && overlap(outs[i], range_of(k_weight, D * 2))) return FN_ERR_INVALID;
+      for (int j = i + 1; j < no; ++j)
+        if (overlap(outs[i], outs[j])) return FN_ERR_INVALID;
+    }
+  }
+  if (M == 0) return FN_OK;
+  const int sms = sm_count();
+  if (sms <= 0) return FN_ERR_CUDA;
+  fn::QKParams p;
+  p.qkv = static_cast<const uint4*>(qkv);
+  p.M = M;
+  p.row_vec = row_stride / 8;
+  p.Hq = Hq;
+  p.Hk = Hk;
+  p.dv = D / 8;
+  p.qw = static_cast<const uint4*>(q_weight);
+  p.kw = static_cast<const uint4*>(k_weight);
+  p.eps = eps;
+  p.out_q = static_cast<uint4*>(out_q);
+  p.out_k = static_cast<uint4*>(out_k);
+  p.out_g = static_cast<uint4*>(out_gate);
+  const int64_t items = M * (Hq + Hk);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc;
+  const int nv = D / 8;
+  if (nv <= 32) rc = launch_qk_v<1>(p, items, sms, st);
+  else if (nv <= 64) rc = launch_qk_v<2>(p, items, sms, st);
+  else rc = launch_qk_v<4>(p, items, sms, st);
+  if (rc == FN_OK) tl_variant = FN_VARIANT_QK_WARP;
+  return rc;
+}
+
+}  // extern "C"

@@ -1,0 +1,85 @@
+// QK Gemma-RMSNorm + gate extraction, sm_100a (sglang PR #27656, "Motivation":
+// one kernel in place of the q copy, the gate copy and the q/k norm).
+//
+// One warp per (token, head).  A q head and its gate are adjacent in the
+// interleaved row ([q_h, gate_h] = 2D contiguous elements), so the warp that
+// normalizes q_h also copies gate_h; k heads get their own warps.  Rows are
+// addressed through row_stride, so no contiguous copy of the projection output
+// is ever made.  With head_dim 256 each lane holds one 16-byte vector.
+#pragma once
+#include "fn_device.cuh"
+
+namespace fn {
+
+struct QKParams {
+  const uint4* qkv;
+  int64_t M;
+  int64_t row_vec;  // row stride in 16-byte vectors
+  int Hq, Hk;
+  int dv;           // head_dim / 8
+  const uint4* qw;
+  const uint4* kw;
+  float eps;
+  uint4* out_q;
+  uint4* out_k;
+  uint4* out_g;
+};
+
+template <int VPL>
+__global__ void __launch_bounds__(256) qk_kernel(const __grid_constant__ QKParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int heads = p.Hq + p.Hk;
+  if (item >= p.M * heads) return;  // warp-uniform
+  const int64_t m = item / heads;
+  const int j = (int)(item - m * heads);
+  const bool isq = j < p.Hq;
+  const uint4* row = p.qkv + m * p.row_vec;
+  const uint4* src = isq ? row + (int64_t)(2 * j) * p.dv
+                         : row + (int64_t)(2 * p.Hq + (j - p.Hq)) * p.dv;
+  const uint4* w = isq ? p.qw : p.kw;
+  uint4* dst = isq ? p.out_q + (m * p.Hq + j) * p.dv
+                   : p.out_k + (m * p.Hk + (j - p.Hq)) * p.dv;
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+
+  uint4 x[VPL], wv[VPL], g[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int v = lane + 32 * i;
+    const bool ok = v < p.dv;
+    x[i] = ok ? ld_stream_nc(src + v) : zero;
+    g[i] = (ok && isq) ? ld_stream_nc(src + p.dv + v) : zero;
+    wv[i] = ok ? ld_keep(w + v) : zero;
+  }
+  if (isq) {
+    uint4* gdst = p.out_g + (m * p.Hq + j) * p.dv;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i)
+      if (lane + 32 * i < p.dv) st_stream(gdst + lane + 32 * i, g[i]);
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const float a = bf_lo(word(x[i], c)), b = bf_hi(word(x[i], c));
+      ss = fmaf(a, a, ss);
+      ss = fmaf(b, b, ss);
+    }
+  ss = warp_sum(ss);
+  const float rstd = (float)(1.0 / sqrt((double)ss / (double)(p.dv * 8) + (double)p.eps));
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    uint4 y;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint32_t xw = word(x[i], c), ww = word(wv[i], c);
+      const float y0 = (bf_lo(xw) * rstd) * (1.f + bf_lo(ww));
+      const float y1 = (bf_hi(xw) * rstd) * (1.f + bf_hi(ww));
+      set_word(y, c, pack_bf16x2(y0, y1));
+    }
+    if (lane + 32 * i < p.dv) st_stream(dst + lane + 32 * i, y);
+  }
+}
+
+}  // namespace fn

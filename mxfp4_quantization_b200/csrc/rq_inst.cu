@@ -1,0 +1,45 @@
+// One instantiation unit of the rmsnorm_quant kernels: the mode and the
+// partial-count bound come from -DFN_INST_MODE / -DFN_INST_MAXP.
+#include "rq_kernel.cuh"
+
+#ifndef FN_INST_MODE
+#error "FN_INST_MODE is required"
+#endif
+#ifndef FN_INST_MAXP
+#error "FN_INST_MAXP is required"
+#endif
+
+#define FN_CAT_(a, b, c) a##_##b##_##c
+#define FN_CAT(a, b, c) FN_CAT_(a, b, c)
+
+namespace fn {
+
+RQKernel FN_CAT(rq_pick, FN_INST_MODE, FN_INST_MAXP)(int V, bool cluster, bool norm) {
+  constexpr int MODE = FN_INST_MODE, MAXP = FN_INST_MAXP;
+  if (cluster) {
+    if (!norm) return nullptr;
+    return rq_kernel<MODE, MAXP, 1, true, true>;
+  }
+  if (!norm) {
+    if constexpr (MAXP != 1) {
+      return nullptr;
+    } else {
+      switch (V) {
+        case 1: return rq_kernel<MODE, 1, 1, false, false>;
+        case 2: return rq_kernel<MODE, 1, 2, false, false>;
+        case 4: return rq_kernel<MODE, 1, 4, false, false>;
+        case 8: return rq_kernel<MODE, 1, 8, false, false>;
+        default: return rq_kernel<MODE, 1, 16, false, false>;
+      }
+    }
+  }
+  switch (V) {
+    case 1: return rq_kernel<MODE, MAXP, 1, true, false>;
+    case 2: return rq_kernel<MODE, MAXP, 2, true, false>;
+    case 4: return rq_kernel<MODE, MAXP, 4, true, false>;
+    case 8: return rq_kernel<MODE, MAXP, 8, true, false>;
+    default: return rq_kernel<MODE, MAXP, 16, true, false>;
+  }
+}
+
+}  // namespace fn

@@ -1,0 +1,47 @@
+// Parameter block shared by the host dispatch and the rmsnorm_quant kernels.
+#pragma once
+#include <cstdint>
+#include <vector_types.h>
+
+namespace fn {
+
+enum : int { MODE_TOKEN = 0, MODE_G128 = 1, MODE_MX = 2 };
+
+struct RQParams {
+  const uint4* parts[8];   // P bf16 [M, H] inputs (as 16-byte vectors)
+  const uint4* residual;   // bf16 [M, H] or nullptr
+  const uint4* weight;     // bf16 [H]
+  uint4* out_residual;     // bf16 [M, H] or nullptr (may equal residual)
+  uint4* out_y;            // bf16 [M, H] or nullptr
+  uint8_t* out_q;          // codes
+  void* out_scale;         // fp32 or E8M0 bytes
+  int64_t M;
+  int nvec;                // H / 8
+  int seg;                 // vectors of a row handled by one block
+  int P;                   // partial count, <= MAXP
+  float eps;
+};
+
+// A kernel instance: every (mode, partial bound, vectors per thread, norm,
+// cluster) combination has the same signature.
+using RQKernel = void (*)(const RQParams);
+
+// Per-(mode, partial bound) instantiation units, each compiled separately
+// (rq_inst.cu) so the library builds in parallel.  `V` is ignored for
+// cluster launches (always one vector per thread there).
+#define FN_RQ_DECL(MODE, MAXP) RQKernel rq_pick_##MODE##_##MAXP(int V, bool cluster, bool norm);
+FN_RQ_DECL(0, 1)
+FN_RQ_DECL(0, 2)
+FN_RQ_DECL(0, 4)
+FN_RQ_DECL(0, 8)
+FN_RQ_DECL(1, 1)
+FN_RQ_DECL(1, 2)
+FN_RQ_DECL(1, 4)
+FN_RQ_DECL(1, 8)
+FN_RQ_DECL(2, 1)
+FN_RQ_DECL(2, 2)
+FN_RQ_DECL(2, 4)
+FN_RQ_DECL(2, 8)
+#undef FN_RQ_DECL
+
+}  // namespace fn

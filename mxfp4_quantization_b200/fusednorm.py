@@ -1,0 +1,270 @@
+"""Python binding of libfusednorm.so (argument marshalling only).
+
+Two layers:
+  * `fn_rmsnorm_quant`, `fn_quant`, `fn_qk_norm_gate`, `fn_status_string`,
+    `fn_last_variant`, `fn_last_launch`, `fn_version`: the C ABI of
+    include/fusednorm.h one to one, taking raw device addresses (ints) and
+    returning the status code.
+  * `rmsnorm_quant`, `quant`, `qk_norm_gate`: take torch CUDA tensors, allocate
+    the outputs with torch (device memory is torch's plumbing), call the C
+    ABI on the current stream, and raise `FusedNormError` on a non-zero status.
+    Every step of the computation runs in the library's kernels.
+
+There is no fallback: if the library is missing, importing this module fails.
+"""
+import ctypes
+import os
+from collections import namedtuple
+from typing import Optional, Sequence, Union
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfusednorm.so")
+
+FN_FP8_PER_TOKEN = 0
+FN_FP8_PER_GROUP128 = 1
+FN_MXFP4 = 2
+
+FN_OK = 0
+FN_ERR_INVALID = -1
+FN_ERR_ALIGN = -2
+FN_ERR_UNSUPPORTED = -3
+FN_ERR_CUDA = -4
+FN_ERR_TIMEOUT = -5
+
+FN_VARIANT_NONE = 0
+FN_VARIANT_ROW_CTA = 1
+FN_VARIANT_ROW_CLUSTER = 2
+FN_VARIANT_QUANT_ONLY = 3
+FN_VARIANT_QK_WARP = 4
+
+FN_MAX_PARTS = 8
+FN_MAX_H = 32768
+FN_MAX_HEAD_DIM = 1024
+
+MODES = {"fp8_per_token": FN_FP8_PER_TOKEN, "fp8_per_group128": FN_FP8_PER_GROUP128,
+         "mxfp4": FN_MXFP4}
+
+# The exported symbols of include/fusednorm.h.
+ABI_SYMBOLS = ("fn_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate", "fn_status_string",
+               "fn_last_variant", "fn_last_launch", "fn_version")
+
+
+class FusedNormError(RuntimeError):
+    def __init__(self, func: str, status: int):
+        super().__init__(f"{func}: {fn_status_string(status)} (status {status})")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python -m mxfp4_quantization_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.fn_rmsnorm_quant.argtypes = [ctypes.POINTER(vp), i32, vp, vp, ctypes.c_float, i32, i64,
+                                     i64, vp, vp, vp, vp, vp]
+    lib.fn_rmsnorm_quant.restype = i32
+    lib.fn_quant.argtypes = [vp, i32, i64, i64, vp, vp, vp]
+    lib.fn_quant.restype = i32
+    lib.fn_qk_norm_gate.argtypes = [vp, i64, i64, i32, i32, i32, vp, vp, ctypes.c_float, vp, vp,
+                                    vp, vp]
+    lib.fn_qk_norm_gate.restype = i32
+    lib.fn_status_string.argtypes = [i32]
+    lib.fn_status_string.restype = ctypes.c_char_p
+    lib.fn_last_variant.argtypes = []
+    lib.fn_last_variant.restype = i32
+    lib.fn_last_launch.argtypes = [ctypes.POINTER(ctypes.c_int32)]
+    lib.fn_last_launch.restype = None
+    lib.fn_version.argtypes = []
+    lib.fn_version.restype = i32
+    return lib
+
+
+_lib = _load()
+
+
+# ---- the C ABI, one to one --------------------------------------------------------
+
+
+def fn_rmsnorm_quant(x_parts: Sequence[int], num_parts: int, residual: Optional[int],
+                     weight: int, eps: float, mode: int, M: int, H: int, out_q: int,
+                     out_scale: int, out_residual: Optional[int], out_y: Optional[int],
+                     stream: Optional[int]) -> int:
+    arr = (ctypes.c_void_p * max(1, len(x_parts)))(*x_parts)
+    return _lib.fn_rmsnorm_quant(arr, num_parts, residual, weight, eps, mode, M, H, out_q,
+                                 out_scale, out_residual, out_y, stream)
+
+
+def fn_quant(y: int, mode: int, M: int, H: int, out_q: int, out_scale: int,
+             stream: Optional[int]) -> int:
+    return _lib.fn_quant(y, mode, M, H, out_q, out_scale, stream)
+
+
+def fn_qk_norm_gate(qkv: int, M: int, row_stride: int, Hq: int, Hk: int, D: int,
+                    q_weight: Optional[int], k_weight: Optional[int], eps: float,
+                    out_q: Optional[int], out_k: Optional[int], out_gate: Optional[int],
+                    stream: Optional[int]) -> int:
+    return _lib.fn_qk_norm_gate(qkv, M, row_stride, Hq, Hk, D, q_weight, k_weight, eps, out_q,
+                                out_k, out_gate, stream)
+
+
+def fn_status_string(status: int) -> str:
+    return _lib.fn_status_string(status).decode()
+
+
+def fn_last_variant() -> int:
+    return _lib.fn_last_variant()
+
+
+def fn_last_launch():
+    out = (ctypes.c_int32 * 4)()
+    _lib.fn_last_launch(out)
+    return tuple(out)
+
+
+def fn_version() -> int:
+    return _lib.fn_version()
+
+
+# ---- tensor API ----------------------------------------------------------------------
+
+RMSNormQuantOutput = namedtuple("RMSNormQuantOutput", "q scale residual_out y")
+QKOutput = namedtuple("QKOutput", "q k gate")
+
+
+def _mode(mode: Union[int, str]) -> int:
+    return MODES[mode] if isinstance(mode, str) else int(mode)
+
+
+def _rows(t: torch.Tensor, name: str, H: Optional[int] = None) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if H is not None and t.shape[-1] != H:
+        raise ValueError(f"{name} has last dim {t.shape[-1]}, expected {H}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.reshape(-1, t.shape[-1])
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def alloc_outputs(mode: int, M: int, H: int, device) -> tuple:
+    """Codes and scales for `mode`: FP8 codes as float8_e4m3fn [M, H]; MXFP4 codes
+    as uint8 [M, H/2]; scales fp32 [M, 1] / fp32 [M, H/128] / uint8 E8M0 [M, H/32]."""
+    if mode == FN_MXFP4:
+        return (torch.empty((M, H // 2), dtype=torch.uint8, device=device),
+                torch.empty((M, H // 32), dtype=torch.uint8, device=device))
+    q = torch.empty((M, H), dtype=torch.float8_e4m3fn, device=device)
+    if mode == FN_FP8_PER_TOKEN:
+        return q, torch.empty((M, 1), dtype=torch.float32, device=device)
+    return q, torch.empty((M, H // 128), dtype=torch.float32, device=device)
+
+
+def rmsnorm_quant(x: Union[torch.Tensor, Sequence[torch.Tensor]], weight: torch.Tensor,
+                  eps: float, mode: Union[int, str], residual: Optional[torch.Tensor] = None,
+                  *, in_place: bool = False, out_residual: Optional[torch.Tensor] = None,
+                  emit_y: bool = False, out_q: Optional[torch.Tensor] = None,
+                  out_scale: Optional[torch.Tensor] = None,
+                  out_y: Optional[torch.Tensor] = None) -> RMSNormQuantOutput:
+    """Fused (sum of partials) + residual add + RMSNorm + quantization.
+
+    x: a bf16 CUDA tensor [..., H] or a list of up to 8 such partial tensors
+    (summed in the kernel).  With `in_place`, residual_out is written into
+    `residual`.  Returns (q, scale, residual_out, y); y is None unless
+    `emit_y` (or `out_y`) asks for the bf16 normed row.
+    """
+    parts = list(x) if isinstance(x, (list, tuple)) else [x]
+    if not 1 <= len(parts) <= FN_MAX_PARTS:
+        raise ValueError("between 1 and 8 partial tensors")
+    H = parts[0].shape[-1]
+    lead = parts[0].shape[:-1]
+    rows = [_rows(p, f"x[{i}]", H) for i, p in enumerate(parts)]
+    for r in rows:
+        if r.shape != rows[0].shape:
+            raise ValueError("all partials must have the same shape")
+    M = rows[0].shape[0]
+    w = _rows(weight, "weight", H)
+    m = _mode(mode)
+    dev = rows[0].device
+    res = None if residual is None else _rows(residual, "residual", H)
+    if res is not None and res.shape[0] != M:
+        raise ValueError("residual rows differ from x rows")
+    if in_place:
+        if res is None:
+            raise ValueError("in_place needs a residual")
+        r_out = res
+    elif out_residual is not None:
+        r_out = _rows(out_residual, "out_residual", H)
+    elif res is not None:
+        r_out = torch.empty_like(res)
+    else:
+        r_out = None
+    if out_q is None or out_scale is None:
+        q, s = alloc_outputs(m, M, H, dev)
+        out_q = q if out_q is None else out_q
+        out_scale = s if out_scale is None else out_scale
+    if out_y is None and emit_y:
+        out_y = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+    st = fn_rmsnorm_quant([r.data_ptr() for r in rows], len(rows), _ptr(res), w.data_ptr(),
+                          float(eps), m, M, H, out_q.data_ptr(), out_scale.data_ptr(),
+                          _ptr(r_out), _ptr(out_y), _stream(dev))
+    if st != FN_OK:
+        raise FusedNormError("fn_rmsnorm_quant", st)
+    ro = None if r_out is None else r_out.view(*lead, H)
+    yo = None if out_y is None else out_y.view(*lead, H)
+    return RMSNormQuantOutput(out_q, out_scale, ro, yo)
+
+
+def quant(y: torch.Tensor, mode: Union[int, str], *, out_q: Optional[torch.Tensor] = None,
+          out_scale: Optional[torch.Tensor] = None):
+    """Quantization step alone on bf16 rows [..., H]; returns (q, scale)."""
+    rows = _rows(y, "y")
+    M, H = rows.shape
+    m = _mode(mode)
+    if out_q is None or out_scale is None:
+        q, s = alloc_outputs(m, M, H, rows.device)
+        out_q = q if out_q is None else out_q
+        out_scale = s if out_scale is None else out_scale
+    st = fn_quant(rows.data_ptr(), m, M, H, out_q.data_ptr(), out_scale.data_ptr(),
+                  _stream(rows.device))
+    if st != FN_OK:
+        raise FusedNormError("fn_quant", st)
+    return out_q, out_scale
+
+
+def qk_norm_gate(qkv: torch.Tensor, Hq: int, Hk: int, D: int, q_weight: torch.Tensor,
+                 k_weight: torch.Tensor, eps: float, *,
+                 out: Optional[QKOutput] = None) -> QKOutput:
+    """Gemma (1 + w) RMSNorm of q and k heads read from the interleaved
+    [q_h0, gate_h0, q_h1, gate_h1, ..., k..., v...] rows of `qkv` [M, row_stride]
+    (any row stride, last dim contiguous); returns contiguous q [M,Hq,D],
+    k [M,Hk,D] and gate [M,Hq,D]."""
+    if not qkv.is_cuda or qkv.dtype != torch.bfloat16:
+        raise TypeError("qkv must be a bf16 CUDA tensor")
+    if qkv.dim() != 2 or qkv.stride(1) != 1:
+        raise ValueError("qkv must be [M, row] with a contiguous last dim")
+    M, row_stride = qkv.shape[0], qkv.stride(0)
+    if qkv.shape[1] < (2 * Hq + Hk) * D:
+        raise ValueError("qkv rows are too short for the heads")
+    qw = _rows(q_weight, "q_weight", D)
+    kw = _rows(k_weight, "k_weight", D)
+    dev = qkv.device
+    if out is None:
+        out = QKOutput(torch.empty((M, Hq, D), dtype=torch.bfloat16, device=dev),
+                       torch.empty((M, Hk, D), dtype=torch.bfloat16, device=dev),
+                       torch.empty((M, Hq, D), dtype=torch.bfloat16, device=dev))
+    st = fn_qk_norm_gate(qkv.data_ptr(), M, row_stride, Hq, Hk, D, qw.data_ptr(),
+                         kw.data_ptr(), float(eps), out.q.data_ptr(), out.k.data_ptr(),
+                         out.gate.data_ptr(), _stream(dev))
+    if st != FN_OK:
+        raise FusedNormError("fn_qk_norm_gate", st)
+    return out

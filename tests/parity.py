@@ -1,0 +1,116 @@
+"""Comparison of the CUDA path with the oracle (host side, numpy).
+
+Criteria (the tolerances of the fused path):
+  residual_out   bit-exact.
+  y              within 1 bf16 ulp of the oracle (the GPU reduces mean(h^2) in
+                 fp32 in another order than the oracle's fp64 sum).
+  quant stage    fed the GPU's own y, the oracle reproduces the GPU's codes and
+                 scales bit for bit.
+  end to end     against the oracle run from the inputs: in groups whose scale
+                 agrees, codes may differ only where y differs, by one code
+                 step at most, and (over at least 1000 codes) in at most 0.1 %
+                 of positions; a group whose scale differs must have a 1-ulp
+                 difference of its amax element, and the count is reported
+                 separately.
+"""
+import numpy as np
+
+import oracle
+
+MX, G128, TOKEN = oracle.MXFP4, oracle.FP8_PER_GROUP128, oracle.FP8_PER_TOKEN
+
+
+def bf16_ord(bits):
+    b = np.asarray(bits).astype(np.int64)
+    return np.where(b & 0x8000, -(b & 0x7FFF), b & 0x7FFF)
+
+
+def ulp_diff(a, b):
+    return np.abs(bf16_ord(a) - bf16_ord(b))
+
+
+def unpack_e2m1(packed):
+    p = np.asarray(packed)
+    return np.stack([p & 0xF, p >> 4], axis=-1).reshape(p.shape[0], -1)
+
+
+def code_ord(codes, mode):
+    c = np.asarray(codes).astype(np.int64)
+    if mode == MX:
+        return np.where(c & 0x8, -(c & 0x7), c & 0x7)
+    return np.where(c & 0x80, -(c & 0x7F), c & 0x7F)
+
+
+def group_size(mode, H):
+    return 32 if mode == MX else 128 if mode == G128 else H
+
+
+def bf16_bits_to_f32(bits):
+    return (np.asarray(bits, dtype=np.uint32) << 16).astype(np.uint32).view(np.float32)
+
+
+def compare_quant_stage(y_bits, q, s, mode):
+    """GPU codes/scales vs the oracle fed the GPU's y: bit-exact."""
+    rq, rs = oracle.quant_rows(y_bits, mode)
+    q = np.asarray(q).reshape(rq.shape)
+    s = np.asarray(s).reshape(rs.shape)
+    bad_q = np.argwhere(q != rq)
+    assert bad_q.size == 0, f"quant stage codes differ at {bad_q[:5].tolist()}"
+    if mode == MX:
+        assert np.array_equal(s, rs), f"E8M0 scales differ at {np.argwhere(s != rs)[:5].tolist()}"
+    else:
+        assert np.array_equal(s.view(np.uint32), rs.view(np.uint32)), \
+            f"fp32 scales differ at {np.argwhere(s.view(np.uint32) != rs.view(np.uint32))[:5].tolist()}"
+
+
+def compare_end_to_end(mode, H, y_gpu, q_gpu, s_gpu, y_orc, q_orc, s_orc):
+    """Returns stats; asserts the end-to-end criterion."""
+    M = y_gpu.shape[0]
+    G = group_size(mode, H)
+    ng = H // G
+    if mode == MX:
+        cg, co = unpack_e2m1(q_gpu), unpack_e2m1(q_orc)
+        sg, so = np.asarray(s_gpu).reshape(M, ng), np.asarray(s_orc).reshape(M, ng)
+        s_eq = sg == so
+    else:
+        cg, co = np.asarray(q_gpu).reshape(M, H), np.asarray(q_orc).reshape(M, H)
+        sg = np.asarray(s_gpu, dtype=np.float32).reshape(M, ng)
+        so = np.asarray(s_orc, dtype=np.float32).reshape(M, ng)
+        s_eq = sg.view(np.uint32) == so.view(np.uint32)
+    y_flip = ulp_diff(y_gpu, y_orc) != 0
+    elem_s_eq = np.repeat(s_eq, G, axis=1)
+    dcode = np.abs(code_ord(cg, mode) - code_ord(co, mode))
+    in_eq = elem_s_eq
+    diff = (dcode != 0) & in_eq
+    n = int(in_eq.sum())
+    stats = {"codes": int(cg.size), "codes_diff": int(diff.sum()),
+             "max_step": int(dcode[in_eq].max()) if n else 0,
+             "groups": int(s_eq.size), "scale_diff": int((~s_eq).sum()),
+             "y_flips": int(y_flip.sum())}
+    assert stats["max_step"] <= 1, f"code differs by {stats['max_step']} steps"
+    assert not np.any(diff & ~y_flip), "a code differs where y agrees"
+    if n >= 1000:
+        assert stats["codes_diff"] <= 1e-3 * n, f"{stats['codes_diff']} of {n} codes differ"
+    yg = np.abs(bf16_bits_to_f32(y_gpu)).reshape(M, ng, G)
+    yo = np.abs(bf16_bits_to_f32(y_orc)).reshape(M, ng, G)
+    for m, g in np.argwhere(~s_eq):
+        ag, ao = yg[m, g].max(), yo[m, g].max()
+        ag_b = np.array([ag], np.float32).view(np.uint32) >> 16
+        ao_b = np.array([ao], np.float32).view(np.uint32) >> 16
+        assert abs(int(ag_b[0]) - int(ao_b[0])) == 1, \
+            f"scale of group ({m},{g}) differs without a 1-ulp amax difference"
+    return stats
+
+
+def check_rmsnorm(mode, eps, parts_bits, res_bits, w_bits, gpu):
+    """gpu: dict of numpy arrays q, scale, residual_out (or None), y for the same rows."""
+    orc = oracle.rmsnorm_quant(parts_bits, res_bits, w_bits, eps, mode)
+    M, H = parts_bits[0].shape
+    if gpu.get("residual_out") is not None:
+        bad = np.argwhere(gpu["residual_out"] != orc["residual_out"])
+        assert bad.size == 0, f"residual_out differs at {bad[:5].tolist()}"
+    d = ulp_diff(gpu["y"], orc["y"])
+    assert d.max(initial=0) <= 1, f"y differs by {d.max()} ulp at {np.argwhere(d > 1)[:5].tolist()}"
+    compare_quant_stage(gpu["y"], gpu["q"], gpu["scale"], mode)
+    return compare_end_to_end(mode, H, gpu["y"], gpu["q"], gpu["scale"], orc["y"], orc["q"],
+                              orc["scale"])

@@ -1,0 +1,141 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+symbol include/fusednorm.h declares, and rejects bad arguments before any CUDA
+call.  Pointers here are fake addresses: a rejected call never dereferences
+or launches anything, and a call that wrongly got through would reach the CUDA
+runtime, find no device and return FN_ERR_CUDA, failing the test."""
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fusednorm.h")
+
+
+@pytest.fixture(scope="module")
+def fnb():
+    from mxfp4_quantization_b200.build import build_library
+    build_library()
+    from mxfp4_quantization_b200 import fusednorm
+    return fusednorm
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"FN_API\s+[\w\s\*]+?\b(fn_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_abi():
+    assert declared_symbols() == sorted(["fn_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate",
+                                         "fn_status_string", "fn_last_variant",
+                                         "fn_last_launch", "fn_version"])
+
+
+def test_library_exports_every_declared_symbol(fnb):
+    out = subprocess.run(["nm", "-D", "--defined-only", fnb.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (fn_\w+)", out))
+    missing = set(declared_symbols()) - exported
+    assert not missing, f"not exported: {missing}"
+    assert set(fnb.ABI_SYMBOLS) == set(declared_symbols())
+    # nothing but the ABI leaks out with default visibility
+    assert exported == set(declared_symbols())
+
+
+def test_header_constants_match_binding(fnb):
+    src = open(HEADER).read()
+    for name in ("FN_FP8_PER_TOKEN", "FN_FP8_PER_GROUP128", "FN_MXFP4", "FN_ERR_INVALID",
+                 "FN_ERR_ALIGN", "FN_ERR_UNSUPPORTED", "FN_ERR_CUDA", "FN_VARIANT_ROW_CTA",
+                 "FN_VARIANT_ROW_CLUSTER", "FN_VARIANT_QUANT_ONLY", "FN_VARIANT_QK_WARP"):
+        m = re.search(rf"\b{name}\s*=\s*(-?\d+)", src)
+        assert m and int(m.group(1)) == getattr(fnb, name), name
+    for name in ("FN_MAX_PARTS", "FN_MAX_H", "FN_MAX_HEAD_DIM"):
+        m = re.search(rf"#define {name} (\d+)", src)
+        assert int(m.group(1)) == getattr(fnb, name), name
+
+
+def test_status_strings(fnb):
+    assert fnb.fn_status_string(0) == "ok"
+    for s in (-1, -2, -3, -4, -5):
+        assert fnb.fn_status_string(s) and fnb.fn_status_string(s) != "unknown status"
+    assert fnb.fn_status_string(17) == "unknown status"
+    assert fnb.fn_version() >= 100
+
+
+BASE = 0x7F0000000000
+
+
+def rq(fnb, **kw):
+    a = dict(x_parts=[BASE], num_parts=1, residual=BASE + (1 << 32), weight=BASE + (2 << 32),
+             eps=1e-6, mode=0, M=4, H=256, out_q=BASE + (3 << 32), out_scale=BASE + (4 << 32),
+             out_residual=BASE + (5 << 32), out_y=None, stream=None)
+    a.update(kw)
+    return fnb.fn_rmsnorm_quant(a["x_parts"], a["num_parts"], a["residual"], a["weight"],
+                                a["eps"], a["mode"], a["M"], a["H"], a["out_q"], a["out_scale"],
+                                a["out_residual"], a["out_y"], a["stream"])
+
+
+def test_rmsnorm_quant_rejects_bad_arguments(fnb):
+    E, A, U = fnb.FN_ERR_INVALID, fnb.FN_ERR_ALIGN, fnb.FN_ERR_UNSUPPORTED
+    cases = [
+        (dict(num_parts=0), E), (dict(num_parts=9, x_parts=[BASE] * 9), E),
+        (dict(mode=3), E), (dict(mode=-1), E), (dict(M=-1), E), (dict(H=0), E),
+        (dict(H=12), E), (dict(mode=1, H=192), E), (dict(mode=2, H=48), E),
+        (dict(H=32776), U), (dict(eps=float("nan")), E), (dict(eps=-1.0), E),
+        (dict(weight=None), E), (dict(out_q=None), E), (dict(out_scale=None), E),
+        (dict(out_residual=None), E), (dict(x_parts=[None]), E),
+        (dict(x_parts=[BASE + 8]), A), (dict(weight=BASE + (2 << 32) + 2), A),
+        (dict(out_q=BASE + (3 << 32) + 4), A), (dict(out_scale=BASE + (4 << 32) + 2), A),
+        (dict(out_y=BASE + (6 << 32) + 8), A),
+        # outputs overlapping inputs or each other
+        (dict(out_q=BASE + 64), E), (dict(out_y=BASE + (1 << 32)), E),
+        (dict(out_scale=BASE + (3 << 32) + 256), E),
+        (dict(out_residual=BASE + (1 << 32) + 16), E),
+    ]
+    for kw, want in cases:
+        assert rq(fnb, **kw) == want, kw
+        assert fnb.fn_last_variant() == fnb.FN_VARIANT_NONE
+
+
+def test_rmsnorm_quant_accepts_empty_and_in_place(fnb):
+    assert rq(fnb, M=0) == fnb.FN_OK
+    assert fnb.fn_last_variant() == fnb.FN_VARIANT_NONE
+    # in-place residual is the one allowed overlap; mxfp4 codes need 4-byte alignment only
+    assert rq(fnb, M=0, out_residual=BASE + (1 << 32)) == fnb.FN_OK
+    assert rq(fnb, M=0, mode=2, out_q=BASE + (3 << 32) + 4, out_scale=BASE + (4 << 32) + 1) == 0
+    assert rq(fnb, M=0, residual=None, out_residual=None) == fnb.FN_OK
+
+
+def test_quant_rejects_bad_arguments(fnb):
+    q = fnb.fn_quant
+    assert q(BASE, 0, 0, 256, BASE + (1 << 32), BASE + (2 << 32), None) == fnb.FN_OK
+    assert q(None, 0, 4, 256, BASE + (1 << 32), BASE + (2 << 32), None) == fnb.FN_ERR_INVALID
+    assert q(BASE + 8, 0, 4, 256, BASE + (1 << 32), BASE + (2 << 32), None) == fnb.FN_ERR_ALIGN
+    assert q(BASE, 1, 4, 64, BASE + (1 << 32), BASE + (2 << 32), None) == fnb.FN_ERR_INVALID
+    assert q(BASE, 0, 4, 256, BASE + 512, BASE + (2 << 32), None) == fnb.FN_ERR_INVALID
+
+
+def qk(fnb, **kw):
+    a = dict(qkv=BASE, M=4, row_stride=18432, Hq=32, Hk=4, D=256, q_weight=BASE + (1 << 32),
+             k_weight=BASE + (2 << 32), eps=1e-6, out_q=BASE + (3 << 32),
+             out_k=BASE + (4 << 32), out_gate=BASE + (5 << 32), stream=None)
+    a.update(kw)
+    return fnb.fn_qk_norm_gate(a["qkv"], a["M"], a["row_stride"], a["Hq"], a["Hk"], a["D"],
+                               a["q_weight"], a["k_weight"], a["eps"], a["out_q"], a["out_k"],
+                               a["out_gate"], a["stream"])
+
+
+def test_qk_norm_gate_rejects_bad_arguments(fnb):
+    E, A, U = fnb.FN_ERR_INVALID, fnb.FN_ERR_ALIGN, fnb.FN_ERR_UNSUPPORTED
+    cases = [
+        (dict(M=-1), E), (dict(D=12), E), (dict(D=0), E), (dict(D=2048, row_stride=1 << 20), U),
+        (dict(row_stride=18436), E), (dict(row_stride=8192), E), (dict(Hq=0, Hk=0), E),
+        (dict(q_weight=None), E), (dict(out_k=None), E), (dict(eps=float("inf")), E),
+        (dict(qkv=BASE + 8), A), (dict(out_gate=BASE + (5 << 32) + 4), A),
+        (dict(out_q=BASE + 1024), E), (dict(out_k=BASE + (3 << 32) + 16), E),
+    ]
+    for kw, want in cases:
+        assert qk(fnb, **kw) == want, kw
+    assert qk(fnb, M=0) == fnb.FN_OK
+    assert qk(fnb, M=0, Hk=0, k_weight=None, out_k=None) == fnb.FN_OK

@@ -1,0 +1,78 @@
+"""fn_quant (the quantization stage alone) against the oracle, bit for bit,
+over every finite bf16 value and the rounding corner cases of E4M3 / E2M1 /
+E8M0.  The fused kernel runs the same device code for its quantization stage."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests import gpu_util, parity
+from tests.oracle_pins import all_finite_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fnb():
+    return gpu_util.lib()
+
+
+def exhaustive_rows(H, seed):
+    """All finite bf16 patterns, shuffled into rows of H, plus corner rows."""
+    b, _ = all_finite_bf16()
+    rng = np.random.default_rng(seed)
+    shuffled = rng.permutation(b)
+    sorted_runs = np.sort(b)  # consecutive patterns share a group: many near-ties
+    rows = [shuffled, sorted_runs]
+    # MX tie blocks: amax 5 * 2^k puts the E2M1 midpoints at 0.25..5 * 2^k
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -0.75, -1.25, -1.75, -2.5,
+                     -3.5, -5.0, 0.1, -0.1, 6.0, 7.0, -7.5, 0.0], dtype=np.float64)
+    tie_blocks = []
+    for k in range(-124, 124, 3):
+        blk = np.zeros(32)
+        blk[:ties.size] = ties * 2.0 ** k
+        tie_blocks.append(blk)
+    tb = torch.from_numpy(np.concatenate(tie_blocks).astype(np.float32)).to(torch.bfloat16)
+    rows.append(tb.view(torch.int16).numpy().view(np.uint16))
+    rows.append(np.zeros(H * 2, dtype=np.uint16))                    # zero groups
+    rows.append(np.full(H, 0x8000, dtype=np.uint16))                 # -0 everywhere
+    rows.append(rng.integers(1, 0x80, H * 2).astype(np.uint16))      # subnormals only
+    rows.append((rng.integers(1, 0x80, H) | 0x8000).astype(np.uint16))
+    flat = np.concatenate(rows)
+    pad = (-flat.size) % H
+    flat = np.concatenate([flat, np.zeros(pad, dtype=np.uint16)])
+    return flat.reshape(-1, H)
+
+
+@pytest.mark.parametrize("mode", [oracle.FP8_PER_TOKEN, oracle.FP8_PER_GROUP128, oracle.MXFP4])
+@pytest.mark.parametrize("H", [128, 4096])
+def test_quant_stage_exhaustive(fnb, mode, H):
+    y = exhaustive_rows(H, seed=H + mode)
+    yt = torch.from_numpy(y.view(np.int16)).view(torch.bfloat16).cuda()
+    M = y.shape[0]
+    q_shape = (M, H // 2) if mode == oracle.MXFP4 else (M, H)
+    s_shape = oracle.scale_shape(mode, M, H)
+    gq = gpu_util.Guarded(q_shape, torch.uint8)
+    gs = gpu_util.Guarded(s_shape, torch.uint8 if mode == oracle.MXFP4 else torch.float32)
+    fnb.quant(yt, mode, out_q=gq.t, out_scale=gs.t)
+    assert fnb.fn_last_variant() == fnb.FN_VARIANT_QUANT_ONLY
+    torch.cuda.synchronize()
+    assert gq.intact() and gs.intact(), "write outside an output"
+    parity.compare_quant_stage(y, gpu_util.u8(gq.t), gpu_util.scale_np(gs.t, mode), mode)
+
+
+def test_negative_tiny_values_keep_their_sign(fnb):
+    """A negative value that rounds to zero gives the -0 code (0x80 / 0x8)."""
+    y = np.zeros((1, 128), dtype=np.float32)
+    y[0, 0] = 448.0
+    y[0, 1:8] = -1e-6
+    y[0, 8] = -0.0
+    yb = torch.from_numpy(y).to(torch.bfloat16)
+    yt = yb.cuda()
+    for mode in (oracle.FP8_PER_GROUP128, oracle.MXFP4):
+        q, s = fnb.quant(yt, mode)
+        torch.cuda.synchronize()
+        parity.compare_quant_stage(gpu_util.bits(yb), gpu_util.u8(q), gpu_util.scale_np(s, mode),
+                                   mode)
+    q, _ = fnb.quant(yt, oracle.FP8_PER_GROUP128)
+    assert np.all(gpu_util.u8(q)[0, 1:9] == 0x80)

@@ -1,0 +1,228 @@
+"""Fused (partial sum) + residual + RMSNorm + quantization on the GPU against
+the oracle: residual bit-exact, y within 1 ulp, quantization stage bit-exact
+on the GPU's y, end-to-end code criterion (tests/parity.py)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mxfp4_quantization_b200 import synth
+from tests import gpu_util, parity
+
+pytestmark = pytest.mark.gpu
+
+TOKEN, G128, MX = synth.FP8_PER_TOKEN, synth.FP8_PER_GROUP128, synth.MXFP4
+
+
+@pytest.fixture(scope="module")
+def fnb():
+    return gpu_util.lib()
+
+
+def run(fnb, wl, M=None, in_place=False, guarded=True, emit_y=True, device_inputs=None):
+    """Run the fused kernel on `wl`'s inputs (drawn on the CPU unless given)."""
+    M = wl.M if M is None else M
+    inp = wl.inputs(device="cpu", M=M) if device_inputs is None else device_inputs
+    parts = [p.cuda() for p in inp["parts"]]
+    res = None if inp["residual"] is None else inp["residual"].cuda()
+    w = inp["weight"].cuda()
+    H = wl.H
+    q_shape = (M, H // 2) if wl.mode == MX else (M, H)
+    s_shape = oracle.scale_shape(wl.mode, M, H)
+    gq = gpu_util.Guarded(q_shape, torch.uint8)
+    gs = gpu_util.Guarded(s_shape, torch.uint8 if wl.mode == MX else torch.float32)
+    gy = gpu_util.Guarded((M, H), torch.bfloat16) if emit_y else None
+    gr = gpu_util.Guarded((M, H), torch.bfloat16) if (res is not None and not in_place) else None
+    out = fnb.rmsnorm_quant(parts, w, wl.eps, wl.mode, residual=res, in_place=in_place,
+                            out_residual=None if gr is None else gr.t, out_q=gq.t,
+                            out_scale=gs.t, out_y=None if gy is None else gy.t)
+    variant, launch = fnb.fn_last_variant(), fnb.fn_last_launch()
+    torch.cuda.synchronize()
+    for g in (gq, gs, gy, gr):
+        assert g is None or g.intact(), "write outside an output"
+    gpu = {"q": gpu_util.u8(gq.t), "scale": gpu_util.scale_np(gs.t, wl.mode),
+           "residual_out": gpu_util.bits(out.residual_out),
+           "y": gpu_util.bits(gy.t) if gy is not None else None}
+    return inp, gpu, variant, launch
+
+
+def check(wl, inp, gpu):
+    parts = [gpu_util.bits(p) for p in inp["parts"]]
+    res = gpu_util.bits(inp["residual"])
+    return parity.check_rmsnorm(wl.mode, wl.eps, parts, res, gpu_util.bits(inp["weight"]), gpu)
+
+
+# (M, H, P, residual): several tiles, ragged tails, the cluster/row switch,
+# the largest H, P up to 8.
+SHAPES = [
+    (1, 7168, 1, True), (5, 7168, 4, True), (16, 2048, 1, True), (16, 7168, 2, True),
+    (17, 7168, 4, True), (19, 7168, 1, True), (37, 8192, 1, True), (150, 7168, 4, True),
+    (64, 4096, 3, False), (33, 1024, 8, True), (7, 32768, 1, True), (200, 2176, 5, True),
+    (3, 128, 1, True), (75, 1152, 6, False), (40, 16384, 2, True), (300, 256, 7, True),
+]
+
+
+@pytest.mark.parametrize("mode", [TOKEN, G128, MX], ids=["token", "g128", "mxfp4"])
+@pytest.mark.parametrize("M,H,P,has_res", SHAPES, ids=[f"M{s[0]}_H{s[1]}_P{s[2]}_{'r' if s[3] else 'nr'}" for s in SHAPES])
+def test_parity(fnb, mode, M, H, P, has_res):
+    wl = synth.RowWorkload("case", M=M, H=H, P=P, mode=mode, eps=1e-6 if H % 3 else 1e-5,
+                           seed=M * 31 + H + P, residual=has_res, outlier_frac=0.01,
+                           channel_decades=1.0 if P > 1 else 0.0)
+    inp, gpu, variant, launch = run(fnb, wl)
+    assert variant in (fnb.FN_VARIANT_ROW_CTA, fnb.FN_VARIANT_ROW_CLUSTER)
+    check(wl, inp, gpu)
+
+
+@pytest.mark.parametrize("mode,H", [(TOKEN, 8), (TOKEN, 24), (MX, 32), (MX, 96), (G128, 128)])
+def test_smallest_rows(fnb, mode, H):
+    wl = synth.RowWorkload("small", M=9, H=H, P=2, mode=mode, eps=1e-6, seed=H)
+    inp, gpu, _, _ = run(fnb, wl)
+    check(wl, inp, gpu)
+
+
+@pytest.mark.parametrize("mode", [TOKEN, G128, MX])
+def test_in_place_residual(fnb, mode):
+    wl = synth.RowWorkload("inplace", M=48, H=8192, P=1, mode=mode, eps=1e-5, seed=5, x_std=2.0)
+    inp = wl.inputs(device="cpu")
+    inp_copy = {"parts": [p.clone() for p in inp["parts"]], "residual": inp["residual"].clone(),
+                "weight": inp["weight"]}
+    dev = {"parts": inp["parts"], "residual": inp["residual"], "weight": inp["weight"]}
+    parts = [p.cuda() for p in dev["parts"]]
+    res = dev["residual"].cuda()
+    w = dev["weight"].cuda()
+    out = fnb.rmsnorm_quant(parts, w, wl.eps, mode, residual=res, in_place=True, emit_y=True)
+    torch.cuda.synchronize()
+    assert out.residual_out.data_ptr() == res.data_ptr()
+    gpu = {"q": gpu_util.u8(out.q), "scale": gpu_util.scale_np(out.scale, mode),
+           "residual_out": gpu_util.bits(res), "y": gpu_util.bits(out.y)}
+    check(wl, inp_copy, gpu)
+
+
+def test_dispatch(fnb):
+    """Small M takes the cluster kernel, large M one block per row."""
+    for M, want in ((1, fnb.FN_VARIANT_ROW_CLUSTER), (16, fnb.FN_VARIANT_ROW_CLUSTER),
+                    (512, fnb.FN_VARIANT_ROW_CTA)):
+        wl = synth.decode(M, MX) if M <= 16 else synth.RowWorkload("big", M=M, H=7168, P=1,
+                                                                     mode=MX, eps=1e-6)
+        _, _, variant, launch = run(fnb, wl)
+        assert variant == want, (M, variant, launch)
+        if want == fnb.FN_VARIANT_ROW_CLUSTER:
+            assert launch[2] >= 2 and launch[0] == M * launch[2]
+
+
+def test_empty_and_rejected_calls_touch_nothing(fnb):
+    w = torch.ones(256, dtype=torch.bfloat16, device="cuda")
+    x = torch.ones((4, 256), dtype=torch.bfloat16, device="cuda")
+    gq = gpu_util.Guarded((4, 256), torch.uint8)
+    gs = gpu_util.Guarded((4,), torch.float32)
+    st = fnb.fn_rmsnorm_quant([x.data_ptr()], 1, None, w.data_ptr(), 1e-6, TOKEN, 0, 256,
+                              gq.t.data_ptr(), gs.t.data_ptr(), None, None, None)
+    assert st == fnb.FN_OK and fnb.fn_last_variant() == fnb.FN_VARIANT_NONE
+    st = fnb.fn_rmsnorm_quant([x.data_ptr()], 1, None, w.data_ptr(), 1e-6, G128, 4, 200,
+                              gq.t.data_ptr(), gs.t.data_ptr(), None, None, None)
+    assert st == fnb.FN_ERR_INVALID
+    torch.cuda.synchronize()
+    assert gq.untouched() and gs.untouched()
+    with pytest.raises(fnb.FusedNormError):
+        fnb.rmsnorm_quant(x, w, 1e-6, MX, out_q=x.view(torch.uint8)[:, :128],
+                          out_scale=gs.t.view(torch.uint8))
+
+
+def test_replays_are_bit_identical(fnb):
+    wl = synth.RowWorkload("det", M=300, H=7168, P=4, mode=MX, eps=1e-6, seed=9,
+                           channel_decades=1.0)
+    inp = wl.inputs(device="cuda")
+    outs = []
+    for _ in range(3):
+        o = fnb.rmsnorm_quant(inp["parts"], inp["weight"], wl.eps, MX, residual=inp["residual"],
+                              emit_y=True)
+        outs.append([t.clone() for t in o])
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        for a, b in zip(outs[0], o):
+            assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+
+
+def test_graph_capture(fnb):
+    """The call is capturable in a CUDA graph and replays to the same bits."""
+    wl = synth.decode(16, TOKEN)
+    inp = wl.inputs(device="cuda")
+    x, r, w = inp["parts"][0], inp["residual"], inp["weight"]
+    eager = fnb.rmsnorm_quant(x, w, wl.eps, TOKEN, residual=r)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            cap = fnb.rmsnorm_quant(x, w, wl.eps, TOKEN, residual=r)
+    g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(eager[:3], cap[:3]):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+
+
+def _sampled_full_size(fnb, wl, n_rows=48):
+    """Full-size workload on the device in the launch shape the benchmark times
+    (no y side output), then with y for the oracle's sampled rows."""
+    inp = wl.inputs(device="cuda")
+    parts, w = inp["parts"], inp["weight"]
+    res = inp["residual"]
+    res0 = res.clone()
+    o1 = fnb.rmsnorm_quant(parts, w, wl.eps, wl.mode, residual=res, in_place=wl.in_place)
+    launch_bench = fnb.fn_last_launch()
+    q1, s1 = o1.q.clone(), o1.scale.clone()
+    r1 = o1.residual_out.clone()
+    # second run from the original residual, with the y side output
+    res2 = res0.clone()
+    o2 = fnb.rmsnorm_quant(parts, w, wl.eps, wl.mode, residual=res2, in_place=wl.in_place,
+                           emit_y=True)
+    assert fnb.fn_last_launch() == launch_bench
+    torch.cuda.synchronize()
+    assert torch.equal(q1.view(torch.uint8), o2.q.view(torch.uint8))
+    assert torch.equal(s1.view(torch.uint8), o2.scale.view(torch.uint8))
+    assert torch.equal(r1, o2.residual_out)
+    # properties at full size: every non-zero group's amax element encodes +-448 (FP8)
+    # and every E8M0 code is finite
+    if wl.mode == MX:
+        assert int(o2.scale.max()) <= 252
+    else:
+        G = wl.H if wl.mode == TOKEN else 128
+        y = o2.y.float().view(wl.M, -1, G).abs()
+        idx = y.argmax(dim=-1, keepdim=True)
+        codes = o2.q.view(torch.uint8).view(wl.M, -1, G).gather(-1, idx)
+        nz = y.amax(dim=-1, keepdim=True) > 0
+        assert bool(((codes & 0x7F) == 0x7E)[nz].all())
+    g = torch.Generator().manual_seed(1)
+    rows = torch.cat([torch.tensor([0, wl.M - 1]), torch.randint(1, wl.M - 1, (n_rows - 2,),
+                                                                  generator=g)]).tolist()
+    sel = torch.tensor(rows, device="cuda")
+    gpu = {"q": gpu_util.u8(o2.q.index_select(0, sel)),
+           "scale": gpu_util.scale_np(o2.scale.index_select(0, sel), wl.mode),
+           "residual_out": gpu_util.bits(o2.residual_out.index_select(0, sel)),
+           "y": gpu_util.bits(o2.y.index_select(0, sel))}
+    parts_b = [gpu_util.bits(p.index_select(0, sel)) for p in parts]
+    return parity.check_rmsnorm(wl.mode, wl.eps, parts_b, gpu_util.bits(res0.index_select(0, sel)),
+                                gpu_util.bits(w), gpu)
+
+
+def test_prefill_mxfp4_full_size(fnb):
+    _sampled_full_size(fnb, synth.PREFILL_MXFP4)
+
+
+def test_prefill_group128_full_size(fnb):
+    _sampled_full_size(fnb, synth.PREFILL_GROUP128)
+
+
+def test_per_token_small_config(fnb):
+    wl = synth.PER_TOKEN_SMALL
+    inp, gpu, variant, _ = run(fnb, wl)
+    check(wl, inp, gpu)
+
+
+@pytest.mark.parametrize("M", synth.DECODE_M)
+@pytest.mark.parametrize("mode", [TOKEN, G128, MX])
+def test_decode_sweep_config(fnb, M, mode):
+    wl = synth.decode(M, mode)
+    inp, gpu, variant, _ = run(fnb, wl)
+    assert variant == fnb.FN_VARIANT_ROW_CLUSTER
+    check(wl, inp, gpu)
