@@ -492,7 +492,9 @@ def main_arm(args):
     from mxfp4_quantization_b200 import fusednorm as fn
     from mxfp4_quantization_b200 import synth
 
-    wl = synth.PREFILL_MXFP4
+    wl = synth.PREFILL_MXFP4 if args.workload == "prefill_mxfp4" else synth.PREFILL_GROUP128
+    mode_name = {synth.MXFP4: "mxfp4", synth.FP8_PER_GROUP128: "fp8_per_group128",
+                 synth.FP8_PER_TOKEN: "fp8_per_token"}[wl.mode]
     seed = rank_seed(wl.seed, rank)
     step, stream, keep = make_row_call(fn, wl, device, seed)
     clocks = ClockSampler(local)
@@ -518,7 +520,7 @@ def main_arm(args):
 
     extra = None
     cpu = None
-    if world == 1 and not args.no_extras:
+    if world == 1 and not args.no_extras and args.workload == "prefill_mxfp4":
         extra = secondary_workloads(fn, device, peak)
     if world == 1 and not args.no_cpu_baseline:
         rate, rows, el = oracle_rows_per_s(256, args.cpu_seconds, 3 * args.cpu_seconds)
@@ -533,17 +535,19 @@ def main_arm(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": {"workload": "prefill_mxfp4", "M": wl.M, "H": wl.H, "P": wl.P,
-                       "mode": "mxfp4", "eps": wl.eps, "rows_per_gpu": wl.M,
-                       "io": "bf16 in; E2M1 codes + E8M0 scales + bf16 residual out",
-                       "l2": "inputs larger than L2 (587 MB per step), no flush",
+            "config": {"workload": wl.name, "M": wl.M, "H": wl.H, "P": wl.P,
+                       "mode": mode_name, "eps": wl.eps, "rows_per_gpu": wl.M,
+                       "in_place": wl.in_place,
+                       "io": "bf16 in; codes + scales + bf16 residual out",
+                       "l2": f"inputs larger than L2 ({wl.M * wl.H * 2 * (wl.P + 1) / 1e6:.0f} MB"
+                             " read per step), no flush",
                        "parallelism": f"dp{world} (independent rows, no collective)"},
             "hbm_GB_s": achieved, "frac_of_peak": achieved / peak,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
-                         "traffic": measured_traffic("rq_mxfp4_p4_h7168"),
+                         "traffic": measured_traffic(wl.name),
                          "algorithmic_bytes_per_launch": bytes_call,
-                         "kernel": "rq_kernel<MXFP4, P<=4, V=4>",
+                         "kernel": "rq_kernel (one block per row)",
                          "launch": list(launch), "variant": variant},
             "e2e": {"value": aggregate(wl.M, world, e2e_ms_max), "unit": "rows/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -567,6 +571,8 @@ def parse(argv=None):
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", choices=["prefill_mxfp4", "prefill_group128"],
+                    default="prefill_mxfp4", help="the workload a step runs")
     ap.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

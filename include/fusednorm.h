@@ -33,7 +33,9 @@
  *    (a cudaStream_t passed as void*; NULL means the legacy default stream).
  *  - All argument checks run on the host before anything is launched; on any
  *    error nothing is launched and no output is touched.  M == 0 returns
- *    FN_OK and launches nothing.
+ *    FN_OK and launches nothing once the sizes and the mode are valid; the
+ *    data pointers are not examined then and may be NULL (an empty torch
+ *    tensor has a NULL data pointer).
  *  - A launch that the CUDA runtime rejects returns FN_ERR_CUDA.
  *  - Calls are thread-safe.  The kernels contain no spin-waits and no flags
  *    shared between thread blocks.

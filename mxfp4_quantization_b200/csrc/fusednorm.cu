@@ -197,10 +197,11 @@ int fn_rmsnorm_quant(const void* const* x_parts, int num_parts, const void* resi
   int rc = check_mode_shape(mode, M, H);
   if (rc != FN_OK) return rc;
   if (!std::isfinite(eps) || eps < 0.f) return FN_ERR_INVALID;
+  if (M == 0) return FN_OK;  // nothing to read or write: data pointers may be NULL
   if (!weight || !out_q || !out_scale) return FN_ERR_INVALID;
   if (residual && !out_residual) return FN_ERR_INVALID;
   for (int p = 0; p < num_parts; ++p) {
-    if (!x_parts[p]) return FN_ERR_INVALID;
+    if (!x_parts[p]) return FN_ERR_INVALID;  // (M > 0 here)
     if (!aligned(x_parts[p], 16)) return FN_ERR_ALIGN;
   }
   if (!aligned(weight, 16) || (residual && !aligned(residual, 16)) ||
@@ -255,6 +256,7 @@ int fn_quant(const void* y, int mode, int64_t M, int64_t H, void* out_q, void* o
   tl_variant = FN_VARIANT_NONE;
   int rc = check_mode_shape(mode, M, H);
   if (rc != FN_OK) return rc;
+  if (M == 0) return FN_OK;
   if (!y || !out_q || !out_scale) return FN_ERR_INVALID;
   if (!aligned(y, 16)) return FN_ERR_ALIGN;
   if ((rc = check_outputs_align(mode, out_q, out_scale)) != FN_OK) return rc;
@@ -284,6 +286,7 @@ int fn_qk_norm_gate(const void* qkv, int64_t M, int64_t row_stride, int Hq, int 
   if (D > FN_MAX_HEAD_DIM) return FN_ERR_UNSUPPORTED;
   if (row_stride % 8 || row_stride < (int64_t)(2 * Hq + Hk) * D) return FN_ERR_INVALID;
   if (!std::isfinite(eps) || eps < 0.f) return FN_ERR_INVALID;
+  if (M == 0) return FN_OK;
   if (!qkv || (Hq > 0 && (!q_weight || !out_q || !out_gate)) || (Hk > 0 && (!k_weight || !out_k)))
     return FN_ERR_INVALID;
   if (!aligned(qkv, 16) || (q_weight && !aligned(q_weight, 16)) ||

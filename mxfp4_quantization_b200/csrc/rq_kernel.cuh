@@ -27,27 +27,46 @@ namespace fn {
 
 namespace cg = cooperative_groups;
 
-// Sum (or max) of one value per thread over the block and, with CL, over the
-// cluster.  The combination order is fixed (warps in index order, cluster
-// ranks in rank order), so every block of a cluster gets the same bits.
-template <bool IS_MAX, bool CL>
-__device__ __forceinline__ float row_reduce(float v, float* red, float* cl_slot) {
-  v = IS_MAX ? warp_max(v) : warp_sum(v);
+// Cluster barrier halves (all threads of every block of the cluster take part).
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Sum of `s` and max of `m` over the block and, with CL, over the cluster.
+// The combination order is fixed (warps in index order, cluster ranks in rank
+// order), so every block of a cluster gets the same bits.  With CL the caller
+// must call cluster_wait() once before exiting: the last arrive here tells the
+// peers this block is done reading their shared memory, and the wait keeps
+// this block's own slot alive until every peer has read it.
+template <bool CL, bool WANT_MAX>
+__device__ __forceinline__ float2 row_reduce(float s, float m, float2* red, float2* cl_slot) {
+  s = warp_sum(s);
+  if (WANT_MAX) m = warp_max(m);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  if (lane == 0) red[warp] = v;
+  if (lane == 0) red[warp] = make_float2(s, m);
   __syncthreads();
-  float t = red[0];
-  for (int i = 1; i < nw; ++i) t = IS_MAX ? fmaxf(t, red[i]) : t + red[i];
+  float2 t = red[0];
+  for (int i = 1; i < nw; ++i) {
+    const float2 o = red[i];
+    t.x += o.x;
+    if (WANT_MAX) t.y = fmaxf(t.y, o.y);
+  }
   if constexpr (CL) {
     cg::cluster_group cl = cg::this_cluster();
     if (threadIdx.x == 0) *cl_slot = t;
-    cl.sync();
+    cluster_arrive();
+    cluster_wait();
     const unsigned nb = cl.num_blocks();
-    float u = *cl.map_shared_rank(cl_slot, 0);
+    float2 u = *cl.map_shared_rank(cl_slot, 0);
     for (unsigned c = 1; c < nb; ++c) {
-      const float o = *cl.map_shared_rank(cl_slot, c);
-      u = IS_MAX ? fmaxf(u, o) : u + o;
+      const float2 o = *cl.map_shared_rank(cl_slot, c);
+      u.x += o.x;
+      if (WANT_MAX) u.y = fmaxf(u.y, o.y);
     }
+    cluster_arrive();
     t = u;
   }
   return t;
@@ -56,9 +75,8 @@ __device__ __forceinline__ float row_reduce(float v, float* red, float* cl_slot)
 template <int MODE, int MAXP, int V, bool NORM, bool CL>
 __global__ void __launch_bounds__(CL ? 512 : 256)
     rq_kernel(const __grid_constant__ RQParams prm) {
-  __shared__ float red_ss[32];
-  __shared__ float red_amax[32];
-  __shared__ float cl_ss, cl_amax;
+  __shared__ float2 red[32];
+  __shared__ float2 cl_slot;
 
   const int T = blockDim.x, t = threadIdx.x, lane = t & 31;
   int64_t row;
@@ -93,10 +111,14 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
   }
 
   // ---- 2. h = bf16(((x0 + x1) + ...) + r), residual_out, sum of squares ----------
+  // Also max |h * w| for the per-token scale: h * w is exact in fp32 (two
+  // 8-bit significands), y = bf16(fl(h * w) * rstd) is monotone in |h * w|, so
+  // max |y| = bf16(fl(max |h * w| * rstd)) comes out of the same reduction.
   uint4 yv[V];
+  float row_amax = 0.f;
   if constexpr (NORM) {
     uint4 hv[V];
-    float ss = 0.f;
+    float ss = 0.f, pmax = 0.f;
 #pragma unroll
     for (int k = 0; k < V; ++k) {
 #pragma unroll
@@ -118,24 +140,29 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
         const float h0 = bf_lo(hw), h1 = bf_hi(hw);
         ss = fmaf(h0, h0, ss);
         ss = fmaf(h1, h1, ss);
+        if (MODE == MODE_TOKEN) {
+          const uint32_t ww = word(win[k], i);
+          pmax = fmaxf(pmax, fmaxf(fabsf(h0 * bf_lo(ww)), fabsf(h1 * bf_hi(ww))));
+        }
       }
       const int v = seg_base + t + k * T;
       if (v < seg_end && prm.out_residual != nullptr) st_stream(prm.out_residual + rowv + v, hv[k]);
     }
 
     // ---- 3. rstd = 1 / sqrt(mean(h^2) + eps) --------------------------------------
-    const float tot = row_reduce<false, CL>(ss, red_ss, &cl_ss);
+    const float2 tot = row_reduce<CL, MODE == MODE_TOKEN>(ss, pmax, red, &cl_slot);
     const float rstd =
-        (float)(1.0 / sqrt((double)tot / (double)(prm.nvec * 8) + (double)prm.eps));
+        (float)(1.0 / sqrt((double)tot.x / (double)(prm.nvec * 8) + (double)prm.eps));
+    if (MODE == MODE_TOKEN) row_amax = __uint_as_float(pack_bf16x2(tot.y * rstd, 0.f) << 16);
 
-    // ---- 4. y = bf16(h * rstd * w) ------------------------------------------------
+    // ---- 4. y = bf16(fl(h * w) * rstd) --------------------------------------------
 #pragma unroll
     for (int k = 0; k < V; ++k) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint32_t hw = word(hv[k], i), ww = word(win[k], i);
-        const float y0 = (bf_lo(hw) * rstd) * bf_lo(ww);
-        const float y1 = (bf_hi(hw) * rstd) * bf_hi(ww);
+        const float y0 = (bf_lo(hw) * bf_lo(ww)) * rstd;
+        const float y1 = (bf_hi(hw) * bf_hi(ww)) * rstd;
         set_word(yv[k], i, pack_bf16x2(y0, y1));
       }
       const int v = seg_base + t + k * T;
@@ -144,6 +171,15 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
   } else {
 #pragma unroll
     for (int k = 0; k < V; ++k) yv[k] = xin[0][k];
+    if (MODE == MODE_TOKEN) {
+      float am = 0.f;
+#pragma unroll
+      for (int k = 0; k < V; ++k)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          am = fmaxf(am, fmaxf(fabsf(bf_lo(word(yv[k], i))), fabsf(bf_hi(word(yv[k], i)))));
+      row_amax = row_reduce<CL, true>(0.f, am, red, &cl_slot).y;
+    }
   }
 
   // ---- 5. quantize y ----------------------------------------------------------------
@@ -151,14 +187,7 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
   if constexpr (MODE == MODE_TOKEN || MODE == MODE_G128) {
     float scale_tok = 1.f;
     if constexpr (MODE == MODE_TOKEN) {
-      float am = 0.f;
-#pragma unroll
-      for (int k = 0; k < V; ++k)
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          am = fmaxf(am, fmaxf(fabsf(bf_lo(word(yv[k], i))), fabsf(bf_hi(word(yv[k], i)))));
-      const float amax = row_reduce<true, CL>(am, red_amax, &cl_amax);
-      scale_tok = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+      scale_tok = row_amax == 0.f ? 1.f : __fdiv_rn(row_amax, 448.f);
       if (rank == 0 && t == 0) static_cast<float*>(prm.out_scale)[row] = scale_tok;
     }
 #pragma unroll
@@ -211,8 +240,8 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
   }
 
   if constexpr (CL) {
-    // No block may leave while a peer can still read its shared-memory slots.
-    cg::this_cluster().sync();
+    // No block may leave while a peer can still read its shared-memory slot.
+    cluster_wait();
   }
 }
 
