@@ -380,11 +380,29 @@ def secondary_workloads(fn, device, peak):
     del keep
     torch.cuda.empty_cache()
 
+    # the large-M kernels side by side (the library picks one by shape)
+    cmp = {}
+    for wl in (synth.PREFILL_MXFP4, synth.PREFILL_GROUP128):
+        step, stream, keep = make_row_call(fn, wl, device, wl.seed)
+        b = wl.bytes_per_call()
+        row = {}
+        for name, v in (("row_cta", fn.FN_VARIANT_ROW_CTA), ("row_tma", fn.FN_VARIANT_ROW_TMA)):
+            with fn.prefer_variant(v):
+                ms = time_steps(step, 100, 5, device, stream)
+                got = fn.fn_last_variant()
+            row[name] = {"us_per_call": ms * 1e3, "GB_s": b / (ms * 1e-3) / 1e9,
+                         "frac_of_peak": b / (ms * 1e-3) / 1e9 / peak, "variant": got,
+                         "launch": list(fn.fn_last_launch())}
+        cmp[wl.name] = row
+        del keep
+        torch.cuda.empty_cache()
+    res["large_m_kernels"] = cmp
+
     def small(wl, per_call_bytes, make):
         n_sets = max(64, int(2 * L2_BYTES / per_call_bytes) + 1)
         n_sets = min(n_sets, 8192)
         us, eager = time_graph_calls(make, n_sets, 7, device)
-        return {"us_per_call_graph": us, "us_eager_device": eager, "calls_per_graph": n_sets,
+        return {"us_per_call_graph": us, "us_single_call_events": eager, "calls_per_graph": n_sets,
                 "GB_s": per_call_bytes / (us * 1e-6) / 1e9}
 
     wl = synth.PER_TOKEN_SMALL
@@ -498,11 +516,13 @@ def main_arm(args):
     seed = rank_seed(wl.seed, rank)
     step, stream, keep = make_row_call(fn, wl, device, seed)
     clocks = ClockSampler(local)
-    # warm-up outside the sampled region, then sample clocks over the timed steps
+    # the sampler needs a moment to start; it runs over the warm-up and the
+    # timed steps, and only samples taken while steps run are kept
+    clocks.start()
+    time.sleep(0.5)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(device)
-    clocks.start()
     ms = time_steps(step, args.steps, 0, device, stream)
     clk = clocks.stop()
     variant, launch = fn.fn_last_variant(), fn.fn_last_launch()
@@ -568,7 +588,7 @@ def main_arm(args):
 def parse(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--steps", type=int, default=12000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", choices=["prefill_mxfp4", "prefill_group128"],

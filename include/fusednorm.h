@@ -37,8 +37,9 @@
  *    data pointers are not examined then and may be NULL (an empty torch
  *    tensor has a NULL data pointer).
  *  - A launch that the CUDA runtime rejects returns FN_ERR_CUDA.
- *  - Calls are thread-safe.  The kernels contain no spin-waits and no flags
- *    shared between thread blocks.
+ *  - Calls are thread-safe.  No kernel waits on another thread block.  The
+ *    TMA-staged kernel waits on its own bulk copies with a bounded poll
+ *    (see fn_device_status).
  */
 #ifndef FUSEDNORM_H
 #define FUSEDNORM_H
@@ -68,7 +69,7 @@ typedef enum {
     FN_ERR_ALIGN = -2,       /* a pointer or stride breaks the alignment rule      */
     FN_ERR_UNSUPPORTED = -3, /* valid request outside the built shapes (e.g. H)    */
     FN_ERR_CUDA = -4,        /* the CUDA runtime rejected the launch               */
-    FN_ERR_TIMEOUT = -5      /* reserved: no kernel here waits on another          */
+    FN_ERR_TIMEOUT = -5      /* a bounded device wait gave up (fn_device_status)   */
 } fn_status;
 
 /* Which kernel the calling thread's last successful call launched. */
@@ -77,7 +78,8 @@ typedef enum {
     FN_VARIANT_ROW_CTA = 1,     /* one thread block per row                        */
     FN_VARIANT_ROW_CLUSTER = 2, /* a cluster of 2..8 blocks per row (small M)      */
     FN_VARIANT_QUANT_ONLY = 3,  /* fn_quant                                        */
-    FN_VARIANT_QK_WARP = 4      /* fn_qk_norm_gate: one warp per (token, head)     */
+    FN_VARIANT_QK_WARP = 4,     /* fn_qk_norm_gate: one warp per (token, head)     */
+    FN_VARIANT_ROW_TMA = 5      /* persistent blocks, rows staged by bulk copies  */
 } fn_variant;
 
 #define FN_MAX_PARTS 8
@@ -159,9 +161,25 @@ FN_API const char* fn_status_string(int status);
 FN_API int fn_last_variant(void);
 
 /* Launch shape of the calling thread's last launch: out[0] grid blocks,
- * out[1] threads per block, out[2] blocks per cluster (1 = none),
- * out[3] elements per thread-vector group (vectors of 8 bf16 per thread). */
+ * out[1] threads per block, out[2] blocks per cluster (FN_VARIANT_ROW_TMA:
+ * shared-memory stages), out[3] 16-byte vectors per thread per tensor. */
 FN_API void fn_last_launch(int32_t out[4]);
+
+/* Thread-local kernel preference for fn_rmsnorm_quant: FN_VARIANT_NONE (the
+ * default) lets the library choose by M, H and P; FN_VARIANT_ROW_CTA,
+ * FN_VARIANT_ROW_CLUSTER or FN_VARIANT_ROW_TMA asks for that kernel where the
+ * shape allows it (the cluster kernel needs a row that splits into 2..8
+ * group-aligned segments with M * blocks <= SMs, the TMA kernel at least two
+ * row stages in shared memory).  Every kernel computes the same bits.
+ * Returns the previous preference. */
+FN_API int fn_prefer_variant(int variant);
+
+/* Reads and clears the library's device status word on the current device
+ * (synchronizes `stream`).  FN_ERR_TIMEOUT means a kernel's bounded wait for
+ * its own bulk copies gave up since the last call, so that call's outputs are
+ * not valid; FN_OK otherwise.  The word is a static device variable of the
+ * library, not an allocation. */
+FN_API int fn_device_status(void* stream);
 
 /* Library ABI version (major * 100 + minor). */
 FN_API int fn_version(void);

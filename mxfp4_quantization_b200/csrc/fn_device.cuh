@@ -58,6 +58,23 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return d;
 }
 
+// Packed bf16 add, one rounding of the exact sum.  For two bf16 operands this
+// equals rounding their fp32 sum to bf16: if the fp32 sum is inexact the
+// operands' exponents differ by more than 16, so the smaller one moves the
+// larger by less than 2^-15 of it, far from any bf16 rounding midpoint.
+__device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Packed max of |a| and |b| (exact: max only selects).
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a & 0x7FFF7FFFu), "r"(b & 0x7FFF7FFFu));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t word(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
@@ -67,6 +84,62 @@ __device__ __forceinline__ void set_word(uint4& v, int i, uint32_t w) {
   else if (i == 1) v.y = w;
   else if (i == 2) v.z = w;
   else v.w = w;
+}
+
+// ---- mixed bf16 / fp32 and packed fp32 arithmetic (sm_100) ---------------------
+
+// acc + x, x the low (HI = false) or high bf16 half of w, rounded once to fp32:
+// the same value as adding x converted to fp32.
+template <bool HI>
+__device__ __forceinline__ float add_bf16(uint32_t w, float acc) {
+  float d;
+  if (HI)
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.bf16 %0, h, %2;\n\t}"
+        : "=f"(d) : "r"(w), "f"(acc));
+  else
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.bf16 %0, l, %2;\n\t}"
+        : "=f"(d) : "r"(w), "f"(acc));
+  return d;
+}
+
+// a * b + c for the low (HI = false) or high bf16 halves of a and b, rounded
+// once to fp32.  The product of two bf16 is exact in fp32, so with c = -0 this
+// is exactly a * b (and its sign for zeros).
+template <bool HI>
+__device__ __forceinline__ float fma_bf16(uint32_t a, uint32_t b, float c) {
+  float d;
+  if (HI)
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, ah, bh, %3;\n\t}"
+        : "=f"(d) : "r"(a), "r"(b), "f"(c));
+  else
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %3;\n\t}"
+        : "=f"(d) : "r"(a), "r"(b), "f"(c));
+  return d;
+}
+
+// Element-wise a * b and a * b + c on fp32 pairs, each rounded once.
+__device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fma_f32x2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mov.b64 c, {%6, %7};\n\tfma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+// max |y| over the 8 bf16 of a vector, as fp32.
+__device__ __forceinline__ float vec_absmax(const uint4& y) {
+  const uint32_t m = absmax_bf16x2(absmax_bf16x2(y.x, y.y), absmax_bf16x2(y.z, y.w));
+  return fmaxf(bf_lo(m), bf_hi(m));
 }
 
 // ---- FP8 E4M3 -----------------------------------------------------------------

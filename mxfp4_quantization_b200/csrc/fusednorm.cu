@@ -5,6 +5,8 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
+#include <mutex>
 
 #include "fusednorm.h"
 #include "qk_kernel.cuh"
@@ -14,6 +16,41 @@ namespace {
 
 thread_local int tl_variant = FN_VARIANT_NONE;
 thread_local int32_t tl_launch[4] = {0, 0, 0, 0};
+thread_local int tl_prefer = FN_VARIANT_NONE;
+
+}  // namespace
+
+// Library status word, one per device that loads the library: a kernel whose
+// bounded wait gives up sets it (it is never part of a computation).
+__device__ int fn_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mu;
+int* g_status_ptr[kMaxDevices];
+int g_smem_optin[kMaxDevices];
+
+// Per-device facts fetched once with the device current: the device address
+// of the status word and the opt-in shared memory per block.
+bool device_facts(int* dev_out, int** status, int* smem_optin) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, fn_status_word) != cudaSuccess) return false;
+    int optin = 0;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return false;
+    g_smem_optin[dev] = optin;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  *dev_out = dev;
+  *status = g_status_ptr[dev];
+  *smem_optin = g_smem_optin[dev];
+  return true;
+}
 
 struct Range {
   uintptr_t lo, hi;  // [lo, hi)
@@ -53,12 +90,44 @@ RQKernel pick_kernel(int mode, int P, int V, bool cluster, bool norm) {
   return nullptr;
 }
 
-// Smallest power-of-two V in {1..16} with ceil(nvec / V) <= 256 threads.
-int row_vectors_per_thread(int nvec) {
+using fn::RQTmaKernel;
+
+RQTmaKernel pick_tma_kernel(int mode, int P, int V) {
+  const int maxp = P == 1 ? 1 : P == 2 ? 2 : P <= 4 ? 4 : 8;
+#define FN_CASE(MODE, MAXP) \
+  if (mode == MODE && maxp == MAXP) return fn::rq_tma_pick_##MODE##_##MAXP(V);
+  FN_CASE(0, 1) FN_CASE(0, 2) FN_CASE(0, 4) FN_CASE(0, 8)
+  FN_CASE(1, 1) FN_CASE(1, 2) FN_CASE(1, 4) FN_CASE(1, 8)
+  FN_CASE(2, 1) FN_CASE(2, 2) FN_CASE(2, 4) FN_CASE(2, 8)
+#undef FN_CASE
+  return nullptr;
+}
+
+// Smallest power-of-two V in {1..vmax} with ceil(nvec / V) <= max_threads.
+int vectors_per_thread(int nvec, int max_threads, int vmax) {
   int V = 1;
-  while (V < 16 && (nvec + V - 1) / V > 256) V *= 2;
+  while (V < vmax && (nvec + V - 1) / V > max_threads) V *= 2;
   return V;
 }
+
+int row_vectors_per_thread(int nvec) { return vectors_per_thread(nvec, 256, 16); }
+
+constexpr int kTmaMaxStages = 8;
+constexpr int kTmaStaticSmem = 2 * 32 * 8;  // the kernel's double-buffered reduction slots
+
+// Stages of the TMA ring that fit in shared memory (0 when fewer than 2 fit).
+int tma_stages(int64_t stage_bytes, int smem_optin) {
+  const int64_t avail = (int64_t)smem_optin - kTmaStaticSmem - 1024;
+  int n = (int)std::min<int64_t>(kTmaMaxStages, avail / (stage_bytes + 8));
+  return n >= 2 ? n : 0;
+}
+
+// Whether a large-M call should take the TMA ring.  Measured on B200: with
+// three or more row tensors (partials + residual) a register-resident row is
+// too big for enough rows to be in flight per SM and the ring wins (MXFP4,
+// H=7168, P=4: 113 us vs 121 us); with two the register kernel keeps four
+// rows per SM in flight and wins (group-128, H=8192, P=1: 289 us vs 448 us).
+bool want_tma(int64_t M, int sms, int ntensor) { return M >= 2 * (int64_t)sms && ntensor >= 3; }
 
 // Cluster size for a small-M launch: the largest C in 2..8 that splits the
 // row into equal segments aligned to the quantization group, each at most 512
@@ -107,8 +176,42 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, vo
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   fn::RQParams p = prm;
 
-  const int C = norm ? pick_cluster(M, nvec, mode, sms) : 0;
-  if (C >= 2) {
+  int dev = 0, smem_optin = 0;
+  if (!device_facts(&dev, &p.status, &smem_optin)) return FN_ERR_CUDA;
+
+  const int pref = tl_prefer;
+  int C = norm ? pick_cluster(M, nvec, mode, sms) : 0;
+  if (pref == FN_VARIANT_ROW_CTA || pref == FN_VARIANT_ROW_TMA) C = 0;
+
+  const int ntensor = P + (prm.residual ? 1 : 0);
+  const int64_t stage_bytes = (int64_t)ntensor * nvec * 16;
+  const int nst = tma_stages(stage_bytes, smem_optin);
+  const bool tma = norm && nst > 0 && pref != FN_VARIANT_ROW_CTA &&
+                   pref != FN_VARIANT_ROW_CLUSTER &&
+                   (pref == FN_VARIANT_ROW_TMA || (C < 2 && want_tma(M, sms, ntensor)));
+
+  if (tma) {
+    const int V = vectors_per_thread(nvec, 512, 8);
+    const int threads = round32((nvec + V - 1) / V);
+    if ((nvec + V - 1) / V > 512) return FN_ERR_UNSUPPORTED;
+    RQTmaKernel k = pick_tma_kernel(mode, P, V);
+    if (!k) return FN_ERR_UNSUPPORTED;
+    const size_t smem = (size_t)nst * (size_t)(stage_bytes + 8);
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+      (void)cudaGetLastError();
+      return FN_ERR_CUDA;
+    }
+    const int64_t grid = std::min<int64_t>(M, sms);
+    p.seg = nvec;
+    k<<<(unsigned)grid, threads, smem, st>>>(p, nst);
+    if (cudaGetLastError() != cudaSuccess) return FN_ERR_CUDA;
+    tl_variant = FN_VARIANT_ROW_TMA;
+    tl_launch[0] = (int32_t)grid;
+    tl_launch[1] = threads;
+    tl_launch[2] = nst;
+    tl_launch[3] = V;
+  } else if (C >= 2) {
     p.seg = nvec / C;
     const int threads = round32(p.seg);
     RQKernel k = pick_kernel(mode, P, 1, true, true);
@@ -171,6 +274,24 @@ extern "C" {
 int fn_version(void) { return 100; }
 
 int fn_last_variant(void) { return tl_variant; }
+
+int fn_prefer_variant(int variant) {
+  const int old = tl_prefer;
+  tl_prefer = variant;
+  return old;
+}
+
+int fn_device_status(void* stream) {
+  int dev = 0, optin = 0;
+  int* p = nullptr;
+  if (!device_facts(&dev, &p, &optin)) return FN_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int h = 0;
+  if (cudaMemcpyAsync(&h, p, sizeof h, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemsetAsync(p, 0, sizeof h, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+    return FN_ERR_CUDA;
+  return h ? FN_ERR_TIMEOUT : FN_OK;
+}
 
 void fn_last_launch(int32_t out[4]) {
   if (out) std::memcpy(out, tl_launch, sizeof tl_launch);

@@ -42,4 +42,14 @@ RQKernel FN_CAT(rq_pick, FN_INST_MODE, FN_INST_MAXP)(int V, bool cluster, bool n
   }
 }
 
+RQTmaKernel FN_CAT(rq_tma_pick, FN_INST_MODE, FN_INST_MAXP)(int V) {
+  constexpr int MODE = FN_INST_MODE, MAXP = FN_INST_MAXP;
+  switch (V) {
+    case 1: return rq_tma_kernel<MODE, MAXP, 1>;
+    case 2: return rq_tma_kernel<MODE, MAXP, 2>;
+    case 4: return rq_tma_kernel<MODE, MAXP, 4>;
+    default: return rq_tma_kernel<MODE, MAXP, 8>;
+  }
+}
+
 }  // namespace fn

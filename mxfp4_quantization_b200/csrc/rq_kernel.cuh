@@ -6,16 +6,17 @@
 // the quantization of the bf16 normed row that sgl-amd-mono PR #26's monokernel
 // notes call bit-exact against stand-alone quantization.
 //
-// HBM-bound, no tensor cores.  One row is owned by one thread block (large M)
-// or by a cluster of 2..8 blocks that exchange their partial sums through
-// distributed shared memory (small M).  Each thread owns V 16-byte vectors of
-// the row (8 bf16 each), vector index seg_base + threadIdx.x + k * blockDim.x,
-// so a warp touches 512 contiguous bytes per tensor per k.  Every load of the
-// row is issued before the first arithmetic; the row then lives in registers
-// (as packed bf16) until its codes are stored, so each byte of HBM is read
-// once and written once.
-//
-// MX blocks (32 elements) are 4 adjacent lanes, FP8 groups (128) are 16
+// HBM-bound, no tensor cores.  Three kernels share the per-vector stages below:
+//  * rq_kernel, CL = false: one thread block per row.  Every load of the row
+//    is issued before the first arithmetic; the row then lives in registers.
+//  * rq_kernel, CL = true (small M): a cluster of 2..8 blocks per row; the
+//    blocks exchange their partial sums through distributed shared memory.
+//  * rq_tma_kernel (large M): one persistent block per SM; a ring of shared
+//    memory stages is filled by bulk asynchronous copies (cp.async.bulk, the
+//    TMA engine, no multicast) several rows ahead of the row being computed.
+// A thread owns 16-byte vectors (8 bf16) with index seg_base + threadIdx.x +
+// k * blockDim.x, so a warp touches 512 contiguous bytes per tensor per k.
+// MX blocks (32 elements) are 4 adjacent lanes and FP8 groups (128) 16
 // adjacent lanes: their amax is a 2- or 4-step xor shuffle.
 #pragma once
 #include <cooperative_groups.h>
@@ -26,6 +27,168 @@
 namespace fn {
 
 namespace cg = cooperative_groups;
+
+// ---------------------------------------------------------------------------
+// per-vector stages
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = bf_lo(word(v, i));
+    f[2 * i + 1] = bf_hi(word(v, i));
+  }
+}
+
+// h = bf16(((x_0 + x_1) + ...) + r) for one vector, every add in fp32.
+template <int MAXP>
+__device__ __forceinline__ uint4 sum_vec(const uint4 (&x)[MAXP], const uint4& r, int P,
+                                         bool has_res) {
+  uint4 h;
+  if constexpr (MAXP == 1) {
+    h = has_res ? make_uint4(add_bf16x2(x[0].x, r.x), add_bf16x2(x[0].y, r.y),
+                             add_bf16x2(x[0].z, r.z), add_bf16x2(x[0].w, r.w))
+                : x[0];
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float a0 = bf_lo(word(x[0], i)), a1 = bf_hi(word(x[0], i));
+#pragma unroll
+      for (int p = 1; p < MAXP; ++p) {
+        if (p < P) {
+          a0 = add_bf16<false>(word(x[p], i), a0);
+          a1 = add_bf16<true>(word(x[p], i), a1);
+        }
+      }
+      if (has_res) {
+        a0 = add_bf16<false>(word(r, i), a0);
+        a1 = add_bf16<true>(word(r, i), a1);
+      }
+      set_word(h, i, pack_bf16x2(a0, a1));
+    }
+  }
+  return h;
+}
+
+// Sum of squares of h (two fp32 accumulators), and (per-token mode) max |h * w|.
+// h * w is exact in fp32 (two 8-bit significands) and y = bf16(fl(h * w) * rstd)
+// is monotone in |h * w|, so max |y| = bf16(fl(max |h * w| * rstd)) falls out
+// of the same reduction as the sum of squares.
+template <bool WANT_PMAX>
+__device__ __forceinline__ void stats_vec(const uint4& h, const uint4& w, float2& ss,
+                                          float& pmax) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t hw = word(h, i);
+    ss.x = fma_bf16<false>(hw, hw, ss.x);
+    ss.y = fma_bf16<true>(hw, hw, ss.y);
+    if (WANT_PMAX) {
+      const uint32_t ww = word(w, i);
+      pmax = fmaxf(pmax, fmaxf(fabsf(fma_bf16<false>(hw, ww, -0.f)),
+                               fabsf(fma_bf16<true>(hw, ww, -0.f))));
+    }
+  }
+}
+
+// y = bf16(fl(h * w) * rstd).
+__device__ __forceinline__ uint4 norm_vec(const uint4& h, const uint4& w, float rstd) {
+  uint4 y;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t hw = word(h, i), ww = word(w, i);
+    const float2 p = make_float2(fma_bf16<false>(hw, ww, -0.f), fma_bf16<true>(hw, ww, -0.f));
+    const float2 q = mul_f32x2(p, make_float2(rstd, rstd));
+    set_word(y, i, pack_bf16x2(q.x, q.y));
+  }
+  return y;
+}
+
+// FP8 scale of a group (or row) amax: amax / 448 (IEEE division), 1 for zero.
+__device__ __forceinline__ float fp8_scale(float amax) {
+  return amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+}
+
+// Eight E4M3 codes of fl32(y / s), the IEEE quotient.
+//
+// Fast path, for s >= 2^-120: with r = RN(1/s) and r_lo = RN(RN(1 - s r) r)
+// (so that r + r_lo carries 1/s to about 2^-46), q = RN(|y| r + RN(|y| r_lo))
+// has the same E4M3 code as RN(|y| / s) for every bf16 y with |y| <= amax and
+// every bf16 amax with s = RN(amax / 448) >= 2^-120; this was checked
+// exhaustively over all such (amax, y) pairs (tests/quotient_proof.c).  The
+// code is computed from |y| and y's sign bit is copied onto it, which also
+// gives -0 the code 0x80.  If any lane of the warp has s < 2^-120 the whole
+// warp takes the IEEE division instead (warp-uniform branch).  All 32 lanes
+// must call.
+__device__ __forceinline__ uint2 e4m3_codes(const uint4& y, float s) {
+  uint32_t c[4];
+  if (!__any_sync(0xffffffffu, !(s >= 0x1p-120f))) {
+    const float r = __frcp_rn(s);
+    const float r_lo = fmaf(-s, r, 1.f) * r;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t a = word(y, i) & 0x7FFF7FFFu;
+      const float2 ya = make_float2(bf_lo(a), bf_hi(a));
+      const float2 t = mul_f32x2(ya, make_float2(r_lo, r_lo));
+      const float2 q = fma_f32x2(ya, make_float2(r, r), t);
+      c[i] = cvt_e4m3x2(q.x, q.y);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t a = word(y, i) & 0x7FFF7FFFu;
+      c[i] = cvt_e4m3x2(__fdiv_rn(bf_lo(a), s), __fdiv_rn(bf_hi(a), s));
+    }
+  }
+  // byte k of code word j takes the sign of element 4j + k: the sign bits sit
+  // at bits 15 and 31 of each y word, i.e. in bytes 1 and 3
+  const uint32_t s0 = __byte_perm(y.x, y.y, 0x7531) & 0x80808080u;
+  const uint32_t s1 = __byte_perm(y.z, y.w, 0x7531) & 0x80808080u;
+  return make_uint2((c[0] | (c[1] << 16)) | s0, (c[2] | (c[3] << 16)) | s1);
+}
+
+// E2M1 codes of y * 2^-e for the 8 bf16 of a vector (inv_bf16 = 2^-e as a bf16
+// bit pattern in both halves): each product is exact, computed by the mixed
+// bf16 FMA with a -0 addend (which keeps the sign of zeros).
+__device__ __forceinline__ uint32_t e2m1_codes(const uint4& y, uint32_t inv_bf16) {
+  float f[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = fma_bf16<false>(word(y, i), inv_bf16, -0.f);
+    f[2 * i + 1] = fma_bf16<true>(word(y, i), inv_bf16, -0.f);
+  }
+  return cvt_e2m1x8(f);
+}
+
+// Quantize vector v of a row (y: 8 bf16) and store its codes and, from the
+// group's first lane, its scale.  All 32 lanes must call (shuffles); `ok`
+// masks the stores of lanes past the row end (whole groups, by alignment).
+template <int MODE>
+__device__ __forceinline__ void quant_store(const uint4& y, bool ok, int lane, int64_t row, int v,
+                                            int H, float scale_tok, uint8_t* out_q,
+                                            void* out_scale) {
+  if constexpr (MODE == MODE_TOKEN || MODE == MODE_G128) {
+    float s = scale_tok;
+    if constexpr (MODE == MODE_G128) {
+      s = fp8_scale(group_max<16>(vec_absmax(y)));
+      if (ok && (lane & 15) == 0) static_cast<float*>(out_scale)[row * (H / 128) + v / 16] = s;
+    }
+    const uint2 c = e4m3_codes(y, s);
+    if (ok) st_stream(reinterpret_cast<uint2*>(out_q + row * (int64_t)H) + v, c);
+  } else {
+    float inv;
+    const uint32_t code = mx_scale(group_max<4>(vec_absmax(y)), inv);
+    const uint32_t inv_b = __float_as_uint(inv) >> 16;  // 2^-e is exact in bf16
+    const uint32_t q = e2m1_codes(y, inv_b | (inv_b << 16));
+    if (ok) {
+      st_stream(reinterpret_cast<uint32_t*>(out_q + row * (int64_t)(H / 2)) + v, q);
+      if ((lane & 3) == 0) static_cast<uint8_t*>(out_scale)[row * (H / 32) + v / 4] = (uint8_t)code;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// reductions
+// ---------------------------------------------------------------------------
 
 // Cluster barrier halves (all threads of every block of the cluster take part).
 __device__ __forceinline__ void cluster_arrive() {
@@ -72,6 +235,19 @@ __device__ __forceinline__ float2 row_reduce(float s, float m, float2* red, floa
   return t;
 }
 
+__device__ __forceinline__ float row_rstd(float ss, int H, float eps) {
+  return (float)(1.0 / sqrt((double)ss / (double)H + (double)eps));
+}
+
+// bf16(fl(pmax * rstd)): the row's max |y| (see stats_vec).
+__device__ __forceinline__ float row_amax_from_pmax(float pmax, float rstd) {
+  return bf_lo(pack_bf16x2(pmax * rstd, 0.f));
+}
+
+// ---------------------------------------------------------------------------
+// register-resident kernel: one row per block (CL = false) or per cluster
+// ---------------------------------------------------------------------------
+
 template <int MODE, int MAXP, int V, bool NORM, bool CL>
 __global__ void __launch_bounds__(CL ? 512 : 256)
     rq_kernel(const __grid_constant__ RQParams prm) {
@@ -90,11 +266,12 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
   }
   const int seg_base = rank * prm.seg, seg_end = seg_base + prm.seg;
   const int64_t rowv = row * (int64_t)prm.nvec;
+  const int H = prm.nvec * 8;
   const bool has_res = NORM && prm.residual != nullptr;
   const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
 
   // ---- 1. issue every load of this block's part of the row -------------------
-  uint4 xin[MAXP][V];
+  uint4 xin[V][MAXP];
   uint4 rin[V];
   uint4 win[V];
 #pragma unroll
@@ -103,146 +280,206 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
     const bool ok = v < seg_end;
 #pragma unroll
     for (int p = 0; p < MAXP; ++p)
-      xin[p][k] = (ok && p < prm.P) ? ld_stream_nc(prm.parts[p] + rowv + v) : zero;
+      xin[k][p] = (ok && p < prm.P) ? ld_stream_nc(prm.parts[p] + rowv + v) : zero;
     if constexpr (NORM) {
       rin[k] = (ok && has_res) ? ld_stream(prm.residual + rowv + v) : zero;
       win[k] = ok ? ld_keep(prm.weight + v) : zero;
     }
   }
 
-  // ---- 2. h = bf16(((x0 + x1) + ...) + r), residual_out, sum of squares ----------
-  // Also max |h * w| for the per-token scale: h * w is exact in fp32 (two
-  // 8-bit significands), y = bf16(fl(h * w) * rstd) is monotone in |h * w|, so
-  // max |y| = bf16(fl(max |h * w| * rstd)) comes out of the same reduction.
   uint4 yv[V];
-  float row_amax = 0.f;
+  float scale_tok = 1.f;
   if constexpr (NORM) {
+    // ---- 2. h, residual_out, statistics --------------------------------------------
     uint4 hv[V];
-    float ss = 0.f, pmax = 0.f;
+    float2 ss = make_float2(0.f, 0.f);
+    float pmax = 0.f;
 #pragma unroll
     for (int k = 0; k < V; ++k) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float a0 = bf_lo(word(xin[0][k], i)), a1 = bf_hi(word(xin[0][k], i));
-#pragma unroll
-        for (int p = 1; p < MAXP; ++p) {
-          if (p < prm.P) {
-            a0 += bf_lo(word(xin[p][k], i));
-            a1 += bf_hi(word(xin[p][k], i));
-          }
-        }
-        if (has_res) {
-          a0 += bf_lo(word(rin[k], i));
-          a1 += bf_hi(word(rin[k], i));
-        }
-        const uint32_t hw = pack_bf16x2(a0, a1);
-        set_word(hv[k], i, hw);
-        const float h0 = bf_lo(hw), h1 = bf_hi(hw);
-        ss = fmaf(h0, h0, ss);
-        ss = fmaf(h1, h1, ss);
-        if (MODE == MODE_TOKEN) {
-          const uint32_t ww = word(win[k], i);
-          pmax = fmaxf(pmax, fmaxf(fabsf(h0 * bf_lo(ww)), fabsf(h1 * bf_hi(ww))));
-        }
-      }
+      hv[k] = sum_vec<MAXP>(xin[k], rin[k], prm.P, has_res);
+      stats_vec<MODE == MODE_TOKEN>(hv[k], win[k], ss, pmax);
       const int v = seg_base + t + k * T;
       if (v < seg_end && prm.out_residual != nullptr) st_stream(prm.out_residual + rowv + v, hv[k]);
     }
-
-    // ---- 3. rstd = 1 / sqrt(mean(h^2) + eps) --------------------------------------
-    const float2 tot = row_reduce<CL, MODE == MODE_TOKEN>(ss, pmax, red, &cl_slot);
-    const float rstd =
-        (float)(1.0 / sqrt((double)tot.x / (double)(prm.nvec * 8) + (double)prm.eps));
-    if (MODE == MODE_TOKEN) row_amax = __uint_as_float(pack_bf16x2(tot.y * rstd, 0.f) << 16);
-
-    // ---- 4. y = bf16(fl(h * w) * rstd) --------------------------------------------
+    // ---- 3. rstd (and the per-token amax) ---------------------------------------------
+    const float2 tot = row_reduce<CL, MODE == MODE_TOKEN>(ss.x + ss.y, pmax, red, &cl_slot);
+    const float rstd = row_rstd(tot.x, H, prm.eps);
+    if (MODE == MODE_TOKEN) scale_tok = fp8_scale(row_amax_from_pmax(tot.y, rstd));
+    // ---- 4. y = bf16(fl(h * w) * rstd) ----------------------------------------------
 #pragma unroll
     for (int k = 0; k < V; ++k) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t hw = word(hv[k], i), ww = word(win[k], i);
-        const float y0 = (bf_lo(hw) * bf_lo(ww)) * rstd;
-        const float y1 = (bf_hi(hw) * bf_hi(ww)) * rstd;
-        set_word(yv[k], i, pack_bf16x2(y0, y1));
-      }
+      yv[k] = norm_vec(hv[k], win[k], rstd);
       const int v = seg_base + t + k * T;
       if (v < seg_end && prm.out_y != nullptr) st_stream(prm.out_y + rowv + v, yv[k]);
     }
   } else {
 #pragma unroll
-    for (int k = 0; k < V; ++k) yv[k] = xin[0][k];
+    for (int k = 0; k < V; ++k) yv[k] = xin[k][0];
     if (MODE == MODE_TOKEN) {
       float am = 0.f;
 #pragma unroll
-      for (int k = 0; k < V; ++k)
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          am = fmaxf(am, fmaxf(fabsf(bf_lo(word(yv[k], i))), fabsf(bf_hi(word(yv[k], i)))));
-      row_amax = row_reduce<CL, true>(0.f, am, red, &cl_slot).y;
+      for (int k = 0; k < V; ++k) am = fmaxf(am, vec_absmax(yv[k]));
+      scale_tok = fp8_scale(row_reduce<CL, true>(0.f, am, red, &cl_slot).y);
     }
   }
+  if (MODE == MODE_TOKEN && rank == 0 && t == 0) static_cast<float*>(prm.out_scale)[row] = scale_tok;
 
   // ---- 5. quantize y ----------------------------------------------------------------
-  const int H = prm.nvec * 8;
-  if constexpr (MODE == MODE_TOKEN || MODE == MODE_G128) {
-    float scale_tok = 1.f;
-    if constexpr (MODE == MODE_TOKEN) {
-      scale_tok = row_amax == 0.f ? 1.f : __fdiv_rn(row_amax, 448.f);
-      if (rank == 0 && t == 0) static_cast<float*>(prm.out_scale)[row] = scale_tok;
-    }
 #pragma unroll
-    for (int k = 0; k < V; ++k) {
-      const int v = seg_base + t + k * T;
-      float scale = scale_tok;
-      if constexpr (MODE == MODE_G128) {
-        float am = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          am = fmaxf(am, fmaxf(fabsf(bf_lo(word(yv[k], i))), fabsf(bf_hi(word(yv[k], i)))));
-        const float amax = group_max<16>(am);
-        scale = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
-        if (v < seg_end && (lane & 15) == 0)
-          static_cast<float*>(prm.out_scale)[row * (H / 128) + v / 16] = scale;
-      }
-      uint32_t c[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        c[i] = cvt_e4m3x2(__fdiv_rn(bf_lo(word(yv[k], i)), scale),
-                          __fdiv_rn(bf_hi(word(yv[k], i)), scale));
-      if (v < seg_end)
-        st_stream(reinterpret_cast<uint2*>(prm.out_q + row * (int64_t)H) + v,
-                  make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16)));
-    }
-  } else {  // MODE_MX
-#pragma unroll
-    for (int k = 0; k < V; ++k) {
-      const int v = seg_base + t + k * T;
-      float f[8];
-      float am = 0.f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        f[2 * i] = bf_lo(word(yv[k], i));
-        f[2 * i + 1] = bf_hi(word(yv[k], i));
-        am = fmaxf(am, fmaxf(fabsf(f[2 * i]), fabsf(f[2 * i + 1])));
-      }
-      const float amax = group_max<4>(am);
-      float inv;
-      const uint32_t code = mx_scale(amax, inv);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) f[i] *= inv;  // exact: a power of two
-      const uint32_t q = cvt_e2m1x8(f);
-      if (v < seg_end) {
-        st_stream(reinterpret_cast<uint32_t*>(prm.out_q + row * (int64_t)(H / 2)) + v, q);
-        if ((lane & 3) == 0)
-          static_cast<uint8_t*>(prm.out_scale)[row * (H / 32) + v / 4] = (uint8_t)code;
-      }
-    }
+  for (int k = 0; k < V; ++k) {
+    const int v = seg_base + t + k * T;
+    quant_store<MODE>(yv[k], v < seg_end, lane, row, v, H, scale_tok, prm.out_q, prm.out_scale);
   }
 
   if constexpr (CL) {
     // No block may leave while a peer can still read its shared-memory slot.
     cluster_wait();
   }
+}
+
+// ---------------------------------------------------------------------------
+// TMA-staged persistent kernel (large M)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// Wait for the phase with the given parity to complete.  Bounded: gives up
+// after `limit` polls and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
+  const uint32_t a = smem_addr(bar);
+  for (uint32_t it = 0; it < limit; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+// Bulk asynchronous copy global -> this block's shared memory (no multicast);
+// completion is counted in bytes on `bar`.  16-byte aligned, size % 16 == 0.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+constexpr uint32_t kWaitLimit = 1u << 24;
+
+// Shared memory: nstages stages of (P + has_res) row segments of H bf16, then
+// one mbarrier per stage.  Block b handles rows b, b + gridDim.x, ...; the
+// copies of the next nstages rows are in flight while a row is computed.  A
+// stage is refilled as soon as the block has read it into registers (after
+// the sum-of-squares reduction's barrier), before rstd, y and the codes.
+template <int MODE, int MAXP, int V>
+__global__ void __launch_bounds__(512, 1)
+    rq_tma_kernel(const __grid_constant__ RQParams prm, int nstages) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float2 red[2][32];
+
+  const int T = blockDim.x, t = threadIdx.x, lane = t & 31;
+  const int nvec = prm.nvec, H = nvec * 8;
+  const bool has_res = prm.residual != nullptr;
+  const int ntensor = prm.P + (has_res ? 1 : 0);
+  const uint32_t seg_bytes = (uint32_t)H * 2u;
+  const uint32_t stage_bytes = seg_bytes * (uint32_t)ntensor;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)nstages * stage_bytes);
+  const int64_t M = prm.M;
+  const int64_t first = blockIdx.x, step = gridDim.x;
+  const int64_t nrows = first < M ? (M - first + step - 1) / step : 0;
+
+  // The weight stays in registers for every row this block handles.
+  uint4 wv[V];
+#pragma unroll
+  for (int k = 0; k < V; ++k) {
+    const int v = t + k * T;
+    wv[k] = v < nvec ? ld_keep(prm.weight + v) : make_uint4(0u, 0u, 0u, 0u);
+  }
+
+  auto issue = [&](int64_t i) {
+    const int s = (int)(i % nstages);
+    const int64_t row = first + i * step;
+    uint8_t* dst = smem + (size_t)s * stage_bytes;
+    mbar_expect_tx(&full[s], stage_bytes);
+    for (int p = 0; p < prm.P; ++p)
+      bulk_load(dst + (size_t)p * seg_bytes, prm.parts[p] + row * nvec, seg_bytes, &full[s]);
+    if (has_res)
+      bulk_load(dst + (size_t)prm.P * seg_bytes, prm.residual + row * nvec, seg_bytes, &full[s]);
+  };
+
+  if (t == 0) {
+    for (int s = 0; s < nstages; ++s) mbar_init(&full[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int64_t i = 0; i < nrows && i < nstages; ++i) issue(i);
+  }
+  __syncthreads();
+
+  bool timed_out = false;
+  for (int64_t i = 0; i < nrows; ++i) {
+    const int s = (int)(i % nstages);
+    const int64_t row = first + i * step;
+    const int64_t rowv = row * nvec;
+    if (!mbar_wait(&full[s], (uint32_t)((i / nstages) & 1), kWaitLimit)) timed_out = true;
+    const uint4* st = reinterpret_cast<const uint4*>(smem + (size_t)s * stage_bytes);
+
+    uint4 hv[V];
+    float2 ss = make_float2(0.f, 0.f);
+    float pmax = 0.f;
+#pragma unroll
+    for (int k = 0; k < V; ++k) {
+      const int v = t + k * T;
+      const bool ok = v < nvec;
+      uint4 x[MAXP];
+#pragma unroll
+      for (int p = 0; p < MAXP; ++p)
+        x[p] = (ok && p < prm.P) ? st[p * nvec + v] : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 r = (ok && has_res) ? st[prm.P * nvec + v] : make_uint4(0u, 0u, 0u, 0u);
+      hv[k] = sum_vec<MAXP>(x, r, prm.P, has_res);
+      stats_vec<MODE == MODE_TOKEN>(hv[k], wv[k], ss, pmax);
+      if (ok && prm.out_residual != nullptr) st_stream(prm.out_residual + rowv + v, hv[k]);
+    }
+    const float2 tot =
+        row_reduce<false, MODE == MODE_TOKEN>(ss.x + ss.y, pmax, red[i & 1], nullptr);
+    // every thread has read stage s: refill it with the row nstages ahead
+    if (t == 0 && i + nstages < nrows) issue(i + nstages);
+
+    const float rstd = row_rstd(tot.x, H, prm.eps);
+    float scale_tok = 1.f;
+    if (MODE == MODE_TOKEN) {
+      scale_tok = fp8_scale(row_amax_from_pmax(tot.y, rstd));
+      if (t == 0) static_cast<float*>(prm.out_scale)[row] = scale_tok;
+    }
+#pragma unroll
+    for (int k = 0; k < V; ++k) {
+      const int v = t + k * T;
+      const bool ok = v < nvec;
+      const uint4 y = norm_vec(hv[k], wv[k], rstd);
+      if (ok && prm.out_y != nullptr) st_stream(prm.out_y + rowv + v, y);
+      quant_store<MODE>(y, ok, lane, row, v, H, scale_tok, prm.out_q, prm.out_scale);
+    }
+  }
+  if (timed_out && prm.status != nullptr) atomicExch(prm.status, 1);
 }
 
 }  // namespace fn

@@ -20,6 +20,7 @@ struct RQParams {
   int seg;                 // vectors of a row handled by one block
   int P;                   // partial count, <= MAXP
   float eps;
+  int* status;             // library status word: set to 1 if a bounded wait gave up
 };
 
 // A kernel instance: every (mode, partial bound, vectors per thread, norm,
@@ -29,7 +30,12 @@ using RQKernel = void (*)(const RQParams);
 // Per-(mode, partial bound) instantiation units, each compiled separately
 // (rq_inst.cu) so the library builds in parallel.  `V` is ignored for
 // cluster launches (always one vector per thread there).
-#define FN_RQ_DECL(MODE, MAXP) RQKernel rq_pick_##MODE##_##MAXP(int V, bool cluster, bool norm);
+// The TMA-staged persistent kernel takes the stage count as a second argument.
+using RQTmaKernel = void (*)(const RQParams, int);
+
+#define FN_RQ_DECL(MODE, MAXP)                                          \
+  RQKernel rq_pick_##MODE##_##MAXP(int V, bool cluster, bool norm); \
+  RQTmaKernel rq_tma_pick_##MODE##_##MAXP(int V);
 FN_RQ_DECL(0, 1)
 FN_RQ_DECL(0, 2)
 FN_RQ_DECL(0, 4)

@@ -37,6 +37,7 @@ FN_VARIANT_ROW_CTA = 1
 FN_VARIANT_ROW_CLUSTER = 2
 FN_VARIANT_QUANT_ONLY = 3
 FN_VARIANT_QK_WARP = 4
+FN_VARIANT_ROW_TMA = 5
 
 FN_MAX_PARTS = 8
 FN_MAX_H = 32768
@@ -47,7 +48,8 @@ MODES = {"fp8_per_token": FN_FP8_PER_TOKEN, "fp8_per_group128": FN_FP8_PER_GROUP
 
 # The exported symbols of include/fusednorm.h.
 ABI_SYMBOLS = ("fn_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate", "fn_status_string",
-               "fn_last_variant", "fn_last_launch", "fn_version")
+               "fn_last_variant", "fn_last_launch", "fn_prefer_variant", "fn_device_status",
+               "fn_version")
 
 
 class FusedNormError(RuntimeError):
@@ -76,6 +78,10 @@ def _load():
     lib.fn_last_variant.restype = i32
     lib.fn_last_launch.argtypes = [ctypes.POINTER(ctypes.c_int32)]
     lib.fn_last_launch.restype = None
+    lib.fn_prefer_variant.argtypes = [i32]
+    lib.fn_prefer_variant.restype = i32
+    lib.fn_device_status.argtypes = [vp]
+    lib.fn_device_status.restype = i32
     lib.fn_version.argtypes = []
     lib.fn_version.restype = i32
     return lib
@@ -123,8 +129,36 @@ def fn_last_launch():
     return tuple(out)
 
 
+def fn_prefer_variant(variant: int) -> int:
+    return _lib.fn_prefer_variant(variant)
+
+
+def fn_device_status(stream: Optional[int]) -> int:
+    return _lib.fn_device_status(stream)
+
+
 def fn_version() -> int:
     return _lib.fn_version()
+
+
+class prefer_variant:
+    """Context manager: ask fn_rmsnorm_quant for one kernel on this thread."""
+
+    def __init__(self, variant: int):
+        self.variant = variant
+
+    def __enter__(self):
+        self.old = fn_prefer_variant(self.variant)
+        return self
+
+    def __exit__(self, *exc):
+        fn_prefer_variant(self.old)
+        return False
+
+
+def device_status() -> int:
+    """fn_device_status on the current stream."""
+    return fn_device_status(torch.cuda.current_stream().cuda_stream)
 
 
 # ---- tensor API ----------------------------------------------------------------------

@@ -1,0 +1,81 @@
+/*
+ * Exhaustive check of the E4M3 quotient used by the FP8 kernels.
+ *
+ * The kernels need code = E4M3_rn_satfinite(RN(y / s)) for a bf16 element y of
+ * a group whose bf16 amax gives the scale s = RN(amax / 448).  Instead of an
+ * IEEE division per element they compute, from |y| and once per group
+ *     r    = RN(1 / s)
+ *     r_lo = RN(RN(1 - s r) * r)          (1 - s r by one fused multiply-add)
+ *     q    = RN(|y| r + RN(|y| r_lo))      (one multiply, one fused multiply-add)
+ * and copy y's sign onto the code.  This program runs every positive finite
+ * bf16 amax with s >= 2^-120 against every bf16 |y| <= amax (about 5.3e8
+ * pairs) and counts the pairs whose E4M3 codes differ.  It exits 0 iff there
+ * are none.  argv[1] (optional) strides the amax loop for a quicker run.
+ *
+ * Build: cc -O2 -ffp-contract=off -o quotient_proof quotient_proof.c -lm
+ * (fmaf must be the correctly rounded fused multiply-add: glibc's is.)
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+static float from_bf16(uint32_t b)
+{
+    uint32_t u = b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* E4M3 ("fn") code of a non-negative float: nearest even on the grid with 3
+ * mantissa bits and minimum normal exponent -6, saturating at 448. */
+static int e4m3_code(float v)
+{
+    double a = (double)v;
+    if (a == 0.0)
+        return 0;
+    int e;
+    (void)frexp(a, &e);
+    int ex = e - 1 < -6 ? -6 : e - 1;
+    double quantum = ldexp(1.0, ex - 3);
+    double r = nearbyint(a / quantum) * quantum;
+    if (r > 448.0)
+        r = 448.0;
+    if (r == 0.0)
+        return 0;
+    (void)frexp(r, &e);
+    ex = e - 1;
+    if (ex < -6)
+        return (int)(r / ldexp(1.0, -9));
+    return ((ex + 7) << 3) | (int)((r / ldexp(1.0, ex) - 1.0) * 8.0);
+}
+
+int main(int argc, char** argv)
+{
+    uint32_t stride = argc > 1 ? (uint32_t)strtoul(argv[1], NULL, 10) : 1u;
+    if (stride == 0)
+        stride = 1;
+    long pairs = 0, bad = 0;
+    for (uint32_t ab = 1; ab < 0x7F80u; ab += stride) {
+        const float amax = from_bf16(ab);
+        const float s = amax / 448.0f;
+        if (!(s >= 0x1p-120f))
+            continue;
+        const float r = 1.0f / s;
+        const float r_lo = fmaf(-s, r, 1.0f) * r;
+        for (uint32_t yb = 0; yb <= ab; ++yb) {
+            const float y = from_bf16(yb);
+            const float q = fmaf(y, r, y * r_lo);
+            if (e4m3_code(q) != e4m3_code(y / s)) {
+                if (bad < 10)
+                    printf("mismatch: amax=%a y=%a q=%a y/s=%a\n", amax, y, q, y / s);
+                ++bad;
+            }
+            ++pairs;
+        }
+    }
+    printf("pairs %ld mismatches %ld\n", pairs, bad);
+    return bad != 0;
+}

@@ -29,7 +29,8 @@ def declared_symbols():
 def test_header_declares_the_abi():
     assert declared_symbols() == sorted(["fn_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate",
                                          "fn_status_string", "fn_last_variant",
-                                         "fn_last_launch", "fn_version"])
+                                         "fn_last_launch", "fn_prefer_variant",
+                                         "fn_device_status", "fn_version"])
 
 
 def test_library_exports_every_declared_symbol(fnb):
@@ -47,7 +48,8 @@ def test_header_constants_match_binding(fnb):
     src = open(HEADER).read()
     for name in ("FN_FP8_PER_TOKEN", "FN_FP8_PER_GROUP128", "FN_MXFP4", "FN_ERR_INVALID",
                  "FN_ERR_ALIGN", "FN_ERR_UNSUPPORTED", "FN_ERR_CUDA", "FN_VARIANT_ROW_CTA",
-                 "FN_VARIANT_ROW_CLUSTER", "FN_VARIANT_QUANT_ONLY", "FN_VARIANT_QK_WARP"):
+                 "FN_VARIANT_ROW_CLUSTER", "FN_VARIANT_QUANT_ONLY", "FN_VARIANT_QK_WARP",
+                 "FN_VARIANT_ROW_TMA", "FN_ERR_TIMEOUT"):
         m = re.search(rf"\b{name}\s*=\s*(-?\d+)", src)
         assert m and int(m.group(1)) == getattr(fnb, name), name
     for name in ("FN_MAX_PARTS", "FN_MAX_H", "FN_MAX_HEAD_DIM"):
@@ -139,3 +141,14 @@ def test_qk_norm_gate_rejects_bad_arguments(fnb):
         assert qk(fnb, **kw) == want, kw
     assert qk(fnb, M=0) == fnb.FN_OK
     assert qk(fnb, M=0, Hk=0, k_weight=None, out_k=None) == fnb.FN_OK
+
+
+def test_prefer_variant_is_thread_local_and_returns_previous(fnb):
+    import threading
+    assert fnb.fn_prefer_variant(fnb.FN_VARIANT_ROW_TMA) == fnb.FN_VARIANT_NONE
+    seen = []
+    th = threading.Thread(target=lambda: seen.append(fnb.fn_prefer_variant(0)))
+    th.start()
+    th.join()
+    assert seen == [fnb.FN_VARIANT_NONE]
+    assert fnb.fn_prefer_variant(fnb.FN_VARIANT_NONE) == fnb.FN_VARIANT_ROW_TMA

@@ -76,3 +76,20 @@ def test_negative_tiny_values_keep_their_sign(fnb):
                                    mode)
     q, _ = fnb.quant(yt, oracle.FP8_PER_GROUP128)
     assert np.all(gpu_util.u8(q)[0, 1:9] == 0x80)
+
+
+@pytest.mark.parametrize("mode", [oracle.FP8_PER_TOKEN, oracle.FP8_PER_GROUP128, oracle.MXFP4])
+def test_quant_stage_random_scales(fnb, mode):
+    """Many groups, each with its own magnitude 2^U(-130, 120): the FP8
+    quotient's fast path (reciprocal multiply) and its exact fallbacks
+    (near-midpoint, E4M3-subnormal, tiny scale) all against IEEE division."""
+    g = torch.Generator().manual_seed(77 + mode)
+    M, H = 4096, 1024
+    mag = torch.pow(2.0, torch.randint(-130, 120, (M, H // 128, 1), generator=g).float())
+    y = (torch.randn((M, H // 128, 128), generator=g) * mag).reshape(M, H)
+    y[::7, 5] = 0.0
+    y[::11, 9] = -0.0
+    yb = y.to(torch.bfloat16)
+    q, s = fnb.quant(yb.cuda(), mode)
+    torch.cuda.synchronize()
+    parity.compare_quant_stage(gpu_util.bits(yb), gpu_util.u8(q), gpu_util.scale_np(s, mode), mode)

@@ -19,8 +19,10 @@ def fnb():
     return gpu_util.lib()
 
 
-def run(fnb, wl, M=None, in_place=False, guarded=True, emit_y=True, device_inputs=None):
-    """Run the fused kernel on `wl`'s inputs (drawn on the CPU unless given)."""
+def run(fnb, wl, M=None, in_place=False, guarded=True, emit_y=True, device_inputs=None,
+        variant=0):
+    """Run the fused kernel on `wl`'s inputs (drawn on the CPU unless given),
+    asking for kernel `variant` (0: the library's choice)."""
     M = wl.M if M is None else M
     inp = wl.inputs(device="cpu", M=M) if device_inputs is None else device_inputs
     parts = [p.cuda() for p in inp["parts"]]
@@ -33,11 +35,13 @@ def run(fnb, wl, M=None, in_place=False, guarded=True, emit_y=True, device_input
     gs = gpu_util.Guarded(s_shape, torch.uint8 if wl.mode == MX else torch.float32)
     gy = gpu_util.Guarded((M, H), torch.bfloat16) if emit_y else None
     gr = gpu_util.Guarded((M, H), torch.bfloat16) if (res is not None and not in_place) else None
-    out = fnb.rmsnorm_quant(parts, w, wl.eps, wl.mode, residual=res, in_place=in_place,
-                            out_residual=None if gr is None else gr.t, out_q=gq.t,
-                            out_scale=gs.t, out_y=None if gy is None else gy.t)
+    with fnb.prefer_variant(variant):
+        out = fnb.rmsnorm_quant(parts, w, wl.eps, wl.mode, residual=res, in_place=in_place,
+                                out_residual=None if gr is None else gr.t, out_q=gq.t,
+                                out_scale=gs.t, out_y=None if gy is None else gy.t)
     variant, launch = fnb.fn_last_variant(), fnb.fn_last_launch()
     torch.cuda.synchronize()
+    assert fnb.device_status() == fnb.FN_OK
     for g in (gq, gs, gy, gr):
         assert g is None or g.intact(), "write outside an output"
     gpu = {"q": gpu_util.u8(gq.t), "scale": gpu_util.scale_np(gs.t, wl.mode),
@@ -62,14 +66,26 @@ SHAPES = [
 ]
 
 
+VARIANTS = {"auto": 0, "cta": 1, "cluster": 2, "tma": 5}
+
+
+def tma_fits(H, P, has_res):
+    return (P + (1 if has_res else 0)) * H * 2 * 2 <= 220 * 1024
+
+
+@pytest.mark.parametrize("variant", ["auto", "cta", "tma"])
 @pytest.mark.parametrize("mode", [TOKEN, G128, MX], ids=["token", "g128", "mxfp4"])
 @pytest.mark.parametrize("M,H,P,has_res", SHAPES, ids=[f"M{s[0]}_H{s[1]}_P{s[2]}_{'r' if s[3] else 'nr'}" for s in SHAPES])
-def test_parity(fnb, mode, M, H, P, has_res):
+def test_parity(fnb, mode, M, H, P, has_res, variant):
     wl = synth.RowWorkload("case", M=M, H=H, P=P, mode=mode, eps=1e-6 if H % 3 else 1e-5,
                            seed=M * 31 + H + P, residual=has_res, outlier_frac=0.01,
                            channel_decades=1.0 if P > 1 else 0.0)
-    inp, gpu, variant, launch = run(fnb, wl)
-    assert variant in (fnb.FN_VARIANT_ROW_CTA, fnb.FN_VARIANT_ROW_CLUSTER)
+    inp, gpu, got, launch = run(fnb, wl, variant=VARIANTS[variant])
+    assert got in (fnb.FN_VARIANT_ROW_CTA, fnb.FN_VARIANT_ROW_CLUSTER, fnb.FN_VARIANT_ROW_TMA)
+    if variant == "cta":
+        assert got == fnb.FN_VARIANT_ROW_CTA
+    if variant == "tma" and tma_fits(H, P, has_res):
+        assert got == fnb.FN_VARIANT_ROW_TMA, launch
     check(wl, inp, gpu)
 
 
@@ -80,8 +96,9 @@ def test_smallest_rows(fnb, mode, H):
     check(wl, inp, gpu)
 
 
+@pytest.mark.parametrize("variant", ["auto", "cta", "tma", "cluster"])
 @pytest.mark.parametrize("mode", [TOKEN, G128, MX])
-def test_in_place_residual(fnb, mode):
+def test_in_place_residual(fnb, mode, variant):
     wl = synth.RowWorkload("inplace", M=48, H=8192, P=1, mode=mode, eps=1e-5, seed=5, x_std=2.0)
     inp = wl.inputs(device="cpu")
     inp_copy = {"parts": [p.clone() for p in inp["parts"]], "residual": inp["residual"].clone(),
@@ -90,7 +107,8 @@ def test_in_place_residual(fnb, mode):
     parts = [p.cuda() for p in dev["parts"]]
     res = dev["residual"].cuda()
     w = dev["weight"].cuda()
-    out = fnb.rmsnorm_quant(parts, w, wl.eps, mode, residual=res, in_place=True, emit_y=True)
+    with fnb.prefer_variant(VARIANTS[variant]):
+        out = fnb.rmsnorm_quant(parts, w, wl.eps, mode, residual=res, in_place=True, emit_y=True)
     torch.cuda.synchronize()
     assert out.residual_out.data_ptr() == res.data_ptr()
     gpu = {"q": gpu_util.u8(out.q), "scale": gpu_util.scale_np(out.scale, mode),
@@ -100,9 +118,10 @@ def test_in_place_residual(fnb, mode):
 
 def test_dispatch(fnb):
     """Small M takes the cluster kernel, large M one block per row."""
-    for M, want in ((1, fnb.FN_VARIANT_ROW_CLUSTER), (16, fnb.FN_VARIANT_ROW_CLUSTER),
-                    (512, fnb.FN_VARIANT_ROW_CTA)):
-        wl = synth.decode(M, MX) if M <= 16 else synth.RowWorkload("big", M=M, H=7168, P=1,
+    for M, P, want in ((1, 1, fnb.FN_VARIANT_ROW_CLUSTER), (16, 1, fnb.FN_VARIANT_ROW_CLUSTER),
+                       (200, 4, fnb.FN_VARIANT_ROW_CTA), (512, 1, fnb.FN_VARIANT_ROW_CTA),
+                       (512, 4, fnb.FN_VARIANT_ROW_TMA)):
+        wl = synth.decode(M, MX) if M <= 16 else synth.RowWorkload("big", M=M, H=7168, P=P,
                                                                      mode=MX, eps=1e-6)
         _, _, variant, launch = run(fnb, wl)
         assert variant == want, (M, variant, launch)
@@ -128,14 +147,17 @@ def test_empty_and_rejected_calls_touch_nothing(fnb):
                           out_scale=gs.t.view(torch.uint8))
 
 
-def test_replays_are_bit_identical(fnb):
+@pytest.mark.parametrize("variant", ["cta", "tma"])
+def test_replays_are_bit_identical(fnb, variant):
     wl = synth.RowWorkload("det", M=300, H=7168, P=4, mode=MX, eps=1e-6, seed=9,
                            channel_decades=1.0)
     inp = wl.inputs(device="cuda")
     outs = []
     for _ in range(3):
-        o = fnb.rmsnorm_quant(inp["parts"], inp["weight"], wl.eps, MX, residual=inp["residual"],
-                              emit_y=True)
+        with fnb.prefer_variant(VARIANTS[variant]):
+            o = fnb.rmsnorm_quant(inp["parts"], inp["weight"], wl.eps, MX,
+                                  residual=inp["residual"], emit_y=True)
+        assert fnb.fn_last_variant() == VARIANTS[variant]
         outs.append([t.clone() for t in o])
     torch.cuda.synchronize()
     for o in outs[1:]:
