@@ -26,7 +26,6 @@ import statistics
 import subprocess
 import sys
 import tempfile
-import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -92,15 +91,20 @@ def aggregate(rows_per_rank: int, world: int, ms_per_step_max: float) -> float:
 
 
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples of the SM clock and throttle reasons (read only).
+    `mark_start()` / `mark_end()` bracket the timed region; only samples taken
+    inside it are summarised."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, device_index: int, period_ms: int = 50):
         self.proc = None
         self.out = None
         self.dev = device_index
         self.period = period_ms
+        self.t0 = self.t1 = None
 
     def _uuid(self):
         import torch
@@ -122,10 +126,19 @@ class ClockSampler:
         except (OSError, FileNotFoundError):
             self.proc = None
 
+    def mark_start(self):
+        import datetime
+        self.t0 = datetime.datetime.now()
+
+    def mark_end(self):
+        import datetime
+        self.t1 = datetime.datetime.now()
+
     def stop(self):
+        import datetime
         if self.proc is None:
             return None
-        time.sleep(self.period / 1000.0)
+        time.sleep(2 * self.period / 1000.0)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -134,21 +147,26 @@ class ClockSampler:
         self.out.seek(0)
         rows = [ln.strip().split(", ") for ln in self.out.read().splitlines() if ln.strip()]
         os.unlink(self.out.name)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons, n_all = [], [], set(), 0
         for r in rows:
             try:
-                sm.append(float(r[0]))
-                mx.append(float(r[1]))
+                ts = datetime.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f")
+                smv, mxv = float(r[1]), float(r[2])
             except (ValueError, IndexError):
                 continue
-            for n, v in zip(names, r[4:8]):
+            n_all += 1
+            if self.t0 and self.t1 and not (self.t0 <= ts <= self.t1):
+                continue
+            sm.append(smv)
+            mx.append(mxv)
+            for n, v in zip(self.REASONS, r[5:9]):
                 if v.strip().lower() == "active":
                     reasons.add(n)
         if not sm:
-            return None
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "samples_total": n_all}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "samples_total": n_all}
 
 
 # ---------------------------------------------------------------------------
@@ -156,7 +174,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 
-def time_steps(fn_step, steps: int, warmup: int, device, stream):
+def time_steps(fn_step, steps: int, warmup: int, device, stream, clocks=None):
     """Untimed warm-up, then `steps` calls bracketed by a barrier and a
     synchronize, timed with CUDA events on the launching stream.
     Returns ms per step on this rank."""
@@ -168,11 +186,15 @@ def time_steps(fn_step, steps: int, warmup: int, device, stream):
     torch.cuda.synchronize(device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    if clocks is not None:
+        clocks.mark_start()
     e0.record(stream)
     for _ in range(steps):
         fn_step()
     e1.record(stream)
     torch.cuda.synchronize(device)
+    if clocks is not None:
+        clocks.mark_end()
     barrier(device)
     return e0.elapsed_time(e1) / steps
 
@@ -523,7 +545,7 @@ def main_arm(args):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(device)
-    ms = time_steps(step, args.steps, 0, device, stream)
+    ms = time_steps(step, args.steps, 0, device, stream, clocks)
     clk = clocks.stop()
     variant, launch = fn.fn_last_variant(), fn.fn_last_launch()
     ms_max = dist_max(ms, device)
