@@ -162,7 +162,8 @@ FN_API int fn_last_variant(void);
 
 /* Launch shape of the calling thread's last launch: out[0] grid blocks,
  * out[1] threads per block, out[2] blocks per cluster (FN_VARIANT_ROW_TMA:
- * shared-memory stages), out[3] 16-byte vectors per thread per tensor. */
+ * 10 * shared-memory stages + row groups), out[3] 16-byte vectors per
+ * thread per tensor. */
 FN_API void fn_last_launch(int32_t out[4]);
 
 /* Thread-local kernel preference for fn_rmsnorm_quant: FN_VARIANT_NONE (the

@@ -113,7 +113,7 @@ int vectors_per_thread(int nvec, int max_threads, int vmax) {
 int row_vectors_per_thread(int nvec) { return vectors_per_thread(nvec, 256, 16); }
 
 constexpr int kTmaMaxStages = 8;
-constexpr int kTmaStaticSmem = 2 * 32 * 8;  // the kernel's double-buffered reduction slots
+constexpr int kTmaStaticSmem = 2 * 2 * 16 * 8 + 8 * 4;  // reduction slots and stage tags
 
 // Stages of the TMA ring that fit in shared memory (0 when fewer than 2 fit).
 int tma_stages(int64_t stage_bytes, int smem_optin) {
@@ -191,9 +191,13 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, vo
                    (pref == FN_VARIANT_ROW_TMA || (C < 2 && want_tma(M, sms, ntensor)));
 
   if (tma) {
-    const int V = vectors_per_thread(nvec, 512, 8);
-    const int threads = round32((nvec + V - 1) / V);
-    if ((nvec + V - 1) / V > 512) return FN_ERR_UNSUPPORTED;
+    // Two row groups of up to 256 threads each, so one group's per-row latency
+    // (reduction, rstd, scales) overlaps the other's arithmetic.
+    const int V = vectors_per_thread(nvec, 256, 8);
+    const int group_threads = round32((nvec + V - 1) / V);
+    const int groups = (int)std::min<int64_t>(2, (M + sms - 1) / sms);
+    const int threads = group_threads * groups;
+    if (group_threads > 256) return FN_ERR_UNSUPPORTED;
     RQTmaKernel k = pick_tma_kernel(mode, P, V);
     if (!k) return FN_ERR_UNSUPPORTED;
     const size_t smem = (size_t)nst * (size_t)(stage_bytes + 8);
@@ -204,12 +208,12 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, vo
     }
     const int64_t grid = std::min<int64_t>(M, sms);
     p.seg = nvec;
-    k<<<(unsigned)grid, threads, smem, st>>>(p, nst);
+    k<<<(unsigned)grid, threads, smem, st>>>(p, nst, groups);
     if (cudaGetLastError() != cudaSuccess) return FN_ERR_CUDA;
     tl_variant = FN_VARIANT_ROW_TMA;
     tl_launch[0] = (int32_t)grid;
     tl_launch[1] = threads;
-    tl_launch[2] = nst;
+    tl_launch[2] = nst * 10 + groups;
     tl_launch[3] = V;
   } else if (C >= 2) {
     p.seg = nvec / C;
@@ -369,6 +373,7 @@ int fn_rmsnorm_quant(const void* const* x_parts, int num_parts, const void* resi
   prm.nvec = (int)(H / 8);
   prm.P = num_parts;
   prm.eps = eps;
+  prm.inv_h = 1.0f / (float)H;
   return launch_rq(prm, mode, num_parts, M, true, stream, FN_VARIANT_ROW_CTA);
 }
 
@@ -446,6 +451,7 @@ int fn_qk_norm_gate(const void* qkv, int64_t M, int64_t row_stride, int Hq, int 
   p.qw = static_cast<const uint4*>(q_weight);
   p.kw = static_cast<const uint4*>(k_weight);
   p.eps = eps;
+  p.inv_d = 1.0f / (float)D;
   p.out_q = static_cast<uint4*>(out_q);
   p.out_k = static_cast<uint4*>(out_k);
   p.out_g = static_cast<uint4*>(out_gate);

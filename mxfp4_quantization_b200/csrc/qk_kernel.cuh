@@ -20,6 +20,7 @@ struct QKParams {
   const uint4* qw;
   const uint4* kw;
   float eps;
+  float inv_d;      // 1 / head_dim
   uint4* out_q;
   uint4* out_k;
   uint4* out_g;
@@ -67,7 +68,11 @@ __global__ void __launch_bounds__(256) qk_kernel(const __grid_constant__ QKParam
       ss = fmaf(b, b, ss);
     }
   ss = warp_sum(ss);
-  const float rstd = (float)(1.0 / sqrt((double)ss / (double)(p.dv * 8) + (double)p.eps));
+  // 1 / sqrt(mean + eps): hardware reciprocal square root plus one
+  // Newton-Raphson step, r <- r (3 - x r^2) / 2 (about one fp32 ulp)
+  const float xm = fmaf(ss, p.inv_d, p.eps);
+  const float r0 = rsqrtf(xm);
+  const float rstd = r0 * fmaf(-0.5f * xm * r0, r0, 1.5f);
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     uint4 y;

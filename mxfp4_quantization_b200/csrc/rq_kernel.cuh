@@ -235,8 +235,13 @@ __device__ __forceinline__ float2 row_reduce(float s, float m, float2* red, floa
   return t;
 }
 
-__device__ __forceinline__ float row_rstd(float ss, int H, float eps) {
-  return (float)(1.0 / sqrt((double)ss / (double)H + (double)eps));
+// 1 / sqrt(mean(h^2) + eps) in fp32: the hardware reciprocal square root
+// refined by one Newton-Raphson step, r <- r (3 - x r^2) / 2, which brings it
+// to about one fp32 ulp (the normed row is specified to 1 bf16 ulp).
+__device__ __forceinline__ float row_rstd(float ss, float inv_h, float eps) {
+  const float x = fmaf(ss, inv_h, eps);
+  const float r = rsqrtf(x);
+  return r * fmaf(-0.5f * x * r, r, 1.5f);
 }
 
 // bf16(fl(pmax * rstd)): the row's max |y| (see stats_vec).
@@ -303,7 +308,7 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
     }
     // ---- 3. rstd (and the per-token amax) ---------------------------------------------
     const float2 tot = row_reduce<CL, MODE == MODE_TOKEN>(ss.x + ss.y, pmax, red, &cl_slot);
-    const float rstd = row_rstd(tot.x, H, prm.eps);
+    const float rstd = row_rstd(tot.x, prm.inv_h, prm.eps);
     if (MODE == MODE_TOKEN) scale_tok = fp8_scale(row_amax_from_pmax(tot.y, rstd));
     // ---- 4. y = bf16(fl(h * w) * rstd) ----------------------------------------------
 #pragma unroll
@@ -387,18 +392,73 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 
 constexpr uint32_t kWaitLimit = 1u << 24;
 
+// Row index published per stage (release) and read before the parity wait
+// (acquire): see rq_tma_kernel.
+__device__ __forceinline__ void tag_store(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int tag_load(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)) : "memory");
+  return v;
+}
+
+// Wait (bounded) until `tag` holds `want`.
+__device__ __forceinline__ bool tag_wait(const int* tag, int want, uint32_t limit) {
+  for (uint32_t it = 0; it < limit; ++it)
+    if (tag_load(tag) == want) return true;
+  return false;
+}
+
+// Named barrier over the `count` threads of one row group (id 1 + group).
+__device__ __forceinline__ void group_barrier(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Sum of `s` and max of `m` over one row group of `tg` threads (whole warps),
+// combined in a fixed order (warps in index order).
+template <bool WANT_MAX>
+__device__ __forceinline__ float2 group_reduce(float s, float m, float2* red, int g, int tg,
+                                               int t) {
+  s = warp_sum(s);
+  if (WANT_MAX) m = warp_max(m);
+  const int lane = t & 31, warp = t >> 5, nw = tg >> 5;
+  if (lane == 0) red[warp] = make_float2(s, m);
+  group_barrier(1 + g, tg);
+  float2 r = red[0];
+  for (int i = 1; i < nw; ++i) {
+    const float2 o = red[i];
+    r.x += o.x;
+    if (WANT_MAX) r.y = fmaxf(r.y, o.y);
+  }
+  return r;
+}
+
 // Shared memory: nstages stages of (P + has_res) row segments of H bf16, then
-// one mbarrier per stage.  Block b handles rows b, b + gridDim.x, ...; the
-// copies of the next nstages rows are in flight while a row is computed.  A
-// stage is refilled as soon as the block has read it into registers (after
-// the sum-of-squares reduction's barrier), before rstd, y and the codes.
+// one mbarrier per stage.  Block b handles rows b, b + gridDim.x, ...; its
+// threads form `groups` row groups of blockDim.x / groups threads (whole
+// warps) that take the block's rows in turn, each group synchronising on its
+// own named barrier, so one group's reduction and scale latency overlaps the
+// other's arithmetic.  The copies of the next rows are in flight while rows
+// are computed: a stage is refilled, by the group that read it, as soon as
+// that group has it in registers (after the sum-of-squares barrier), before
+// rstd, y and the codes.
+//
+// A stage is consumed by the groups in turn (row i by group i % groups), so a
+// group skips phases of a stage's mbarrier, and a parity wait alone could be
+// satisfied by an older completed phase of the same parity.  Each stage
+// therefore carries the index of the row last issued into it; a group first
+// waits (bounded) for its row's index there, which also proves that the
+// stage's previous row has been consumed, and only then waits on the parity.
 template <int MODE, int MAXP, int V>
 __global__ void __launch_bounds__(512, 1)
-    rq_tma_kernel(const __grid_constant__ RQParams prm, int nstages) {
+    rq_tma_kernel(const __grid_constant__ RQParams prm, int nstages, int groups) {
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float2 red[2][32];
+  __shared__ float2 red[2][2][16];  // [group][buffer][warp]
+  __shared__ int issued[8];         // row index last issued into each stage
 
-  const int T = blockDim.x, t = threadIdx.x, lane = t & 31;
+  const int tg = blockDim.x / groups;
+  const int g = threadIdx.x / tg, t = threadIdx.x - g * tg, lane = threadIdx.x & 31;
   const int nvec = prm.nvec, H = nvec * 8;
   const bool has_res = prm.residual != nullptr;
   const int ntensor = prm.P + (has_res ? 1 : 0);
@@ -409,11 +469,11 @@ __global__ void __launch_bounds__(512, 1)
   const int64_t first = blockIdx.x, step = gridDim.x;
   const int64_t nrows = first < M ? (M - first + step - 1) / step : 0;
 
-  // The weight stays in registers for every row this block handles.
+  // The weight stays in registers for every row this group handles.
   uint4 wv[V];
 #pragma unroll
   for (int k = 0; k < V; ++k) {
-    const int v = t + k * T;
+    const int v = t + k * tg;
     wv[k] = v < nvec ? ld_keep(prm.weight + v) : make_uint4(0u, 0u, 0u, 0u);
   }
 
@@ -426,21 +486,28 @@ __global__ void __launch_bounds__(512, 1)
       bulk_load(dst + (size_t)p * seg_bytes, prm.parts[p] + row * nvec, seg_bytes, &full[s]);
     if (has_res)
       bulk_load(dst + (size_t)prm.P * seg_bytes, prm.residual + row * nvec, seg_bytes, &full[s]);
+    tag_store(&issued[s], (int)i);
   };
 
-  if (t == 0) {
-    for (int s = 0; s < nstages; ++s) mbar_init(&full[s], 1);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < nstages; ++s) {
+      mbar_init(&full[s], 1);
+      issued[s] = -1;
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     for (int64_t i = 0; i < nrows && i < nstages; ++i) issue(i);
   }
   __syncthreads();
 
   bool timed_out = false;
-  for (int64_t i = 0; i < nrows; ++i) {
+  int buf = 0;
+  for (int64_t i = g; i < nrows; i += groups, buf ^= 1) {
     const int s = (int)(i % nstages);
     const int64_t row = first + i * step;
     const int64_t rowv = row * nvec;
-    if (!mbar_wait(&full[s], (uint32_t)((i / nstages) & 1), kWaitLimit)) timed_out = true;
+    if (!tag_wait(&issued[s], (int)i, kWaitLimit) ||
+        !mbar_wait(&full[s], (uint32_t)((i / nstages) & 1), kWaitLimit))
+      timed_out = true;
     const uint4* st = reinterpret_cast<const uint4*>(smem + (size_t)s * stage_bytes);
 
     uint4 hv[V];
@@ -448,7 +515,7 @@ __global__ void __launch_bounds__(512, 1)
     float pmax = 0.f;
 #pragma unroll
     for (int k = 0; k < V; ++k) {
-      const int v = t + k * T;
+      const int v = t + k * tg;
       const bool ok = v < nvec;
       uint4 x[MAXP];
 #pragma unroll
@@ -460,11 +527,11 @@ __global__ void __launch_bounds__(512, 1)
       if (ok && prm.out_residual != nullptr) st_stream(prm.out_residual + rowv + v, hv[k]);
     }
     const float2 tot =
-        row_reduce<false, MODE == MODE_TOKEN>(ss.x + ss.y, pmax, red[i & 1], nullptr);
-    // every thread has read stage s: refill it with the row nstages ahead
+        group_reduce<MODE == MODE_TOKEN>(ss.x + ss.y, pmax, red[g][buf], g, tg, t);
+    // the whole group has read stage s: refill it with the row nstages ahead
     if (t == 0 && i + nstages < nrows) issue(i + nstages);
 
-    const float rstd = row_rstd(tot.x, H, prm.eps);
+    const float rstd = row_rstd(tot.x, prm.inv_h, prm.eps);
     float scale_tok = 1.f;
     if (MODE == MODE_TOKEN) {
       scale_tok = fp8_scale(row_amax_from_pmax(tot.y, rstd));
@@ -472,7 +539,7 @@ __global__ void __launch_bounds__(512, 1)
     }
 #pragma unroll
     for (int k = 0; k < V; ++k) {
-      const int v = t + k * T;
+      const int v = t + k * tg;
       const bool ok = v < nvec;
       const uint4 y = norm_vec(hv[k], wv[k], rstd);
       if (ok && prm.out_y != nullptr) st_stream(prm.out_y + rowv + v, y);

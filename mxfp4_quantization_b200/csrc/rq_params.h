@@ -20,6 +20,7 @@ struct RQParams {
   int seg;                 // vectors of a row handled by one block
   int P;                   // partial count, <= MAXP
   float eps;
+  float inv_h;             // 1 / H (fp32), for the mean of squares
   int* status;             // library status word: set to 1 if a bounded wait gave up
 };
 
@@ -30,8 +31,9 @@ using RQKernel = void (*)(const RQParams);
 // Per-(mode, partial bound) instantiation units, each compiled separately
 // (rq_inst.cu) so the library builds in parallel.  `V` is ignored for
 // cluster launches (always one vector per thread there).
-// The TMA-staged persistent kernel takes the stage count as a second argument.
-using RQTmaKernel = void (*)(const RQParams, int);
+// The TMA-staged persistent kernel takes the stage count and the number of row
+// groups per block as further arguments.
+using RQTmaKernel = void (*)(const RQParams, int, int);
 
 #define FN_RQ_DECL(MODE, MAXP)                                          \
   RQKernel rq_pick_##MODE##_##MAXP(int V, bool cluster, bool norm); \
