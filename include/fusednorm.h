@@ -182,6 +182,15 @@ FN_API int fn_prefer_variant(int variant);
  * library, not an allocation. */
 FN_API int fn_device_status(void* stream);
 
+/* Test hook for the failure path (thread-local, off by default).  While on,
+ * FN_VARIANT_ROW_TMA launches make every stage's mbarrier expect 16 bytes more
+ * than its copies bring, so the kernel's bounded waits run out: each thread
+ * gives up after one second, stops waiting and issuing, and the block
+ * finishes; nothing faults or hangs.  Outputs of such a call are not valid and
+ * the next fn_device_status returns FN_ERR_TIMEOUT.  No page describes this:
+ * it exists to test the timeout path.  Returns the previous setting. */
+FN_API int fn_debug_stall_copies(int on);
+
 /* Library ABI version (major * 100 + minor). */
 FN_API int fn_version(void);
 

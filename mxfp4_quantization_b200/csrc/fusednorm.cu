@@ -17,6 +17,7 @@ namespace {
 thread_local int tl_variant = FN_VARIANT_NONE;
 thread_local int32_t tl_launch[4] = {0, 0, 0, 0};
 thread_local int tl_prefer = FN_VARIANT_NONE;
+thread_local int tl_stall_copies = 0;
 
 }  // namespace
 
@@ -208,6 +209,7 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, vo
     }
     const int64_t grid = std::min<int64_t>(M, sms);
     p.seg = nvec;
+    p.debug_extra_tx = tl_stall_copies ? 16u : 0u;
     k<<<(unsigned)grid, threads, smem, st>>>(p, nst, groups);
     if (cudaGetLastError() != cudaSuccess) return FN_ERR_CUDA;
     tl_variant = FN_VARIANT_ROW_TMA;
@@ -282,6 +284,12 @@ int fn_last_variant(void) { return tl_variant; }
 int fn_prefer_variant(int variant) {
   const int old = tl_prefer;
   tl_prefer = variant;
+  return old;
+}
+
+int fn_debug_stall_copies(int on) {
+  const int old = tl_stall_copies;
+  tl_stall_copies = on ? 1 : 0;
   return old;
 }
 

@@ -361,22 +361,28 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
-// Wait for the phase with the given parity to complete.  Bounded: gives up
-// after `limit` polls and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase with the given parity to complete.  Bounded in time:
+// gives up and returns false once `deadline` (globaltimer ns) has passed.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t deadline) {
   const uint32_t a = smem_addr(bar);
-  for (uint32_t it = 0; it < limit; ++it) {
+  while (true) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(a), "r"(parity)
+        : "r"(a), "r"(parity), "r"(20000u)
         : "memory");
     if (done) return true;
+    if (global_ns() > deadline) return false;
   }
-  return false;
 }
 
 // Bulk asynchronous copy global -> this block's shared memory (no multicast);
@@ -390,7 +396,9 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-constexpr uint32_t kWaitLimit = 1u << 24;
+// A wait on the block's own bulk copies gives up after this long (one second;
+// a healthy copy lands in microseconds).
+constexpr uint64_t kWaitNs = 1000000000ull;
 
 // Row index published per stage (release) and read before the parity wait
 // (acquire): see rq_tma_kernel.
@@ -403,11 +411,13 @@ __device__ __forceinline__ int tag_load(const int* p) {
   return v;
 }
 
-// Wait (bounded) until `tag` holds `want`.
-__device__ __forceinline__ bool tag_wait(const int* tag, int want, uint32_t limit) {
-  for (uint32_t it = 0; it < limit; ++it)
+// Wait (bounded in time, see mbar_wait) until `tag` holds `want`.
+__device__ __forceinline__ bool tag_wait(const int* tag, int want, uint64_t deadline) {
+  while (true) {
     if (tag_load(tag) == want) return true;
-  return false;
+    if (global_ns() > deadline) return false;
+    __nanosleep(64);
+  }
 }
 
 // Named barrier over the `count` threads of one row group (id 1 + group).
@@ -481,7 +491,7 @@ __global__ void __launch_bounds__(512, 1)
     const int s = (int)(i % nstages);
     const int64_t row = first + i * step;
     uint8_t* dst = smem + (size_t)s * stage_bytes;
-    mbar_expect_tx(&full[s], stage_bytes);
+    mbar_expect_tx(&full[s], stage_bytes + prm.debug_extra_tx);
     for (int p = 0; p < prm.P; ++p)
       bulk_load(dst + (size_t)p * seg_bytes, prm.parts[p] + row * nvec, seg_bytes, &full[s]);
     if (has_res)
@@ -499,15 +509,24 @@ __global__ void __launch_bounds__(512, 1)
   }
   __syncthreads();
 
+  // After a wait gives up, the thread stops waiting and its group stops
+  // issuing copies (the stage's mbarrier would be left with an open phase);
+  // it still takes part in every barrier, so the block finishes, and the
+  // status word records the failure.  No copy is left in flight: every copy
+  // issued was for a row whose wait either completed or gave up on its phase
+  // having already received all its bytes.
   bool timed_out = false;
   int buf = 0;
   for (int64_t i = g; i < nrows; i += groups, buf ^= 1) {
     const int s = (int)(i % nstages);
     const int64_t row = first + i * step;
     const int64_t rowv = row * nvec;
-    if (!tag_wait(&issued[s], (int)i, kWaitLimit) ||
-        !mbar_wait(&full[s], (uint32_t)((i / nstages) & 1), kWaitLimit))
-      timed_out = true;
+    if (!timed_out) {
+      const uint64_t deadline = global_ns() + kWaitNs;
+      if (!tag_wait(&issued[s], (int)i, deadline) ||
+          !mbar_wait(&full[s], (uint32_t)((i / nstages) & 1), deadline))
+        timed_out = true;
+    }
     const uint4* st = reinterpret_cast<const uint4*>(smem + (size_t)s * stage_bytes);
 
     uint4 hv[V];
@@ -529,7 +548,7 @@ __global__ void __launch_bounds__(512, 1)
     const float2 tot =
         group_reduce<MODE == MODE_TOKEN>(ss.x + ss.y, pmax, red[g][buf], g, tg, t);
     // the whole group has read stage s: refill it with the row nstages ahead
-    if (t == 0 && i + nstages < nrows) issue(i + nstages);
+    if (t == 0 && !timed_out && i + nstages < nrows) issue(i + nstages);
 
     const float rstd = row_rstd(tot.x, prm.inv_h, prm.eps);
     float scale_tok = 1.f;

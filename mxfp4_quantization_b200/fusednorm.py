@@ -49,7 +49,7 @@ MODES = {"fp8_per_token": FN_FP8_PER_TOKEN, "fp8_per_group128": FN_FP8_PER_GROUP
 # The exported symbols of include/fusednorm.h.
 ABI_SYMBOLS = ("fn_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate", "fn_status_string",
                "fn_last_variant", "fn_last_launch", "fn_prefer_variant", "fn_device_status",
-               "fn_version")
+               "fn_debug_stall_copies", "fn_version")
 
 
 class FusedNormError(RuntimeError):
@@ -82,6 +82,8 @@ def _load():
     lib.fn_prefer_variant.restype = i32
     lib.fn_device_status.argtypes = [vp]
     lib.fn_device_status.restype = i32
+    lib.fn_debug_stall_copies.argtypes = [i32]
+    lib.fn_debug_stall_copies.restype = i32
     lib.fn_version.argtypes = []
     lib.fn_version.restype = i32
     return lib
@@ -135,6 +137,10 @@ def fn_prefer_variant(variant: int) -> int:
 
 def fn_device_status(stream: Optional[int]) -> int:
     return _lib.fn_device_status(stream)
+
+
+def fn_debug_stall_copies(on: int) -> int:
+    return _lib.fn_debug_stall_copies(on)
 
 
 def fn_version() -> int:

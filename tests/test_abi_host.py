@@ -30,7 +30,8 @@ def test_header_declares_the_abi():
     assert declared_symbols() == sorted(["fn_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate",
                                          "fn_status_string", "fn_last_variant",
                                          "fn_last_launch", "fn_prefer_variant",
-                                         "fn_device_status", "fn_version"])
+                                         "fn_device_status", "fn_debug_stall_copies",
+                                         "fn_version"])
 
 
 def test_library_exports_every_declared_symbol(fnb):

@@ -250,3 +250,27 @@ def test_decode_sweep_config(fnb, M, mode):
     inp, gpu, variant, _ = run(fnb, wl)
     assert variant == fnb.FN_VARIANT_ROW_CLUSTER
     check(wl, inp, gpu)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(fnb):
+    """Failure path of the TMA kernel without a fault: the test hook makes its
+    stage barriers expect more bytes than arrive, the bounded waits give up
+    after about a second, the call completes, and the status word says so.
+    The next ordinary call works and the status is clean again."""
+    wl = synth.RowWorkload("stall", M=300, H=1024, P=3, mode=MX, eps=1e-6, seed=13)
+    inp = wl.inputs(device="cuda")
+    assert fnb.device_status() == fnb.FN_OK
+    old = fnb.fn_debug_stall_copies(1)
+    try:
+        with fnb.prefer_variant(fnb.FN_VARIANT_ROW_TMA):
+            fnb.rmsnorm_quant(inp["parts"], inp["weight"], wl.eps, MX, residual=inp["residual"])
+            assert fnb.fn_last_variant() == fnb.FN_VARIANT_ROW_TMA
+    finally:
+        fnb.fn_debug_stall_copies(old)
+    torch.cuda.synchronize()
+    assert fnb.device_status() == fnb.FN_ERR_TIMEOUT
+    assert fnb.device_status() == fnb.FN_OK  # read-and-clear
+    # the context is still usable and the kernel correct
+    inp2, gpu, variant, _ = run(fnb, wl, variant=fnb.FN_VARIANT_ROW_TMA)
+    assert variant == fnb.FN_VARIANT_ROW_TMA
+    check(wl, inp2, gpu)
