@@ -424,7 +424,7 @@ def secondary_workloads(fn, device, peak):
         n_sets = max(64, int(2 * L2_BYTES / per_call_bytes) + 1)
         n_sets = min(n_sets, 8192)
         us, eager = time_graph_calls(make, n_sets, 7, device)
-        return {"us_per_call_graph": us, "us_single_call_events": eager, "calls_per_graph": n_sets,
+        return {"us_per_call_graph": us, "us_single_call_host_to_device": eager, "calls_per_graph": n_sets,
                 "GB_s": per_call_bytes / (us * 1e-6) / 1e9}
 
     wl = synth.PER_TOKEN_SMALL
@@ -589,7 +589,10 @@ def main_arm(args):
                          "frac": achieved / peak, "peak_kind": peak_kind,
                          "traffic": measured_traffic(wl.name),
                          "algorithmic_bytes_per_launch": bytes_call,
-                         "kernel": "rq_kernel (one block per row)",
+                         "kernel": {fn.FN_VARIANT_ROW_TMA: "rq_tma_kernel (TMA-staged, persistent)",
+                                    fn.FN_VARIANT_ROW_CTA: "rq_kernel (one block per row)",
+                                    fn.FN_VARIANT_ROW_CLUSTER: "rq_kernel (cluster per row)"}.get(
+                                        variant, str(variant)),
                          "launch": list(launch), "variant": variant},
             "e2e": {"value": aggregate(wl.M, world, e2e_ms_max), "unit": "rows/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
