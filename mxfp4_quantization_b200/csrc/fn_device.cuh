@@ -27,6 +27,12 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   return r;
 }
 
+// Bulk prefetch of a contiguous global range into L2 (nothing to wait for).
+// 16-byte aligned, size % 16 == 0.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Small, reused operand (the norm weight): normal cached read-only load.
 __device__ __forceinline__ uint4 ld_keep(const uint4* p) { return __ldg(p); }
 

@@ -114,6 +114,13 @@ int vectors_per_thread(int nvec, int max_threads, int vmax) {
 int row_vectors_per_thread(int nvec) { return vectors_per_thread(nvec, 256, 16); }
 
 constexpr int kTmaMaxStages = 8;
+// L2 prefetch distance, in rows, of the one-block-per-row kernel, in units of
+// SMs: a block starts the row 2 * #SMs blocks later towards L2, about one
+// wave ahead.  Measured on B200 (prefill MXFP4 H=7168 P=4 / group-128
+// H=8192 P=1): 0 -> 121.8 / 315 us, 2 SMs' worth -> 114.6 / 281-305 us;
+// 4 SMs' worth and more is slower again.  The TMA ring gains nothing from it
+// (120 -> 128 us with any distance), so it does not prefetch.
+constexpr int kRowPrefetchSms = 2;
 constexpr int kTmaStaticSmem = 2 * 2 * 16 * 8 + 8 * 4;  // reduction slots and stage tags
 
 // Stages of the TMA ring that fit in shared memory (0 when fewer than 2 fit).
@@ -123,12 +130,10 @@ int tma_stages(int64_t stage_bytes, int smem_optin) {
   return n >= 2 ? n : 0;
 }
 
-// Whether a large-M call should take the TMA ring.  Measured on B200: with
-// three or more row tensors (partials + residual) a register-resident row is
-// too big for enough rows to be in flight per SM and the ring wins (MXFP4,
-// H=7168, P=4: 113 us vs 121 us); with two the register kernel keeps four
-// rows per SM in flight and wins (group-128, H=8192, P=1: 289 us vs 448 us).
-bool want_tma(int64_t M, int sms, int ntensor) { return M >= 2 * (int64_t)sms && ntensor >= 3; }
+// The TMA ring is taken only on request (fn_prefer_variant): with the L2
+// prefetch above, one block per row keeps enough bytes in flight and is the
+// faster large-M kernel on B200 for every shape measured (MXFP4 H=7168 P=4:
+// 114.6 us vs 120.1 us; group-128 H=8192 P=1: 281-305 us vs 395 us).
 
 // Cluster size for a small-M launch: the largest C in 2..8 that splits the
 // row into equal segments aligned to the quantization group, each at most 512
@@ -189,7 +194,7 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, vo
   const int nst = tma_stages(stage_bytes, smem_optin);
   const bool tma = norm && nst > 0 && pref != FN_VARIANT_ROW_CTA &&
                    pref != FN_VARIANT_ROW_CLUSTER &&
-                   (pref == FN_VARIANT_ROW_TMA || (C < 2 && want_tma(M, sms, ntensor)));
+                   pref == FN_VARIANT_ROW_TMA;
 
   if (tma) {
     // Two row groups of up to 256 threads each, so one group's per-row latency
@@ -210,6 +215,7 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, vo
     const int64_t grid = std::min<int64_t>(M, sms);
     p.seg = nvec;
     p.debug_extra_tx = tl_stall_copies ? 16u : 0u;
+    p.prefetch_rows = 0;
     k<<<(unsigned)grid, threads, smem, st>>>(p, nst, groups);
     if (cudaGetLastError() != cudaSuccess) return FN_ERR_CUDA;
     tl_variant = FN_VARIANT_ROW_TMA;
@@ -246,6 +252,7 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, vo
   } else {
     const int V = row_vectors_per_thread(nvec);
     p.seg = nvec;
+    p.prefetch_rows = M > (int64_t)kRowPrefetchSms * sms ? kRowPrefetchSms * sms : 0;
     const int threads = round32((nvec + V - 1) / V);
     RQKernel k = pick_kernel(mode, P, V, false, norm);
     if (!k) return FN_ERR_UNSUPPORTED;

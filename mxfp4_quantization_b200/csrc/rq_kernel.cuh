@@ -103,47 +103,56 @@ __device__ __forceinline__ uint4 norm_vec(const uint4& h, const uint4& w, float 
   return y;
 }
 
-// FP8 scale of a group (or row) amax: amax / 448 (IEEE division), 1 for zero.
-__device__ __forceinline__ float fp8_scale(float amax) {
-  return amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+// FP8 scale of a group (or row) and the reciprocal pair the codes use.
+struct Fp8Scale {
+  float s;         // RN(amax / 448), 1 for an all-zero group
+  float r, r_lo;   // RN(1/s), RN(RN(1 - s r) r)
+  bool exact_div;  // the fast quotient is not proven here: use the IEEE division
+};
+
+// The formulas themselves (IEEE division and reciprocal).
+__device__ __forceinline__ Fp8Scale fp8_scale_direct(float amax) {
+  Fp8Scale c;
+  c.s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+  c.exact_div = !(c.s >= 0x1p-120f);
+  c.r = c.exact_div ? 1.f : __frcp_rn(c.s);
+  c.r_lo = fmaf(-c.s, c.r, 1.f) * c.r;
+  return c;
 }
 
 // Eight E4M3 codes of fl32(y / s), the IEEE quotient.
 //
-// Fast path, for s >= 2^-120: with r = RN(1/s) and r_lo = RN(RN(1 - s r) r)
-// (so that r + r_lo carries 1/s to about 2^-46), q = RN(|y| r + RN(|y| r_lo))
-// has the same E4M3 code as RN(|y| / s) for every bf16 y with |y| <= amax and
-// every bf16 amax with s = RN(amax / 448) >= 2^-120; this was checked
-// exhaustively over all such (amax, y) pairs (tests/quotient_proof.c).  The
-// code is computed from |y| and y's sign bit is copied onto it, which also
-// gives -0 the code 0x80.  If any lane of the warp has s < 2^-120 the whole
-// warp takes the IEEE division instead (warp-uniform branch).  All 32 lanes
-// must call.
-__device__ __forceinline__ uint2 e4m3_codes(const uint4& y, float s) {
-  uint32_t c[4];
-  if (!__any_sync(0xffffffffu, !(s >= 0x1p-120f))) {
-    const float r = __frcp_rn(s);
-    const float r_lo = fmaf(-s, r, 1.f) * r;
+// Fast path: with r = RN(1/s) and r_lo = RN(RN(1 - s r) r) (r + r_lo carries
+// 1/s to about 2^-46), q = RN(|y| r + RN(|y| r_lo)) has the same E4M3 code as
+// RN(|y| / s) for every bf16 y with |y| <= amax and every bf16 amax with
+// s = RN(amax / 448) >= 2^-120: checked exhaustively over all such (amax, y)
+// pairs by tests/quotient_proof.c.  The code is computed from |y| and y's
+// sign bit is copied onto it, which also gives -0 the code 0x80.  If any lane
+// of the warp needs the IEEE division the whole warp takes it (warp-uniform
+// branch).  All 32 lanes must call.
+__device__ __forceinline__ uint2 e4m3_codes(const uint4& y, const Fp8Scale& c) {
+  uint32_t q8[4];
+  if (!__any_sync(0xffffffffu, c.exact_div)) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint32_t a = word(y, i) & 0x7FFF7FFFu;
       const float2 ya = make_float2(bf_lo(a), bf_hi(a));
-      const float2 t = mul_f32x2(ya, make_float2(r_lo, r_lo));
-      const float2 q = fma_f32x2(ya, make_float2(r, r), t);
-      c[i] = cvt_e4m3x2(q.x, q.y);
+      const float2 t = mul_f32x2(ya, make_float2(c.r_lo, c.r_lo));
+      const float2 q = fma_f32x2(ya, make_float2(c.r, c.r), t);
+      q8[i] = cvt_e4m3x2(q.x, q.y);
     }
   } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint32_t a = word(y, i) & 0x7FFF7FFFu;
-      c[i] = cvt_e4m3x2(__fdiv_rn(bf_lo(a), s), __fdiv_rn(bf_hi(a), s));
+      q8[i] = cvt_e4m3x2(__fdiv_rn(bf_lo(a), c.s), __fdiv_rn(bf_hi(a), c.s));
     }
   }
   // byte k of code word j takes the sign of element 4j + k: the sign bits sit
   // at bits 15 and 31 of each y word, i.e. in bytes 1 and 3
   const uint32_t s0 = __byte_perm(y.x, y.y, 0x7531) & 0x80808080u;
   const uint32_t s1 = __byte_perm(y.z, y.w, 0x7531) & 0x80808080u;
-  return make_uint2((c[0] | (c[1] << 16)) | s0, (c[2] | (c[3] << 16)) | s1);
+  return make_uint2((q8[0] | (q8[1] << 16)) | s0, (q8[2] | (q8[3] << 16)) | s1);
 }
 
 // E2M1 codes of y * 2^-e for the 8 bf16 of a vector (inv_bf16 = 2^-e as a bf16
@@ -162,18 +171,19 @@ __device__ __forceinline__ uint32_t e2m1_codes(const uint4& y, uint32_t inv_bf16
 // Quantize vector v of a row (y: 8 bf16) and store its codes and, from the
 // group's first lane, its scale.  All 32 lanes must call (shuffles); `ok`
 // masks the stores of lanes past the row end (whole groups, by alignment).
+// `tok` is the row's scale (per-token mode).
 template <int MODE>
 __device__ __forceinline__ void quant_store(const uint4& y, bool ok, int lane, int64_t row, int v,
-                                            int H, float scale_tok, uint8_t* out_q,
+                                            int H, const Fp8Scale& tok, uint8_t* out_q,
                                             void* out_scale) {
   if constexpr (MODE == MODE_TOKEN || MODE == MODE_G128) {
-    float s = scale_tok;
+    Fp8Scale c = tok;
     if constexpr (MODE == MODE_G128) {
-      s = fp8_scale(group_max<16>(vec_absmax(y)));
-      if (ok && (lane & 15) == 0) static_cast<float*>(out_scale)[row * (H / 128) + v / 16] = s;
+      c = fp8_scale_direct(group_max<16>(vec_absmax(y)));
+      if (ok && (lane & 15) == 0) static_cast<float*>(out_scale)[row * (H / 128) + v / 16] = c.s;
     }
-    const uint2 c = e4m3_codes(y, s);
-    if (ok) st_stream(reinterpret_cast<uint2*>(out_q + row * (int64_t)H) + v, c);
+    const uint2 q = e4m3_codes(y, c);
+    if (ok) st_stream(reinterpret_cast<uint2*>(out_q + row * (int64_t)H) + v, q);
   } else {
     float inv;
     const uint32_t code = mx_scale(group_max<4>(vec_absmax(y)), inv);
@@ -275,6 +285,15 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
   const bool has_res = NORM && prm.residual != nullptr;
   const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
 
+  // The block `prefetch_rows` rows later in launch order will most likely run
+  // next on this SM's slot: start its row towards L2 now.
+  if (!CL && prm.prefetch_rows > 0 && t == 0 && row + prm.prefetch_rows < prm.M) {
+    const int64_t prow = (row + prm.prefetch_rows) * (int64_t)prm.nvec;
+    const uint32_t bytes = (uint32_t)prm.nvec * 16u;
+    for (int p = 0; p < prm.P; ++p) bulk_prefetch_l2(prm.parts[p] + prow, bytes);
+    if (prm.residual != nullptr) bulk_prefetch_l2(prm.residual + prow, bytes);
+  }
+
   // ---- 1. issue every load of this block's part of the row -------------------
   uint4 xin[V][MAXP];
   uint4 rin[V];
@@ -293,7 +312,7 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
   }
 
   uint4 yv[V];
-  float scale_tok = 1.f;
+  Fp8Scale scale_tok = {1.f, 1.f, 0.f, false};
   if constexpr (NORM) {
     // ---- 2. h, residual_out, statistics --------------------------------------------
     uint4 hv[V];
@@ -309,7 +328,7 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
     // ---- 3. rstd (and the per-token amax) ---------------------------------------------
     const float2 tot = row_reduce<CL, MODE == MODE_TOKEN>(ss.x + ss.y, pmax, red, &cl_slot);
     const float rstd = row_rstd(tot.x, prm.inv_h, prm.eps);
-    if (MODE == MODE_TOKEN) scale_tok = fp8_scale(row_amax_from_pmax(tot.y, rstd));
+    if (MODE == MODE_TOKEN) scale_tok = fp8_scale_direct(row_amax_from_pmax(tot.y, rstd));
     // ---- 4. y = bf16(fl(h * w) * rstd) ----------------------------------------------
 #pragma unroll
     for (int k = 0; k < V; ++k) {
@@ -324,10 +343,11 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
       float am = 0.f;
 #pragma unroll
       for (int k = 0; k < V; ++k) am = fmaxf(am, vec_absmax(yv[k]));
-      scale_tok = fp8_scale(row_reduce<CL, true>(0.f, am, red, &cl_slot).y);
+      scale_tok = fp8_scale_direct(row_reduce<CL, true>(0.f, am, red, &cl_slot).y);
     }
   }
-  if (MODE == MODE_TOKEN && rank == 0 && t == 0) static_cast<float*>(prm.out_scale)[row] = scale_tok;
+  if (MODE == MODE_TOKEN && rank == 0 && t == 0)
+    static_cast<float*>(prm.out_scale)[row] = scale_tok.s;
 
   // ---- 5. quantize y ----------------------------------------------------------------
 #pragma unroll
@@ -497,6 +517,14 @@ __global__ void __launch_bounds__(512, 1)
     if (has_res)
       bulk_load(dst + (size_t)prm.P * seg_bytes, prm.residual + row * nvec, seg_bytes, &full[s]);
     tag_store(&issued[s], (int)i);
+    // start the row prefetch_rows further on towards L2, so that its copy
+    // into shared memory finds it there
+    const int64_t ip = i + prm.prefetch_rows;
+    if (prm.prefetch_rows > 0 && ip < nrows) {
+      const int64_t prow = first + ip * step;
+      for (int p = 0; p < prm.P; ++p) bulk_prefetch_l2(prm.parts[p] + prow * nvec, seg_bytes);
+      if (has_res) bulk_prefetch_l2(prm.residual + prow * nvec, seg_bytes);
+    }
   };
 
   if (threadIdx.x == 0) {
@@ -551,10 +579,10 @@ __global__ void __launch_bounds__(512, 1)
     if (t == 0 && !timed_out && i + nstages < nrows) issue(i + nstages);
 
     const float rstd = row_rstd(tot.x, prm.inv_h, prm.eps);
-    float scale_tok = 1.f;
+    Fp8Scale scale_tok = {1.f, 1.f, 0.f, false};
     if (MODE == MODE_TOKEN) {
-      scale_tok = fp8_scale(row_amax_from_pmax(tot.y, rstd));
-      if (t == 0) static_cast<float*>(prm.out_scale)[row] = scale_tok;
+      scale_tok = fp8_scale_direct(row_amax_from_pmax(tot.y, rstd));
+      if (t == 0) static_cast<float*>(prm.out_scale)[row] = scale_tok.s;
     }
 #pragma unroll
     for (int k = 0; k < V; ++k) {

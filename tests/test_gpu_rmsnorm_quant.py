@@ -122,7 +122,7 @@ def test_dispatch(fnb):
     """Small M takes the cluster kernel, large M one block per row."""
     for M, P, want in ((1, 1, fnb.FN_VARIANT_ROW_CLUSTER), (16, 1, fnb.FN_VARIANT_ROW_CLUSTER),
                        (200, 4, fnb.FN_VARIANT_ROW_CTA), (512, 1, fnb.FN_VARIANT_ROW_CTA),
-                       (512, 4, fnb.FN_VARIANT_ROW_TMA)):
+                       (512, 4, fnb.FN_VARIANT_ROW_CTA)):
         wl = synth.decode(M, MX) if M <= 16 else synth.RowWorkload("big", M=M, H=7168, P=P,
                                                                      mode=MX, eps=1e-6)
         _, _, variant, launch = run(fnb, wl)
