@@ -236,6 +236,19 @@ def hbm_peak():
 # ---------------------------------------------------------------------------
 
 
+MODE_NAMES = {0: "fp8_per_token", 1: "fp8_per_group128", 2: "mxfp4"}
+
+
+def workload_config(wl, world: int) -> dict:
+    """The `config` object of the JSON line (both arms)."""
+    return {"workload": wl.name, "M": wl.M, "H": wl.H, "P": wl.P, "mode": MODE_NAMES[wl.mode],
+            "eps": wl.eps, "rows_per_gpu": wl.M, "in_place": wl.in_place,
+            "io": "bf16 in; codes + scales + bf16 residual out",
+            "l2": f"inputs larger than L2 ({wl.M * wl.H * 2 * (wl.P + 1) / 1e6:.0f} MB read per"
+                  " step), no flush",
+            "parallelism": f"dp{world} (independent rows, no collective)"}
+
+
 def make_row_call(fn, wl, device, seed):
     import torch
     from mxfp4_quantization_b200 import synth
@@ -455,12 +468,17 @@ def secondary_workloads(fn, device, peak):
 # ---------------------------------------------------------------------------
 
 
-def oracle_rows_per_s(rows: int, min_seconds: float, max_seconds: float, seed: int = 3):
-    """The oracle, as it stands, single-threaded, on `rows` rows of the prefill
-    MXFP4 recipe, repeated until `min_seconds` have passed."""
+def pick_workload(name: str):
+    from mxfp4_quantization_b200 import synth
+    return synth.PREFILL_MXFP4 if name == "prefill_mxfp4" else synth.PREFILL_GROUP128
+
+
+def oracle_rows_per_s(rows: int, min_seconds: float, max_seconds: float, workload: str):
+    """The oracle, as it stands, single-threaded, on `rows` rows of the
+    workload's recipe, repeated until `min_seconds` have passed."""
     import oracle
     from mxfp4_quantization_b200 import synth
-    wl = synth.RowWorkload(**{**synth.PREFILL_MXFP4.__dict__, "seed": seed})
+    wl = pick_workload(workload)
     inp = wl.inputs(device="cpu", M=rows)
     parts = [synth.to_bits(p) for p in inp["parts"]]
     res, w = synth.to_bits(inp["residual"]), synth.to_bits(inp["weight"])
@@ -481,8 +499,8 @@ def reference_arm(args):
     import oracle
     from mxfp4_quantization_b200 import synth
     oracle.load()
-    wl = synth.PREFILL_MXFP4
-    rate, _, _ = oracle_rows_per_s(8, 0.5, 5.0)
+    wl = pick_workload(args.workload)
+    rate, _, _ = oracle_rows_per_s(8, 0.5, 5.0, args.workload)
     budget_s = 90.0
     rows_per_step = int(max(1, min(wl.M, rate * budget_s / max(1, args.steps + args.warmup))))
     inp = synth.RowWorkload(**{**wl.__dict__}).inputs(device="cpu", M=rows_per_step)
@@ -495,14 +513,13 @@ def reference_arm(args):
         oracle.rmsnorm_quant(parts, res, w, wl.eps, wl.mode)
     el = time.perf_counter() - t0
     value = rows_per_step * args.steps / el
-    sample = (f"{rows_per_step} rows of the prefill MXFP4 workload (H=7168, P=4) per step, "
+    sample = (f"{rows_per_step} rows of the {wl.name} workload (H={wl.H}, P={wl.P}) per step, "
               f"single-threaded oracle")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "prefill_mxfp4", "M": wl.M, "H": wl.H, "P": wl.P,
-                       "mode": "mxfp4", "rows_per_step": rows_per_step},
+            "config": {**workload_config(wl, world), "rows_per_step": rows_per_step},
             "cpu_baseline": {"value": value, "unit": "rows/s", "cores": 1, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0,
@@ -532,9 +549,7 @@ def main_arm(args):
     from mxfp4_quantization_b200 import fusednorm as fn
     from mxfp4_quantization_b200 import synth
 
-    wl = synth.PREFILL_MXFP4 if args.workload == "prefill_mxfp4" else synth.PREFILL_GROUP128
-    mode_name = {synth.MXFP4: "mxfp4", synth.FP8_PER_GROUP128: "fp8_per_group128",
-                 synth.FP8_PER_TOKEN: "fp8_per_token"}[wl.mode]
+    wl = pick_workload(args.workload)
     seed = rank_seed(wl.seed, rank)
     step, stream, keep = make_row_call(fn, wl, device, seed)
     clocks = ClockSampler(local)
@@ -565,9 +580,10 @@ def main_arm(args):
     if world == 1 and not args.no_extras and args.workload == "prefill_mxfp4":
         extra = secondary_workloads(fn, device, peak)
     if world == 1 and not args.no_cpu_baseline:
-        rate, rows, el = oracle_rows_per_s(256, args.cpu_seconds, 3 * args.cpu_seconds)
+        rate, rows, el = oracle_rows_per_s(256, args.cpu_seconds, 3 * args.cpu_seconds,
+                                           args.workload)
         cpu = {"value": rate, "unit": "rows/s", "cores": 1, "kind": "oracle",
-               "sample": f"{rows} rows (256 rows of the prefill MXFP4 recipe, H=7168, P=4, "
+               "sample": f"{rows} rows (256 rows of the {wl.name} recipe, H={wl.H}, P={wl.P}, "
                          f"repeated) in {el:.1f} s, single-threaded; "
                          f"host has {os.cpu_count()} cores"}
 
@@ -577,13 +593,7 @@ def main_arm(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": {"workload": wl.name, "M": wl.M, "H": wl.H, "P": wl.P,
-                       "mode": mode_name, "eps": wl.eps, "rows_per_gpu": wl.M,
-                       "in_place": wl.in_place,
-                       "io": "bf16 in; codes + scales + bf16 residual out",
-                       "l2": f"inputs larger than L2 ({wl.M * wl.H * 2 * (wl.P + 1) / 1e6:.0f} MB"
-                             " read per step), no flush",
-                       "parallelism": f"dp{world} (independent rows, no collective)"},
+            "config": workload_config(wl, world),
             "hbm_GB_s": achieved, "frac_of_peak": achieved / peak,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
