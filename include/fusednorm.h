@@ -82,6 +82,25 @@ typedef enum {
     FN_VARIANT_ROW_TMA = 5      /* persistent blocks, rows staged by bulk copies  */
 } fn_variant;
 
+/* Scale-layout flags, OR-ed into `mode` (fn_rmsnorm_quant, fn_quant).  No
+ * flag: scales row-major as listed below.  These lay the scales out for the
+ * GEMM that consumes the quantized tuple (the pages' "pre-shuffled" scales for
+ * the consumer, sglang PR #29723, "Modifications"; the layouts themselves are
+ * this architecture's, not the pages'):
+ *  FN_SCALE_SWIZZLE_32_4_4  (FN_MXFP4 only) E8M0 scales in the tiling that
+ *      block-scaled matrix multiplies read on B200: the [M, H/32] scale
+ *      matrix padded to [roundup(M,128), roundup(H/32,4)] and cut into
+ *      128 x 4 tiles of 512 bytes, tiles in row-tile-major order; inside a
+ *      tile, row r and group c sit at byte (r % 32) * 16 + (r / 32) * 4 + c.
+ *      out_scale must hold roundup(M,128) * roundup(H/32,4) bytes; padding
+ *      entries are not written.
+ *  FN_SCALE_MN_MAJOR  (FN_FP8_PER_GROUP128 only) fp32 scales group-major:
+ *      scale of row m, group g at out_scale[g * roundup(M,4) + m];
+ *      out_scale must hold (H/128) * roundup(M,4) floats; padding not written. */
+#define FN_MODE_MASK 0xFF
+#define FN_SCALE_SWIZZLE_32_4_4 0x100
+#define FN_SCALE_MN_MAJOR 0x200
+
 #define FN_MAX_PARTS 8
 #define FN_MAX_H 32768
 #define FN_MAX_HEAD_DIM 1024
@@ -105,7 +124,7 @@ typedef enum {
  * residual     bf16 [M, H], or NULL (no residual add).
  * weight       bf16 [H].
  * eps          finite, >= 0.
- * mode         fn_mode.
+ * mode         fn_mode, optionally OR-ed with one FN_SCALE_* layout flag.
  * M, H         M >= 0; H % 8 == 0, 8 <= H <= FN_MAX_H; H % 128 == 0 for
  *              FN_FP8_PER_GROUP128, H % 32 == 0 for FN_MXFP4.
  * out_q        FP8: u8 [M, H]; MXFP4: u8 [M, H/2].

@@ -150,32 +150,69 @@ int pick_cluster(int64_t M, int nvec, int mode, int sms) {
   return 0;
 }
 
-int check_mode_shape(int mode, int64_t M, int64_t H) {
-  if (mode < FN_FP8_PER_TOKEN || mode > FN_MXFP4) return FN_ERR_INVALID;
+// `mode` carries the quantization (low byte) and scale-layout flags.
+struct ModeInfo {
+  int q = -1;       // FN_FP8_PER_TOKEN / FN_FP8_PER_GROUP128 / FN_MXFP4
+  int layout = 0;   // fn::SCALE_ROW_MAJOR / SCALE_SWIZZLE_32_4_4 / SCALE_MN_MAJOR
+};
+
+int parse_mode(int mode, ModeInfo* mi) {
+  const int q = mode & FN_MODE_MASK, flags = mode & ~FN_MODE_MASK;
+  if (q < FN_FP8_PER_TOKEN || q > FN_MXFP4) return FN_ERR_INVALID;
+  mi->q = q;
+  mi->layout = fn::SCALE_ROW_MAJOR;
+  if (flags == FN_SCALE_SWIZZLE_32_4_4) {
+    if (q != FN_MXFP4) return FN_ERR_INVALID;
+    mi->layout = fn::SCALE_SWIZZLE_32_4_4;
+  } else if (flags == FN_SCALE_MN_MAJOR) {
+    if (q != FN_FP8_PER_GROUP128) return FN_ERR_INVALID;
+    mi->layout = fn::SCALE_MN_MAJOR;
+  } else if (flags != 0) {
+    return FN_ERR_INVALID;
+  }
+  return FN_OK;
+}
+
+int check_mode_shape(const ModeInfo& mi, int64_t M, int64_t H) {
   if (M < 0 || H <= 0 || H % 8) return FN_ERR_INVALID;
-  if (mode == FN_FP8_PER_GROUP128 && H % 128) return FN_ERR_INVALID;
-  if (mode == FN_MXFP4 && H % 32) return FN_ERR_INVALID;
+  if (mi.q == FN_FP8_PER_GROUP128 && H % 128) return FN_ERR_INVALID;
+  if (mi.q == FN_MXFP4 && H % 32) return FN_ERR_INVALID;
   if (H > FN_MAX_H) return FN_ERR_UNSUPPORTED;
   if (M > (int64_t)INT32_MAX / 8) return FN_ERR_UNSUPPORTED;  // grid size
   return FN_OK;
 }
 
-int64_t code_bytes(int mode, int64_t M, int64_t H) { return mode == FN_MXFP4 ? M * H / 2 : M * H; }
+int64_t code_bytes(const ModeInfo& mi, int64_t M, int64_t H) {
+  return mi.q == FN_MXFP4 ? M * H / 2 : M * H;
+}
 
-int64_t scale_bytes(int mode, int64_t M, int64_t H) {
-  if (mode == FN_FP8_PER_TOKEN) return M * 4;
-  if (mode == FN_FP8_PER_GROUP128) return M * (H / 128) * 4;
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// Bytes of the scale buffer, including a layout's padding.
+int64_t scale_bytes(const ModeInfo& mi, int64_t M, int64_t H) {
+  if (mi.q == FN_FP8_PER_TOKEN) return M * 4;
+  if (mi.q == FN_FP8_PER_GROUP128)
+    return (mi.layout == fn::SCALE_MN_MAJOR ? round_up(M, 4) : M) * (H / 128) * 4;
+  if (mi.layout == fn::SCALE_SWIZZLE_32_4_4) return round_up(M, 128) * round_up(H / 32, 4);
   return M * (H / 32);
 }
 
-int check_outputs_align(int mode, const void* out_q, const void* out_scale) {
-  if (!aligned(out_q, mode == FN_MXFP4 ? 4 : 8)) return FN_ERR_ALIGN;
-  if (mode != FN_MXFP4 && !aligned(out_scale, 4)) return FN_ERR_ALIGN;
+// The kernel's scale-index parameter for a layout.
+int64_t scale_ld(const ModeInfo& mi, int64_t M, int64_t H) {
+  if (mi.layout == fn::SCALE_SWIZZLE_32_4_4) return round_up(H / 32, 4) / 4;  // column tiles
+  if (mi.layout == fn::SCALE_MN_MAJOR) return round_up(M, 4);
+  return 0;
+}
+
+int check_outputs_align(const ModeInfo& mi, const void* out_q, const void* out_scale) {
+  if (!aligned(out_q, mi.q == FN_MXFP4 ? 4 : 8)) return FN_ERR_ALIGN;
+  if (mi.q != FN_MXFP4 && !aligned(out_scale, 4)) return FN_ERR_ALIGN;
   return FN_OK;
 }
 
 int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, void* stream,
               int variant_if_norm) {
+  // `mode` is the quantization alone here (the layout travels in prm)
   const int nvec = prm.nvec;
   const int sms = sm_count();
   if (sms <= 0) return FN_ERR_CUDA;
@@ -334,8 +371,10 @@ int fn_rmsnorm_quant(const void* const* x_parts, int num_parts, const void* resi
                      void* stream) {
   tl_variant = FN_VARIANT_NONE;
   if (!x_parts || num_parts < 1 || num_parts > FN_MAX_PARTS) return FN_ERR_INVALID;
-  int rc = check_mode_shape(mode, M, H);
+  ModeInfo mi;
+  int rc = parse_mode(mode, &mi);
   if (rc != FN_OK) return rc;
+  if ((rc = check_mode_shape(mi, M, H)) != FN_OK) return rc;
   if (!std::isfinite(eps) || eps < 0.f) return FN_ERR_INVALID;
   if (M == 0) return FN_OK;  // nothing to read or write: data pointers may be NULL
   if (!weight || !out_q || !out_scale) return FN_ERR_INVALID;
@@ -347,13 +386,13 @@ int fn_rmsnorm_quant(const void* const* x_parts, int num_parts, const void* resi
   if (!aligned(weight, 16) || (residual && !aligned(residual, 16)) ||
       (out_residual && !aligned(out_residual, 16)) || (out_y && !aligned(out_y, 16)))
     return FN_ERR_ALIGN;
-  if ((rc = check_outputs_align(mode, out_q, out_scale)) != FN_OK) return rc;
+  if ((rc = check_outputs_align(mi, out_q, out_scale)) != FN_OK) return rc;
 
   const int64_t row_bytes = M * H * 2;
   Range outs[4];
   int no = 0;
-  outs[no++] = range_of(out_q, code_bytes(mode, M, H));
-  outs[no++] = range_of(out_scale, scale_bytes(mode, M, H));
+  outs[no++] = range_of(out_q, code_bytes(mi, M, H));
+  outs[no++] = range_of(out_scale, scale_bytes(mi, M, H));
   if (out_residual) outs[no++] = range_of(out_residual, row_bytes);
   if (out_y) outs[no++] = range_of(out_y, row_bytes);
   if (M > 0) {
@@ -389,22 +428,26 @@ int fn_rmsnorm_quant(const void* const* x_parts, int num_parts, const void* resi
   prm.P = num_parts;
   prm.eps = eps;
   prm.inv_h = 1.0f / (float)H;
-  return launch_rq(prm, mode, num_parts, M, true, stream, FN_VARIANT_ROW_CTA);
+  prm.scale_layout = mi.layout;
+  prm.scale_ld = scale_ld(mi, M, H);
+  return launch_rq(prm, mi.q, num_parts, M, true, stream, FN_VARIANT_ROW_CTA);
 }
 
 int fn_quant(const void* y, int mode, int64_t M, int64_t H, void* out_q, void* out_scale,
              void* stream) {
   tl_variant = FN_VARIANT_NONE;
-  int rc = check_mode_shape(mode, M, H);
+  ModeInfo mi;
+  int rc = parse_mode(mode, &mi);
   if (rc != FN_OK) return rc;
+  if ((rc = check_mode_shape(mi, M, H)) != FN_OK) return rc;
   if (M == 0) return FN_OK;
   if (!y || !out_q || !out_scale) return FN_ERR_INVALID;
   if (!aligned(y, 16)) return FN_ERR_ALIGN;
-  if ((rc = check_outputs_align(mode, out_q, out_scale)) != FN_OK) return rc;
+  if ((rc = check_outputs_align(mi, out_q, out_scale)) != FN_OK) return rc;
   if (M > 0) {
     const Range in = range_of(y, M * H * 2);
-    const Range q = range_of(out_q, code_bytes(mode, M, H));
-    const Range s = range_of(out_scale, scale_bytes(mode, M, H));
+    const Range q = range_of(out_q, code_bytes(mi, M, H));
+    const Range s = range_of(out_scale, scale_bytes(mi, M, H));
     if (overlap(in, q) || overlap(in, s) || overlap(q, s)) return FN_ERR_INVALID;
   }
   if (M == 0) return FN_OK;
@@ -416,7 +459,9 @@ int fn_quant(const void* y, int mode, int64_t M, int64_t H, void* out_q, void* o
   prm.M = M;
   prm.nvec = (int)(H / 8);
   prm.P = 1;
-  return launch_rq(prm, mode, 1, M, false, stream, FN_VARIANT_QUANT_ONLY);
+  prm.scale_layout = mi.layout;
+  prm.scale_ld = scale_ld(mi, M, H);
+  return launch_rq(prm, mi.q, 1, M, false, stream, FN_VARIANT_QUANT_ONLY);
 }
 
 int fn_qk_norm_gate(const void* qkv, int64_t M, int64_t row_stride, int Hq, int Hk, int D,

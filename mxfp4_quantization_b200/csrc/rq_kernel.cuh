@@ -168,6 +168,20 @@ __device__ __forceinline__ uint32_t e2m1_codes(const uint4& y, uint32_t inv_bf16
   return cvt_e2m1x8(f);
 }
 
+// Byte offset (MX) or element index (FP8 groups) of the scale of group `g`
+// of row `row` in the requested layout (row-major unless a flag asks
+// otherwise).  The 32x4x4 swizzle is the tiling of block-scaled matrix
+// multiplies on this architecture: 128 rows x 4 groups per 512-byte tile,
+// tiles in row-tile-major order, and inside a tile row r, group c at
+// (r % 32) * 16 + (r / 32) * 4 + c.
+__device__ __forceinline__ int64_t scale_index(int layout, int64_t ld, int64_t row, int64_t g,
+                                               int64_t groups_per_row) {
+  if (layout == SCALE_SWIZZLE_32_4_4)
+    return ((row >> 7) * ld + (g >> 2)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (g & 3);
+  if (layout == SCALE_MN_MAJOR) return g * ld + row;
+  return row * groups_per_row + g;
+}
+
 // Quantize vector v of a row (y: 8 bf16) and store its codes and, from the
 // group's first lane, its scale.  All 32 lanes must call (shuffles); `ok`
 // masks the stores of lanes past the row end (whole groups, by alignment).
@@ -175,12 +189,13 @@ __device__ __forceinline__ uint32_t e2m1_codes(const uint4& y, uint32_t inv_bf16
 template <int MODE>
 __device__ __forceinline__ void quant_store(const uint4& y, bool ok, int lane, int64_t row, int v,
                                             int H, const Fp8Scale& tok, uint8_t* out_q,
-                                            void* out_scale) {
+                                            void* out_scale, int layout, int64_t ld) {
   if constexpr (MODE == MODE_TOKEN || MODE == MODE_G128) {
     Fp8Scale c = tok;
     if constexpr (MODE == MODE_G128) {
       c = fp8_scale_direct(group_max<16>(vec_absmax(y)));
-      if (ok && (lane & 15) == 0) static_cast<float*>(out_scale)[row * (H / 128) + v / 16] = c.s;
+      if (ok && (lane & 15) == 0)
+        static_cast<float*>(out_scale)[scale_index(layout, ld, row, v / 16, H / 128)] = c.s;
     }
     const uint2 q = e4m3_codes(y, c);
     if (ok) st_stream(reinterpret_cast<uint2*>(out_q + row * (int64_t)H) + v, q);
@@ -191,7 +206,9 @@ __device__ __forceinline__ void quant_store(const uint4& y, bool ok, int lane, i
     const uint32_t q = e2m1_codes(y, inv_b | (inv_b << 16));
     if (ok) {
       st_stream(reinterpret_cast<uint32_t*>(out_q + row * (int64_t)(H / 2)) + v, q);
-      if ((lane & 3) == 0) static_cast<uint8_t*>(out_scale)[row * (H / 32) + v / 4] = (uint8_t)code;
+      if ((lane & 3) == 0)
+        static_cast<uint8_t*>(out_scale)[scale_index(layout, ld, row, v / 4, H / 32)] =
+            (uint8_t)code;
     }
   }
 }
@@ -353,7 +370,8 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
 #pragma unroll
   for (int k = 0; k < V; ++k) {
     const int v = seg_base + t + k * T;
-    quant_store<MODE>(yv[k], v < seg_end, lane, row, v, H, scale_tok, prm.out_q, prm.out_scale);
+    quant_store<MODE>(yv[k], v < seg_end, lane, row, v, H, scale_tok, prm.out_q, prm.out_scale,
+                      prm.scale_layout, prm.scale_ld);
   }
 
   if constexpr (CL) {
@@ -590,7 +608,8 @@ __global__ void __launch_bounds__(512, 1)
       const bool ok = v < nvec;
       const uint4 y = norm_vec(hv[k], wv[k], rstd);
       if (ok && prm.out_y != nullptr) st_stream(prm.out_y + rowv + v, y);
-      quant_store<MODE>(y, ok, lane, row, v, H, scale_tok, prm.out_q, prm.out_scale);
+      quant_store<MODE>(y, ok, lane, row, v, H, scale_tok, prm.out_q, prm.out_scale,
+                        prm.scale_layout, prm.scale_ld);
     }
   }
   if (timed_out && prm.status != nullptr) atomicExch(prm.status, 1);

@@ -7,6 +7,9 @@ namespace fn {
 
 enum : int { MODE_TOKEN = 0, MODE_G128 = 1, MODE_MX = 2 };
 
+// Scale layouts (include/fusednorm.h, FN_SCALE_*).
+enum : int { SCALE_ROW_MAJOR = 0, SCALE_SWIZZLE_32_4_4 = 1, SCALE_MN_MAJOR = 2 };
+
 struct RQParams {
   const uint4* parts[8];   // P bf16 [M, H] inputs (as 16-byte vectors)
   const uint4* residual;   // bf16 [M, H] or nullptr
@@ -24,6 +27,8 @@ struct RQParams {
   int* status;             // library status word: set to 1 if a bounded wait gave up
   uint32_t debug_extra_tx; // test hook: extra bytes each TMA stage expects (0 normally)
   int prefetch_rows;       // L2 prefetch distance in rows of this block (0: none)
+  int scale_layout;        // SCALE_*
+  int64_t scale_ld;        // swizzled: column tiles per row tile; MN-major: row stride
 };
 
 // A kernel instance: every (mode, partial bound, vectors per thread, norm,

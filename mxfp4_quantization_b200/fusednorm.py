@@ -39,6 +39,10 @@ FN_VARIANT_QUANT_ONLY = 3
 FN_VARIANT_QK_WARP = 4
 FN_VARIANT_ROW_TMA = 5
 
+FN_MODE_MASK = 0xFF
+FN_SCALE_SWIZZLE_32_4_4 = 0x100
+FN_SCALE_MN_MAJOR = 0x200
+
 FN_MAX_PARTS = 8
 FN_MAX_H = 32768
 FN_MAX_HEAD_DIM = 1024
@@ -197,15 +201,29 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _round_up(x: int, m: int) -> int:
+    return (x + m - 1) // m * m
+
+
 def alloc_outputs(mode: int, M: int, H: int, device) -> tuple:
-    """Codes and scales for `mode`: FP8 codes as float8_e4m3fn [M, H]; MXFP4 codes
-    as uint8 [M, H/2]; scales fp32 [M, 1] / fp32 [M, H/128] / uint8 E8M0 [M, H/32]."""
-    if mode == FN_MXFP4:
-        return (torch.empty((M, H // 2), dtype=torch.uint8, device=device),
-                torch.empty((M, H // 32), dtype=torch.uint8, device=device))
+    """Codes and scales for `mode` (with its layout flag, if any): FP8 codes as
+    float8_e4m3fn [M, H]; MXFP4 codes as uint8 [M, H/2]; scales fp32 [M, 1] /
+    fp32 [M, H/128] / uint8 E8M0 [M, H/32] row-major, or, with a layout flag,
+    the padded buffer that layout needs (zero-filled: padding is not written):
+    uint8 [roundup(M,128) * roundup(H/32,4)] for FN_SCALE_SWIZZLE_32_4_4,
+    fp32 [H/128, roundup(M,4)] for FN_SCALE_MN_MAJOR."""
+    q_mode, flags = mode & FN_MODE_MASK, mode & ~FN_MODE_MASK
+    if q_mode == FN_MXFP4:
+        q = torch.empty((M, H // 2), dtype=torch.uint8, device=device)
+        if flags == FN_SCALE_SWIZZLE_32_4_4:
+            n = _round_up(M, 128) * _round_up(H // 32, 4)
+            return q, torch.zeros((n,), dtype=torch.uint8, device=device)
+        return q, torch.empty((M, H // 32), dtype=torch.uint8, device=device)
     q = torch.empty((M, H), dtype=torch.float8_e4m3fn, device=device)
-    if mode == FN_FP8_PER_TOKEN:
+    if q_mode == FN_FP8_PER_TOKEN:
         return q, torch.empty((M, 1), dtype=torch.float32, device=device)
+    if flags == FN_SCALE_MN_MAJOR:
+        return q, torch.zeros((H // 128, _round_up(M, 4)), dtype=torch.float32, device=device)
     return q, torch.empty((M, H // 128), dtype=torch.float32, device=device)
 
 

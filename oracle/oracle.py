@@ -185,3 +185,41 @@ def qk_norm_gate(qkv, row_stride: int, Hq: int, Hk: int, D: int, q_weight, k_wei
     if rc != 0:
         raise OracleError("orc_qk_norm_gate rejected the shape")
     return {"q": q, "k": k, "gate": g}
+
+
+# ---- scale layouts ------------------------------------------------------------
+
+SCALE_SWIZZLE_32_4_4 = 0x100
+SCALE_MN_MAJOR = 0x200
+
+
+def _round_up(x, m):
+    return (x + m - 1) // m * m
+
+
+def place_scales(scales, layout: int, fill=0):
+    """Row-major scales [M, G] -> the flat buffer of `layout`.
+
+    SCALE_SWIZZLE_32_4_4: [M, G] padded to [roundup(M,128), roundup(G,4)] and
+    cut into 128 x 4 tiles of 512 entries, tiles in row-tile-major order;
+    inside a tile, row r and group c sit at (r % 32) * 16 + (r // 32) * 4 + c.
+    SCALE_MN_MAJOR: [G, roundup(M,4)], entry (g, m) = scale of row m, group g.
+    Padding entries hold `fill`.
+    """
+    scales = np.asarray(scales)
+    M, G = scales.shape
+    if layout == SCALE_SWIZZLE_32_4_4:
+        Mp, Gp = _round_up(M, 128), _round_up(G, 4)
+        out = np.full(Mp * Gp, fill, dtype=scales.dtype)
+        ct = Gp // 4
+        for m in range(M):
+            for g in range(G):
+                off = ((m // 128) * ct + g // 4) * 512 + (m % 32) * 16 + ((m % 128) // 32) * 4 + g % 4
+                out[off] = scales[m, g]
+        return out
+    if layout == SCALE_MN_MAJOR:
+        Mp = _round_up(M, 4)
+        out = np.full((G, Mp), fill, dtype=scales.dtype)
+        out[:, :M] = scales.T
+        return out.reshape(-1)
+    raise OracleError(f"unknown scale layout {layout:#x}")

@@ -478,3 +478,23 @@ def pin_qk_layout(lib):
 ALL_PINS = [pin_e4m3_decode, pin_e4m3_encode, pin_e2m1, pin_bf16_rounding, pin_mx_scale,
             pin_worked_rows, pin_rstd_closed_form, pin_quant_stage_random,
             pin_full_path_bruteforce, pin_partial_sum_order, pin_qk_layout]
+
+
+def pin_scale_layouts(lib):
+    """The placement of scales in the GEMM layouts: the 32x4x4 swizzle against
+    a library's own implementation of that layout (quack.mx_utils.to_blocked),
+    the M-major layout against a plain transpose."""
+    from quack.mx_utils import to_blocked
+    rng = np.random.default_rng(3)
+    for M, G in ((1, 1), (5, 7), (128, 4), (130, 9), (300, 224), (257, 56)):
+        a = rng.integers(0, 255, (M, G)).astype(np.uint8)
+        mine = oracle.place_scales(a, oracle.SCALE_SWIZZLE_32_4_4)
+        ref = to_blocked(torch.from_numpy(a)).numpy().reshape(-1)
+        assert np.array_equal(mine, ref), f"swizzled layout {M}x{G}"
+        f = rng.standard_normal((M, G)).astype(np.float32)
+        mm = oracle.place_scales(f, oracle.SCALE_MN_MAJOR).reshape(G, -1)
+        assert mm.shape[1] == (M + 3) // 4 * 4
+        assert np.array_equal(mm[:, :M], f.T) and np.all(mm[:, M:] == 0), f"M-major {M}x{G}"
+
+
+ALL_PINS.append(pin_scale_layouts)

@@ -153,3 +153,20 @@ def test_prefer_variant_is_thread_local_and_returns_previous(fnb):
     th.join()
     assert seen == [fnb.FN_VARIANT_NONE]
     assert fnb.fn_prefer_variant(fnb.FN_VARIANT_NONE) == fnb.FN_VARIANT_ROW_TMA
+
+
+def test_scale_layout_flags(fnb):
+    E = fnb.FN_ERR_INVALID
+    SW, MN = fnb.FN_SCALE_SWIZZLE_32_4_4, fnb.FN_SCALE_MN_MAJOR
+    # each flag only with its mode, no unknown flags, no two flags
+    assert rq(fnb, M=0, mode=fnb.FN_MXFP4 | SW) == fnb.FN_OK
+    assert rq(fnb, M=0, mode=fnb.FN_FP8_PER_GROUP128 | MN) == fnb.FN_OK
+    assert rq(fnb, M=0, mode=fnb.FN_FP8_PER_TOKEN | SW) == E
+    assert rq(fnb, M=0, mode=fnb.FN_MXFP4 | MN) == E
+    assert rq(fnb, M=0, mode=fnb.FN_MXFP4 | SW | MN) == E
+    assert rq(fnb, M=0, mode=fnb.FN_MXFP4 | 0x400) == E
+    # the padded scale buffer counts in the overlap check: M=4, H=256 swizzled
+    # needs 128 * 8 bytes of scales, so codes 512 bytes after it overlap
+    assert rq(fnb, mode=fnb.FN_MXFP4 | SW, out_q=BASE + (4 << 32) + 512) == E
+    assert fnb.fn_quant(BASE, fnb.FN_FP8_PER_TOKEN | MN, 4, 256, BASE + (1 << 32),
+                        BASE + (2 << 32), None) == E
