@@ -273,9 +273,14 @@ def make_row_call(fn, wl, device, seed):
 
 
 def e2e_row(fn, wl, device, steps, warmup, seed):
-    """Rows/s through the public tensor API from pinned host memory: each step
-    copies the step's inputs host->device, runs the fused call and reads the
-    quantized tuple (codes, scales, residual_out) back to pinned host memory."""
+    """Rows/s through the public tensor API from pinned host memory: every
+    step copies its inputs host->device, runs the fused call and reads the
+    quantized tuple (codes, scales, residual_out) back to pinned host memory.
+    Steps are pipelined the way a serving loop would run them: two device
+    buffer sets, host->device copies on one stream, the kernel on a second,
+    device->host copies on a third, so that step i+1's inputs travel while
+    step i computes and its results travel back (PCIe is full duplex).
+    Returns (ms per step, h2d bytes per step, d2h bytes per step)."""
     import torch
     from mxfp4_quantization_b200 import synth
     wl = synth.RowWorkload(**{**wl.__dict__, "seed": seed})
@@ -283,30 +288,66 @@ def e2e_row(fn, wl, device, steps, warmup, seed):
     h_parts = [p.to("cpu").pin_memory() for p in src["parts"]]
     h_res = src["residual"].to("cpu").pin_memory()
     w = src["weight"]
-    d_parts = [torch.empty_like(p) for p in src["parts"]]
-    d_res = torch.empty_like(src["residual"])
-    q, s = fn.alloc_outputs(wl.mode, wl.M, wl.H, device)
-    d_rout = torch.empty_like(d_res)
-    h_q = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
-    h_s = torch.empty(s.shape, dtype=s.dtype, pin_memory=True)
-    h_rout = torch.empty(d_rout.shape, dtype=d_rout.dtype, pin_memory=True)
+    sets = []
+    for _ in range(2):
+        q, s = fn.alloc_outputs(wl.mode, wl.M, wl.H, device)
+        sets.append({"parts": [torch.empty_like(p) for p in src["parts"]],
+                     "res": torch.empty_like(src["residual"]),
+                     "rout": torch.empty_like(src["residual"]), "q": q, "s": s})
+    q0, s0 = sets[0]["q"], sets[0]["s"]
+    h_q = torch.empty(q0.shape, dtype=q0.dtype, pin_memory=True)
+    h_s = torch.empty(s0.shape, dtype=s0.dtype, pin_memory=True)
+    h_rout = torch.empty(sets[0]["rout"].shape, dtype=torch.bfloat16, pin_memory=True)
     del src
     h2d = sum(p.numel() * p.element_size() for p in h_parts) + h_res.numel() * 2
-    d2h = q.numel() * q.element_size() + s.numel() * s.element_size() + d_rout.numel() * 2
-    stream = torch.cuda.current_stream(device)
+    d2h = q0.numel() * q0.element_size() + s0.numel() * s0.element_size() + h_rout.numel() * 2
+    s_in, s_cmp, s_out = (torch.cuda.Stream(device) for _ in range(3))
+    in_done = [torch.cuda.Event() for _ in range(2)]
+    cmp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
+    for e in cmp_done + out_done:
+        e.record(torch.cuda.current_stream(device))
 
-    def step():
-        for hp, dp in zip(h_parts, d_parts):
-            dp.copy_(hp, non_blocking=True)
-        d_res.copy_(h_res, non_blocking=True)
-        fn.rmsnorm_quant(d_parts, w, wl.eps, wl.mode, residual=d_res, out_residual=d_rout,
-                         out_q=q, out_scale=s)
-        h_q.copy_(q, non_blocking=True)
-        h_s.copy_(s, non_blocking=True)
-        h_rout.copy_(d_rout, non_blocking=True)
+    def step(i):
+        b = i & 1
+        st = sets[b]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(cmp_done[b])  # this set's inputs were consumed two steps ago
+            for hp, dp in zip(h_parts, st["parts"]):
+                dp.copy_(hp, non_blocking=True)
+            st["res"].copy_(h_res, non_blocking=True)
+            in_done[b].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(in_done[b])
+            s_cmp.wait_event(out_done[b])  # and its outputs were read back
+            fn.rmsnorm_quant(st["parts"], w, wl.eps, wl.mode, residual=st["res"],
+                             out_residual=st["rout"], out_q=st["q"], out_scale=st["s"])
+            cmp_done[b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(cmp_done[b])
+            h_q.copy_(st["q"], non_blocking=True)
+            h_s.copy_(st["s"], non_blocking=True)
+            h_rout.copy_(st["rout"], non_blocking=True)
+            out_done[b].record(s_out)
 
-    ms = time_steps(step, steps, warmup, device, stream)
-    return ms, h2d, d2h
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    s_cmp.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(steps):
+        step(i)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_cmp)
+    e1.record(s_out)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
 def time_graph_calls(make_calls, n_sets, replays, device):
@@ -378,21 +419,37 @@ def decode_calls(fn, wl, device):
     return make
 
 
-def qk_calls(fn, wl, device):
+def qk_calls(fn, wl, device, fp8=False):
     import torch
 
     def make(n):
         inp = wl.inputs(device=device)
         calls = []
+        bf, f8, f32 = torch.bfloat16, torch.uint8, torch.float32
         for i in range(n):
             qkv = inp["qkv"].roll(i, 0).clone()
-            out = fn.QKOutput(torch.empty((wl.M, wl.Hq, wl.D), dtype=torch.bfloat16, device=device),
-                              torch.empty((wl.M, wl.Hk, wl.D), dtype=torch.bfloat16, device=device),
-                              torch.empty((wl.M, wl.Hq, wl.D), dtype=torch.bfloat16, device=device))
+            if fp8:
+                bufs = [torch.empty((wl.M, wl.Hq, wl.D), dtype=f8, device=device),
+                        torch.empty((wl.M, wl.Hq), dtype=f32, device=device),
+                        torch.empty((wl.M, wl.Hk, wl.D), dtype=f8, device=device),
+                        torch.empty((wl.M, wl.Hk), dtype=f32, device=device),
+                        torch.empty((wl.M, wl.Hq, wl.D), dtype=bf, device=device)]
 
-            def call(qkv=qkv, out=out):
-                fn.qk_norm_gate(qkv, wl.Hq, wl.Hk, wl.D, inp["q_weight"], inp["k_weight"],
-                                wl.eps, out=out)
+                def call(qkv=qkv, bufs=bufs):
+                    st = fn.fn_qk_norm_gate_fp8(
+                        qkv.data_ptr(), wl.M, qkv.stride(0), wl.Hq, wl.Hk, wl.D,
+                        inp["q_weight"].data_ptr(), inp["k_weight"].data_ptr(), wl.eps,
+                        *[b.data_ptr() for b in bufs], None, None,
+                        torch.cuda.current_stream(device).cuda_stream)
+                    assert st == fn.FN_OK
+            else:
+                out = fn.QKOutput(torch.empty((wl.M, wl.Hq, wl.D), dtype=bf, device=device),
+                                  torch.empty((wl.M, wl.Hk, wl.D), dtype=bf, device=device),
+                                  torch.empty((wl.M, wl.Hq, wl.D), dtype=bf, device=device))
+
+                def call(qkv=qkv, out=out):
+                    fn.qk_norm_gate(qkv, wl.Hq, wl.Hk, wl.D, inp["q_weight"], inp["k_weight"],
+                                    wl.eps, out=out)
             calls.append(call)
         return calls
     return make
@@ -459,6 +516,9 @@ def secondary_workloads(fn, device, peak):
     for M in synth.QK_M:
         wl = synth.qk_prologue(M)
         qk[f"m{M}"] = small(wl, wl.bytes_per_call(), qk_calls(fn, wl, device))
+        # FP8 epilogue: codes (1 byte) and a scale per head replace the bf16 q, k
+        b8 = wl.bytes_per_call() - M * (wl.Hq + wl.Hk) * (wl.D - 4)
+        qk[f"m{M}_fp8"] = small(wl, b8, qk_calls(fn, wl, device, fp8=True))
     res["qk_prologue"] = qk
     return res
 
@@ -571,7 +631,7 @@ def main_arm(args):
     del keep
     torch.cuda.empty_cache()
 
-    e2e_steps = max(3, min(args.steps, 10))
+    e2e_steps = max(4, min(args.steps, 20))
     e2e_ms, h2d, d2h = e2e_row(fn, wl, device, e2e_steps, 2, seed)
     e2e_ms_max = dist_max(e2e_ms, device)
 
@@ -606,7 +666,9 @@ def main_arm(args):
                          "launch": list(launch), "variant": variant},
             "e2e": {"value": aggregate(wl.M, world, e2e_ms_max), "unit": "rows/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": e2e_steps},
+                    "steps": e2e_steps,
+                    "method": "public tensor API; pinned host buffers; copies in, kernel and "
+                              "copies out on three streams, two buffer sets (steps pipelined)"},
             "gpu_launches": args.steps,
             "clocks": clk,
             "cpu_baseline": cpu,

@@ -79,7 +79,8 @@ typedef enum {
     FN_VARIANT_ROW_CLUSTER = 2, /* a cluster of 2..8 blocks per row (small M)      */
     FN_VARIANT_QUANT_ONLY = 3,  /* fn_quant                                        */
     FN_VARIANT_QK_WARP = 4,     /* fn_qk_norm_gate: one warp per (token, head)     */
-    FN_VARIANT_ROW_TMA = 5      /* persistent blocks, rows staged by bulk copies  */
+    FN_VARIANT_ROW_TMA = 5,     /* persistent blocks, rows staged by bulk copies  */
+    FN_VARIANT_QK_WARP_FP8 = 6  /* fn_qk_norm_gate_fp8                             */
 } fn_variant;
 
 /* Scale-layout flags, OR-ed into `mode` (fn_rmsnorm_quant, fn_quant).  No
@@ -172,6 +173,24 @@ FN_API int fn_quant(const void* y, int mode, int64_t M, int64_t H, void* out_q, 
 FN_API int fn_qk_norm_gate(const void* qkv, int64_t M, int64_t row_stride, int Hq, int Hk, int D,
                     const void* q_weight, const void* k_weight, float eps, void* out_q,
                     void* out_k, void* out_gate, void* stream);
+
+/*
+ * fn_qk_norm_gate with an FP8 epilogue for an FP8 attention consumer (the
+ * pages' MXFP4-AttnFP8 serving runs attention in FP8; sglang PR #29723,
+ * "Speed Tests").  Each normed q and k head (D values) is quantized with the
+ * per-token rule of fn_rmsnorm_quant applied to the head vector: scale =
+ * amax / 448 (fp32 division, 1.0 for an all-zero head), code = E4M3 of
+ * y / scale, nearest even, saturating.
+ * out_q8     u8 E4M3 [M, Hq, D], 8-byte aligned;  out_q_scale fp32 [M, Hq].
+ * out_k8     u8 E4M3 [M, Hk, D], 8-byte aligned;  out_k_scale fp32 [M, Hk].
+ * out_gate   bf16 [M, Hq, D] as in fn_qk_norm_gate.
+ * out_q, out_k  the bf16 normed heads as in fn_qk_norm_gate, or NULL.
+ * Other arguments, checks and errors as fn_qk_norm_gate.
+ */
+FN_API int fn_qk_norm_gate_fp8(const void* qkv, int64_t M, int64_t row_stride, int Hq, int Hk,
+                               int D, const void* q_weight, const void* k_weight, float eps,
+                               void* out_q8, void* out_q_scale, void* out_k8, void* out_k_scale,
+                               void* out_gate, void* out_q, void* out_k, void* stream);
 
 /* Static, NUL-terminated description of a status code. */
 FN_API const char* fn_status_string(int status);

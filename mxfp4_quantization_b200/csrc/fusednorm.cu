@@ -304,17 +304,103 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, vo
   return FN_OK;
 }
 
-template <int VPL>
+template <int VPL, bool FP8>
 int launch_qk_v(const fn::QKParams& p, int64_t items, int sms, cudaStream_t st) {
   const int wpb = items <= (int64_t)8 * sms ? 1 : 8;
   const int64_t blocks = (items + wpb - 1) / wpb;
-  fn::qk_kernel<VPL><<<(unsigned)blocks, wpb * 32, 0, st>>>(p);
+  fn::qk_kernel<VPL, FP8><<<(unsigned)blocks, wpb * 32, 0, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return FN_ERR_CUDA;
   tl_launch[0] = (int32_t)blocks;
   tl_launch[1] = wpb * 32;
   tl_launch[2] = 1;
   tl_launch[3] = VPL;
   return FN_OK;
+}
+
+
+// Shared body of fn_qk_norm_gate and fn_qk_norm_gate_fp8 (fp8 when out_q8 or
+// out_k8 is given; the bf16 q / k outputs are then optional).
+int qk_impl(const void* qkv, int64_t M, int64_t row_stride, int Hq, int Hk, int D,
+            const void* q_weight, const void* k_weight, float eps, void* out_q, void* out_k,
+            void* out_gate, void* out_q8, void* out_qs, void* out_k8, void* out_ks,
+            void* stream) {
+  tl_variant = FN_VARIANT_NONE;
+  const bool fp8 = out_q8 != nullptr || out_k8 != nullptr;
+  if (M < 0 || Hq < 0 || Hk < 0 || Hq + Hk < 1 || D <= 0 || D % 8) return FN_ERR_INVALID;
+  if (D > FN_MAX_HEAD_DIM) return FN_ERR_UNSUPPORTED;
+  if (row_stride % 8 || row_stride < (int64_t)(2 * Hq + Hk) * D) return FN_ERR_INVALID;
+  if (!std::isfinite(eps) || eps < 0.f) return FN_ERR_INVALID;
+  if (M == 0) return FN_OK;
+  if (!qkv || (Hq > 0 && (!q_weight || !out_gate || (!out_q && !fp8))) ||
+      (Hk > 0 && (!k_weight || (!out_k && !fp8))))
+    return FN_ERR_INVALID;
+  if (!aligned(qkv, 16) || (q_weight && !aligned(q_weight, 16)) ||
+      (k_weight && !aligned(k_weight, 16)) || (out_q && !aligned(out_q, 16)) ||
+      (out_k && !aligned(out_k, 16)) || (out_gate && !aligned(out_gate, 16)) ||
+      (out_q8 && !aligned(out_q8, 8)) || (out_k8 && !aligned(out_k8, 8)) ||
+      (out_qs && !aligned(out_qs, 4)) || (out_ks && !aligned(out_ks, 4)))
+    return FN_ERR_ALIGN;
+  if (M > (int64_t)INT32_MAX / 8 || (int64_t)M * (Hq + Hk) > (int64_t)INT32_MAX)
+    return FN_ERR_UNSUPPORTED;
+  {
+    const Range in = range_of(qkv, ((M - 1) * row_stride + (int64_t)(2 * Hq + Hk) * D) * 2);
+    Range outs[7];
+    int no = 0;
+    if (Hq > 0) {
+      if (out_q) outs[no++] = range_of(out_q, M * Hq * D * 2);
+      outs[no++] = range_of(out_gate, M * Hq * D * 2);
+      if (out_q8) outs[no++] = range_of(out_q8, M * Hq * D);
+      if (out_qs) outs[no++] = range_of(out_qs, M * Hq * 4);
+    }
+    if (Hk > 0) {
+      if (out_k) outs[no++] = range_of(out_k, M * Hk * D * 2);
+      if (out_k8) outs[no++] = range_of(out_k8, M * Hk * D);
+      if (out_ks) outs[no++] = range_of(out_ks, M * Hk * 4);
+    }
+    for (int i = 0; i < no; ++i) {
+      if (overlap(outs[i], in)) return FN_ERR_INVALID;
+      if (q_weight && overlap(outs[i], range_of(q_weight, D * 2))) return FN_ERR_INVALID;
+      if (k_weight && overlap(outs[i], range_of(k_weight, D * 2))) return FN_ERR_INVALID;
+      for (int j = i + 1; j < no; ++j)
+        if (overlap(outs[i], outs[j])) return FN_ERR_INVALID;
+    }
+  }
+  const int sms = sm_count();
+  if (sms <= 0) return FN_ERR_CUDA;
+  fn::QKParams p;
+  std::memset(&p, 0, sizeof p);
+  p.qkv = static_cast<const uint4*>(qkv);
+  p.M = M;
+  p.row_vec = row_stride / 8;
+  p.Hq = Hq;
+  p.Hk = Hk;
+  p.dv = D / 8;
+  p.qw = static_cast<const uint4*>(q_weight);
+  p.kw = static_cast<const uint4*>(k_weight);
+  p.eps = eps;
+  p.inv_d = 1.0f / (float)D;
+  p.out_q = static_cast<uint4*>(out_q);
+  p.out_k = static_cast<uint4*>(out_k);
+  p.out_g = static_cast<uint4*>(out_gate);
+  p.out_q8 = static_cast<uint8_t*>(out_q8);
+  p.out_qs = static_cast<float*>(out_qs);
+  p.out_k8 = static_cast<uint8_t*>(out_k8);
+  p.out_ks = static_cast<float*>(out_ks);
+  const int64_t items = M * (Hq + Hk);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc;
+  const int nv = D / 8;
+  if (fp8) {
+    if (nv <= 32) rc = launch_qk_v<1, true>(p, items, sms, st);
+    else if (nv <= 64) rc = launch_qk_v<2, true>(p, items, sms, st);
+    else rc = launch_qk_v<4, true>(p, items, sms, st);
+  } else {
+    if (nv <= 32) rc = launch_qk_v<1, false>(p, items, sms, st);
+    else if (nv <= 64) rc = launch_qk_v<2, false>(p, items, sms, st);
+    else rc = launch_qk_v<4, false>(p, items, sms, st);
+  }
+  if (rc == FN_OK) tl_variant = fp8 ? FN_VARIANT_QK_WARP_FP8 : FN_VARIANT_QK_WARP;
+  return rc;
 }
 
 }  // namespace
@@ -467,63 +553,19 @@ int fn_quant(const void* y, int mode, int64_t M, int64_t H, void* out_q, void* o
 int fn_qk_norm_gate(const void* qkv, int64_t M, int64_t row_stride, int Hq, int Hk, int D,
                     const void* q_weight, const void* k_weight, float eps, void* out_q,
                     void* out_k, void* out_gate, void* stream) {
+  return qk_impl(qkv, M, row_stride, Hq, Hk, D, q_weight, k_weight, eps, out_q, out_k, out_gate,
+                 nullptr, nullptr, nullptr, nullptr, stream);
+}
+
+int fn_qk_norm_gate_fp8(const void* qkv, int64_t M, int64_t row_stride, int Hq, int Hk, int D,
+                        const void* q_weight, const void* k_weight, float eps, void* out_q8,
+                        void* out_q_scale, void* out_k8, void* out_k_scale, void* out_gate,
+                        void* out_q, void* out_k, void* stream) {
   tl_variant = FN_VARIANT_NONE;
-  if (M < 0 || Hq < 0 || Hk < 0 || Hq + Hk < 1 || D <= 0 || D % 8) return FN_ERR_INVALID;
-  if (D > FN_MAX_HEAD_DIM) return FN_ERR_UNSUPPORTED;
-  if (row_stride % 8 || row_stride < (int64_t)(2 * Hq + Hk) * D) return FN_ERR_INVALID;
-  if (!std::isfinite(eps) || eps < 0.f) return FN_ERR_INVALID;
-  if (M == 0) return FN_OK;
-  if (!qkv || (Hq > 0 && (!q_weight || !out_q || !out_gate)) || (Hk > 0 && (!k_weight || !out_k)))
+  if (M > 0 && ((Hq > 0 && (!out_q8 || !out_q_scale)) || (Hk > 0 && (!out_k8 || !out_k_scale))))
     return FN_ERR_INVALID;
-  if (!aligned(qkv, 16) || (q_weight && !aligned(q_weight, 16)) ||
-      (k_weight && !aligned(k_weight, 16)) || (out_q && !aligned(out_q, 16)) ||
-      (out_k && !aligned(out_k, 16)) || (out_gate && !aligned(out_gate, 16)))
-    return FN_ERR_ALIGN;
-  if (M > (int64_t)INT32_MAX / 8 || (int64_t)M * (Hq + Hk) > (int64_t)INT32_MAX)
-    return FN_ERR_UNSUPPORTED;
-  if (M > 0) {
-    const Range in = range_of(qkv, ((M - 1) * row_stride + (int64_t)(2 * Hq + Hk) * D) * 2);
-    Range outs[3];
-    int no = 0;
-    if (Hq > 0) {
-      outs[no++] = range_of(out_q, M * Hq * D * 2);
-      outs[no++] = range_of(out_gate, M * Hq * D * 2);
-    }
-    if (Hk > 0) outs[no++] = range_of(out_k, M * Hk * D * 2);
-    for (int i = 0; i < no; ++i) {
-      if (overlap(outs[i], in)) return FN_ERR_INVALID;
-      if (q_weight && overlap(outs[i], range_of(q_weight, D * 2))) return FN_ERR_INVALID;
-      if (k_weight && overlap(outs[i], range_of(k_weight, D * 2))) return FN_ERR_INVALID;
-      for (int j = i + 1; j < no; ++j)
-        if (overlap(outs[i], outs[j])) return FN_ERR_INVALID;
-    }
-  }
-  if (M == 0) return FN_OK;
-  const int sms = sm_count();
-  if (sms <= 0) return FN_ERR_CUDA;
-  fn::QKParams p;
-  p.qkv = static_cast<const uint4*>(qkv);
-  p.M = M;
-  p.row_vec = row_stride / 8;
-  p.Hq = Hq;
-  p.Hk = Hk;
-  p.dv = D / 8;
-  p.qw = static_cast<const uint4*>(q_weight);
-  p.kw = static_cast<const uint4*>(k_weight);
-  p.eps = eps;
-  p.inv_d = 1.0f / (float)D;
-  p.out_q = static_cast<uint4*>(out_q);
-  p.out_k = static_cast<uint4*>(out_k);
-  p.out_g = static_cast<uint4*>(out_gate);
-  const int64_t items = M * (Hq + Hk);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int rc;
-  const int nv = D / 8;
-  if (nv <= 32) rc = launch_qk_v<1>(p, items, sms, st);
-  else if (nv <= 64) rc = launch_qk_v<2>(p, items, sms, st);
-  else rc = launch_qk_v<4>(p, items, sms, st);
-  if (rc == FN_OK) tl_variant = FN_VARIANT_QK_WARP;
-  return rc;
+  return qk_impl(qkv, M, row_stride, Hq, Hk, D, q_weight, k_weight, eps, out_q, out_k, out_gate,
+                 out_q8, out_q_scale, out_k8, out_k_scale, stream);
 }
 
 }  // extern "C"

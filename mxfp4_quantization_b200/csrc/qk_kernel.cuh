@@ -8,6 +8,7 @@
 // is ever made.  With head_dim 256 each lane holds one 16-byte vector.
 #pragma once
 #include "fn_device.cuh"
+#include "quant.cuh"
 
 namespace fn {
 
@@ -21,12 +22,19 @@ struct QKParams {
   const uint4* kw;
   float eps;
   float inv_d;      // 1 / head_dim
-  uint4* out_q;
+  uint4* out_q;     // bf16 outputs (optional when FP8 codes are written)
   uint4* out_k;
   uint4* out_g;
+  uint8_t* out_q8;  // E4M3 codes [M, Hq, D] and fp32 scales [M, Hq] (FP8 kernel)
+  float* out_qs;
+  uint8_t* out_k8;  // E4M3 codes [M, Hk, D] and fp32 scales [M, Hk]
+  float* out_ks;
 };
 
-template <int VPL>
+// FP8: also quantize each normed q and k head to E4M3 with one fp32 scale per
+// (token, head) — the per-token rule of the row kernels (scale = amax / 448)
+// applied to each head vector, for an FP8 attention consumer.
+template <int VPL, bool FP8>
 __global__ void __launch_bounds__(256) qk_kernel(const __grid_constant__ QKParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -39,8 +47,9 @@ __global__ void __launch_bounds__(256) qk_kernel(const __grid_constant__ QKParam
   const uint4* src = isq ? row + (int64_t)(2 * j) * p.dv
                          : row + (int64_t)(2 * p.Hq + (j - p.Hq)) * p.dv;
   const uint4* w = isq ? p.qw : p.kw;
-  uint4* dst = isq ? p.out_q + (m * p.Hq + j) * p.dv
-                   : p.out_k + (m * p.Hk + (j - p.Hq)) * p.dv;
+  const int64_t head = isq ? m * p.Hq + j : m * p.Hk + (j - p.Hq);  // output head index
+  uint4* dst = isq ? p.out_q : p.out_k;
+  if (dst != nullptr) dst += head * p.dv;
   const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
 
   uint4 x[VPL], wv[VPL], g[VPL];
@@ -73,17 +82,30 @@ __global__ void __launch_bounds__(256) qk_kernel(const __grid_constant__ QKParam
   const float xm = fmaf(ss, p.inv_d, p.eps);
   const float r0 = rsqrtf(xm);
   const float rstd = r0 * fmaf(-0.5f * xm * r0, r0, 1.5f);
+  uint4 y[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
-    uint4 y;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const uint32_t xw = word(x[i], c), ww = word(wv[i], c);
       const float y0 = (bf_lo(xw) * rstd) * (1.f + bf_lo(ww));
       const float y1 = (bf_hi(xw) * rstd) * (1.f + bf_hi(ww));
-      set_word(y, c, pack_bf16x2(y0, y1));
+      set_word(y[i], c, pack_bf16x2(y0, y1));
     }
-    if (lane + 32 * i < p.dv) st_stream(dst + lane + 32 * i, y);
+    if (dst != nullptr && lane + 32 * i < p.dv) st_stream(dst + lane + 32 * i, y[i]);
+  }
+  if constexpr (FP8) {
+    float am = 0.f;  // lanes past the head hold y = 0
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) am = fmaxf(am, vec_absmax(y[i]));
+    const Fp8Scale sc = fp8_scale_direct(warp_max(am));
+    uint8_t* codes = (isq ? p.out_q8 : p.out_k8) + head * (int64_t)p.dv * 8;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const uint2 q = e4m3_codes(y[i], sc);  // every lane takes part
+      if (lane + 32 * i < p.dv) st_stream(reinterpret_cast<uint2*>(codes) + lane + 32 * i, q);
+    }
+    if (lane == 0) (isq ? p.out_qs : p.out_ks)[head] = sc.s;
   }
 }
 

@@ -1,0 +1,60 @@
+// FP8 E4M3 quantization of 8-element bf16 vectors, shared by the row kernels
+// and the QK prologue: the group scale and the division-free codes.
+#pragma once
+#include "fn_device.cuh"
+
+namespace fn {
+
+// FP8 scale of a group (or row) and the reciprocal pair the codes use.
+struct Fp8Scale {
+  float s;         // RN(amax / 448), 1 for an all-zero group
+  float r, r_lo;   // RN(1/s), RN(RN(1 - s r) r)
+  bool exact_div;  // the fast quotient is not proven here: use the IEEE division
+};
+
+// The formulas themselves (IEEE division and reciprocal).
+__device__ __forceinline__ Fp8Scale fp8_scale_direct(float amax) {
+  Fp8Scale c;
+  c.s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+  c.exact_div = !(c.s >= 0x1p-120f);
+  c.r = c.exact_div ? 1.f : __frcp_rn(c.s);
+  c.r_lo = fmaf(-c.s, c.r, 1.f) * c.r;
+  return c;
+}
+
+// Eight E4M3 codes of fl32(y / s), the IEEE quotient.
+//
+// Fast path: with r = RN(1/s) and r_lo = RN(RN(1 - s r) r) (r + r_lo carries
+// 1/s to about 2^-46), q = RN(|y| r + RN(|y| r_lo)) has the same E4M3 code as
+// RN(|y| / s) for every bf16 y with |y| <= amax and every bf16 amax with
+// s = RN(amax / 448) >= 2^-120: checked exhaustively over all such (amax, y)
+// pairs by tests/quotient_proof.c.  The code is computed from |y| and y's
+// sign bit is copied onto it, which also gives -0 the code 0x80.  If any lane
+// of the warp needs the IEEE division the whole warp takes it (warp-uniform
+// branch).  All 32 lanes must call.
+__device__ __forceinline__ uint2 e4m3_codes(const uint4& y, const Fp8Scale& c) {
+  uint32_t q8[4];
+  if (!__any_sync(0xffffffffu, c.exact_div)) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t a = word(y, i) & 0x7FFF7FFFu;
+      const float2 ya = make_float2(bf_lo(a), bf_hi(a));
+      const float2 t = mul_f32x2(ya, make_float2(c.r_lo, c.r_lo));
+      const float2 q = fma_f32x2(ya, make_float2(c.r, c.r), t);
+      q8[i] = cvt_e4m3x2(q.x, q.y);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t a = word(y, i) & 0x7FFF7FFFu;
+      q8[i] = cvt_e4m3x2(__fdiv_rn(bf_lo(a), c.s), __fdiv_rn(bf_hi(a), c.s));
+    }
+  }
+  // byte k of code word j takes the sign of element 4j + k: the sign bits sit
+  // at bits 15 and 31 of each y word, i.e. in bytes 1 and 3
+  const uint32_t s0 = __byte_perm(y.x, y.y, 0x7531) & 0x80808080u;
+  const uint32_t s1 = __byte_perm(y.z, y.w, 0x7531) & 0x80808080u;
+  return make_uint2((q8[0] | (q8[1] << 16)) | s0, (q8[2] | (q8[3] << 16)) | s1);
+}
+
+}  // namespace fn

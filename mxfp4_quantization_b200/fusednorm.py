@@ -38,6 +38,7 @@ FN_VARIANT_ROW_CLUSTER = 2
 FN_VARIANT_QUANT_ONLY = 3
 FN_VARIANT_QK_WARP = 4
 FN_VARIANT_ROW_TMA = 5
+FN_VARIANT_QK_WARP_FP8 = 6
 
 FN_MODE_MASK = 0xFF
 FN_SCALE_SWIZZLE_32_4_4 = 0x100
@@ -51,7 +52,8 @@ MODES = {"fp8_per_token": FN_FP8_PER_TOKEN, "fp8_per_group128": FN_FP8_PER_GROUP
          "mxfp4": FN_MXFP4}
 
 # The exported symbols of include/fusednorm.h.
-ABI_SYMBOLS = ("fn_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate", "fn_status_string",
+ABI_SYMBOLS = ("fn_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate", "fn_qk_norm_gate_fp8",
+               "fn_status_string",
                "fn_last_variant", "fn_last_launch", "fn_prefer_variant", "fn_device_status",
                "fn_debug_stall_copies", "fn_version")
 
@@ -76,6 +78,9 @@ def _load():
     lib.fn_qk_norm_gate.argtypes = [vp, i64, i64, i32, i32, i32, vp, vp, ctypes.c_float, vp, vp,
                                     vp, vp]
     lib.fn_qk_norm_gate.restype = i32
+    lib.fn_qk_norm_gate_fp8.argtypes = [vp, i64, i64, i32, i32, i32, vp, vp, ctypes.c_float, vp,
+                                        vp, vp, vp, vp, vp, vp, vp]
+    lib.fn_qk_norm_gate_fp8.restype = i32
     lib.fn_status_string.argtypes = [i32]
     lib.fn_status_string.restype = ctypes.c_char_p
     lib.fn_last_variant.argtypes = []
@@ -119,6 +124,17 @@ def fn_qk_norm_gate(qkv: int, M: int, row_stride: int, Hq: int, Hk: int, D: int,
                     stream: Optional[int]) -> int:
     return _lib.fn_qk_norm_gate(qkv, M, row_stride, Hq, Hk, D, q_weight, k_weight, eps, out_q,
                                 out_k, out_gate, stream)
+
+
+def fn_qk_norm_gate_fp8(qkv: int, M: int, row_stride: int, Hq: int, Hk: int, D: int,
+                        q_weight: Optional[int], k_weight: Optional[int], eps: float,
+                        out_q8: Optional[int], out_q_scale: Optional[int], out_k8: Optional[int],
+                        out_k_scale: Optional[int], out_gate: Optional[int],
+                        out_q: Optional[int], out_k: Optional[int],
+                        stream: Optional[int]) -> int:
+    return _lib.fn_qk_norm_gate_fp8(qkv, M, row_stride, Hq, Hk, D, q_weight, k_weight, eps,
+                                    out_q8, out_q_scale, out_k8, out_k_scale, out_gate, out_q,
+                                    out_k, stream)
 
 
 def fn_status_string(status: int) -> str:
@@ -175,6 +191,7 @@ def device_status() -> int:
 
 RMSNormQuantOutput = namedtuple("RMSNormQuantOutput", "q scale residual_out y")
 QKOutput = namedtuple("QKOutput", "q k gate")
+QKFp8Output = namedtuple("QKFp8Output", "q8 q_scale k8 k_scale gate q k")
 
 
 def _mode(mode: Union[int, str]) -> int:
@@ -325,4 +342,36 @@ def qk_norm_gate(qkv: torch.Tensor, Hq: int, Hk: int, D: int, q_weight: torch.Te
                          out.gate.data_ptr(), _stream(dev))
     if st != FN_OK:
         raise FusedNormError("fn_qk_norm_gate", st)
+    return out
+
+
+def qk_norm_gate_fp8(qkv: torch.Tensor, Hq: int, Hk: int, D: int, q_weight: torch.Tensor,
+                     k_weight: torch.Tensor, eps: float, *, emit_bf16: bool = False) -> QKFp8Output:
+    """qk_norm_gate with E4M3 q and k (one fp32 scale per token and head);
+    returns (q8 [M,Hq,D] float8_e4m3fn, q_scale [M,Hq], k8, k_scale, gate [M,Hq,D]
+    bf16, q, k) where q and k are the bf16 normed heads if `emit_bf16`."""
+    if not qkv.is_cuda or qkv.dtype != torch.bfloat16:
+        raise TypeError("qkv must be a bf16 CUDA tensor")
+    if qkv.dim() != 2 or qkv.stride(1) != 1:
+        raise ValueError("qkv must be [M, row] with a contiguous last dim")
+    M, row_stride = qkv.shape[0], qkv.stride(0)
+    if qkv.shape[1] < (2 * Hq + Hk) * D:
+        raise ValueError("qkv rows are too short for the heads")
+    qw = _rows(q_weight, "q_weight", D)
+    kw = _rows(k_weight, "k_weight", D)
+    dev = qkv.device
+    f8, f32, bf = torch.float8_e4m3fn, torch.float32, torch.bfloat16
+    out = QKFp8Output(torch.empty((M, Hq, D), dtype=f8, device=dev),
+                      torch.empty((M, Hq), dtype=f32, device=dev),
+                      torch.empty((M, Hk, D), dtype=f8, device=dev),
+                      torch.empty((M, Hk), dtype=f32, device=dev),
+                      torch.empty((M, Hq, D), dtype=bf, device=dev),
+                      torch.empty((M, Hq, D), dtype=bf, device=dev) if emit_bf16 else None,
+                      torch.empty((M, Hk, D), dtype=bf, device=dev) if emit_bf16 else None)
+    st = fn_qk_norm_gate_fp8(qkv.data_ptr(), M, row_stride, Hq, Hk, D, qw.data_ptr(),
+                             kw.data_ptr(), float(eps), out.q8.data_ptr(), out.q_scale.data_ptr(),
+                             out.k8.data_ptr(), out.k_scale.data_ptr(), out.gate.data_ptr(),
+                             _ptr(out.q), _ptr(out.k), _stream(dev))
+    if st != FN_OK:
+        raise FusedNormError("fn_qk_norm_gate_fp8", st)
     return out

@@ -14,5 +14,5 @@ from .oracle import (  # noqa: F401
     FP8_PER_TOKEN, FP8_PER_GROUP128, MXFP4, OracleError, load, bf16_from_double,
     bf16_to_double, e4m3_encode, e4m3_decode, e2m1_encode, e2m1_decode,
     mx_scale_code, rstd, quant_rows, rmsnorm_quant, qk_norm_gate, scale_shape,
-    code_shape, place_scales, SCALE_SWIZZLE_32_4_4, SCALE_MN_MAJOR,
+    code_shape, place_scales, qk_norm_gate_fp8, SCALE_SWIZZLE_32_4_4, SCALE_MN_MAJOR,
 )

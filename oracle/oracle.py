@@ -54,6 +54,12 @@ def load(path: str = LIB):
                                      ctypes.c_int, ctypes.c_int, _u16p, _u16p,
                                      ctypes.c_float, _u16p, _u16p, _u16p]
     lib.orc_qk_norm_gate.restype = ctypes.c_int
+    _f32p = ctypes.POINTER(ctypes.c_float)
+    lib.orc_qk_norm_gate_fp8.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, _u16p, _u16p,
+                                         ctypes.c_float, _u8p, _f32p, _u8p, _f32p, _u16p,
+                                         _u16p, _u16p]
+    lib.orc_qk_norm_gate_fp8.restype = ctypes.c_int
     if path == LIB:
         _lib = lib
     return lib
@@ -185,6 +191,27 @@ def qk_norm_gate(qkv, row_stride: int, Hq: int, Hk: int, D: int, q_weight, k_wei
     if rc != 0:
         raise OracleError("orc_qk_norm_gate rejected the shape")
     return {"q": q, "k": k, "gate": g}
+
+
+def qk_norm_gate_fp8(qkv, row_stride: int, Hq: int, Hk: int, D: int, q_weight, k_weight,
+                     eps: float, lib=None):
+    """Returns dict(q8, qs, k8, ks, gate, q, k) (see orc_qk_norm_gate_fp8)."""
+    lib = lib or load()
+    x = _u16(qkv)
+    M = x.shape[0]
+    f32p = ctypes.POINTER(ctypes.c_float)
+    out = {"q8": np.zeros((M, Hq, D), np.uint8), "qs": np.zeros((M, Hq), np.float32),
+           "k8": np.zeros((M, Hk, D), np.uint8), "ks": np.zeros((M, Hk), np.float32),
+           "gate": np.zeros((M, Hq, D), np.uint16), "q": np.zeros((M, Hq, D), np.uint16),
+           "k": np.zeros((M, Hk, D), np.uint16)}
+    rc = lib.orc_qk_norm_gate_fp8(_p16(x), M, row_stride, Hq, Hk, D, _p16(_u16(q_weight)),
+                                  _p16(_u16(k_weight)), eps, _p8(out["q8"]),
+                                  out["qs"].ctypes.data_as(f32p), _p8(out["k8"]),
+                                  out["ks"].ctypes.data_as(f32p), _p16(out["gate"]),
+                                  _p16(out["q"]), _p16(out["k"]))
+    if rc != 0:
+        raise OracleError("orc_qk_norm_gate_fp8 rejected the shape")
+    return out
 
 
 # ---- scale layouts ------------------------------------------------------------

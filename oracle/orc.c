@@ -411,3 +411,42 @@ int orc_qk_norm_gate(const uint16_t* qkv, int64_t M, int64_t row_stride, int Hq,
     }
     return ORC_OK;
 }
+
+/*
+ * The QK prologue with E4M3 q and k for an FP8 attention consumer (reading:
+ * the per-token FP8 rule of [AR] applied to each normed head vector of D
+ * values — scale = fl32(amax / 448), code = e4m3(fl32(y / scale)), scale 1
+ * for an all-zero head).  q8 [M,Hq,D] with scales qs [M,Hq]; k8 [M,Hk,D]
+ * with ks [M,Hk]; gate as orc_qk_norm_gate.  out_q / out_k may be NULL.
+ */
+int orc_qk_norm_gate_fp8(const uint16_t* qkv, int64_t M, int64_t row_stride, int Hq, int Hk,
+                         int D, const uint16_t* q_weight, const uint16_t* k_weight, float eps,
+                         uint8_t* q8, float* qs, uint8_t* k8, float* ks, uint16_t* out_gate,
+                         uint16_t* out_q, uint16_t* out_k)
+{
+    if (M < 0 || Hq < 0 || Hk < 0 || D <= 0 || row_stride < (int64_t)(2 * Hq + Hk) * D)
+        return ORC_BAD;
+    uint16_t* y = (uint16_t*)malloc((size_t)D * sizeof(uint16_t));
+    if (!y)
+        return ORC_BAD;
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t* row = qkv + m * row_stride;
+        for (int h = 0; h < Hq; ++h) {
+            const int64_t o = m * Hq + h;
+            gemma_norm_head(row + (int64_t)2 * h * D, q_weight, D, eps, y);
+            quant_fp8_group(y, D, q8 + o * D, qs + o);
+            if (out_q)
+                memcpy(out_q + o * D, y, (size_t)D * sizeof(uint16_t));
+            memcpy(out_gate + o * D, row + (int64_t)(2 * h + 1) * D, (size_t)D * sizeof(uint16_t));
+        }
+        for (int h = 0; h < Hk; ++h) {
+            const int64_t o = m * Hk + h;
+            gemma_norm_head(row + (int64_t)2 * Hq * D + (int64_t)h * D, k_weight, D, eps, y);
+            quant_fp8_group(y, D, k8 + o * D, ks + o);
+            if (out_k)
+                memcpy(out_k + o * D, y, (size_t)D * sizeof(uint16_t));
+        }
+    }
+    free(y);
+    return ORC_OK;
+}

@@ -498,3 +498,30 @@ def pin_scale_layouts(lib):
 
 
 ALL_PINS.append(pin_scale_layouts)
+
+
+def pin_qk_fp8(lib):
+    """The FP8 QK prologue is the bf16 prologue followed by the per-token FP8
+    quantization of each head vector (two pinned pieces composed), and its
+    gate is the same bit copy."""
+    M, Hq, Hk, D = 3, 4, 2, 64
+    stride = (2 * Hq + 2 * Hk) * D
+    g = torch.Generator().manual_seed(8)
+    x = bf16_bits_from_torch((torch.randn((M, stride), generator=g) *
+                              torch.pow(10.0, torch.rand((M, 1), generator=g) * 4 - 2)).to(torch.bfloat16))
+    x[1, 2 * D:3 * D] = 0  # an all-zero q head: scale 1, codes 0
+    qw = bf16_bits_from_torch((0.1 * torch.randn((D,), generator=g)).to(torch.bfloat16))
+    kw = bf16_bits_from_torch((0.1 * torch.randn((D,), generator=g)).to(torch.bfloat16))
+    base = oracle.qk_norm_gate(x, stride, Hq, Hk, D, qw, kw, 1e-6, lib)
+    f8 = oracle.qk_norm_gate_fp8(x, stride, Hq, Hk, D, qw, kw, 1e-6, lib)
+    for name, H in (("q", Hq), ("k", Hk)):
+        y = base[name].reshape(M * H, D)
+        assert np.array_equal(f8[name].reshape(M * H, D), y)
+        rq, rs = oracle.quant_rows(y, oracle.FP8_PER_TOKEN, lib)
+        assert np.array_equal(f8[name + "8"].reshape(M * H, D), rq), f"{name} codes"
+        assert np.array_equal(f8[name + "s"].reshape(-1), rs), f"{name} scales"
+    assert np.array_equal(f8["gate"], base["gate"])
+    assert f8["qs"][1, 1] == 1.0 and np.all(f8["q8"][1, 1] == 0)
+
+
+ALL_PINS.append(pin_qk_fp8)

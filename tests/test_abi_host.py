@@ -28,6 +28,7 @@ def declared_symbols():
 
 def test_header_declares_the_abi():
     assert declared_symbols() == sorted(["fn_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate",
+                                         "fn_qk_norm_gate_fp8",
                                          "fn_status_string", "fn_last_variant",
                                          "fn_last_launch", "fn_prefer_variant",
                                          "fn_device_status", "fn_debug_stall_copies",
@@ -50,7 +51,7 @@ def test_header_constants_match_binding(fnb):
     for name in ("FN_FP8_PER_TOKEN", "FN_FP8_PER_GROUP128", "FN_MXFP4", "FN_ERR_INVALID",
                  "FN_ERR_ALIGN", "FN_ERR_UNSUPPORTED", "FN_ERR_CUDA", "FN_VARIANT_ROW_CTA",
                  "FN_VARIANT_ROW_CLUSTER", "FN_VARIANT_QUANT_ONLY", "FN_VARIANT_QK_WARP",
-                 "FN_VARIANT_ROW_TMA", "FN_ERR_TIMEOUT"):
+                 "FN_VARIANT_ROW_TMA", "FN_VARIANT_QK_WARP_FP8", "FN_ERR_TIMEOUT"):
         m = re.search(rf"\b{name}\s*=\s*(-?\d+)", src)
         assert m and int(m.group(1)) == getattr(fnb, name), name
     for name in ("FN_MAX_PARTS", "FN_MAX_H", "FN_MAX_HEAD_DIM"):
@@ -170,3 +171,20 @@ def test_scale_layout_flags(fnb):
     assert rq(fnb, mode=fnb.FN_MXFP4 | SW, out_q=BASE + (4 << 32) + 512) == E
     assert fnb.fn_quant(BASE, fnb.FN_FP8_PER_TOKEN | MN, 4, 256, BASE + (1 << 32),
                         BASE + (2 << 32), None) == E
+
+
+def test_qk_fp8_rejects_bad_arguments(fnb):
+    def q8(**kw):
+        a = dict(qkv=BASE, M=4, row_stride=18432, Hq=32, Hk=4, D=256, qw=BASE + (1 << 32),
+                 kw=BASE + (2 << 32), eps=1e-6, q8=BASE + (3 << 32), qs=BASE + (4 << 32),
+                 k8=BASE + (5 << 32), ks=BASE + (6 << 32), g=BASE + (7 << 32), q=None, k=None)
+        a.update(kw)
+        return fnb.fn_qk_norm_gate_fp8(a["qkv"], a["M"], a["row_stride"], a["Hq"], a["Hk"],
+                                       a["D"], a["qw"], a["kw"], a["eps"], a["q8"], a["qs"],
+                                       a["k8"], a["ks"], a["g"], a["q"], a["k"], None)
+    E, A = fnb.FN_ERR_INVALID, fnb.FN_ERR_ALIGN
+    assert q8(M=0) == fnb.FN_OK
+    assert q8(q8=None) == E and q8(ks=None) == E and q8(g=None) == E
+    assert q8(q8=BASE + (3 << 32) + 4) == A and q8(qs=BASE + (4 << 32) + 2) == A
+    assert q8(qs=BASE + (3 << 32) + 64) == E          # scales inside the q codes
+    assert q8(k8=BASE + 100 * 2 * 256) == E           # codes inside qkv
