@@ -91,6 +91,18 @@ RQKernel pick_kernel(int mode, int P, int V, bool cluster, bool norm) {
   return nullptr;
 }
 
+// The exact-cover instance for a row of T * V vectors, or nullptr.
+RQKernel pick_exact_kernel(int mode, int P, int T, int V) {
+  const int maxp = P == 1 ? 1 : P == 2 ? 2 : P <= 4 ? 4 : 8;
+#define FN_CASE(MODE, MAXP) \
+  if (mode == MODE && maxp == MAXP) return fn::rq_exact_pick_##MODE##_##MAXP(T, V);
+  FN_CASE(0, 1) FN_CASE(0, 2) FN_CASE(0, 4) FN_CASE(0, 8)
+  FN_CASE(1, 1) FN_CASE(1, 2) FN_CASE(1, 4) FN_CASE(1, 8)
+  FN_CASE(2, 1) FN_CASE(2, 2) FN_CASE(2, 4) FN_CASE(2, 8)
+#undef FN_CASE
+  return nullptr;
+}
+
 using fn::RQTmaKernel;
 
 RQTmaKernel pick_tma_kernel(int mode, int P, int V) {
@@ -291,7 +303,8 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, vo
     p.seg = nvec;
     p.prefetch_rows = M > (int64_t)kRowPrefetchSms * sms ? kRowPrefetchSms * sms : 0;
     const int threads = round32((nvec + V - 1) / V);
-    RQKernel k = pick_kernel(mode, P, V, false, norm);
+    RQKernel k = norm && threads * V == nvec ? pick_exact_kernel(mode, P, threads, V) : nullptr;
+    if (!k) k = pick_kernel(mode, P, V, false, norm);
     if (!k) return FN_ERR_UNSUPPORTED;
     k<<<(unsigned)M, threads, 0, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return FN_ERR_CUDA;

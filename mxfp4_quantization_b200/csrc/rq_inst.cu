@@ -42,6 +42,18 @@ RQKernel FN_CAT(rq_pick, FN_INST_MODE, FN_INST_MAXP)(int V, bool cluster, bool n
   }
 }
 
+// Exact-cover instances (one block of T threads per row of T * V vectors):
+// T = 224 serves H = 3584, 7168, 14336; T = 256 serves H = 4096, 8192, 16384.
+RQKernel FN_CAT(rq_exact_pick, FN_INST_MODE, FN_INST_MAXP)(int T, int V) {
+  constexpr int MODE = FN_INST_MODE, MAXP = FN_INST_MAXP;
+#define FN_EXACT(TT, VV) \
+  if (T == TT && V == VV) return rq_kernel<MODE, MAXP, VV, true, false, TT>;
+  FN_EXACT(224, 2) FN_EXACT(224, 4) FN_EXACT(224, 8)
+  FN_EXACT(256, 2) FN_EXACT(256, 4) FN_EXACT(256, 8)
+#undef FN_EXACT
+  return nullptr;
+}
+
 RQTmaKernel FN_CAT(rq_tma_pick, FN_INST_MODE, FN_INST_MAXP)(int V) {
   constexpr int MODE = FN_INST_MODE, MAXP = FN_INST_MAXP;
   switch (V) {

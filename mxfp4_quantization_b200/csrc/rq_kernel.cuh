@@ -229,13 +229,19 @@ __device__ __forceinline__ float row_amax_from_pmax(float pmax, float rstd) {
 // register-resident kernel: one row per block (CL = false) or per cluster
 // ---------------------------------------------------------------------------
 
-template <int MODE, int MAXP, int V, bool NORM, bool CL>
+// TB > 0 marks an exact-cover instance: the block has TB threads and the row
+// is exactly TB * V vectors (H = 8 * TB * V), so every offset is a
+// compile-time constant and no access needs a bounds test.  TB = 0 reads the
+// block size and the row length at run time.
+template <int MODE, int MAXP, int V, bool NORM, bool CL, int TB = 0>
 __global__ void __launch_bounds__(CL ? 512 : 256)
     rq_kernel(const __grid_constant__ RQParams prm) {
+  static_assert(TB == 0 || (!CL && NORM), "exact-cover instances are one block per row");
   __shared__ float2 red[32];
   __shared__ float2 cl_slot;
 
-  const int T = blockDim.x, t = threadIdx.x, lane = t & 31;
+  const int T = TB ? TB : (int)blockDim.x, t = threadIdx.x, lane = t & 31;
+  const int nvec = TB ? TB * V : prm.nvec;
   int64_t row;
   int rank = 0;
   if constexpr (CL) {
@@ -245,17 +251,17 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
   } else {
     row = blockIdx.x;
   }
-  const int seg_base = rank * prm.seg, seg_end = seg_base + prm.seg;
-  const int64_t rowv = row * (int64_t)prm.nvec;
-  const int H = prm.nvec * 8;
+  const int seg_base = TB ? 0 : rank * prm.seg, seg_end = TB ? nvec : seg_base + prm.seg;
+  const int64_t rowv = row * (int64_t)nvec;
+  const int H = nvec * 8;
   const bool has_res = NORM && prm.residual != nullptr;
   const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
 
   // The block `prefetch_rows` rows later in launch order will most likely run
   // next on this SM's slot: start its row towards L2 now.
   if (!CL && prm.prefetch_rows > 0 && t == 0 && row + prm.prefetch_rows < prm.M) {
-    const int64_t prow = (row + prm.prefetch_rows) * (int64_t)prm.nvec;
-    const uint32_t bytes = (uint32_t)prm.nvec * 16u;
+    const int64_t prow = (row + prm.prefetch_rows) * (int64_t)nvec;
+    const uint32_t bytes = (uint32_t)nvec * 16u;
     for (int p = 0; p < prm.P; ++p) bulk_prefetch_l2(prm.parts[p] + prow, bytes);
     if (prm.residual != nullptr) bulk_prefetch_l2(prm.residual + prow, bytes);
   }
@@ -267,7 +273,7 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
 #pragma unroll
   for (int k = 0; k < V; ++k) {
     const int v = seg_base + t + k * T;
-    const bool ok = v < seg_end;
+    const bool ok = TB || v < seg_end;
 #pragma unroll
     for (int p = 0; p < MAXP; ++p)
       xin[k][p] = (ok && p < prm.P) ? ld_stream_nc(prm.parts[p] + rowv + v) : zero;
@@ -289,7 +295,8 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
       hv[k] = sum_vec<MAXP>(xin[k], rin[k], prm.P, has_res);
       stats_vec<MODE == MODE_TOKEN>(hv[k], win[k], ss, pmax);
       const int v = seg_base + t + k * T;
-      if (v < seg_end && prm.out_residual != nullptr) st_stream(prm.out_residual + rowv + v, hv[k]);
+      if ((TB || v < seg_end) && prm.out_residual != nullptr)
+        st_stream(prm.out_residual + rowv + v, hv[k]);
     }
     // ---- 3. rstd (and the per-token amax) ---------------------------------------------
     const float2 tot = row_reduce<CL, MODE == MODE_TOKEN>(ss.x + ss.y, pmax, red, &cl_slot);
@@ -300,7 +307,7 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
     for (int k = 0; k < V; ++k) {
       yv[k] = norm_vec(hv[k], win[k], rstd);
       const int v = seg_base + t + k * T;
-      if (v < seg_end && prm.out_y != nullptr) st_stream(prm.out_y + rowv + v, yv[k]);
+      if ((TB || v < seg_end) && prm.out_y != nullptr) st_stream(prm.out_y + rowv + v, yv[k]);
     }
   } else {
 #pragma unroll
@@ -319,7 +326,7 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
 #pragma unroll
   for (int k = 0; k < V; ++k) {
     const int v = seg_base + t + k * T;
-    quant_store<MODE>(yv[k], v < seg_end, lane, row, v, H, scale_tok, prm.out_q, prm.out_scale,
+    quant_store<MODE>(yv[k], TB || v < seg_end, lane, row, v, H, scale_tok, prm.out_q, prm.out_scale,
                       prm.scale_layout, prm.scale_ld);
   }
 

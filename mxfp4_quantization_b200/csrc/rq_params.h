@@ -44,6 +44,7 @@ using RQTmaKernel = void (*)(const RQParams, int, int);
 
 #define FN_RQ_DECL(MODE, MAXP)                                          \
   RQKernel rq_pick_##MODE##_##MAXP(int V, bool cluster, bool norm); \
+  RQKernel rq_exact_pick_##MODE##_##MAXP(int T, int V);             \
   RQTmaKernel rq_tma_pick_##MODE##_##MAXP(int V);
 FN_RQ_DECL(0, 1)
 FN_RQ_DECL(0, 2)

@@ -63,6 +63,7 @@ SHAPES = [
     (17, 7168, 4, True), (19, 7168, 1, True), (37, 8192, 1, True), (150, 7168, 4, True),
     (64, 4096, 3, False), (33, 1024, 8, True), (7, 32768, 1, True), (200, 2176, 5, True),
     (3, 128, 1, True), (75, 1152, 6, False), (40, 16384, 2, True), (300, 256, 7, True),
+    (45, 3584, 8, True), (9, 14336, 3, False), (21, 6144, 2, True),
     # many rows per block: the persistent kernels wrap their stage ring many times
     (1500, 7168, 4, True), (2400, 1024, 3, True),
 ]
