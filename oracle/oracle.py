@@ -10,6 +10,10 @@ FP8_PER_TOKEN = 0
 FP8_PER_GROUP128 = 1
 MXFP4 = 2
 
+# storage format of the 16-bit tensors
+IO_BF16 = 0
+IO_FP16 = 1
+
 _lib = None
 
 _u16p = ctypes.POINTER(ctypes.c_uint16)
@@ -31,6 +35,10 @@ def load(path: str = LIB):
     lib.orc_bf16_to_double.restype = ctypes.c_double
     lib.orc_bf16_from_double.argtypes = [ctypes.c_double]
     lib.orc_bf16_from_double.restype = ctypes.c_uint16
+    lib.orc_fp16_to_double.argtypes = [ctypes.c_uint16]
+    lib.orc_fp16_to_double.restype = ctypes.c_double
+    lib.orc_fp16_from_double.argtypes = [ctypes.c_double]
+    lib.orc_fp16_from_double.restype = ctypes.c_uint16
     lib.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
     lib.orc_e4m3_decode.restype = ctypes.c_double
     lib.orc_e4m3_encode.argtypes = [ctypes.c_double]
@@ -41,14 +49,15 @@ def load(path: str = LIB):
     lib.orc_e2m1_encode.restype = ctypes.c_uint8
     lib.orc_mx_scale_code.argtypes = [ctypes.c_double]
     lib.orc_mx_scale_code.restype = ctypes.c_uint8
-    lib.orc_rstd.argtypes = [_u16p, ctypes.c_int64, ctypes.c_float]
+    lib.orc_rstd.argtypes = [_u16p, ctypes.c_int64, ctypes.c_float, ctypes.c_int]
     lib.orc_rstd.restype = ctypes.c_double
     lib.orc_quant_rows.argtypes = [_u16p, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
-                                   _u8p, ctypes.c_void_p]
+                                   _u8p, ctypes.c_void_p, ctypes.c_int]
     lib.orc_quant_rows.restype = ctypes.c_int
     lib.orc_rmsnorm_quant.argtypes = [ctypes.POINTER(_u16p), ctypes.c_int, _u16p, _u16p,
                                       ctypes.c_float, ctypes.c_int, ctypes.c_int64,
-                                      ctypes.c_int64, _u8p, ctypes.c_void_p, _u16p, _u16p]
+                                      ctypes.c_int64, _u8p, ctypes.c_void_p, _u16p, _u16p,
+                                      ctypes.c_int]
     lib.orc_rmsnorm_quant.restype = ctypes.c_int
     lib.orc_qk_norm_gate.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                                      ctypes.c_int, ctypes.c_int, _u16p, _u16p,
@@ -105,6 +114,17 @@ def bf16_from_double(v, lib=None):
                     dtype=np.uint16).reshape(np.shape(v))
 
 
+def fp16_to_double(bits, lib=None):
+    lib = lib or load()
+    return np.array([lib.orc_fp16_to_double(int(b)) for b in np.ravel(bits)]).reshape(np.shape(bits))
+
+
+def fp16_from_double(v, lib=None):
+    lib = lib or load()
+    return np.array([lib.orc_fp16_from_double(float(x)) for x in np.ravel(v)],
+                    dtype=np.uint16).reshape(np.shape(v))
+
+
 def e4m3_encode(v, lib=None):
     lib = lib or load()
     return np.array([lib.orc_e4m3_encode(float(x)) for x in np.ravel(v)],
@@ -135,30 +155,33 @@ def mx_scale_code(amax, lib=None):
 
 # ---- row operations ---------------------------------------------------------
 
-def rstd(h_bits, eps: float, lib=None) -> float:
+def rstd(h_bits, eps: float, lib=None, io: int = IO_BF16) -> float:
     lib = lib or load()
     h = _u16(h_bits)
-    return lib.orc_rstd(_p16(h), h.size, eps)
+    return lib.orc_rstd(_p16(h), h.size, eps, io)
 
 
-def quant_rows(y_bits, mode: int, lib=None):
-    """Quantize bf16 rows [M, H]; returns (codes, scales)."""
+def quant_rows(y_bits, mode: int, lib=None, io: int = IO_BF16):
+    """Quantize 16-bit rows [M, H] (bf16, or binary16 with io=IO_FP16);
+    returns (codes, scales)."""
     lib = lib or load()
     y = _u16(y_bits)
     M, H = y.shape
     q = np.zeros(code_shape(mode, M, H), dtype=np.uint8)
     s = np.zeros(scale_shape(mode, M, H), dtype=_scale_dtype(mode))
-    rc = lib.orc_quant_rows(_p16(y), mode, M, H, _p8(q), s.ctypes.data_as(ctypes.c_void_p))
+    rc = lib.orc_quant_rows(_p16(y), mode, M, H, _p8(q), s.ctypes.data_as(ctypes.c_void_p), io)
     if rc != 0:
         raise OracleError(f"orc_quant_rows rejected mode={mode} H={H}")
     return q, s
 
 
-def rmsnorm_quant(parts, residual, weight, eps: float, mode: int, lib=None):
+def rmsnorm_quant(parts, residual, weight, eps: float, mode: int, lib=None,
+                  io: int = IO_BF16):
     """Unfused reference sequence over [M, H] rows.
 
     parts: list of P uint16 [M, H] arrays; residual: uint16 [M, H] or None;
-    weight: uint16 [H].  Returns dict(q, scale, residual_out, y).
+    weight: uint16 [H]; all bf16 bit patterns, or binary16 with io=IO_FP16.
+    Returns dict(q, scale, residual_out, y).
     """
     lib = lib or load()
     parts = [_u16(p) for p in parts]
@@ -171,7 +194,7 @@ def rmsnorm_quant(parts, residual, weight, eps: float, mode: int, lib=None):
     r_out = np.zeros((M, H), dtype=np.uint16)
     y = np.zeros((M, H), dtype=np.uint16)
     rc = lib.orc_rmsnorm_quant(arr, len(parts), _p16(res), _p16(w), eps, mode, M, H, _p8(q),
-                               s.ctypes.data_as(ctypes.c_void_p), _p16(r_out), _p16(y))
+                               s.ctypes.data_as(ctypes.c_void_p), _p16(r_out), _p16(y), io)
     if rc != 0:
         raise OracleError(f"orc_rmsnorm_quant rejected P={len(parts)} mode={mode} H={H}")
     return {"q": q, "scale": s, "residual_out": r_out, "y": y}

@@ -42,6 +42,13 @@
  *  A8  all-zero MX block: scale code 0 (2^-127), codes 0.
  *  A9  element 2i in the low nibble of byte i; scales row-major.
  *  A11 a NaN or infinite MX block amax gives scale code 0xFF.
+ *  A17 fp16 input/output ([AR] review: the producer's activation dtype is
+ *      carried through the quantized tuple, FP16 beside BF16): with
+ *      io = ORC_IO_FP16 every 16-bit tensor (partials, residual, weight,
+ *      residual_out, y, the rows given to orc_quant_rows) is IEEE binary16
+ *      instead of bf16, and every "bf16(...)" rounding above is a binary16
+ *      rounding (nearest even, subnormals kept, overflow to infinity).
+ *      Codes and scales are unchanged.
  *
  * Build: plain C99, -O2 -ffp-contract=off, no fast-math, x86-64 SSE float
  * arithmetic (FLT_EVAL_METHOD == 0), so `float` operations are IEEE binary32
@@ -65,6 +72,10 @@
 #define ORC_OK 0
 #define ORC_BAD -1
 
+/* Storage format of the 16-bit tensors (A17). */
+#define ORC_IO_BF16 0
+#define ORC_IO_FP16 1
+
 /* ------------------------------------------------------------------ */
 /* Number formats                                                       */
 /* ------------------------------------------------------------------ */
@@ -76,14 +87,6 @@ double orc_bf16_to_double(uint16_t b)
     float f;
     memcpy(&f, &u, sizeof f);
     return (double)f;
-}
-
-static float bf16_to_float(uint16_t b)
-{
-    uint32_t u = (uint32_t)b << 16;
-    float f;
-    memcpy(&f, &u, sizeof f);
-    return f;
 }
 
 /*
@@ -122,6 +125,61 @@ uint16_t orc_bf16_from_double(double v)
     uint32_t u;
     memcpy(&u, &f, sizeof u);
     return (uint16_t)(u >> 16);
+}
+
+/* IEEE binary16: 1 sign, 5 exponent (bias 15), 10 mantissa bits; exponent
+ * field 0 holds zero and the subnormals m 2^-24; field 31 holds infinity
+ * (m == 0) and NaN. */
+double orc_fp16_to_double(uint16_t b)
+{
+    int s = b >> 15, e = (b >> 10) & 0x1F, m = b & 0x3FF;
+    double mag;
+    if (e == 31)
+        mag = m ? NAN : INFINITY;
+    else if (e == 0)
+        mag = ldexp((double)m, -24);
+    else
+        mag = ldexp(1024.0 + m, e - 25);
+    return s ? -mag : mag;
+}
+
+/* IEEE round-to-nearest-even of a double to binary16 (11 significant bits,
+ * emin -14, subnormals kept); magnitudes that round beyond the largest
+ * finite value 65504 become infinity. */
+uint16_t orc_fp16_from_double(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000 : 0x0000;
+    if (isnan(v))
+        return (uint16_t)(sign | 0x7E00u);
+    double r = fabs(round_to_grid(v, 10, -14));
+    if (r >= 65536.0)
+        return (uint16_t)(sign | 0x7C00u);
+    if (r == 0.0)
+        return sign;
+    int e2;
+    (void)frexp(r, &e2);
+    int ex = e2 - 1;
+    if (ex < -14) /* subnormal: r = m 2^-24 */
+        return (uint16_t)(sign | (uint16_t)(r / 0x1p-24));
+    int m = (int)((r / ldexp(1.0, ex) - 1.0) * 1024.0);
+    return (uint16_t)(sign | ((ex + 15) << 10) | m);
+}
+
+/* The value of a stored 16-bit element, and the rounding of a value to the
+ * storage format. */
+static double elem_to_double(int io, uint16_t b)
+{
+    return io == ORC_IO_FP16 ? orc_fp16_to_double(b) : orc_bf16_to_double(b);
+}
+
+static float elem_to_float(int io, uint16_t b)
+{
+    return (float)elem_to_double(io, b); /* exact: both formats fit binary32 */
+}
+
+static uint16_t elem_from_double(int io, double v)
+{
+    return io == ORC_IO_FP16 ? orc_fp16_from_double(v) : orc_bf16_from_double(v);
 }
 
 /* OCP E4M3 "fn": 1 sign, 4 exponent (bias 7), 3 mantissa bits; no infinity;
@@ -213,18 +271,18 @@ uint8_t orc_mx_scale_code(double amax)
 /* quantization of the bf16 row, [OCP])                                 */
 /* ------------------------------------------------------------------ */
 
-/* FP8 E4M3 of one group of n bf16 values with one fp32 scale (A5-A7). */
-static void quant_fp8_group(const uint16_t* y, int64_t n, uint8_t* q, float* scale_out)
+/* FP8 E4M3 of one group of n 16-bit values with one fp32 scale (A5-A7). */
+static void quant_fp8_group(const uint16_t* y, int64_t n, uint8_t* q, float* scale_out, int io)
 {
     float amax = 0.0f;
     for (int64_t j = 0; j < n; ++j) {
-        float a = fabsf(bf16_to_float(y[j]));
+        float a = fabsf(elem_to_float(io, y[j]));
         if (a > amax)
             amax = a;
     }
     float scale = (amax == 0.0f) ? 1.0f : amax / 448.0f; /* one binary32 division */
     for (int64_t j = 0; j < n; ++j) {
-        float t = bf16_to_float(y[j]) / scale;            /* one binary32 division */
+        float t = elem_to_float(io, y[j]) / scale;        /* one binary32 division */
         q[j] = orc_e4m3_encode((double)t);
     }
     *scale_out = scale;
@@ -232,12 +290,12 @@ static void quant_fp8_group(const uint16_t* y, int64_t n, uint8_t* q, float* sca
 
 /* MXFP4 of one 32-element block: E8M0 scale code, then E2M1 codes of
  * y_j * 2^-e, packed two per byte, element 2i in the low nibble (A9). */
-static void quant_mx_block(const uint16_t* y, uint8_t* packed, uint8_t* scale_code)
+static void quant_mx_block(const uint16_t* y, uint8_t* packed, uint8_t* scale_code, int io)
 {
     double amax = 0.0;
     int any_nan = 0;
     for (int j = 0; j < 32; ++j) {
-        double a = fabs(orc_bf16_to_double(y[j]));
+        double a = fabs(elem_to_double(io, y[j]));
         if (isnan(a))
             any_nan = 1;
         else if (a > amax)
@@ -248,8 +306,8 @@ static void quant_mx_block(const uint16_t* y, uint8_t* packed, uint8_t* scale_co
     uint8_t sc = orc_mx_scale_code(amax);
     int e = (int)sc - 127;
     for (int i = 0; i < 16; ++i) {
-        double v0 = ldexp(orc_bf16_to_double(y[2 * i]), -e);     /* exact */
-        double v1 = ldexp(orc_bf16_to_double(y[2 * i + 1]), -e); /* exact */
+        double v0 = ldexp(elem_to_double(io, y[2 * i]), -e);     /* exact */
+        double v1 = ldexp(elem_to_double(io, y[2 * i + 1]), -e); /* exact */
         uint8_t c0 = orc_e2m1_encode(v0), c1 = orc_e2m1_encode(v1);
         packed[i] = (uint8_t)(c0 | (c1 << 4));
     }
@@ -257,32 +315,32 @@ static void quant_mx_block(const uint16_t* y, uint8_t* packed, uint8_t* scale_co
 }
 
 /*
- * Quantize M bf16 rows of length H.
+ * Quantize M rows of length H (bf16, or binary16 with io = ORC_IO_FP16).
  *   mode 0: out_q [M,H] E4M3, out_scale fp32 [M]
  *   mode 1: out_q [M,H] E4M3, out_scale fp32 [M, H/128] row-major
  *   mode 2: out_q [M,H/2] packed E2M1, out_scale u8 E8M0 [M, H/32] row-major
  */
 int orc_quant_rows(const uint16_t* y, int mode, int64_t M, int64_t H,
-                   uint8_t* out_q, void* out_scale)
+                   uint8_t* out_q, void* out_scale, int io)
 {
-    if (M < 0 || H <= 0)
+    if (M < 0 || H <= 0 || (io != ORC_IO_BF16 && io != ORC_IO_FP16))
         return ORC_BAD;
     for (int64_t m = 0; m < M; ++m) {
         const uint16_t* yr = y + m * H;
         if (mode == ORC_FP8_PER_TOKEN) {
-            quant_fp8_group(yr, H, out_q + m * H, (float*)out_scale + m);
+            quant_fp8_group(yr, H, out_q + m * H, (float*)out_scale + m, io);
         } else if (mode == ORC_FP8_PER_GROUP128) {
             if (H % 128)
                 return ORC_BAD;
             for (int64_t g = 0; g < H / 128; ++g)
                 quant_fp8_group(yr + g * 128, 128, out_q + m * H + g * 128,
-                                (float*)out_scale + m * (H / 128) + g);
+                                (float*)out_scale + m * (H / 128) + g, io);
         } else if (mode == ORC_MXFP4) {
             if (H % 32)
                 return ORC_BAD;
             for (int64_t b = 0; b < H / 32; ++b)
                 quant_mx_block(yr + b * 32, out_q + m * (H / 2) + b * 16,
-                               (uint8_t*)out_scale + m * (H / 32) + b);
+                               (uint8_t*)out_scale + m * (H / 32) + b, io);
         } else {
             return ORC_BAD;
         }
@@ -294,12 +352,12 @@ int orc_quant_rows(const uint16_t* y, int mode, int64_t M, int64_t H,
 /* RMSNorm ([AR] "Accuracy Tests": the unfused sequence)                */
 /* ------------------------------------------------------------------ */
 
-/* rstd = 1/sqrt(mean(h^2) + eps) in fp64 over n bf16 values (A1). */
-double orc_rstd(const uint16_t* h, int64_t n, float eps)
+/* rstd = 1/sqrt(mean(h^2) + eps) in fp64 over n 16-bit values (A1). */
+double orc_rstd(const uint16_t* h, int64_t n, float eps, int io)
 {
     double ss = 0.0;
     for (int64_t j = 0; j < n; ++j) {
-        double v = orc_bf16_to_double(h[j]);
+        double v = elem_to_double(io, h[j]);
         ss += v * v;
     }
     return 1.0 / sqrt(ss / (double)n + (double)eps);
@@ -312,13 +370,16 @@ double orc_rstd(const uint16_t* h, int64_t n, float eps)
  *   y  = bf16( h * rstd * w )                                           fp64 (A1, A4)
  *   (q, scale) = quantize(y)                                            (A5-A9)
  * residual may be NULL (no residual add); out_residual and out_y may be NULL.
+ * io = ORC_IO_FP16: every 16-bit tensor and rounding is binary16 (A17).
  */
 int orc_rmsnorm_quant(const uint16_t* const* parts, int P, const uint16_t* residual,
                       const uint16_t* weight, float eps, int mode, int64_t M, int64_t H,
                       uint8_t* out_q, void* out_scale, uint16_t* out_residual,
-                      uint16_t* out_y)
+                      uint16_t* out_y, int io)
 {
     if (P < 1 || P > 8 || M < 0 || H <= 0 || !parts || !weight)
+        return ORC_BAD;
+    if (io != ORC_IO_BF16 && io != ORC_IO_FP16)
         return ORC_BAD;
     if (mode == ORC_FP8_PER_GROUP128 && H % 128)
         return ORC_BAD;
@@ -335,30 +396,30 @@ int orc_rmsnorm_quant(const uint16_t* const* parts, int P, const uint16_t* resid
     }
     for (int64_t m = 0; m < M; ++m) {
         for (int64_t j = 0; j < H; ++j) {
-            float s = bf16_to_float(parts[0][m * H + j]);
+            float s = elem_to_float(io, parts[0][m * H + j]);
             for (int p = 1; p < P; ++p)
-                s = s + bf16_to_float(parts[p][m * H + j]);
+                s = s + elem_to_float(io, parts[p][m * H + j]);
             if (residual)
-                s = s + bf16_to_float(residual[m * H + j]);
-            hbuf[j] = orc_bf16_from_double((double)s);
+                s = s + elem_to_float(io, residual[m * H + j]);
+            hbuf[j] = elem_from_double(io, (double)s);
         }
-        double rstd = orc_rstd(hbuf, H, eps);
+        double rstd = orc_rstd(hbuf, H, eps, io);
         for (int64_t j = 0; j < H; ++j)
-            ybuf[j] = orc_bf16_from_double(orc_bf16_to_double(hbuf[j]) * rstd *
-                                           orc_bf16_to_double(weight[j]));
+            ybuf[j] = elem_from_double(io, elem_to_double(io, hbuf[j]) * rstd *
+                                               elem_to_double(io, weight[j]));
         if (out_residual)
             memcpy(out_residual + m * H, hbuf, (size_t)H * sizeof(uint16_t));
         if (out_y)
             memcpy(out_y + m * H, ybuf, (size_t)H * sizeof(uint16_t));
         int rc;
         if (mode == ORC_FP8_PER_TOKEN)
-            rc = orc_quant_rows(ybuf, mode, 1, H, out_q + m * H, (float*)out_scale + m);
+            rc = orc_quant_rows(ybuf, mode, 1, H, out_q + m * H, (float*)out_scale + m, io);
         else if (mode == ORC_FP8_PER_GROUP128)
             rc = orc_quant_rows(ybuf, mode, 1, H, out_q + m * H,
-                                (float*)out_scale + m * (H / 128));
+                                (float*)out_scale + m * (H / 128), io);
         else
             rc = orc_quant_rows(ybuf, mode, 1, H, out_q + m * (H / 2),
-                                (uint8_t*)out_scale + m * (H / 32));
+                                (uint8_t*)out_scale + m * (H / 32), io);
         if (rc != ORC_OK) {
             free(hbuf);
             free(ybuf);
@@ -378,7 +439,7 @@ int orc_rmsnorm_quant(const uint16_t* const* parts, int P, const uint16_t* resid
 static void gemma_norm_head(const uint16_t* x, const uint16_t* w, int D, float eps,
                             uint16_t* y)
 {
-    double rstd = orc_rstd(x, D, eps);
+    double rstd = orc_rstd(x, D, eps, ORC_IO_BF16);
     for (int d = 0; d < D; ++d)
         y[d] = orc_bf16_from_double(orc_bf16_to_double(x[d]) * rstd *
                                     (1.0 + orc_bf16_to_double(w[d])));
@@ -434,7 +495,7 @@ int orc_qk_norm_gate_fp8(const uint16_t* qkv, int64_t M, int64_t row_stride, int
         for (int h = 0; h < Hq; ++h) {
             const int64_t o = m * Hq + h;
             gemma_norm_head(row + (int64_t)2 * h * D, q_weight, D, eps, y);
-            quant_fp8_group(y, D, q8 + o * D, qs + o);
+            quant_fp8_group(y, D, q8 + o * D, qs + o, ORC_IO_BF16);
             if (out_q)
                 memcpy(out_q + o * D, y, (size_t)D * sizeof(uint16_t));
             memcpy(out_gate + o * D, row + (int64_t)(2 * h + 1) * D, (size_t)D * sizeof(uint16_t));
@@ -442,7 +503,7 @@ int orc_qk_norm_gate_fp8(const uint16_t* qkv, int64_t M, int64_t row_stride, int
         for (int h = 0; h < Hk; ++h) {
             const int64_t o = m * Hk + h;
             gemma_norm_head(row + (int64_t)2 * Hq * D + (int64_t)h * D, k_weight, D, eps, y);
-            quant_fp8_group(y, D, k8 + o * D, ks + o);
+            quant_fp8_group(y, D, k8 + o * D, ks + o, ORC_IO_BF16);
             if (out_k)
                 memcpy(out_k + o * D, y, (size_t)D * sizeof(uint16_t));
         }

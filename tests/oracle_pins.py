@@ -137,10 +137,11 @@ def ref_y_bits(h_vals, w_vals, eps, gemma=False):
     return np.array(out, dtype=np.uint16)
 
 
-def ref_quant_fp8(y_bits, group):
+def ref_quant_fp8(y_bits, group, decode=None):
     """Library formulation: fp32 amax, fp32 amax/448, fp32 y/scale, torch's
-    float8_e4m3fn conversion (nearest-even; never reached above 464 here)."""
-    y = bf16_bits_to_f64(y_bits).astype(np.float32)
+    float8_e4m3fn conversion (nearest-even; never reached above 464 here).
+    `decode` maps the stored bits to values (bf16 by default)."""
+    y = (decode or bf16_bits_to_f64)(y_bits).astype(np.float32)
     M, H = y.shape
     codes = np.zeros((M, H), dtype=np.uint8)
     scales = np.zeros((M, H // group), dtype=np.float32)
@@ -156,8 +157,8 @@ def ref_quant_fp8(y_bits, group):
     return codes, scales
 
 
-def ref_quant_mx(y_bits):
-    y = bf16_bits_to_f64(y_bits)
+def ref_quant_mx(y_bits, decode=None):
+    y = (decode or bf16_bits_to_f64)(y_bits)
     M, H = y.shape
     gv, gc = e2m1_grid_golden()
     packed = np.zeros((M, H // 2), dtype=np.uint8)
@@ -525,3 +526,146 @@ def pin_qk_fp8(lib):
 
 
 ALL_PINS.append(pin_qk_fp8)
+
+
+# ----------------------------------------------------------------------------
+# binary16 input/output
+# ----------------------------------------------------------------------------
+
+
+def fp16_bits_to_f64(bits):
+    """binary16 bit patterns -> values, by numpy's own half-precision type."""
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def nearest_fp16_decimal(x: Decimal) -> int:
+    """binary16 bit pattern nearest to a high-precision value (ties to even;
+    finite values only)."""
+    if x == 0:
+        return 0x8000 if x.is_signed() else 0
+    neg = x < 0
+    ax = -x if neg else x
+    base = int(np.array([np.float16(float(ax))]).view(np.uint16)[0])
+    best = None
+    for b in range(max(base - 2, 0), min(base + 3, 0x7C00)):
+        d = abs(Decimal(float(fp16_bits_to_f64([b])[0])) - ax)
+        key = (d, b & 1)
+        if best is None or key < best[0]:
+            best = (key, b)
+    return best[1] | 0x8000 if neg else best[1]
+
+
+def pin_fp16_format(lib):
+    """binary16 decode and rounding against numpy's float16 and exact
+    Fraction arithmetic: every pattern, random values, ties, overflow and
+    subnormals."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = fp16_bits_to_f64(bits)
+    mine = oracle.fp16_to_double(bits, lib)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(mine), nan), "binary16 NaN patterns"
+    assert np.array_equal(mine[~nan], ref[~nan]), "binary16 decode vs numpy"
+    assert np.array_equal(np.signbit(mine[~nan]), np.signbit(ref[~nan])), "binary16 signed zero"
+    assert np.array_equal(oracle.fp16_from_double(ref[~nan], lib), bits[~nan]), "round trip"
+    # binary32 inputs (so numpy's conversion rounds once) across the range
+    rng = np.random.default_rng(17)
+    f = (rng.standard_normal(40000) * np.exp2(rng.uniform(-30, 18, 40000))).astype(np.float32)
+    with np.errstate(over="ignore"):  # beyond 65520 numpy gives infinity, as it should
+        ref16 = f.astype(np.float16).view(np.uint16)
+    assert np.array_equal(oracle.fp16_from_double(f.astype(np.float64), lib), ref16), \
+        "binary16 rounding vs numpy"
+    # midpoints between neighbours: ties to the even pattern, exactly
+    for b in list(rng.integers(0, 0x7BFF, 300)) + [0, 1, 0x3FF, 0x400, 0x3BFF, 0x7BFE]:
+        b = int(b)
+        lo, hi = fp16_bits_to_f64([b, b + 1])
+        mid = (lo + hi) / 2
+        assert Fraction(mid) == (Fraction(lo) + Fraction(hi)) / 2
+        want_tie = b if b % 2 == 0 else b + 1
+        for sgn, sb in ((1.0, 0), (-1.0, 0x8000)):
+            assert lib.orc_fp16_from_double(sgn * mid) == want_tie | sb, f"tie above {b:#x}"
+            assert lib.orc_fp16_from_double(sgn * np.nextafter(mid, 0)) == b | sb
+            assert lib.orc_fp16_from_double(sgn * np.nextafter(mid, np.inf)) == (b + 1) | sb
+    # overflow: 65520 is the midpoint between 65504 (odd) and 2^16: infinity
+    assert lib.orc_fp16_from_double(65520.0) == 0x7C00
+    assert lib.orc_fp16_from_double(np.nextafter(65520.0, 0)) == 0x7BFF
+    assert lib.orc_fp16_from_double(-1e9) == 0xFC00
+    # subnormals: 2^-25 ties to 0, 3 2^-25 ties to 2 2^-24
+    assert lib.orc_fp16_from_double(2.0 ** -25) == 0
+    assert lib.orc_fp16_from_double(-(2.0 ** -25)) == 0x8000
+    assert lib.orc_fp16_from_double(np.nextafter(2.0 ** -25, 1)) == 1
+    assert lib.orc_fp16_from_double(3 * 2.0 ** -25) == 2
+
+
+def _small_case_fp16(seed, M, H, P, residual):
+    g = torch.Generator().manual_seed(seed)
+    as_bits = lambda t: t.to(torch.float16).contiguous().view(torch.int16).numpy().view(np.uint16)
+    parts = [as_bits(torch.randn((M, H), generator=g) * (torch.rand((M, 1), generator=g) * 8 + 0.1))
+             for _ in range(P)]
+    res = as_bits(torch.randn((M, H), generator=g)) if residual else None
+    w = as_bits(1 + 0.3 * torch.randn((H,), generator=g))
+    return parts, res, w
+
+
+def pin_fp16_path(lib):
+    """io = binary16: the whole unfused sequence recomputed independently
+    (numpy fp32 sums rounded once by numpy, the norm in 60-digit decimal
+    rounded to the nearest binary16, the quantization by the library and
+    brute formulations), the constant-row closed form of W1, and the
+    quantization of binary16 rows with subnormal and near-overflow values."""
+    F16 = oracle.IO_FP16
+    cases = [(1, 2, 32, 1, True, oracle.FP8_PER_TOKEN), (2, 2, 64, 3, True, oracle.MXFP4),
+             (3, 2, 128, 2, False, oracle.FP8_PER_GROUP128), (4, 1, 96, 4, True, oracle.MXFP4)]
+    getcontext().prec = 60
+    for seed, M, H, P, has_res, mode in cases:
+        parts, res, w = _small_case_fp16(seed, M, H, P, has_res)
+        eps = 1e-6 if seed % 2 else 1e-5
+        r = oracle.rmsnorm_quant(parts, res, w, eps, mode, lib, io=F16)
+        acc = fp16_bits_to_f64(parts[0]).astype(np.float32)
+        for p in parts[1:] + ([res] if has_res else []):
+            acc = (acc + fp16_bits_to_f64(p).astype(np.float32)).astype(np.float32)
+        h = acc.astype(np.float16).view(np.uint16)
+        assert np.array_equal(r["residual_out"], h), f"fp16 residual case {seed}"
+        wv = fp16_bits_to_f64(w)
+        y = np.zeros((M, H), dtype=np.uint16)
+        for m in range(M):
+            hv = fp16_bits_to_f64(h[m])
+            rs = decimal_rstd(hv, np.float32(eps))
+            y[m] = [nearest_fp16_decimal(Decimal(float(a)) * rs * Decimal(float(b)))
+                    for a, b in zip(hv, wv)]
+        assert np.array_equal(r["y"], y), f"fp16 y case {seed}"
+        if mode == oracle.MXFP4:
+            rq, rsc = ref_quant_mx(y, fp16_bits_to_f64)
+        else:
+            rq, rsc = ref_quant_fp8(y, H if mode == oracle.FP8_PER_TOKEN else 128, fp16_bits_to_f64)
+        assert np.array_equal(r["q"], rq), f"fp16 codes case {seed}"
+        assert np.array_equal(r["scale"].reshape(rsc.shape), rsc), f"fp16 scales case {seed}"
+    # W1 with binary16 storage: y = 1 exactly, so the same codes and scales
+    w1 = {c["id"]: c for c in json.load(open(os.path.join(GOLDEN, "worked_rows.json")))["cases"]}["W1"]
+    H = w1["H"]
+    x = np.full((1, H), np.float16(w1["x_value"])).view(np.uint16)
+    wt = np.full((H,), np.float16(w1["w_value"])).view(np.uint16)
+    r = oracle.rmsnorm_quant([x], None, wt, w1["eps"], oracle.FP8_PER_TOKEN, lib, io=F16)
+    assert np.all(fp16_bits_to_f64(r["y"]) == w1["y_value"]), "W1 fp16 y"
+    assert r["scale"][0] == np.float32(w1["fp8_per_token"]["scale"])
+    assert np.all(r["q"] == int(w1["fp8_per_token"]["code"], 16))
+    r = oracle.rmsnorm_quant([x], None, wt, w1["eps"], oracle.MXFP4, lib, io=F16)
+    assert np.all(r["scale"] == w1["mxfp4"]["scale_code"])
+    assert np.all(r["q"] == int(w1["mxfp4"]["byte"], 16))
+    # quantization of binary16 rows over the format's whole range
+    rng = np.random.default_rng(23)
+    y = (rng.standard_normal((4, 256)) * np.exp2(rng.integers(-20, 12, (4, 1)))).astype(np.float16)
+    y[1, :32] = np.float16(2.0 ** -24) * rng.integers(-3, 4, 32)  # subnormal block
+    y[2, 7] = np.float16(65504.0)
+    y[3, 100:140] = 0
+    yb = y.view(np.uint16)
+    for mode, group in ((oracle.FP8_PER_TOKEN, 256), (oracle.FP8_PER_GROUP128, 128)):
+        q, sc = oracle.quant_rows(yb, mode, lib, io=F16)
+        rq, rsc = ref_quant_fp8(yb, group, fp16_bits_to_f64)
+        assert np.array_equal(q, rq) and np.array_equal(sc.reshape(rsc.shape), rsc), f"fp16 FP8 {mode}"
+    q, sc = oracle.quant_rows(yb, oracle.MXFP4, lib, io=F16)
+    rq, rsc = ref_quant_mx(yb, fp16_bits_to_f64)
+    assert np.array_equal(q, rq) and np.array_equal(sc, rsc), "fp16 MXFP4"
+    assert sc[2, 0] == 15 - 2 + 127  # amax 65504: floor(log2) = 15
+
+
+ALL_PINS += [pin_fp16_format, pin_fp16_path]

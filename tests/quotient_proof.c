@@ -10,7 +10,10 @@
  * and copy y's sign onto the code.  This program runs every positive finite
  * bf16 amax with s >= 2^-120 against every bf16 |y| <= amax (about 5.3e8
  * pairs) and counts the pairs whose E4M3 codes differ.  It exits 0 iff there
- * are none.  argv[1] (optional) strides the amax loop for a quicker run.
+ * are none.  argv[1] (optional) strides the amax loop for a quicker run;
+ * argv[2] = "fp16" runs the same check over IEEE binary16 amax and y (every
+ * positive finite binary16 amax, whose scale is always above 2^-120, against
+ * every binary16 |y| <= amax: about 5.0e8 pairs).
  *
  * Build: cc -O2 -ffp-contract=off -o quotient_proof quotient_proof.c -lm
  * (fmaf must be the correctly rounded fused multiply-add: glibc's is.)
@@ -27,6 +30,12 @@ static float from_bf16(uint32_t b)
     float f;
     memcpy(&f, &u, sizeof f);
     return f;
+}
+
+static float from_fp16(uint32_t b)
+{
+    int e = (int)(b >> 10) & 0x1F, m = (int)(b & 0x3FF);
+    return e == 0 ? (float)ldexp((double)m, -24) : (float)ldexp(1024.0 + m, e - 25);
 }
 
 /* E4M3 ("fn") code of a non-negative float: nearest even on the grid with 3
@@ -57,16 +66,19 @@ int main(int argc, char** argv)
     uint32_t stride = argc > 1 ? (uint32_t)strtoul(argv[1], NULL, 10) : 1u;
     if (stride == 0)
         stride = 1;
+    const int fp16 = argc > 2 && strcmp(argv[2], "fp16") == 0;
+    float (*from_bits)(uint32_t) = fp16 ? from_fp16 : from_bf16;
+    const uint32_t end = fp16 ? 0x7C00u : 0x7F80u; /* first non-finite pattern */
     long pairs = 0, bad = 0;
-    for (uint32_t ab = 1; ab < 0x7F80u; ab += stride) {
-        const float amax = from_bf16(ab);
+    for (uint32_t ab = 1; ab < end; ab += stride) {
+        const float amax = from_bits(ab);
         const float s = amax / 448.0f;
         if (!(s >= 0x1p-120f))
             continue;
         const float r = 1.0f / s;
         const float r_lo = fmaf(-s, r, 1.0f) * r;
         for (uint32_t yb = 0; yb <= ab; ++yb) {
-            const float y = from_bf16(yb);
+            const float y = from_bits(yb);
             const float q = fmaf(y, r, y * r_lo);
             if (e4m3_code(q) != e4m3_code(y / s)) {
                 if (bad < 10)

@@ -21,15 +21,15 @@ MUTANTS = [
      "return 1.0 / (sqrt(ss / (double)n) + (double)eps);"),
     ("mean_over_n_minus_1", "return 1.0 / sqrt(ss / (double)n + (double)eps);",
      "return 1.0 / sqrt(ss / (double)(n - 1) + (double)eps);"),
-    ("residual_dropped", "s = s + bf16_to_float(residual[m * H + j]);",
-     "s = s + 0.0f * bf16_to_float(residual[m * H + j]);"),
-    ("partials_in_fp64", "float s = bf16_to_float(parts[0][m * H + j]);",
-     "double s = bf16_to_float(parts[0][m * H + j]);"),
+    ("residual_dropped", "s = s + elem_to_float(io, residual[m * H + j]);",
+     "s = s + 0.0f * elem_to_float(io, residual[m * H + j]);"),
+    ("partials_in_fp64", "float s = elem_to_float(io, parts[0][m * H + j]);",
+     "double s = elem_to_float(io, parts[0][m * H + j]);"),
     ("plain_weight_in_gemma", "(1.0 + orc_bf16_to_double(w[d]))", "orc_bf16_to_double(w[d])"),
     ("ties_away_from_zero", "double n = nearbyint(fabs(v) / quantum);",
      "double n = round(fabs(v) / quantum);"),
-    ("reciprocal_multiply", "float t = bf16_to_float(y[j]) / scale;",
-     "float t = bf16_to_float(y[j]) * (1.0f / scale);"),
+    ("reciprocal_multiply", "float t = elem_to_float(io, y[j]) / scale;",
+     "float t = elem_to_float(io, y[j]) * (1.0f / scale);"),
     ("fp8_max_240", "amax / 448.0f", "amax / 240.0f"),
     ("e4m3_no_subnormals", "round_to_grid(v, 3, -6)", "round_to_grid(v, 3, -7)"),
     ("q_from_gate_slot", "gemma_norm_head(row + (int64_t)2 * h * D, q_weight",
@@ -39,8 +39,20 @@ MUTANTS = [
     ("zero_group_scale_zero", "float scale = (amax == 0.0f) ? 1.0f : amax / 448.0f;",
      "float scale = (amax == 0.0f) ? 0.0f : amax / 448.0f;"),
     ("weight_applied_twice",
-     "ybuf[j] = orc_bf16_from_double(orc_bf16_to_double(hbuf[j]) * rstd *",
-     "ybuf[j] = orc_bf16_from_double(orc_bf16_to_double(weight[j]) * orc_bf16_to_double(hbuf[j]) * rstd *"),
+     "ybuf[j] = elem_from_double(io, elem_to_double(io, hbuf[j]) * rstd *",
+     "ybuf[j] = elem_from_double(io, elem_to_double(io, weight[j]) * elem_to_double(io, hbuf[j]) * rstd *"),
+    # binary16 input/output
+    ("fp16_nine_mantissa_bits", "round_to_grid(v, 10, -14)", "round_to_grid(v, 9, -14)"),
+    ("fp16_no_subnormal_grid", "round_to_grid(v, 10, -14)", "round_to_grid(v, 10, -15)"),
+    ("fp16_overflow_saturates", "return (uint16_t)(sign | 0x7C00u);",
+     "return (uint16_t)(sign | 0x7BFFu);"),
+    ("fp16_decode_bias", "mag = ldexp(1024.0 + m, e - 25);", "mag = ldexp(1024.0 + m, e - 24);"),
+    ("fp16_weight_read_as_bf16", "elem_to_double(io, weight[j]));",
+     "orc_bf16_to_double(weight[j]));"),
+    ("fp16_quant_reads_bf16", "float t = elem_to_float(io, y[j]) / scale;",
+     "float t = elem_to_float(ORC_IO_BF16, y[j]) / scale;"),
+    ("fp16_h_rounded_as_bf16", "hbuf[j] = elem_from_double(io, (double)s);",
+     "hbuf[j] = orc_bf16_from_double((double)s);"),
 ]
 
 
