@@ -19,6 +19,7 @@ definition; there is no runnable GPU reference for this path) on the same
 metric, one bounded sample of rows per step.
 """
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -255,14 +256,15 @@ def make_row_call(fn, wl, device, seed):
     wl = synth.RowWorkload(**{**wl.__dict__, "seed": seed})
     inp = wl.inputs(device=device)
     parts, res, w = inp["parts"], inp["residual"], inp["weight"]
-    q, s = fn.alloc_outputs(wl.mode, wl.M, wl.H, device)
+    mode = wl.mode | (fn.FN_IO_FP16 if wl.dtype == torch.float16 else 0)
+    q, s = fn.alloc_outputs(mode, wl.M, wl.H, device)
     r_out = res if wl.in_place else torch.empty_like(res)
     ptrs = [p.data_ptr() for p in parts]
     stream = torch.cuda.current_stream(device)
     sp = stream.cuda_stream
 
     def step():
-        st = fn.fn_rmsnorm_quant(ptrs, len(ptrs), res.data_ptr(), w.data_ptr(), wl.eps, wl.mode,
+        st = fn.fn_rmsnorm_quant(ptrs, len(ptrs), res.data_ptr(), w.data_ptr(), wl.eps, mode,
                                  wl.M, wl.H, q.data_ptr(), s.data_ptr(), r_out.data_ptr(), None,
                                  sp)
         if st != fn.FN_OK:
@@ -489,6 +491,21 @@ def secondary_workloads(fn, device, peak):
         del keep
         torch.cuda.empty_cache()
     res["large_m_kernels"] = cmp
+
+    # the two large-M shapes with float16 rows (FN_IO_FP16: the producer's dtype
+    # carried through the tuple; same bytes per call)
+    f16 = {}
+    for base in (synth.PREFILL_MXFP4, synth.PREFILL_GROUP128):
+        wl = dataclasses.replace(base, name=base.name + "_fp16", dtype=torch.float16)
+        step, stream, keep = make_row_call(fn, wl, device, wl.seed)
+        ms = time_steps(step, 100, 5, device, stream)
+        b = wl.bytes_per_call()
+        f16[wl.name] = {"M": wl.M, "H": wl.H, "P": wl.P, "us_per_call": ms * 1e3,
+                        "GB_s": b / (ms * 1e-3) / 1e9, "frac_of_peak": b / (ms * 1e-3) / 1e9 / peak,
+                        "variant": fn.fn_last_variant(), "launch": list(fn.fn_last_launch())}
+        del keep
+        torch.cuda.empty_cache()
+    res["fp16_rows"] = f16
 
     def small(wl, per_call_bytes, make):
         n_sets = max(64, int(2 * L2_BYTES / per_call_bytes) + 1)

@@ -102,6 +102,15 @@ typedef enum {
 #define FN_SCALE_SWIZZLE_32_4_4 0x100
 #define FN_SCALE_MN_MAJOR 0x200
 
+/* Row-format flag, OR-ed into `mode` (fn_rmsnorm_quant, fn_quant): every
+ * 16-bit tensor of the call (x_parts, residual, weight, out_residual, out_y;
+ * y of fn_quant) is IEEE binary16 instead of bf16, and every "bf16_rn" in the
+ * formulas below is the binary16 rounding (nearest even, subnormals kept,
+ * overflow to infinity).  Codes and scales are unchanged.  This carries an
+ * FP16 producer's dtype through the quantized tuple instead of promoting it to
+ * BF16 (sglang PR #29723, review of the tuple path's output dtype). */
+#define FN_IO_FP16 0x1000
+
 #define FN_MAX_PARTS 8
 #define FN_MAX_H 32768
 #define FN_MAX_HEAD_DIM 1024
@@ -125,7 +134,8 @@ typedef enum {
  * residual     bf16 [M, H], or NULL (no residual add).
  * weight       bf16 [H].
  * eps          finite, >= 0.
- * mode         fn_mode, optionally OR-ed with one FN_SCALE_* layout flag.
+ * mode         fn_mode, optionally OR-ed with one FN_SCALE_* layout flag and
+ *              with FN_IO_FP16 (every "bf16" tensor here is then binary16).
  * M, H         M >= 0; H % 8 == 0, 8 <= H <= FN_MAX_H; H % 128 == 0 for
  *              FN_FP8_PER_GROUP128, H % 32 == 0 for FN_MXFP4.
  * out_q        FP8: u8 [M, H]; MXFP4: u8 [M, H/2].
@@ -146,7 +156,8 @@ FN_API int fn_rmsnorm_quant(const void* const* x_parts, int num_parts, const voi
                      void* stream);
 
 /*
- * The quantization step alone on existing bf16 rows y [M, H] (the third
+ * The quantization step alone on existing bf16 (or, with FN_IO_FP16,
+ * binary16) rows y [M, H] (the third
  * launch of the unfused AllReduce -> RMSNorm -> quantize sequence in sglang
  * PR #29723; the stand-alone row quantization the monokernel notes compare
  * against).  Same modes, layouts, alignment and overlap rules as

@@ -24,9 +24,11 @@ NVCC_FLAGS = ARCH + [
     "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
 ]
 
+# one unit per (quantization mode, partial-count bound, row format: 0 bf16, 1 binary16)
 UNITS = [("fusednorm", "fusednorm.cu", [])] + [
-    (f"rq_{mode}_{maxp}", "rq_inst.cu", [f"-DFN_INST_MODE={mode}", f"-DFN_INST_MAXP={maxp}"])
-    for mode in (0, 1, 2) for maxp in (1, 2, 4, 8)
+    (f"rq_{mode}_{maxp}_{io}", "rq_inst.cu",
+     [f"-DFN_INST_MODE={mode}", f"-DFN_INST_MAXP={maxp}", f"-DFN_INST_IO={io}"])
+    for mode in (0, 1, 2) for maxp in (1, 2, 4, 8) for io in (0, 1)
 ]
 
 

@@ -142,10 +142,124 @@ __device__ __forceinline__ float2 fma_f32x2(float2 a, float2 b, float2 c) {
   return d;
 }
 
-// max |y| over the 8 bf16 of a vector, as fp32.
+// ---- IEEE binary16 -------------------------------------------------------------
+
+__device__ __forceinline__ float f16_lo(uint32_t w) {
+  float d;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.f32.f16 %0, l;\n\t}" : "=f"(d) : "r"(w));
+  return d;
+}
+__device__ __forceinline__ float f16_hi(uint32_t w) {
+  float d;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.f32.f16 %0, h;\n\t}" : "=f"(d) : "r"(w));
+  return d;
+}
+
+// Two fp32 -> packed binary16 pair, each rounded to nearest even (subnormals
+// kept, overflow to infinity).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// Packed binary16 add, one rounding of the exact sum, subnormals kept.  For
+// two binary16 operands this equals rounding their fp32 sum to binary16: the
+// fp32 sum is inexact only if the exponents differ by more than 13, and then
+// the smaller operand moves the larger by under a quarter of its half-ulp, so
+// both roundings return the larger operand.
+__device__ __forceinline__ uint32_t add_f16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t absmax_f16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a & 0x7FFF7FFFu), "r"(b & 0x7FFF7FFFu));
+  return d;
+}
+
+template <bool HI>
+__device__ __forceinline__ float add_f16(uint32_t w, float acc) {
+  float d;
+  if (HI)
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.f16 %0, h, %2;\n\t}"
+        : "=f"(d) : "r"(w), "f"(acc));
+  else
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.f16 %0, l, %2;\n\t}"
+        : "=f"(d) : "r"(w), "f"(acc));
+  return d;
+}
+
+// As fma_bf16: the product of two binary16 (11-bit significands) is exact in
+// fp32.
+template <bool HI>
+__device__ __forceinline__ float fma_f16(uint32_t a, uint32_t b, float c) {
+  float d;
+  if (HI)
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.f16 %0, ah, bh, %3;\n\t}"
+        : "=f"(d) : "r"(a), "r"(b), "f"(c));
+  else
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.f16 %0, al, bl, %3;\n\t}"
+        : "=f"(d) : "r"(a), "r"(b), "f"(c));
+  return d;
+}
+
+// ---- element formats ---------------------------------------------------------------
+// The row kernels are written once over the format of their 16-bit tensors:
+// Bf16, or F16 (IEEE binary16).  Each gives the pair decode, the rounding
+// pack, the packed add and |max|, and the mixed fp32 add and fma on one half.
+
+struct Bf16 {
+  static constexpr bool kF16 = false;
+  static __device__ __forceinline__ float lo(uint32_t w) { return bf_lo(w); }
+  static __device__ __forceinline__ float hi(uint32_t w) { return bf_hi(w); }
+  static __device__ __forceinline__ uint32_t pack(float l, float h) { return pack_bf16x2(l, h); }
+  static __device__ __forceinline__ uint32_t add2(uint32_t a, uint32_t b) {
+    return add_bf16x2(a, b);
+  }
+  static __device__ __forceinline__ uint32_t absmax2(uint32_t a, uint32_t b) {
+    return absmax_bf16x2(a, b);
+  }
+  template <bool HI>
+  static __device__ __forceinline__ float add(uint32_t w, float acc) {
+    return add_bf16<HI>(w, acc);
+  }
+  template <bool HI>
+  static __device__ __forceinline__ float fma(uint32_t a, uint32_t b, float c) {
+    return fma_bf16<HI>(a, b, c);
+  }
+};
+
+struct F16 {
+  static constexpr bool kF16 = true;
+  static __device__ __forceinline__ float lo(uint32_t w) { return f16_lo(w); }
+  static __device__ __forceinline__ float hi(uint32_t w) { return f16_hi(w); }
+  static __device__ __forceinline__ uint32_t pack(float l, float h) { return pack_f16x2(l, h); }
+  static __device__ __forceinline__ uint32_t add2(uint32_t a, uint32_t b) {
+    return add_f16x2(a, b);
+  }
+  static __device__ __forceinline__ uint32_t absmax2(uint32_t a, uint32_t b) {
+    return absmax_f16x2(a, b);
+  }
+  template <bool HI>
+  static __device__ __forceinline__ float add(uint32_t w, float acc) {
+    return add_f16<HI>(w, acc);
+  }
+  template <bool HI>
+  static __device__ __forceinline__ float fma(uint32_t a, uint32_t b, float c) {
+    return fma_f16<HI>(a, b, c);
+  }
+};
+
+// max |y| over the 8 16-bit values of a vector, as fp32.
+template <class IO = Bf16>
 __device__ __forceinline__ float vec_absmax(const uint4& y) {
-  const uint32_t m = absmax_bf16x2(absmax_bf16x2(y.x, y.y), absmax_bf16x2(y.z, y.w));
-  return fmaxf(bf_lo(m), bf_hi(m));
+  const uint32_t m = IO::absmax2(IO::absmax2(y.x, y.y), IO::absmax2(y.z, y.w));
+  return fmaxf(IO::lo(m), IO::hi(m));
 }
 
 // ---- FP8 E4M3 -----------------------------------------------------------------
@@ -200,9 +314,9 @@ __device__ __forceinline__ float group_max(float v) {
   return v;
 }
 
-// MX block exponent from the block amax (a non-negative value of a bf16):
-// e = floor(log2 amax) - 2, clamped to [-127, 127]; zero and bf16 subnormals
-// (binary32 exponent field 0) give -127.  Returns the E8M0 code e + 127, and
+// MX block exponent from the block amax (a non-negative bf16 or binary16
+// value): e = floor(log2 amax) - 2, clamped to [-127, 127]; zero and bf16
+// subnormals (binary32 exponent field 0) give -127.  Returns the E8M0 code e + 127, and
 // 2^-e (always a normal binary32, since e <= 125) in `inv`.  A NaN or
 // infinite amax gives code 0xFF.
 __device__ __forceinline__ uint32_t mx_scale(float amax, float& inv) {

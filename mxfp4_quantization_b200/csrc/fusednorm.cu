@@ -80,10 +80,13 @@ int round32(int x) { return (x + 31) / 32 * 32; }
 using fn::RQKernel;
 
 // Kernel instance for (mode, P, V, cluster, norm).
-RQKernel pick_kernel(int mode, int P, int V, bool cluster, bool norm) {
+// `f16`: binary16 rows (FN_IO_FP16), else bf16.
+RQKernel pick_kernel(int mode, int P, int V, bool cluster, bool norm, bool f16) {
   const int maxp = (!norm || P == 1) ? 1 : P == 2 ? 2 : P <= 4 ? 4 : 8;
-#define FN_CASE(MODE, MAXP) \
-  if (mode == MODE && maxp == MAXP) return fn::rq_pick_##MODE##_##MAXP(V, cluster, norm);
+#define FN_CASE(MODE, MAXP)                                                       \
+  if (mode == MODE && maxp == MAXP)                                               \
+    return f16 ? fn::rq_pick_##MODE##_##MAXP##_1(V, cluster, norm)                \
+               : fn::rq_pick_##MODE##_##MAXP##_0(V, cluster, norm);
   FN_CASE(0, 1) FN_CASE(0, 2) FN_CASE(0, 4) FN_CASE(0, 8)
   FN_CASE(1, 1) FN_CASE(1, 2) FN_CASE(1, 4) FN_CASE(1, 8)
   FN_CASE(2, 1) FN_CASE(2, 2) FN_CASE(2, 4) FN_CASE(2, 8)
@@ -92,10 +95,12 @@ RQKernel pick_kernel(int mode, int P, int V, bool cluster, bool norm) {
 }
 
 // The exact-cover instance for a row of T * V vectors, or nullptr.
-RQKernel pick_exact_kernel(int mode, int P, int T, int V) {
+RQKernel pick_exact_kernel(int mode, int P, int T, int V, bool f16) {
   const int maxp = P == 1 ? 1 : P == 2 ? 2 : P <= 4 ? 4 : 8;
-#define FN_CASE(MODE, MAXP) \
-  if (mode == MODE && maxp == MAXP) return fn::rq_exact_pick_##MODE##_##MAXP(T, V);
+#define FN_CASE(MODE, MAXP)                                                              \
+  if (mode == MODE && maxp == MAXP)                                                      \
+    return f16 ? fn::rq_exact_pick_##MODE##_##MAXP##_1(T, V)                             \
+               : fn::rq_exact_pick_##MODE##_##MAXP##_0(T, V);
   FN_CASE(0, 1) FN_CASE(0, 2) FN_CASE(0, 4) FN_CASE(0, 8)
   FN_CASE(1, 1) FN_CASE(1, 2) FN_CASE(1, 4) FN_CASE(1, 8)
   FN_CASE(2, 1) FN_CASE(2, 2) FN_CASE(2, 4) FN_CASE(2, 8)
@@ -105,10 +110,11 @@ RQKernel pick_exact_kernel(int mode, int P, int T, int V) {
 
 using fn::RQTmaKernel;
 
-RQTmaKernel pick_tma_kernel(int mode, int P, int V) {
+RQTmaKernel pick_tma_kernel(int mode, int P, int V, bool f16) {
   const int maxp = P == 1 ? 1 : P == 2 ? 2 : P <= 4 ? 4 : 8;
-#define FN_CASE(MODE, MAXP) \
-  if (mode == MODE && maxp == MAXP) return fn::rq_tma_pick_##MODE##_##MAXP(V);
+#define FN_CASE(MODE, MAXP)                                                                \
+  if (mode == MODE && maxp == MAXP)                                                        \
+    return f16 ? fn::rq_tma_pick_##MODE##_##MAXP##_1(V) : fn::rq_tma_pick_##MODE##_##MAXP##_0(V);
   FN_CASE(0, 1) FN_CASE(0, 2) FN_CASE(0, 4) FN_CASE(0, 8)
   FN_CASE(1, 1) FN_CASE(1, 2) FN_CASE(1, 4) FN_CASE(1, 8)
   FN_CASE(2, 1) FN_CASE(2, 2) FN_CASE(2, 4) FN_CASE(2, 8)
@@ -162,16 +168,18 @@ int pick_cluster(int64_t M, int nvec, int mode, int sms) {
   return 0;
 }
 
-// `mode` carries the quantization (low byte) and scale-layout flags.
+// `mode` carries the quantization (low byte), scale-layout and row-format flags.
 struct ModeInfo {
   int q = -1;       // FN_FP8_PER_TOKEN / FN_FP8_PER_GROUP128 / FN_MXFP4
   int layout = 0;   // fn::SCALE_ROW_MAJOR / SCALE_SWIZZLE_32_4_4 / SCALE_MN_MAJOR
+  bool f16 = false; // FN_IO_FP16: the 16-bit tensors are IEEE binary16
 };
 
 int parse_mode(int mode, ModeInfo* mi) {
-  const int q = mode & FN_MODE_MASK, flags = mode & ~FN_MODE_MASK;
+  const int q = mode & FN_MODE_MASK, flags = mode & ~(FN_MODE_MASK | FN_IO_FP16);
   if (q < FN_FP8_PER_TOKEN || q > FN_MXFP4) return FN_ERR_INVALID;
   mi->q = q;
+  mi->f16 = (mode & FN_IO_FP16) != 0;
   mi->layout = fn::SCALE_ROW_MAJOR;
   if (flags == FN_SCALE_SWIZZLE_32_4_4) {
     if (q != FN_MXFP4) return FN_ERR_INVALID;
@@ -222,8 +230,8 @@ int check_outputs_align(const ModeInfo& mi, const void* out_q, const void* out_s
   return FN_OK;
 }
 
-int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, void* stream,
-              int variant_if_norm) {
+int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, bool f16,
+              void* stream, int variant_if_norm) {
   // `mode` is the quantization alone here (the layout travels in prm)
   const int nvec = prm.nvec;
   const int sms = sm_count();
@@ -253,7 +261,7 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, vo
     const int groups = (int)std::min<int64_t>(2, (M + sms - 1) / sms);
     const int threads = group_threads * groups;
     if (group_threads > 256) return FN_ERR_UNSUPPORTED;
-    RQTmaKernel k = pick_tma_kernel(mode, P, V);
+    RQTmaKernel k = pick_tma_kernel(mode, P, V, f16);
     if (!k) return FN_ERR_UNSUPPORTED;
     const size_t smem = (size_t)nst * (size_t)(stage_bytes + 8);
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -275,7 +283,7 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, vo
   } else if (C >= 2) {
     p.seg = nvec / C;
     const int threads = round32(p.seg);
-    RQKernel k = pick_kernel(mode, P, 1, true, true);
+    RQKernel k = pick_kernel(mode, P, 1, true, true, f16);
     if (!k) return FN_ERR_UNSUPPORTED;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(M * C));
@@ -303,8 +311,9 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, vo
     p.seg = nvec;
     p.prefetch_rows = M > (int64_t)kRowPrefetchSms * sms ? kRowPrefetchSms * sms : 0;
     const int threads = round32((nvec + V - 1) / V);
-    RQKernel k = norm && threads * V == nvec ? pick_exact_kernel(mode, P, threads, V) : nullptr;
-    if (!k) k = pick_kernel(mode, P, V, false, norm);
+    RQKernel k =
+        norm && threads * V == nvec ? pick_exact_kernel(mode, P, threads, V, f16) : nullptr;
+    if (!k) k = pick_kernel(mode, P, V, false, norm, f16);
     if (!k) return FN_ERR_UNSUPPORTED;
     k<<<(unsigned)M, threads, 0, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return FN_ERR_CUDA;
@@ -529,7 +538,7 @@ int fn_rmsnorm_quant(const void* const* x_parts, int num_parts, const void* resi
   prm.inv_h = 1.0f / (float)H;
   prm.scale_layout = mi.layout;
   prm.scale_ld = scale_ld(mi, M, H);
-  return launch_rq(prm, mi.q, num_parts, M, true, stream, FN_VARIANT_ROW_CTA);
+  return launch_rq(prm, mi.q, num_parts, M, true, mi.f16, stream, FN_VARIANT_ROW_CTA);
 }
 
 int fn_quant(const void* y, int mode, int64_t M, int64_t H, void* out_q, void* out_scale,
@@ -560,7 +569,7 @@ int fn_quant(const void* y, int mode, int64_t M, int64_t H, void* out_q, void* o
   prm.P = 1;
   prm.scale_layout = mi.layout;
   prm.scale_ld = scale_ld(mi, M, H);
-  return launch_rq(prm, mi.q, 1, M, false, stream, FN_VARIANT_QUANT_ONLY);
+  return launch_rq(prm, mi.q, 1, M, false, mi.f16, stream, FN_VARIANT_QUANT_ONLY);
 }
 
 int fn_qk_norm_gate(const void* qkv, int64_t M, int64_t row_stride, int Hq, int Hk, int D,

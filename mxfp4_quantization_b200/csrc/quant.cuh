@@ -1,5 +1,5 @@
-// FP8 E4M3 quantization of 8-element bf16 vectors, shared by the row kernels
-// and the QK prologue: the group scale and the division-free codes.
+// FP8 E4M3 quantization of 8-element bf16 / binary16 vectors, shared by the
+// row kernels and the QK prologue: the group scale and the division-free codes.
 #pragma once
 #include "fn_device.cuh"
 
@@ -27,18 +27,20 @@ __device__ __forceinline__ Fp8Scale fp8_scale_direct(float amax) {
 // Fast path: with r = RN(1/s) and r_lo = RN(RN(1 - s r) r) (r + r_lo carries
 // 1/s to about 2^-46), q = RN(|y| r + RN(|y| r_lo)) has the same E4M3 code as
 // RN(|y| / s) for every bf16 y with |y| <= amax and every bf16 amax with
-// s = RN(amax / 448) >= 2^-120: checked exhaustively over all such (amax, y)
+// s = RN(amax / 448) >= 2^-120, and likewise for every binary16 pair (whose
+// scales are all above 2^-120): checked exhaustively over all such (amax, y)
 // pairs by tests/quotient_proof.c.  The code is computed from |y| and y's
 // sign bit is copied onto it, which also gives -0 the code 0x80.  If any lane
 // of the warp needs the IEEE division the whole warp takes it (warp-uniform
 // branch).  All 32 lanes must call.
+template <class IO = Bf16>
 __device__ __forceinline__ uint2 e4m3_codes(const uint4& y, const Fp8Scale& c) {
   uint32_t q8[4];
   if (!__any_sync(0xffffffffu, c.exact_div)) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint32_t a = word(y, i) & 0x7FFF7FFFu;
-      const float2 ya = make_float2(bf_lo(a), bf_hi(a));
+      const float2 ya = make_float2(IO::lo(a), IO::hi(a));
       const float2 t = mul_f32x2(ya, make_float2(c.r_lo, c.r_lo));
       const float2 q = fma_f32x2(ya, make_float2(c.r, c.r), t);
       q8[i] = cvt_e4m3x2(q.x, q.y);
@@ -47,11 +49,11 @@ __device__ __forceinline__ uint2 e4m3_codes(const uint4& y, const Fp8Scale& c) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint32_t a = word(y, i) & 0x7FFF7FFFu;
-      q8[i] = cvt_e4m3x2(__fdiv_rn(bf_lo(a), c.s), __fdiv_rn(bf_hi(a), c.s));
+      q8[i] = cvt_e4m3x2(__fdiv_rn(IO::lo(a), c.s), __fdiv_rn(IO::hi(a), c.s));
     }
   }
   // byte k of code word j takes the sign of element 4j + k: the sign bits sit
-  // at bits 15 and 31 of each y word, i.e. in bytes 1 and 3
+  // at bits 15 and 31 of each y word (both formats), i.e. in bytes 1 and 3
   const uint32_t s0 = __byte_perm(y.x, y.y, 0x7531) & 0x80808080u;
   const uint32_t s1 = __byte_perm(y.z, y.w, 0x7531) & 0x80808080u;
   return make_uint2((q8[0] | (q8[1] << 16)) | s0, (q8[2] | (q8[3] << 16)) | s1);

@@ -1,5 +1,8 @@
-// One instantiation unit of the rmsnorm_quant kernels: the mode and the
-// partial-count bound come from -DFN_INST_MODE / -DFN_INST_MAXP.
+// One instantiation unit of the rmsnorm_quant kernels: the mode, the
+// partial-count bound and the row format (0 bf16, 1 binary16) come from
+// -DFN_INST_MODE / -DFN_INST_MAXP / -DFN_INST_IO.
+#include <type_traits>
+
 #include "rq_kernel.cuh"
 
 #ifndef FN_INST_MODE
@@ -8,37 +11,42 @@
 #ifndef FN_INST_MAXP
 #error "FN_INST_MAXP is required"
 #endif
+#ifndef FN_INST_IO
+#error "FN_INST_IO is required"
+#endif
 
-#define FN_CAT_(a, b, c) a##_##b##_##c
-#define FN_CAT(a, b, c) FN_CAT_(a, b, c)
+#define FN_CAT_(a, b, c, d) a##_##b##_##c##_##d
+#define FN_CAT4(a, b, c, d) FN_CAT_(a, b, c, d)
+#define FN_CAT(a, b, c) FN_CAT4(a, b, c, FN_INST_IO)
 
 namespace fn {
 
 RQKernel FN_CAT(rq_pick, FN_INST_MODE, FN_INST_MAXP)(int V, bool cluster, bool norm) {
   constexpr int MODE = FN_INST_MODE, MAXP = FN_INST_MAXP;
+  using IO = std::conditional_t<FN_INST_IO == 1, F16, Bf16>;
   if (cluster) {
     if (!norm) return nullptr;
-    return rq_kernel<MODE, MAXP, 1, true, true>;
+    return rq_kernel<MODE, MAXP, 1, true, true, 0, IO>;
   }
   if (!norm) {
     if constexpr (MAXP != 1) {
       return nullptr;
     } else {
       switch (V) {
-        case 1: return rq_kernel<MODE, 1, 1, false, false>;
-        case 2: return rq_kernel<MODE, 1, 2, false, false>;
-        case 4: return rq_kernel<MODE, 1, 4, false, false>;
-        case 8: return rq_kernel<MODE, 1, 8, false, false>;
-        default: return rq_kernel<MODE, 1, 16, false, false>;
+        case 1: return rq_kernel<MODE, 1, 1, false, false, 0, IO>;
+        case 2: return rq_kernel<MODE, 1, 2, false, false, 0, IO>;
+        case 4: return rq_kernel<MODE, 1, 4, false, false, 0, IO>;
+        case 8: return rq_kernel<MODE, 1, 8, false, false, 0, IO>;
+        default: return rq_kernel<MODE, 1, 16, false, false, 0, IO>;
       }
     }
   }
   switch (V) {
-    case 1: return rq_kernel<MODE, MAXP, 1, true, false>;
-    case 2: return rq_kernel<MODE, MAXP, 2, true, false>;
-    case 4: return rq_kernel<MODE, MAXP, 4, true, false>;
-    case 8: return rq_kernel<MODE, MAXP, 8, true, false>;
-    default: return rq_kernel<MODE, MAXP, 16, true, false>;
+    case 1: return rq_kernel<MODE, MAXP, 1, true, false, 0, IO>;
+    case 2: return rq_kernel<MODE, MAXP, 2, true, false, 0, IO>;
+    case 4: return rq_kernel<MODE, MAXP, 4, true, false, 0, IO>;
+    case 8: return rq_kernel<MODE, MAXP, 8, true, false, 0, IO>;
+    default: return rq_kernel<MODE, MAXP, 16, true, false, 0, IO>;
   }
 }
 
@@ -46,8 +54,9 @@ RQKernel FN_CAT(rq_pick, FN_INST_MODE, FN_INST_MAXP)(int V, bool cluster, bool n
 // T = 224 serves H = 3584, 7168, 14336; T = 256 serves H = 4096, 8192, 16384.
 RQKernel FN_CAT(rq_exact_pick, FN_INST_MODE, FN_INST_MAXP)(int T, int V) {
   constexpr int MODE = FN_INST_MODE, MAXP = FN_INST_MAXP;
+  using IO = std::conditional_t<FN_INST_IO == 1, F16, Bf16>;
 #define FN_EXACT(TT, VV) \
-  if (T == TT && V == VV) return rq_kernel<MODE, MAXP, VV, true, false, TT>;
+  if (T == TT && V == VV) return rq_kernel<MODE, MAXP, VV, true, false, TT, IO>;
   FN_EXACT(224, 2) FN_EXACT(224, 4) FN_EXACT(224, 8)
   FN_EXACT(256, 2) FN_EXACT(256, 4) FN_EXACT(256, 8)
 #undef FN_EXACT
@@ -56,11 +65,12 @@ RQKernel FN_CAT(rq_exact_pick, FN_INST_MODE, FN_INST_MAXP)(int T, int V) {
 
 RQTmaKernel FN_CAT(rq_tma_pick, FN_INST_MODE, FN_INST_MAXP)(int V) {
   constexpr int MODE = FN_INST_MODE, MAXP = FN_INST_MAXP;
+  using IO = std::conditional_t<FN_INST_IO == 1, F16, Bf16>;
   switch (V) {
-    case 1: return rq_tma_kernel<MODE, MAXP, 1>;
-    case 2: return rq_tma_kernel<MODE, MAXP, 2>;
-    case 4: return rq_tma_kernel<MODE, MAXP, 4>;
-    default: return rq_tma_kernel<MODE, MAXP, 8>;
+    case 1: return rq_tma_kernel<MODE, MAXP, 1, IO>;
+    case 2: return rq_tma_kernel<MODE, MAXP, 2, IO>;
+    case 4: return rq_tma_kernel<MODE, MAXP, 4, IO>;
+    default: return rq_tma_kernel<MODE, MAXP, 8, IO>;
   }
 }
 

@@ -33,86 +33,99 @@ namespace cg = cooperative_groups;
 // per-vector stages
 // ---------------------------------------------------------------------------
 
-__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = bf_lo(word(v, i));
-    f[2 * i + 1] = bf_hi(word(v, i));
-  }
-}
+// Every stage is written over the element format IO of the 16-bit tensors
+// (Bf16 or F16, fn_device.cuh); "bf16" below reads "IO" for binary16 rows.
 
 // h = bf16(((x_0 + x_1) + ...) + r) for one vector, every add in fp32.
-template <int MAXP>
+template <int MAXP, class IO = Bf16>
 __device__ __forceinline__ uint4 sum_vec(const uint4 (&x)[MAXP], const uint4& r, int P,
                                          bool has_res) {
   uint4 h;
   if constexpr (MAXP == 1) {
-    h = has_res ? make_uint4(add_bf16x2(x[0].x, r.x), add_bf16x2(x[0].y, r.y),
-                             add_bf16x2(x[0].z, r.z), add_bf16x2(x[0].w, r.w))
+    h = has_res ? make_uint4(IO::add2(x[0].x, r.x), IO::add2(x[0].y, r.y),
+                             IO::add2(x[0].z, r.z), IO::add2(x[0].w, r.w))
                 : x[0];
   } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      float a0 = bf_lo(word(x[0], i)), a1 = bf_hi(word(x[0], i));
+      float a0 = IO::lo(word(x[0], i)), a1 = IO::hi(word(x[0], i));
 #pragma unroll
       for (int p = 1; p < MAXP; ++p) {
         if (p < P) {
-          a0 = add_bf16<false>(word(x[p], i), a0);
-          a1 = add_bf16<true>(word(x[p], i), a1);
+          a0 = IO::template add<false>(word(x[p], i), a0);
+          a1 = IO::template add<true>(word(x[p], i), a1);
         }
       }
       if (has_res) {
-        a0 = add_bf16<false>(word(r, i), a0);
-        a1 = add_bf16<true>(word(r, i), a1);
+        a0 = IO::template add<false>(word(r, i), a0);
+        a1 = IO::template add<true>(word(r, i), a1);
       }
-      set_word(h, i, pack_bf16x2(a0, a1));
+      set_word(h, i, IO::pack(a0, a1));
     }
   }
   return h;
 }
 
 // Sum of squares of h (two fp32 accumulators), and (per-token mode) max |h * w|.
-// h * w is exact in fp32 (two 8-bit significands) and y = bf16(fl(h * w) * rstd)
-// is monotone in |h * w|, so max |y| = bf16(fl(max |h * w| * rstd)) falls out
-// of the same reduction as the sum of squares.
-template <bool WANT_PMAX>
+// h * w is exact in fp32 (two 8-bit, or two 11-bit, significands) and
+// y = bf16(fl(h * w) * rstd) is monotone in |h * w|, so
+// max |y| = bf16(fl(max |h * w| * rstd)) falls out of the same reduction as
+// the sum of squares.
+template <bool WANT_PMAX, class IO = Bf16>
 __device__ __forceinline__ void stats_vec(const uint4& h, const uint4& w, float2& ss,
                                           float& pmax) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t hw = word(h, i);
-    ss.x = fma_bf16<false>(hw, hw, ss.x);
-    ss.y = fma_bf16<true>(hw, hw, ss.y);
+    ss.x = IO::template fma<false>(hw, hw, ss.x);
+    ss.y = IO::template fma<true>(hw, hw, ss.y);
     if (WANT_PMAX) {
       const uint32_t ww = word(w, i);
-      pmax = fmaxf(pmax, fmaxf(fabsf(fma_bf16<false>(hw, ww, -0.f)),
-                               fabsf(fma_bf16<true>(hw, ww, -0.f))));
+      pmax = fmaxf(pmax, fmaxf(fabsf(IO::template fma<false>(hw, ww, -0.f)),
+                               fabsf(IO::template fma<true>(hw, ww, -0.f))));
     }
   }
 }
 
 // y = bf16(fl(h * w) * rstd).
+template <class IO = Bf16>
 __device__ __forceinline__ uint4 norm_vec(const uint4& h, const uint4& w, float rstd) {
   uint4 y;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t hw = word(h, i), ww = word(w, i);
-    const float2 p = make_float2(fma_bf16<false>(hw, ww, -0.f), fma_bf16<true>(hw, ww, -0.f));
+    const float2 p = make_float2(IO::template fma<false>(hw, ww, -0.f),
+                                 IO::template fma<true>(hw, ww, -0.f));
     const float2 q = mul_f32x2(p, make_float2(rstd, rstd));
-    set_word(y, i, pack_bf16x2(q.x, q.y));
+    set_word(y, i, IO::pack(q.x, q.y));
   }
   return y;
 }
 
-// E2M1 codes of y * 2^-e for the 8 bf16 of a vector (inv_bf16 = 2^-e as a bf16
-// bit pattern in both halves): each product is exact, computed by the mixed
-// bf16 FMA with a -0 addend (which keeps the sign of zeros).
-__device__ __forceinline__ uint32_t e2m1_codes(const uint4& y, uint32_t inv_bf16) {
+// E2M1 codes of y * 2^-e for the 8 values of a vector (inv = 2^-e); each
+// product is exact and keeps the sign of zeros.  For bf16 rows 2^-e is itself
+// a bf16 (e <= 125), and the mixed bf16 FMA with a -0 addend forms the
+// product in one instruction; a binary16 row's 2^-e can lie outside binary16
+// (up to 2^26), so those products are fp32 multiplies.
+template <class IO = Bf16>
+__device__ __forceinline__ uint32_t e2m1_codes(const uint4& y, float inv) {
   float f[8];
+  if constexpr (!IO::kF16) {
+    const uint32_t ib = __float_as_uint(inv) >> 16;
+    const uint32_t inv2 = ib | (ib << 16);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = fma_bf16<false>(word(y, i), inv_bf16, -0.f);
-    f[2 * i + 1] = fma_bf16<true>(word(y, i), inv_bf16, -0.f);
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = fma_bf16<false>(word(y, i), inv2, -0.f);
+      f[2 * i + 1] = fma_bf16<true>(word(y, i), inv2, -0.f);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 p = mul_f32x2(make_float2(IO::lo(word(y, i)), IO::hi(word(y, i))),
+                                 make_float2(inv, inv));
+      f[2 * i] = p.x;
+      f[2 * i + 1] = p.y;
+    }
   }
   return cvt_e2m1x8(f);
 }
@@ -135,24 +148,23 @@ __device__ __forceinline__ int64_t scale_index(int layout, int64_t ld, int64_t r
 // group's first lane, its scale.  All 32 lanes must call (shuffles); `ok`
 // masks the stores of lanes past the row end (whole groups, by alignment).
 // `tok` is the row's scale (per-token mode).
-template <int MODE>
+template <int MODE, class IO = Bf16>
 __device__ __forceinline__ void quant_store(const uint4& y, bool ok, int lane, int64_t row, int v,
                                             int H, const Fp8Scale& tok, uint8_t* out_q,
                                             void* out_scale, int layout, int64_t ld) {
   if constexpr (MODE == MODE_TOKEN || MODE == MODE_G128) {
     Fp8Scale c = tok;
     if constexpr (MODE == MODE_G128) {
-      c = fp8_scale_direct(group_max<16>(vec_absmax(y)));
+      c = fp8_scale_direct(group_max<16>(vec_absmax<IO>(y)));
       if (ok && (lane & 15) == 0)
         static_cast<float*>(out_scale)[scale_index(layout, ld, row, v / 16, H / 128)] = c.s;
     }
-    const uint2 q = e4m3_codes(y, c);
+    const uint2 q = e4m3_codes<IO>(y, c);
     if (ok) st_stream(reinterpret_cast<uint2*>(out_q + row * (int64_t)H) + v, q);
   } else {
     float inv;
-    const uint32_t code = mx_scale(group_max<4>(vec_absmax(y)), inv);
-    const uint32_t inv_b = __float_as_uint(inv) >> 16;  // 2^-e is exact in bf16
-    const uint32_t q = e2m1_codes(y, inv_b | (inv_b << 16));
+    const uint32_t code = mx_scale(group_max<4>(vec_absmax<IO>(y)), inv);
+    const uint32_t q = e2m1_codes<IO>(y, inv);
     if (ok) {
       st_stream(reinterpret_cast<uint32_t*>(out_q + row * (int64_t)(H / 2)) + v, q);
       if ((lane & 3) == 0)
@@ -221,8 +233,9 @@ __device__ __forceinline__ float row_rstd(float ss, float inv_h, float eps) {
 }
 
 // bf16(fl(pmax * rstd)): the row's max |y| (see stats_vec).
+template <class IO = Bf16>
 __device__ __forceinline__ float row_amax_from_pmax(float pmax, float rstd) {
-  return bf_lo(pack_bf16x2(pmax * rstd, 0.f));
+  return IO::lo(IO::pack(pmax * rstd, 0.f));
 }
 
 // ---------------------------------------------------------------------------
@@ -233,7 +246,7 @@ __device__ __forceinline__ float row_amax_from_pmax(float pmax, float rstd) {
 // is exactly TB * V vectors (H = 8 * TB * V), so every offset is a
 // compile-time constant and no access needs a bounds test.  TB = 0 reads the
 // block size and the row length at run time.
-template <int MODE, int MAXP, int V, bool NORM, bool CL, int TB = 0>
+template <int MODE, int MAXP, int V, bool NORM, bool CL, int TB = 0, class IO = Bf16>
 __global__ void __launch_bounds__(CL ? 512 : 256)
     rq_kernel(const __grid_constant__ RQParams prm) {
   static_assert(TB == 0 || (!CL && NORM), "exact-cover instances are one block per row");
@@ -292,8 +305,8 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
     float pmax = 0.f;
 #pragma unroll
     for (int k = 0; k < V; ++k) {
-      hv[k] = sum_vec<MAXP>(xin[k], rin[k], prm.P, has_res);
-      stats_vec<MODE == MODE_TOKEN>(hv[k], win[k], ss, pmax);
+      hv[k] = sum_vec<MAXP, IO>(xin[k], rin[k], prm.P, has_res);
+      stats_vec<MODE == MODE_TOKEN, IO>(hv[k], win[k], ss, pmax);
       const int v = seg_base + t + k * T;
       if ((TB || v < seg_end) && prm.out_residual != nullptr)
         st_stream(prm.out_residual + rowv + v, hv[k]);
@@ -301,11 +314,11 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
     // ---- 3. rstd (and the per-token amax) ---------------------------------------------
     const float2 tot = row_reduce<CL, MODE == MODE_TOKEN>(ss.x + ss.y, pmax, red, &cl_slot);
     const float rstd = row_rstd(tot.x, prm.inv_h, prm.eps);
-    if (MODE == MODE_TOKEN) scale_tok = fp8_scale_direct(row_amax_from_pmax(tot.y, rstd));
+    if (MODE == MODE_TOKEN) scale_tok = fp8_scale_direct(row_amax_from_pmax<IO>(tot.y, rstd));
     // ---- 4. y = bf16(fl(h * w) * rstd) ----------------------------------------------
 #pragma unroll
     for (int k = 0; k < V; ++k) {
-      yv[k] = norm_vec(hv[k], win[k], rstd);
+      yv[k] = norm_vec<IO>(hv[k], win[k], rstd);
       const int v = seg_base + t + k * T;
       if ((TB || v < seg_end) && prm.out_y != nullptr) st_stream(prm.out_y + rowv + v, yv[k]);
     }
@@ -315,7 +328,7 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
     if (MODE == MODE_TOKEN) {
       float am = 0.f;
 #pragma unroll
-      for (int k = 0; k < V; ++k) am = fmaxf(am, vec_absmax(yv[k]));
+      for (int k = 0; k < V; ++k) am = fmaxf(am, vec_absmax<IO>(yv[k]));
       scale_tok = fp8_scale_direct(row_reduce<CL, true>(0.f, am, red, &cl_slot).y);
     }
   }
@@ -326,8 +339,8 @@ __global__ void __launch_bounds__(CL ? 512 : 256)
 #pragma unroll
   for (int k = 0; k < V; ++k) {
     const int v = seg_base + t + k * T;
-    quant_store<MODE>(yv[k], TB || v < seg_end, lane, row, v, H, scale_tok, prm.out_q, prm.out_scale,
-                      prm.scale_layout, prm.scale_ld);
+    quant_store<MODE, IO>(yv[k], TB || v < seg_end, lane, row, v, H, scale_tok, prm.out_q,
+                          prm.out_scale, prm.scale_layout, prm.scale_ld);
   }
 
   if constexpr (CL) {
@@ -454,7 +467,7 @@ __device__ __forceinline__ float2 group_reduce(float s, float m, float2* red, in
 // therefore carries the index of the row last issued into it; a group first
 // waits (bounded) for its row's index there, which also proves that the
 // stage's previous row has been consumed, and only then waits on the parity.
-template <int MODE, int MAXP, int V>
+template <int MODE, int MAXP, int V, class IO = Bf16>
 __global__ void __launch_bounds__(512, 1)
     rq_tma_kernel(const __grid_constant__ RQParams prm, int nstages, int groups) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -543,8 +556,8 @@ __global__ void __launch_bounds__(512, 1)
       for (int p = 0; p < MAXP; ++p)
         x[p] = (ok && p < prm.P) ? st[p * nvec + v] : make_uint4(0u, 0u, 0u, 0u);
       const uint4 r = (ok && has_res) ? st[prm.P * nvec + v] : make_uint4(0u, 0u, 0u, 0u);
-      hv[k] = sum_vec<MAXP>(x, r, prm.P, has_res);
-      stats_vec<MODE == MODE_TOKEN>(hv[k], wv[k], ss, pmax);
+      hv[k] = sum_vec<MAXP, IO>(x, r, prm.P, has_res);
+      stats_vec<MODE == MODE_TOKEN, IO>(hv[k], wv[k], ss, pmax);
       if (ok && prm.out_residual != nullptr) st_stream(prm.out_residual + rowv + v, hv[k]);
     }
     const float2 tot =
@@ -555,17 +568,17 @@ __global__ void __launch_bounds__(512, 1)
     const float rstd = row_rstd(tot.x, prm.inv_h, prm.eps);
     Fp8Scale scale_tok = {1.f, 1.f, 0.f, false};
     if (MODE == MODE_TOKEN) {
-      scale_tok = fp8_scale_direct(row_amax_from_pmax(tot.y, rstd));
+      scale_tok = fp8_scale_direct(row_amax_from_pmax<IO>(tot.y, rstd));
       if (t == 0) static_cast<float*>(prm.out_scale)[row] = scale_tok.s;
     }
 #pragma unroll
     for (int k = 0; k < V; ++k) {
       const int v = t + k * tg;
       const bool ok = v < nvec;
-      const uint4 y = norm_vec(hv[k], wv[k], rstd);
+      const uint4 y = norm_vec<IO>(hv[k], wv[k], rstd);
       if (ok && prm.out_y != nullptr) st_stream(prm.out_y + rowv + v, y);
-      quant_store<MODE>(y, ok, lane, row, v, H, scale_tok, prm.out_q, prm.out_scale,
-                        prm.scale_layout, prm.scale_ld);
+      quant_store<MODE, IO>(y, ok, lane, row, v, H, scale_tok, prm.out_q, prm.out_scale,
+                            prm.scale_layout, prm.scale_ld);
     }
   }
   if (timed_out && prm.status != nullptr) atomicExch(prm.status, 1);

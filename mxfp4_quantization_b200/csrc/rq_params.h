@@ -42,22 +42,25 @@ using RQKernel = void (*)(const RQParams);
 // groups per block as further arguments.
 using RQTmaKernel = void (*)(const RQParams, int, int);
 
-#define FN_RQ_DECL(MODE, MAXP)                                          \
-  RQKernel rq_pick_##MODE##_##MAXP(int V, bool cluster, bool norm); \
-  RQKernel rq_exact_pick_##MODE##_##MAXP(int T, int V);             \
-  RQTmaKernel rq_tma_pick_##MODE##_##MAXP(int V);
-FN_RQ_DECL(0, 1)
-FN_RQ_DECL(0, 2)
-FN_RQ_DECL(0, 4)
-FN_RQ_DECL(0, 8)
-FN_RQ_DECL(1, 1)
-FN_RQ_DECL(1, 2)
-FN_RQ_DECL(1, 4)
-FN_RQ_DECL(1, 8)
-FN_RQ_DECL(2, 1)
-FN_RQ_DECL(2, 2)
-FN_RQ_DECL(2, 4)
-FN_RQ_DECL(2, 8)
+// IO: 0 = bf16 rows, 1 = binary16 rows.
+#define FN_RQ_DECL(MODE, MAXP, IO)                                          \
+  RQKernel rq_pick_##MODE##_##MAXP##_##IO(int V, bool cluster, bool norm); \
+  RQKernel rq_exact_pick_##MODE##_##MAXP##_##IO(int T, int V);             \
+  RQTmaKernel rq_tma_pick_##MODE##_##MAXP##_##IO(int V);
+#define FN_RQ_DECL_IO(MODE, MAXP) FN_RQ_DECL(MODE, MAXP, 0) FN_RQ_DECL(MODE, MAXP, 1)
+FN_RQ_DECL_IO(0, 1)
+FN_RQ_DECL_IO(0, 2)
+FN_RQ_DECL_IO(0, 4)
+FN_RQ_DECL_IO(0, 8)
+FN_RQ_DECL_IO(1, 1)
+FN_RQ_DECL_IO(1, 2)
+FN_RQ_DECL_IO(1, 4)
+FN_RQ_DECL_IO(1, 8)
+FN_RQ_DECL_IO(2, 1)
+FN_RQ_DECL_IO(2, 2)
+FN_RQ_DECL_IO(2, 4)
+FN_RQ_DECL_IO(2, 8)
+#undef FN_RQ_DECL_IO
 #undef FN_RQ_DECL
 
 }  // namespace fn

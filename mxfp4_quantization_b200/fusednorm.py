@@ -43,6 +43,7 @@ FN_VARIANT_QK_WARP_FP8 = 6
 FN_MODE_MASK = 0xFF
 FN_SCALE_SWIZZLE_32_4_4 = 0x100
 FN_SCALE_MN_MAJOR = 0x200
+FN_IO_FP16 = 0x1000
 
 FN_MAX_PARTS = 8
 FN_MAX_H = 32768
@@ -198,11 +199,12 @@ def _mode(mode: Union[int, str]) -> int:
     return MODES[mode] if isinstance(mode, str) else int(mode)
 
 
-def _rows(t: torch.Tensor, name: str, H: Optional[int] = None) -> torch.Tensor:
+def _rows(t: torch.Tensor, name: str, H: Optional[int] = None,
+          dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
-    if t.dtype != torch.bfloat16:
-        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if H is not None and t.shape[-1] != H:
         raise ValueError(f"{name} has last dim {t.shape[-1]}, expected {H}")
     if not t.is_contiguous():
@@ -222,6 +224,18 @@ def _round_up(x: int, m: int) -> int:
     return (x + m - 1) // m * m
 
 
+def _row_format(t: torch.Tensor, mode: int):
+    """The 16-bit format of a call (bf16, or float16 -> FN_IO_FP16), taken from
+    its first input; every other 16-bit tensor must match it."""
+    if t.dtype not in (torch.bfloat16, torch.float16):
+        raise TypeError(f"rows must be bfloat16 or float16, got {t.dtype}")
+    if t.dtype == torch.float16:
+        return t.dtype, mode | FN_IO_FP16
+    if mode & FN_IO_FP16:
+        raise TypeError("FN_IO_FP16 was asked for but the rows are bfloat16")
+    return t.dtype, mode
+
+
 def alloc_outputs(mode: int, M: int, H: int, device) -> tuple:
     """Codes and scales for `mode` (with its layout flag, if any): FP8 codes as
     float8_e4m3fn [M, H]; MXFP4 codes as uint8 [M, H/2]; scales fp32 [M, 1] /
@@ -229,7 +243,7 @@ def alloc_outputs(mode: int, M: int, H: int, device) -> tuple:
     the padded buffer that layout needs (zero-filled: padding is not written):
     uint8 [roundup(M,128) * roundup(H/32,4)] for FN_SCALE_SWIZZLE_32_4_4,
     fp32 [H/128, roundup(M,4)] for FN_SCALE_MN_MAJOR."""
-    q_mode, flags = mode & FN_MODE_MASK, mode & ~FN_MODE_MASK
+    q_mode, flags = mode & FN_MODE_MASK, mode & (FN_SCALE_SWIZZLE_32_4_4 | FN_SCALE_MN_MAJOR)
     if q_mode == FN_MXFP4:
         q = torch.empty((M, H // 2), dtype=torch.uint8, device=device)
         if flags == FN_SCALE_SWIZZLE_32_4_4:
@@ -252,25 +266,27 @@ def rmsnorm_quant(x: Union[torch.Tensor, Sequence[torch.Tensor]], weight: torch.
                   out_y: Optional[torch.Tensor] = None) -> RMSNormQuantOutput:
     """Fused (sum of partials) + residual add + RMSNorm + quantization.
 
-    x: a bf16 CUDA tensor [..., H] or a list of up to 8 such partial tensors
-    (summed in the kernel).  With `in_place`, residual_out is written into
-    `residual`.  Returns (q, scale, residual_out, y); y is None unless
-    `emit_y` (or `out_y`) asks for the bf16 normed row.
+    x: a bf16 (or float16) CUDA tensor [..., H] or a list of up to 8 such
+    partial tensors (summed in the kernel).  With `in_place`, residual_out is
+    written into `residual`.  Returns (q, scale, residual_out, y); y is None
+    unless `emit_y` (or `out_y`) asks for the normed row.  float16 rows select
+    FN_IO_FP16: residual, weight, residual_out and y are then float16 too, so
+    the producer's dtype is carried through the tuple.
     """
     parts = list(x) if isinstance(x, (list, tuple)) else [x]
     if not 1 <= len(parts) <= FN_MAX_PARTS:
         raise ValueError("between 1 and 8 partial tensors")
     H = parts[0].shape[-1]
     lead = parts[0].shape[:-1]
-    rows = [_rows(p, f"x[{i}]", H) for i, p in enumerate(parts)]
+    dt, m = _row_format(parts[0], _mode(mode))
+    rows = [_rows(p, f"x[{i}]", H, dt) for i, p in enumerate(parts)]
     for r in rows:
         if r.shape != rows[0].shape:
             raise ValueError("all partials must have the same shape")
     M = rows[0].shape[0]
-    w = _rows(weight, "weight", H)
-    m = _mode(mode)
+    w = _rows(weight, "weight", H, dt)
     dev = rows[0].device
-    res = None if residual is None else _rows(residual, "residual", H)
+    res = None if residual is None else _rows(residual, "residual", H, dt)
     if res is not None and res.shape[0] != M:
         raise ValueError("residual rows differ from x rows")
     if in_place:
@@ -278,7 +294,7 @@ def rmsnorm_quant(x: Union[torch.Tensor, Sequence[torch.Tensor]], weight: torch.
             raise ValueError("in_place needs a residual")
         r_out = res
     elif out_residual is not None:
-        r_out = _rows(out_residual, "out_residual", H)
+        r_out = _rows(out_residual, "out_residual", H, dt)
     elif res is not None:
         r_out = torch.empty_like(res)
     else:
@@ -288,7 +304,9 @@ def rmsnorm_quant(x: Union[torch.Tensor, Sequence[torch.Tensor]], weight: torch.
         out_q = q if out_q is None else out_q
         out_scale = s if out_scale is None else out_scale
     if out_y is None and emit_y:
-        out_y = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+        out_y = torch.empty((M, H), dtype=dt, device=dev)
+    elif out_y is not None:
+        out_y = _rows(out_y, "out_y", H, dt)
     st = fn_rmsnorm_quant([r.data_ptr() for r in rows], len(rows), _ptr(res), w.data_ptr(),
                           float(eps), m, M, H, out_q.data_ptr(), out_scale.data_ptr(),
                           _ptr(r_out), _ptr(out_y), _stream(dev))
@@ -301,10 +319,11 @@ def rmsnorm_quant(x: Union[torch.Tensor, Sequence[torch.Tensor]], weight: torch.
 
 def quant(y: torch.Tensor, mode: Union[int, str], *, out_q: Optional[torch.Tensor] = None,
           out_scale: Optional[torch.Tensor] = None):
-    """Quantization step alone on bf16 rows [..., H]; returns (q, scale)."""
-    rows = _rows(y, "y")
+    """Quantization step alone on bf16 (or float16) rows [..., H]; returns
+    (q, scale)."""
+    dt, m = _row_format(y, _mode(mode))
+    rows = _rows(y, "y", None, dt)
     M, H = rows.shape
-    m = _mode(mode)
     if out_q is None or out_scale is None:
         q, s = alloc_outputs(m, M, H, rows.device)
         out_q = q if out_q is None else out_q

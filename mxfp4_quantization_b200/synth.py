@@ -1,6 +1,7 @@
 """Seeded synthetic inputs for the fused RMSNorm + quantization path.
 
-This module only draws random numbers and casts them to bf16 with torch; it
+This module only draws random numbers and casts them to bf16 (or float16)
+with torch; it
 holds none of the method's arithmetic, so both the CUDA path and the CPU
 oracle can be fed from it.  Every tensor gets its own seed, derived from the
 workload seed and the tensor's name, so a sub-range of rows can be regenerated
@@ -46,18 +47,18 @@ def _gen(device, seed: int, name: str) -> torch.Generator:
 
 
 def normal_bf16(shape, seed: int, name: str, std: float = 1.0, mean: float = 0.0,
-                device="cpu") -> torch.Tensor:
+                device="cpu", dtype=torch.bfloat16) -> torch.Tensor:
     g = _gen(device, seed, name)
     t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
-    return (t * std + mean).to(torch.bfloat16)
+    return (t * std + mean).to(dtype)
 
 
 def normal_with_outliers_bf16(shape, seed: int, name: str, frac: float, mult: float,
-                              device="cpu") -> torch.Tensor:
+                              device="cpu", dtype=torch.bfloat16) -> torch.Tensor:
     g = _gen(device, seed, name)
     t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
     mask = torch.rand(shape, generator=g, device=device) < frac
-    return torch.where(mask, t * mult, t).to(torch.bfloat16)
+    return torch.where(mask, t * mult, t).to(dtype)
 
 
 def channel_scale(H: int, seed: int, name: str, decades: float, device="cpu") -> torch.Tensor:
@@ -82,11 +83,12 @@ class RowWorkload:
     channel_decades: float = 0.0
     residual: bool = True
     in_place: bool = False
+    dtype: torch.dtype = torch.bfloat16  # of every 16-bit tensor (float16: binary16 rows)
 
     def inputs(self, device="cpu", rows: Optional[slice] = None, M: Optional[int] = None):
         """Draw the inputs. `M` overrides the row count (same recipe)."""
         M = self.M if M is None else M
-        H, s = self.H, self.seed
+        H, s, dt = self.H, self.seed, self.dtype
         shape = (M, H)
         if self.channel_decades > 0:
             c = channel_scale(H, s, "channel", self.channel_decades, device)
@@ -94,16 +96,17 @@ class RowWorkload:
             for p in range(self.P):
                 g = _gen(device, s, f"part{p}")
                 t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
-                parts.append((t * c[None, :]).to(torch.bfloat16))
+                parts.append((t * c[None, :]).to(dt))
         elif self.outlier_frac > 0:
             parts = [normal_with_outliers_bf16(shape, s, f"part{p}", self.outlier_frac,
-                                               self.outlier_mult, device)
+                                               self.outlier_mult, device, dt)
                      for p in range(self.P)]
         else:
-            parts = [normal_bf16(shape, s, f"part{p}", std=self.x_std, device=device)
+            parts = [normal_bf16(shape, s, f"part{p}", std=self.x_std, device=device, dtype=dt)
                      for p in range(self.P)]
-        residual = normal_bf16(shape, s, "residual", device=device) if self.residual else None
-        weight = normal_bf16((H,), s, "weight", std=0.1, mean=1.0, device=device)
+        residual = (normal_bf16(shape, s, "residual", device=device, dtype=dt)
+                    if self.residual else None)
+        weight = normal_bf16((H,), s, "weight", std=0.1, mean=1.0, device=device, dtype=dt)
         return {"parts": parts, "residual": residual, "weight": weight}
 
     def bytes_per_row(self) -> int:
@@ -180,6 +183,6 @@ PREFILL_GROUP128 = RowWorkload("prefill_group128", M=32768, H=8192, P=1,
 
 
 def to_bits(t: torch.Tensor):
-    """bf16 tensor -> numpy uint16 bit patterns (CPU copy)."""
+    """bf16 / float16 tensor -> numpy uint16 bit patterns (CPU copy)."""
     import numpy as np
     return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)

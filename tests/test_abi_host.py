@@ -188,3 +188,22 @@ def test_qk_fp8_rejects_bad_arguments(fnb):
     assert q8(q8=BASE + (3 << 32) + 4) == A and q8(qs=BASE + (4 << 32) + 2) == A
     assert q8(qs=BASE + (3 << 32) + 64) == E          # scales inside the q codes
     assert q8(k8=BASE + 100 * 2 * 256) == E           # codes inside qkv
+
+
+def test_fp16_row_flag(fnb):
+    """FN_IO_FP16 combines with every mode and layout flag; unknown bits next
+    to it are still rejected; its value matches the header."""
+    m = re.search(r"#define FN_IO_FP16 (0x[0-9A-Fa-f]+)", open(HEADER).read())
+    assert m and int(m.group(1), 16) == fnb.FN_IO_FP16
+    F = fnb.FN_IO_FP16
+    for mode in (fnb.FN_FP8_PER_TOKEN, fnb.FN_FP8_PER_GROUP128, fnb.FN_MXFP4,
+                 fnb.FN_MXFP4 | fnb.FN_SCALE_SWIZZLE_32_4_4,
+                 fnb.FN_FP8_PER_GROUP128 | fnb.FN_SCALE_MN_MAJOR):
+        assert rq(fnb, M=0, mode=mode | F) == fnb.FN_OK
+        assert fnb.fn_quant(BASE, mode | F, 0, 256, BASE + (1 << 32), BASE + (2 << 32),
+                            None) == fnb.FN_OK
+    assert rq(fnb, M=0, mode=fnb.FN_MXFP4 | F | 0x2000) == fnb.FN_ERR_INVALID
+    assert rq(fnb, M=0, mode=fnb.FN_FP8_PER_TOKEN | F | fnb.FN_SCALE_SWIZZLE_32_4_4) == \
+        fnb.FN_ERR_INVALID
+    # the same argument checks apply (here: H not a multiple of 8)
+    assert rq(fnb, mode=fnb.FN_MXFP4 | F, H=12) == fnb.FN_ERR_INVALID

@@ -33,8 +33,8 @@ def run(fnb, wl, M=None, in_place=False, guarded=True, emit_y=True, device_input
     s_shape = oracle.scale_shape(wl.mode, M, H)
     gq = gpu_util.Guarded(q_shape, torch.uint8)
     gs = gpu_util.Guarded(s_shape, torch.uint8 if wl.mode == MX else torch.float32)
-    gy = gpu_util.Guarded((M, H), torch.bfloat16) if emit_y else None
-    gr = gpu_util.Guarded((M, H), torch.bfloat16) if (res is not None and not in_place) else None
+    gy = gpu_util.Guarded((M, H), wl.dtype) if emit_y else None
+    gr = gpu_util.Guarded((M, H), wl.dtype) if (res is not None and not in_place) else None
     with fnb.prefer_variant(variant):
         out = fnb.rmsnorm_quant(parts, w, wl.eps, wl.mode, residual=res, in_place=in_place,
                                 out_residual=None if gr is None else gr.t, out_q=gq.t,
@@ -50,10 +50,15 @@ def run(fnb, wl, M=None, in_place=False, guarded=True, emit_y=True, device_input
     return inp, gpu, variant, launch
 
 
+def io_of(wl):
+    return oracle.IO_FP16 if wl.dtype == torch.float16 else oracle.IO_BF16
+
+
 def check(wl, inp, gpu):
     parts = [gpu_util.bits(p) for p in inp["parts"]]
     res = gpu_util.bits(inp["residual"])
-    return parity.check_rmsnorm(wl.mode, wl.eps, parts, res, gpu_util.bits(inp["weight"]), gpu)
+    return parity.check_rmsnorm(wl.mode, wl.eps, parts, res, gpu_util.bits(inp["weight"]), gpu,
+                                io_of(wl))
 
 
 # (M, H, P, residual): several tiles, ragged tails, the cluster/row switch,
@@ -275,3 +280,75 @@ def test_bounded_wait_reports_timeout_and_context_survives(fnb):
     inp2, gpu, variant, _ = run(fnb, wl, variant=fnb.FN_VARIANT_ROW_TMA)
     assert variant == fnb.FN_VARIANT_ROW_TMA
     check(wl, inp2, gpu)
+
+
+# ---- binary16 rows (FN_IO_FP16) ---------------------------------------------------
+
+F16_SHAPES = [
+    (1, 7168, 1, True), (16, 2048, 1, True), (17, 7168, 4, True), (37, 8192, 1, True),
+    (64, 4096, 3, False), (200, 2176, 5, True), (300, 256, 7, True), (40, 16384, 2, True),
+    (1500, 7168, 4, True), (600, 8192, 1, True),
+]
+
+
+@pytest.mark.parametrize("variant", ["auto", "cta", "tma"])
+@pytest.mark.parametrize("mode", [TOKEN, G128, MX], ids=["token", "g128", "mxfp4"])
+@pytest.mark.parametrize("M,H,P,has_res", F16_SHAPES,
+                         ids=[f"M{s[0]}_H{s[1]}_P{s[2]}" for s in F16_SHAPES])
+def test_fp16_parity(fnb, mode, M, H, P, has_res, variant):
+    """float16 rows: every 16-bit output stays float16, residual_out bit-exact,
+    y within 1 binary16 ulp, the quantization of the GPU's y bit-exact, codes
+    end to end as for bf16, under every kernel."""
+    wl = synth.RowWorkload("fp16", M=M, H=H, P=P, mode=mode, eps=1e-6, seed=M + H + P,
+                           residual=has_res, outlier_frac=0.01,
+                           channel_decades=1.0 if P > 1 else 0.0, dtype=torch.float16)
+    inp, gpu, got, launch = run(fnb, wl, variant=VARIANTS[variant])
+    if variant == "cta":
+        assert got == fnb.FN_VARIANT_ROW_CTA
+    if variant == "tma" and tma_fits(H, P, has_res):
+        assert got == fnb.FN_VARIANT_ROW_TMA, launch
+    check(wl, inp, gpu)
+
+
+def test_fp16_dtype_carried_and_in_place(fnb):
+    wl = synth.RowWorkload("fp16_inplace", M=48, H=8192, P=1, mode=G128, eps=1e-5, seed=6,
+                           x_std=2.0, dtype=torch.float16)
+    inp = wl.inputs(device="cpu")
+    ref_inp = {k: (v if k != "parts" else list(v)) for k, v in inp.items()}
+    ref_inp["residual"] = inp["residual"].clone()
+    parts = [p.cuda() for p in inp["parts"]]
+    res, w = inp["residual"].cuda(), inp["weight"].cuda()
+    out = fnb.rmsnorm_quant(parts, w, wl.eps, G128, residual=res, in_place=True, emit_y=True)
+    torch.cuda.synchronize()
+    assert out.residual_out.dtype == torch.float16 and out.y.dtype == torch.float16
+    assert out.residual_out.data_ptr() == res.data_ptr()
+    gpu = {"q": gpu_util.u8(out.q), "scale": gpu_util.scale_np(out.scale, G128),
+           "residual_out": gpu_util.bits(res), "y": gpu_util.bits(out.y)}
+    check(wl, ref_inp, gpu)
+    # mixed formats are refused before any launch
+    with pytest.raises(TypeError):
+        fnb.rmsnorm_quant(parts, w.to(torch.bfloat16), wl.eps, G128, residual=res)
+    with pytest.raises(TypeError):
+        fnb.rmsnorm_quant([p.to(torch.bfloat16) for p in parts], w.to(torch.bfloat16), wl.eps,
+                          G128 | fnb.FN_IO_FP16)
+
+
+@pytest.mark.parametrize("mode", [TOKEN, G128, MX], ids=["token", "g128", "mxfp4"])
+def test_fp16_quant_only_full_range(fnb, mode):
+    """fn_quant on float16 rows spanning the format: subnormal groups, values
+    next to 65504, zeros, signed zeros; bit-exact against the oracle."""
+    g = torch.Generator().manual_seed(40 + mode)
+    M, H = 37, 1024
+    y = torch.randn((M, H), generator=g) * torch.pow(2.0, torch.randint(-22, 15, (M, 1),
+                                                                         generator=g).float())
+    y = y.clamp(-65504, 65504).to(torch.float16)
+    y[1, :128] = (torch.randint(-6, 7, (128,), generator=g) * 2.0 ** -24).to(torch.float16)
+    y[2, 5] = 65504.0
+    y[3, :256] = 0
+    y[4, :32] = -0.0
+    bits = gpu_util.bits(y)
+    q, s = fnb.quant(y.cuda(), mode)
+    assert fnb.fn_last_variant() == fnb.FN_VARIANT_QUANT_ONLY
+    torch.cuda.synchronize()
+    parity.compare_quant_stage(bits, gpu_util.u8(q), gpu_util.scale_np(s, mode), mode,
+                               oracle.IO_FP16)
