@@ -6,7 +6,9 @@
 #include <cstdint>
 #include <cstring>
 #include <algorithm>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "fusednorm.h"
 #include "qk_kernel.cuh"
@@ -140,6 +142,36 @@ constexpr int kTmaMaxStages = 8;
 // (120 -> 128 us with any distance), so it does not prefetch.
 constexpr int kRowPrefetchSms = 2;
 constexpr int kTmaStaticSmem = 2 * 2 * 16 * 8 + 8 * 4;  // reduction slots and stage tags
+
+// Fewest resident warps per SM the one-block-per-row kernel should run with
+// before its row is split more finely.  Measured on B200 (sustained, power
+// capped): MXFP4 H=7168 P=4 at 224 threads x 4 vectors (114 registers, 2
+// blocks = 14 warps per SM) 118.4 us; at 448 x 2 (28 warps) 115.5 us even at a
+// 70 MHz lower SM clock.  Group-128 H=8192 P=1 already runs 32 warps at 256 x 4
+// (297.2 us) and loses at 512 x 2 (310.6 us): more warps only pay below ~16.
+constexpr int kMinRowWarps = 16;
+
+// Resident warps per SM of `k` at `threads` per block (-1 if the runtime
+// cannot tell), cached per (kernel, block size).
+int resident_warps(RQKernel k, int threads) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> cache;
+  const auto key = std::make_pair(reinterpret_cast<const void*>(k), threads);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  int blocks = 0;
+  int w = -1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, k, threads, 0) == cudaSuccess)
+    w = blocks * (threads / 32);
+  else
+    (void)cudaGetLastError();
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = w;
+  return w;
+}
 
 // Stages of the TMA ring that fit in shared memory (0 when fewer than 2 fit).
 int tma_stages(int64_t stage_bytes, int smem_optin) {
@@ -307,12 +339,25 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, bo
     tl_launch[2] = C;
     tl_launch[3] = 1;
   } else {
-    const int V = row_vectors_per_thread(nvec);
+    int V = row_vectors_per_thread(nvec);
     p.seg = nvec;
     p.prefetch_rows = M > (int64_t)kRowPrefetchSms * sms ? kRowPrefetchSms * sms : 0;
-    const int threads = round32((nvec + V - 1) / V);
+    int threads = round32((nvec + V - 1) / V);
     RQKernel k =
         norm && threads * V == nvec ? pick_exact_kernel(mode, P, threads, V, f16) : nullptr;
+    if (k && V >= 4) {
+      // Many partials held in registers leave room for few blocks per SM:
+      // below kMinRowWarps resident warps, split the row twice as finely.
+      const int w = resident_warps(k, threads);
+      RQKernel k2 = w >= 0 && w < kMinRowWarps
+                        ? pick_exact_kernel(mode, P, 2 * threads, V / 2, f16)
+                        : nullptr;
+      if (k2 && resident_warps(k2, 2 * threads) > w) {
+        k = k2;
+        threads *= 2;
+        V /= 2;
+      }
+    }
     if (!k) k = pick_kernel(mode, P, V, false, norm, f16);
     if (!k) return FN_ERR_UNSUPPORTED;
     k<<<(unsigned)M, threads, 0, st>>>(p);

@@ -245,9 +245,11 @@ __device__ __forceinline__ float row_amax_from_pmax(float pmax, float rstd) {
 // TB > 0 marks an exact-cover instance: the block has TB threads and the row
 // is exactly TB * V vectors (H = 8 * TB * V), so every offset is a
 // compile-time constant and no access needs a bounds test.  TB = 0 reads the
-// block size and the row length at run time.
+// block size and the row length at run time.  Blocks of up to 256 threads
+// keep the whole register file per thread (255); the wide exact-cover
+// instances (TB = 448, 512) and the cluster kernel allow 512 threads.
 template <int MODE, int MAXP, int V, bool NORM, bool CL, int TB = 0, class IO = Bf16>
-__global__ void __launch_bounds__(CL ? 512 : 256)
+__global__ void __launch_bounds__((CL || TB > 256) ? 512 : 256)
     rq_kernel(const __grid_constant__ RQParams prm) {
   static_assert(TB == 0 || (!CL && NORM), "exact-cover instances are one block per row");
   __shared__ float2 red[32];

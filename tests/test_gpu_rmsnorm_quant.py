@@ -137,6 +137,17 @@ def test_dispatch(fnb):
             assert launch[2] >= 2 and launch[0] == M * launch[2]
 
 
+def test_row_split_follows_occupancy(fnb):
+    """One block per row: a row whose partials leave room for few blocks per
+    SM (MXFP4 H=7168 P=4: 224 threads x 4 vectors would give 14 warps) is
+    split twice as finely; group-128 H=8192 P=1 keeps 256 x 4."""
+    for H, P, mode, want in ((7168, 4, MX, [448, 2]), (8192, 1, G128, [256, 4]),
+                             (7168, 1, TOKEN, [224, 4])):
+        wl = synth.RowWorkload("split", M=400, H=H, P=P, mode=mode, eps=1e-6, seed=H + P)
+        _, _, variant, launch = run(fnb, wl, emit_y=False)
+        assert variant == fnb.FN_VARIANT_ROW_CTA and list(launch[1::2]) == want, launch
+
+
 def test_empty_and_rejected_calls_touch_nothing(fnb):
     w = torch.ones(256, dtype=torch.bfloat16, device="cuda")
     x = torch.ones((4, 256), dtype=torch.bfloat16, device="cuda")
