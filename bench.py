@@ -511,8 +511,13 @@ def secondary_workloads(fn, device, peak):
         n_sets = max(64, int(2 * L2_BYTES / per_call_bytes) + 1)
         n_sets = min(n_sets, 8192)
         us, eager = time_graph_calls(make, n_sets, 7, device)
-        return {"us_per_call_graph": us, "us_single_call_host_to_device": eager, "calls_per_graph": n_sets,
-                "GB_s": per_call_bytes / (us * 1e-6) / 1e9}
+        launch = list(fn.fn_last_launch())
+        # the same graph with every call a programmatic dependent of the one before
+        with fn.programmatic_launch(True):
+            us_pdl, _ = time_graph_calls(make, n_sets, 7, device)
+        return {"us_per_call_graph": us, "us_per_call_graph_programmatic": us_pdl,
+                "us_single_call_host_to_device": eager, "calls_per_graph": n_sets,
+                "GB_s": per_call_bytes / (us * 1e-6) / 1e9, "launch": launch}
 
     wl = synth.PER_TOKEN_SMALL
     r = small(wl, wl.bytes_per_call(), decode_calls(fn, wl, device))

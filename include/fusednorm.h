@@ -206,6 +206,17 @@ FN_API int fn_qk_norm_gate_fp8(const void* qkv, int64_t M, int64_t row_stride, i
 /* Static, NUL-terminated description of a status code. */
 FN_API const char* fn_status_string(int status);
 
+/* Thread-local launch mode for the calling thread's later calls (every entry
+ * point): on != 0 launches each kernel as a programmatic dependent of the
+ * work before it on its stream (CUDA programmatic dependent launch, sm_90
+ * and later), so its blocks may be scheduled while the previous kernel
+ * drains; every kernel of this library first waits, on the device, until the
+ * grids it depends on have completed and their writes are visible, so results
+ * are those of ordinary stream order.  Works inside CUDA graph capture.
+ * Default 0.  Returns the previous setting.  (A launch-latency measure for
+ * decode-sized calls; the pages describe no counterpart.) */
+FN_API int fn_programmatic_launch(int on);
+
 /* fn_variant of the calling thread's last call (FN_VARIANT_NONE after an error). */
 FN_API int fn_last_variant(void);
 

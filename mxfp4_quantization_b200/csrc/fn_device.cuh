@@ -6,6 +6,17 @@
 
 namespace fn {
 
+// ---- launch ordering --------------------------------------------------------------
+
+// First statement of every kernel.  Programmatic dependent launch: wait until
+// the grids this one depends on have completed and their writes are visible
+// (at once for an ordinary launch), then allow the next grid on the stream to
+// start launching its blocks (which wait the same way before touching memory).
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- memory -----------------------------------------------------------------
 
 // Read-only input that no output aliases: non-coherent path, no L1 allocation

@@ -20,6 +20,7 @@ thread_local int tl_variant = FN_VARIANT_NONE;
 thread_local int32_t tl_launch[4] = {0, 0, 0, 0};
 thread_local int tl_prefer = FN_VARIANT_NONE;
 thread_local int tl_stall_copies = 0;
+thread_local int tl_pdl = 0;  // launch as a programmatic dependent (fn_programmatic_launch)
 
 }  // namespace
 
@@ -143,6 +144,42 @@ constexpr int kTmaMaxStages = 8;
 constexpr int kRowPrefetchSms = 2;
 constexpr int kTmaStaticSmem = 2 * 2 * 16 * 8 + 8 * 4;  // reduction slots and stage tags
 
+// Launch `k(args...)` on `st`: with a cluster dimension when `cluster` > 1,
+// and, when the calling thread asked for it (fn_programmatic_launch), as a
+// programmatic dependent of the work before it on the stream.  Every kernel
+// starts by waiting for the grids it depends on (griddepcontrol.wait), so the
+// dependent launch only lets its blocks be scheduled early.
+template <typename... KArgs, typename... Args>
+int launch_kernel(void (*k)(KArgs...), unsigned grid, unsigned threads, size_t smem,
+                  cudaStream_t st, int cluster, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = (unsigned)cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (tl_pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = (unsigned)n;
+  if (cudaLaunchKernelEx(&cfg, k, args...) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return FN_ERR_CUDA;
+  }
+  return FN_OK;
+}
+
 // Fewest resident warps per SM the one-block-per-row kernel should run with
 // before its row is split more finely.  Measured on B200 (sustained, power
 // capped): MXFP4 H=7168 P=4 at 224 threads x 4 vectors (114 registers, 2
@@ -171,6 +208,31 @@ int resident_warps(RQKernel k, int threads) {
   std::lock_guard<std::mutex> lock(mu);
   cache[key] = w;
   return w;
+}
+
+// The block for a decode-sized launch (M at most one row per SM): the fewest
+// vectors per thread V <= 4 with at most 512 threads per row, taken from an
+// exact-cover instance or, up to 256 threads, the generic one.  Each thread's
+// chain of dependent steps is then shortest, with no cluster barrier.
+// Measured on B200 (CUDA graph, cold inputs, programmatic launch), H=7168:
+// MXFP4 M=1/16 2.33/2.51 us at 448 x 2 against 2.94/3.31 us for an 8-block
+// cluster and 2.60/2.80 us at 224 x 4; group-128 2.77/2.94 against
+// 3.16/3.54 and 3.31/3.52; per-token 2.32/2.50 against 2.95/3.34 and
+// 2.30/2.51; H=2048 M=16 per-token 2.01 us at 256 x 1 against 3.06 us.
+// nullptr when no such block exists (the cluster kernel is used).
+RQKernel wide_row_block(int mode, int P, int nvec, bool f16, int* T, int* V) {
+  for (int v = 1; v <= 4; v *= 2) {
+    const int t = round32((nvec + v - 1) / v);
+    if (t > 512) continue;
+    RQKernel k = t * v == nvec ? pick_exact_kernel(mode, P, t, v, f16) : nullptr;
+    if (!k && t <= 256) k = pick_kernel(mode, P, v, false, true, f16);
+    if (k) {
+      *T = t;
+      *V = v;
+      return k;
+    }
+  }
+  return nullptr;
 }
 
 // Stages of the TMA ring that fit in shared memory (0 when fewer than 2 fit).
@@ -275,7 +337,12 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, bo
   if (!device_facts(&dev, &p.status, &smem_optin)) return FN_ERR_CUDA;
 
   const int pref = tl_prefer;
-  int C = norm ? pick_cluster(M, nvec, mode, sms) : 0;
+  // Decode-sized M: one wide block per row when one fits (see wide_row_block).
+  int wide_T = 0, wide_V = 0;
+  RQKernel wide_k = nullptr;
+  if (norm && M <= sms && pref != FN_VARIANT_ROW_CLUSTER && pref != FN_VARIANT_ROW_TMA)
+    wide_k = wide_row_block(mode, P, nvec, f16, &wide_T, &wide_V);
+  int C = norm && !wide_k ? pick_cluster(M, nvec, mode, sms) : 0;
   if (pref == FN_VARIANT_ROW_CTA || pref == FN_VARIANT_ROW_TMA) C = 0;
 
   const int ntensor = P + (prm.residual ? 1 : 0);
@@ -305,8 +372,8 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, bo
     p.seg = nvec;
     p.debug_extra_tx = tl_stall_copies ? 16u : 0u;
     p.prefetch_rows = 0;
-    k<<<(unsigned)grid, threads, smem, st>>>(p, nst, groups);
-    if (cudaGetLastError() != cudaSuccess) return FN_ERR_CUDA;
+    if (launch_kernel(k, (unsigned)grid, (unsigned)threads, smem, st, 1, p, nst, groups) != FN_OK)
+      return FN_ERR_CUDA;
     tl_variant = FN_VARIANT_ROW_TMA;
     tl_launch[0] = (int32_t)grid;
     tl_launch[1] = threads;
@@ -317,35 +384,21 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, bo
     const int threads = round32(p.seg);
     RQKernel k = pick_kernel(mode, P, 1, true, true, f16);
     if (!k) return FN_ERR_UNSUPPORTED;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(M * C));
-    cfg.blockDim = dim3((unsigned)threads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, k, p) != cudaSuccess) {
-      (void)cudaGetLastError();
+    if (launch_kernel(k, (unsigned)(M * C), (unsigned)threads, 0, st, C, p) != FN_OK)
       return FN_ERR_CUDA;
-    }
     tl_variant = FN_VARIANT_ROW_CLUSTER;
     tl_launch[0] = (int32_t)(M * C);
     tl_launch[1] = threads;
     tl_launch[2] = C;
     tl_launch[3] = 1;
   } else {
-    int V = row_vectors_per_thread(nvec);
+    int V = wide_k ? wide_V : row_vectors_per_thread(nvec);
     p.seg = nvec;
     p.prefetch_rows = M > (int64_t)kRowPrefetchSms * sms ? kRowPrefetchSms * sms : 0;
-    int threads = round32((nvec + V - 1) / V);
-    RQKernel k =
-        norm && threads * V == nvec ? pick_exact_kernel(mode, P, threads, V, f16) : nullptr;
-    if (k && V >= 4) {
+    int threads = wide_k ? wide_T : round32((nvec + V - 1) / V);
+    RQKernel k = wide_k;
+    if (!k && norm && threads * V == nvec) k = pick_exact_kernel(mode, P, threads, V, f16);
+    if (k && !wide_k && V >= 4) {
       // Many partials held in registers leave room for few blocks per SM:
       // below kMinRowWarps resident warps, split the row twice as finely.
       const int w = resident_warps(k, threads);
@@ -360,8 +413,8 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, bo
     }
     if (!k) k = pick_kernel(mode, P, V, false, norm, f16);
     if (!k) return FN_ERR_UNSUPPORTED;
-    k<<<(unsigned)M, threads, 0, st>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return FN_ERR_CUDA;
+    if (launch_kernel(k, (unsigned)M, (unsigned)threads, 0, st, 1, p) != FN_OK)
+      return FN_ERR_CUDA;
     tl_variant = norm ? variant_if_norm : FN_VARIANT_QUANT_ONLY;
     tl_launch[0] = (int32_t)M;
     tl_launch[1] = threads;
@@ -375,8 +428,9 @@ template <int VPL, bool FP8>
 int launch_qk_v(const fn::QKParams& p, int64_t items, int sms, cudaStream_t st) {
   const int wpb = items <= (int64_t)8 * sms ? 1 : 8;
   const int64_t blocks = (items + wpb - 1) / wpb;
-  fn::qk_kernel<VPL, FP8><<<(unsigned)blocks, wpb * 32, 0, st>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return FN_ERR_CUDA;
+  if (launch_kernel(fn::qk_kernel<VPL, FP8>, (unsigned)blocks, (unsigned)(wpb * 32), 0, st, 1,
+                    p) != FN_OK)
+    return FN_ERR_CUDA;
   tl_launch[0] = (int32_t)blocks;
   tl_launch[1] = wpb * 32;
   tl_launch[2] = 1;
@@ -487,6 +541,12 @@ int fn_prefer_variant(int variant) {
 int fn_debug_stall_copies(int on) {
   const int old = tl_stall_copies;
   tl_stall_copies = on ? 1 : 0;
+  return old;
+}
+
+int fn_programmatic_launch(int on) {
+  const int old = tl_pdl;
+  tl_pdl = on ? 1 : 0;
   return old;
 }
 

@@ -36,6 +36,7 @@ struct QKParams {
 // applied to each head vector, for an FP8 attention consumer.
 template <int VPL, bool FP8>
 __global__ void __launch_bounds__(256) qk_kernel(const __grid_constant__ QKParams p) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int heads = p.Hq + p.Hk;

@@ -52,8 +52,8 @@ RQKernel FN_CAT(rq_pick, FN_INST_MODE, FN_INST_MAXP)(int V, bool cluster, bool n
 
 // Exact-cover instances (one block of T threads per row of T * V vectors):
 // T = 224 serves H = 3584, 7168, 14336; T = 256 serves H = 4096, 8192, 16384;
-// T = 448 and 512 are the same rows split twice as finely (more warps per SM
-// when the partials leave room for few blocks).
+// T = 448 and 512 are the same rows split more finely (more warps per SM when
+// the partials leave room for few blocks; the widest block for decode-sized M).
 RQKernel FN_CAT(rq_exact_pick, FN_INST_MODE, FN_INST_MAXP)(int T, int V) {
   constexpr int MODE = FN_INST_MODE, MAXP = FN_INST_MAXP;
   using IO = std::conditional_t<FN_INST_IO == 1, F16, Bf16>;
@@ -61,7 +61,8 @@ RQKernel FN_CAT(rq_exact_pick, FN_INST_MODE, FN_INST_MAXP)(int T, int V) {
   if (T == TT && V == VV) return rq_kernel<MODE, MAXP, VV, true, false, TT, IO>;
   FN_EXACT(224, 2) FN_EXACT(224, 4) FN_EXACT(224, 8)
   FN_EXACT(256, 2) FN_EXACT(256, 4) FN_EXACT(256, 8)
-  FN_EXACT(448, 2) FN_EXACT(448, 4) FN_EXACT(512, 2) FN_EXACT(512, 4)
+  FN_EXACT(448, 1) FN_EXACT(448, 2) FN_EXACT(448, 4)
+  FN_EXACT(512, 1) FN_EXACT(512, 2) FN_EXACT(512, 4)
 #undef FN_EXACT
   return nullptr;
 }

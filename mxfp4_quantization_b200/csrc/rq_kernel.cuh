@@ -254,6 +254,7 @@ __global__ void __launch_bounds__((CL || TB > 256) ? 512 : 256)
   static_assert(TB == 0 || (!CL && NORM), "exact-cover instances are one block per row");
   __shared__ float2 red[32];
   __shared__ float2 cl_slot;
+  pdl_enter();
 
   const int T = TB ? TB : (int)blockDim.x, t = threadIdx.x, lane = t & 31;
   const int nvec = TB ? TB * V : prm.nvec;
@@ -475,6 +476,7 @@ __global__ void __launch_bounds__(512, 1)
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float2 red[2][2][16];  // [group][buffer][warp]
   __shared__ int issued[8];         // row index last issued into each stage
+  pdl_enter();
 
   const int tg = blockDim.x / groups;
   const int g = threadIdx.x / tg, t = threadIdx.x - g * tg, lane = threadIdx.x & 31;

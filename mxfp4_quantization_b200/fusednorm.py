@@ -56,7 +56,7 @@ MODES = {"fp8_per_token": FN_FP8_PER_TOKEN, "fp8_per_group128": FN_FP8_PER_GROUP
 ABI_SYMBOLS = ("fn_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate", "fn_qk_norm_gate_fp8",
                "fn_status_string",
                "fn_last_variant", "fn_last_launch", "fn_prefer_variant", "fn_device_status",
-               "fn_debug_stall_copies", "fn_version")
+               "fn_debug_stall_copies", "fn_programmatic_launch", "fn_version")
 
 
 class FusedNormError(RuntimeError):
@@ -94,6 +94,8 @@ def _load():
     lib.fn_device_status.restype = i32
     lib.fn_debug_stall_copies.argtypes = [i32]
     lib.fn_debug_stall_copies.restype = i32
+    lib.fn_programmatic_launch.argtypes = [i32]
+    lib.fn_programmatic_launch.restype = i32
     lib.fn_version.argtypes = []
     lib.fn_version.restype = i32
     return lib
@@ -164,8 +166,28 @@ def fn_debug_stall_copies(on: int) -> int:
     return _lib.fn_debug_stall_copies(on)
 
 
+def fn_programmatic_launch(on: int) -> int:
+    return _lib.fn_programmatic_launch(on)
+
+
 def fn_version() -> int:
     return _lib.fn_version()
+
+
+class programmatic_launch:
+    """Context manager: this thread's calls launch their kernels as
+    programmatic dependents of the stream's previous work (see
+    fn_programmatic_launch)."""
+
+    def __init__(self, on: bool = True):
+        self.on = on
+
+    def __enter__(self):
+        self.old = fn_programmatic_launch(1 if self.on else 0)
+        return self
+
+    def __exit__(self, *exc):
+        fn_programmatic_launch(self.old)
 
 
 class prefer_variant:

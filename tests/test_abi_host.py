@@ -32,7 +32,7 @@ def test_header_declares_the_abi():
                                          "fn_status_string", "fn_last_variant",
                                          "fn_last_launch", "fn_prefer_variant",
                                          "fn_device_status", "fn_debug_stall_copies",
-                                         "fn_version"])
+                                         "fn_programmatic_launch", "fn_version"])
 
 
 def test_library_exports_every_declared_symbol(fnb):
@@ -207,3 +207,16 @@ def test_fp16_row_flag(fnb):
         fnb.FN_ERR_INVALID
     # the same argument checks apply (here: H not a multiple of 8)
     assert rq(fnb, mode=fnb.FN_MXFP4 | F, H=12) == fnb.FN_ERR_INVALID
+
+
+def test_programmatic_launch_is_thread_local_and_returns_previous(fnb):
+    import threading
+    assert fnb.fn_programmatic_launch(1) == 0
+    seen = []
+    t = threading.Thread(target=lambda: seen.append(fnb.fn_programmatic_launch(0)))
+    t.start()
+    t.join()
+    assert seen == [0]
+    with fnb.programmatic_launch(False):
+        assert fnb.fn_programmatic_launch(0) == 0
+    assert fnb.fn_programmatic_launch(0) == 1

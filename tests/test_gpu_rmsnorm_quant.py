@@ -125,16 +125,21 @@ def test_in_place_residual(fnb, mode, variant):
 
 
 def test_dispatch(fnb):
-    """Small M takes the cluster kernel, large M one block per row."""
-    for M, P, want in ((1, 1, fnb.FN_VARIANT_ROW_CLUSTER), (16, 1, fnb.FN_VARIANT_ROW_CLUSTER),
-                       (200, 4, fnb.FN_VARIANT_ROW_CTA), (512, 1, fnb.FN_VARIANT_ROW_CTA),
-                       (512, 4, fnb.FN_VARIANT_ROW_CTA)):
-        wl = synth.decode(M, MX) if M <= 16 else synth.RowWorkload("big", M=M, H=7168, P=P,
-                                                                     mode=MX, eps=1e-6)
+    """Decode-sized M takes one wide block per row (448 threads x 2 vectors at
+    H=7168), or the cluster kernel when no block of at most 512 threads and 4
+    vectors covers the row (H=32768); large M one block per row."""
+    CTA, CL = fnb.FN_VARIANT_ROW_CTA, fnb.FN_VARIANT_ROW_CLUSTER
+    for M, H, P, want, shape in ((1, 7168, 1, CTA, [448, 2]), (16, 7168, 1, CTA, [448, 2]),
+                                 (16, 2048, 1, CTA, [256, 1]), (3, 8192, 2, CTA, [512, 2]),
+                                 (2, 32768, 1, CL, None), (200, 7168, 4, CTA, [448, 2]),
+                                 (512, 7168, 1, CTA, [224, 4]), (512, 7168, 4, CTA, [448, 2])):
+        wl = synth.RowWorkload("dispatch", M=M, H=H, P=P, mode=MX, eps=1e-6, seed=M)
         _, _, variant, launch = run(fnb, wl)
-        assert variant == want, (M, variant, launch)
-        if want == fnb.FN_VARIANT_ROW_CLUSTER:
+        assert variant == want, (M, H, variant, launch)
+        if want == CL:
             assert launch[2] >= 2 and launch[0] == M * launch[2]
+        else:
+            assert list(launch[1::2]) == shape, (M, H, launch)
 
 
 def test_row_split_follows_occupancy(fnb):
@@ -260,12 +265,16 @@ def test_per_token_small_config(fnb):
     check(wl, inp, gpu)
 
 
+@pytest.mark.parametrize("variant", ["auto", "cluster"])
 @pytest.mark.parametrize("M", synth.DECODE_M)
 @pytest.mark.parametrize("mode", [TOKEN, G128, MX])
-def test_decode_sweep_config(fnb, M, mode):
+def test_decode_sweep_config(fnb, M, mode, variant):
+    """The decode sweep: the library's choice (one 448-thread block per row)
+    and the cluster kernel on the same rows."""
     wl = synth.decode(M, mode)
-    inp, gpu, variant, _ = run(fnb, wl)
-    assert variant == fnb.FN_VARIANT_ROW_CLUSTER
+    inp, gpu, got, launch = run(fnb, wl, variant=VARIANTS[variant])
+    want = fnb.FN_VARIANT_ROW_CTA if variant == "auto" else fnb.FN_VARIANT_ROW_CLUSTER
+    assert got == want, launch
     check(wl, inp, gpu)
 
 
@@ -363,3 +372,45 @@ def test_fp16_quant_only_full_range(fnb, mode):
     torch.cuda.synchronize()
     parity.compare_quant_stage(bits, gpu_util.u8(q), gpu_util.scale_np(s, mode), mode,
                                oracle.IO_FP16)
+
+
+@pytest.mark.parametrize("M,H,P,mode", [(4, 7168, 1, MX), (16, 2048, 2, TOKEN), (700, 8192, 1, G128),
+                                        (300, 7168, 4, MX)])
+@pytest.mark.parametrize("graph", [False, True])
+def test_programmatic_launch_chain(fnb, M, H, P, mode, graph):
+    """Twelve in-place calls, each reading the residual the previous one wrote,
+    launched as programmatic dependents (eagerly or from a CUDA graph), give
+    the same bits as the same chain in ordinary stream order."""
+    wl = synth.RowWorkload("pdl", M=M, H=H, P=P, mode=mode, eps=1e-6, seed=M + H)
+    inp = wl.inputs(device="cuda")
+
+    def chain(pdl):
+        res = inp["residual"].clone()
+        outs = []
+
+        def body():
+            for _ in range(12):
+                o = fnb.rmsnorm_quant(inp["parts"], inp["weight"], wl.eps, mode, residual=res,
+                                      in_place=True)
+                outs.append((o.q, o.scale))
+
+        with fnb.programmatic_launch(pdl):
+            if graph:
+                s = torch.cuda.Stream()
+                s.wait_stream(torch.cuda.current_stream())
+                with torch.cuda.stream(s):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=s):
+                        body()
+                g.replay()
+            else:
+                body()
+        torch.cuda.synchronize()
+        return res, outs
+
+    r0, o0 = chain(False)
+    r1, o1 = chain(True)
+    assert torch.equal(r0.view(torch.int16), r1.view(torch.int16))
+    for (q0, s0), (q1, s1) in zip(o0, o1):
+        assert torch.equal(q0.view(torch.uint8), q1.view(torch.uint8))
+        assert torch.equal(s0.view(torch.uint8), s1.view(torch.uint8))
