@@ -80,7 +80,8 @@ typedef enum {
     FN_VARIANT_QUANT_ONLY = 3,  /* fn_quant                                        */
     FN_VARIANT_QK_WARP = 4,     /* fn_qk_norm_gate: one warp per (token, head)     */
     FN_VARIANT_ROW_TMA = 5,     /* persistent blocks, rows staged by bulk copies  */
-    FN_VARIANT_QK_WARP_FP8 = 6  /* fn_qk_norm_gate_fp8                             */
+    FN_VARIANT_QK_WARP_FP8 = 6, /* fn_qk_norm_gate_fp8                             */
+    FN_VARIANT_ROW_ALLREDUCE = 7 /* fn_ar_rmsnorm_quant: one block per row of the shard */
 } fn_variant;
 
 /* Scale-layout flags, OR-ed into `mode` (fn_rmsnorm_quant, fn_quant).  No
@@ -154,6 +155,45 @@ FN_API int fn_rmsnorm_quant(const void* const* x_parts, int num_parts, const voi
                      const void* weight, float eps, int mode, int64_t M, int64_t H,
                      void* out_q, void* out_scale, void* out_residual, void* out_y,
                      void* stream);
+
+/*
+ * Fused all-reduce + residual add + RMSNorm + quantization across the
+ * num_ranks ranks of a tensor-parallel group (sglang PR #29723, "Motivation"
+ * and "Modifications": the AllReduce -> RMSNorm -> quantize sequence in one
+ * kernel), two-stage form, one call per rank.  Rank `rank` computes the rows
+ * [M*rank/num_ranks, M*(rank+1)/num_ranks) exactly as fn_rmsnorm_quant with
+ * P = num_ranks partials would (partials summed in rank order, then the
+ * residual), reading each row from every rank's partial buffer, and writes the
+ * results into every rank's output buffers: the reduce-scatter and the
+ * all-gather of the tuple are the kernel's own peer loads and stores.  After
+ * all ranks' calls every rank holds the same outputs for all M rows.
+ * (The one-stage form — each rank computes all rows from all partials and
+ * writes only its own outputs — is fn_rmsnorm_quant given the peer partials.)
+ *
+ * x_parts      HOST array of num_ranks pointers: rank p's partial bf16 [M, H]
+ *              (this rank's own, and peer-mapped memory of the others).
+ * num_ranks    2..8.  rank: 0..num_ranks-1.
+ * residual     this rank's residual replica bf16 [M, H], or NULL.
+ * weight, eps, mode, M, H   as fn_rmsnorm_quant (FN_IO_FP16 is not
+ *              supported here: FN_ERR_UNSUPPORTED).
+ * out_q, out_scale   HOST arrays of num_ranks pointers: rank d's code and
+ *              scale buffers for all M rows (layouts as fn_rmsnorm_quant).
+ * out_residual HOST array of num_ranks pointers to every rank's residual_out
+ *              [M, H] (required when residual != NULL; entry `rank` may be
+ *              `residual` itself, in place), or NULL.
+ * out_y        HOST array of num_ranks bf16 [M, H] pointers, or NULL.
+ * Ordering     the caller orders the call between two group barriers: every
+ *              rank's partial (and residual) complete before any rank's call
+ *              starts, and every rank's call complete before any output is
+ *              read.  The kernel itself never waits on another rank.
+ * Errors       argument checks as fn_rmsnorm_quant, applied to every rank's
+ *              pointers, all before launch; an empty shard returns FN_OK with
+ *              nothing launched.  H above 16384 is FN_ERR_UNSUPPORTED here.
+ */
+FN_API int fn_ar_rmsnorm_quant(const void* const* x_parts, int num_ranks, int rank,
+                               const void* residual, const void* weight, float eps, int mode,
+                               int64_t M, int64_t H, void* const* out_q, void* const* out_scale,
+                               void* const* out_residual, void* const* out_y, void* stream);
 
 /*
  * The quantization step alone on existing bf16 (or, with FN_IO_FP16,

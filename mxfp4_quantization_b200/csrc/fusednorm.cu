@@ -11,6 +11,7 @@
 #include <utility>
 
 #include "fusednorm.h"
+#include "ar_kernel.cuh"
 #include "qk_kernel.cuh"
 #include "rq_params.h"
 
@@ -644,6 +645,106 @@ int fn_rmsnorm_quant(const void* const* x_parts, int num_parts, const void* resi
   prm.scale_layout = mi.layout;
   prm.scale_ld = scale_ld(mi, M, H);
   return launch_rq(prm, mi.q, num_parts, M, true, mi.f16, stream, FN_VARIANT_ROW_CTA);
+}
+
+int fn_ar_rmsnorm_quant(const void* const* x_parts, int num_ranks, int rank, const void* residual,
+                        const void* weight, float eps, int mode, int64_t M, int64_t H,
+                        void* const* out_q, void* const* out_scale, void* const* out_residual,
+                        void* const* out_y, void* stream) {
+  tl_variant = FN_VARIANT_NONE;
+  if (!x_parts || num_ranks < 2 || num_ranks > fn::kMaxRanks || rank < 0 || rank >= num_ranks)
+    return FN_ERR_INVALID;
+  ModeInfo mi;
+  int rc = parse_mode(mode, &mi);
+  if (rc != FN_OK) return rc;
+  if (mi.f16) return FN_ERR_UNSUPPORTED;  // bf16 rows only
+  if ((rc = check_mode_shape(mi, M, H)) != FN_OK) return rc;
+  if (!std::isfinite(eps) || eps < 0.f) return FN_ERR_INVALID;
+  const int64_t row0 = M * rank / num_ranks, row1 = M * (rank + 1) / num_ranks;
+  if (row1 == row0) return FN_OK;  // an empty shard: nothing to read or write
+  if (!weight || !out_q || !out_scale || (residual && !out_residual)) return FN_ERR_INVALID;
+  const int n = num_ranks;
+  for (int d = 0; d < n; ++d) {
+    if (!x_parts[d] || !out_q[d] || !out_scale[d]) return FN_ERR_INVALID;
+    if ((out_residual && !out_residual[d]) || (out_y && !out_y[d])) return FN_ERR_INVALID;
+    if (!aligned(x_parts[d], 16) || (out_residual && !aligned(out_residual[d], 16)) ||
+        (out_y && !aligned(out_y[d], 16)))
+      return FN_ERR_ALIGN;
+    if ((rc = check_outputs_align(mi, out_q[d], out_scale[d])) != FN_OK) return rc;
+  }
+  if (!aligned(weight, 16) || (residual && !aligned(residual, 16))) return FN_ERR_ALIGN;
+
+  // Outputs (every rank's) must not overlap one another or any input; the one
+  // exception is this rank's residual_out on its own residual (in place).
+  const int64_t row_bytes = M * H * 2;
+  Range outs[4 * fn::kMaxRanks];
+  int own_res = -1, no = 0;
+  for (int d = 0; d < n; ++d) {
+    outs[no++] = range_of(out_q[d], code_bytes(mi, M, H));
+    outs[no++] = range_of(out_scale[d], scale_bytes(mi, M, H));
+    if (out_residual) {
+      if (d == rank) own_res = no;
+      outs[no++] = range_of(out_residual[d], row_bytes);
+    }
+    if (out_y) outs[no++] = range_of(out_y[d], row_bytes);
+  }
+  Range ins[fn::kMaxRanks + 1];
+  int ni = 0;
+  for (int d = 0; d < n; ++d) ins[ni++] = range_of(x_parts[d], row_bytes);
+  ins[ni++] = range_of(weight, H * 2);
+  const Range res_in = residual ? range_of(residual, row_bytes) : Range{0, 0};
+  for (int i = 0; i < no; ++i) {
+    for (int j = i + 1; j < no; ++j)
+      if (overlap(outs[i], outs[j])) return FN_ERR_INVALID;
+    for (int j = 0; j < ni; ++j)
+      if (overlap(outs[i], ins[j])) return FN_ERR_INVALID;
+    if (residual && overlap(outs[i], res_in) && !(i == own_res && out_residual[rank] == residual))
+      return FN_ERR_INVALID;
+  }
+
+  const int sms = sm_count();
+  if (sms <= 0) return FN_ERR_CUDA;
+  int dev = 0, smem_optin = 0;
+  fn::ARParams ap;
+  std::memset(&ap, 0, sizeof ap);
+  if (!device_facts(&dev, &ap.rq.status, &smem_optin)) return FN_ERR_CUDA;
+  fn::RQParams& prm = ap.rq;
+  for (int d = 0; d < n; ++d) prm.parts[d] = static_cast<const uint4*>(x_parts[d]);
+  prm.residual = static_cast<const uint4*>(residual);
+  prm.weight = static_cast<const uint4*>(weight);
+  prm.M = M;
+  prm.nvec = (int)(H / 8);
+  prm.seg = prm.nvec;
+  prm.P = n;
+  prm.eps = eps;
+  prm.inv_h = 1.0f / (float)H;
+  prm.scale_layout = mi.layout;
+  prm.scale_ld = scale_ld(mi, M, H);
+  ap.row0 = row0;
+  ap.ndst = n;
+  for (int d = 0; d < n; ++d) {
+    ap.out_q[d] = static_cast<uint8_t*>(out_q[d]);
+    ap.out_scale[d] = out_scale[d];
+    ap.out_residual[d] = out_residual ? static_cast<uint4*>(out_residual[d]) : nullptr;
+    ap.out_y[d] = out_y ? static_cast<uint4*>(out_y[d]) : nullptr;
+  }
+  const int V = vectors_per_thread(prm.nvec, 256, 8);
+  const int threads = round32((prm.nvec + V - 1) / V);
+  if (threads > 256) return FN_ERR_UNSUPPORTED;
+  const int maxp = n == 2 ? 2 : n <= 4 ? 4 : 8;
+  fn::RQArKernel k = mi.q == FN_FP8_PER_TOKEN      ? fn::rq_ar_pick_0(maxp, V)
+                     : mi.q == FN_FP8_PER_GROUP128 ? fn::rq_ar_pick_1(maxp, V)
+                                                   : fn::rq_ar_pick_2(maxp, V);
+  if (!k) return FN_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (launch_kernel(k, (unsigned)(row1 - row0), (unsigned)threads, 0, st, 1, ap) != FN_OK)
+    return FN_ERR_CUDA;
+  tl_variant = FN_VARIANT_ROW_ALLREDUCE;
+  tl_launch[0] = (int32_t)(row1 - row0);
+  tl_launch[1] = threads;
+  tl_launch[2] = 1;
+  tl_launch[3] = V;
+  return FN_OK;
 }
 
 int fn_quant(const void* y, int mode, int64_t M, int64_t H, void* out_q, void* out_scale,

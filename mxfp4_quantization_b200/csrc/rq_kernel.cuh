@@ -144,34 +144,58 @@ __device__ __forceinline__ int64_t scale_index(int layout, int64_t ld, int64_t r
   return row * groups_per_row + g;
 }
 
-// Quantize vector v of a row (y: 8 bf16) and store its codes and, from the
-// group's first lane, its scale.  All 32 lanes must call (shuffles); `ok`
-// masks the stores of lanes past the row end (whole groups, by alignment).
-// `tok` is the row's scale (per-token mode).
+// Codes of one vector (y: 8 values) and, for the group modes, its group's
+// scale.  All 32 lanes must call (shuffles).  `tok` is the row's scale
+// (per-token mode).
+struct QuantVec {
+  uint2 q8;     // FP8: eight E4M3 codes
+  uint32_t q4;  // MXFP4: eight E2M1 codes
+  float s;      // group-128: the group's fp32 scale
+  uint32_t e8;  // MXFP4: the block's E8M0 code
+};
+
+template <int MODE, class IO = Bf16>
+__device__ __forceinline__ QuantVec quant_vec(const uint4& y, const Fp8Scale& tok) {
+  QuantVec r;
+  if constexpr (MODE == MODE_TOKEN || MODE == MODE_G128) {
+    Fp8Scale c = tok;
+    if constexpr (MODE == MODE_G128) c = fp8_scale_direct(group_max<16>(vec_absmax<IO>(y)));
+    r.s = c.s;
+    r.q8 = e4m3_codes<IO>(y, c);
+  } else {
+    float inv;
+    r.e8 = mx_scale(group_max<4>(vec_absmax<IO>(y)), inv);
+    r.q4 = e2m1_codes<IO>(y, inv);
+  }
+  return r;
+}
+
+// Store the codes of vector v of a row and, from the group's first lane, its
+// scale; `ok` masks lanes past the row end (whole groups, by alignment).
+template <int MODE>
+__device__ __forceinline__ void store_quant(const QuantVec& r, bool ok, int lane, int64_t row,
+                                            int v, int H, uint8_t* out_q, void* out_scale,
+                                            int layout, int64_t ld) {
+  if (!ok) return;
+  if constexpr (MODE == MODE_TOKEN || MODE == MODE_G128) {
+    if (MODE == MODE_G128 && (lane & 15) == 0)
+      static_cast<float*>(out_scale)[scale_index(layout, ld, row, v / 16, H / 128)] = r.s;
+    st_stream(reinterpret_cast<uint2*>(out_q + row * (int64_t)H) + v, r.q8);
+  } else {
+    st_stream(reinterpret_cast<uint32_t*>(out_q + row * (int64_t)(H / 2)) + v, r.q4);
+    if ((lane & 3) == 0)
+      static_cast<uint8_t*>(out_scale)[scale_index(layout, ld, row, v / 4, H / 32)] =
+          (uint8_t)r.e8;
+  }
+}
+
+// Quantize vector v of a row and store it (quant_vec, then store_quant).
 template <int MODE, class IO = Bf16>
 __device__ __forceinline__ void quant_store(const uint4& y, bool ok, int lane, int64_t row, int v,
                                             int H, const Fp8Scale& tok, uint8_t* out_q,
                                             void* out_scale, int layout, int64_t ld) {
-  if constexpr (MODE == MODE_TOKEN || MODE == MODE_G128) {
-    Fp8Scale c = tok;
-    if constexpr (MODE == MODE_G128) {
-      c = fp8_scale_direct(group_max<16>(vec_absmax<IO>(y)));
-      if (ok && (lane & 15) == 0)
-        static_cast<float*>(out_scale)[scale_index(layout, ld, row, v / 16, H / 128)] = c.s;
-    }
-    const uint2 q = e4m3_codes<IO>(y, c);
-    if (ok) st_stream(reinterpret_cast<uint2*>(out_q + row * (int64_t)H) + v, q);
-  } else {
-    float inv;
-    const uint32_t code = mx_scale(group_max<4>(vec_absmax<IO>(y)), inv);
-    const uint32_t q = e2m1_codes<IO>(y, inv);
-    if (ok) {
-      st_stream(reinterpret_cast<uint32_t*>(out_q + row * (int64_t)(H / 2)) + v, q);
-      if ((lane & 3) == 0)
-        static_cast<uint8_t*>(out_scale)[scale_index(layout, ld, row, v / 4, H / 32)] =
-            (uint8_t)code;
-    }
-  }
+  store_quant<MODE>(quant_vec<MODE, IO>(y, tok), ok, lane, row, v, H, out_q, out_scale, layout,
+                    ld);
 }
 
 // ---------------------------------------------------------------------------

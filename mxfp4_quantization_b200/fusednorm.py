@@ -39,6 +39,7 @@ FN_VARIANT_QUANT_ONLY = 3
 FN_VARIANT_QK_WARP = 4
 FN_VARIANT_ROW_TMA = 5
 FN_VARIANT_QK_WARP_FP8 = 6
+FN_VARIANT_ROW_ALLREDUCE = 7
 
 FN_MODE_MASK = 0xFF
 FN_SCALE_SWIZZLE_32_4_4 = 0x100
@@ -53,7 +54,8 @@ MODES = {"fp8_per_token": FN_FP8_PER_TOKEN, "fp8_per_group128": FN_FP8_PER_GROUP
          "mxfp4": FN_MXFP4}
 
 # The exported symbols of include/fusednorm.h.
-ABI_SYMBOLS = ("fn_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate", "fn_qk_norm_gate_fp8",
+ABI_SYMBOLS = ("fn_rmsnorm_quant", "fn_ar_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate",
+               "fn_qk_norm_gate_fp8",
                "fn_status_string",
                "fn_last_variant", "fn_last_launch", "fn_prefer_variant", "fn_device_status",
                "fn_debug_stall_copies", "fn_programmatic_launch", "fn_version")
@@ -74,6 +76,10 @@ def _load():
     lib.fn_rmsnorm_quant.argtypes = [ctypes.POINTER(vp), i32, vp, vp, ctypes.c_float, i32, i64,
                                      i64, vp, vp, vp, vp, vp]
     lib.fn_rmsnorm_quant.restype = i32
+    pvp = ctypes.POINTER(vp)
+    lib.fn_ar_rmsnorm_quant.argtypes = [pvp, i32, i32, vp, vp, ctypes.c_float, i32, i64, i64,
+                                        pvp, pvp, pvp, pvp, vp]
+    lib.fn_ar_rmsnorm_quant.restype = i32
     lib.fn_quant.argtypes = [vp, i32, i64, i64, vp, vp, vp]
     lib.fn_quant.restype = i32
     lib.fn_qk_norm_gate.argtypes = [vp, i64, i64, i32, i32, i32, vp, vp, ctypes.c_float, vp, vp,
@@ -114,6 +120,20 @@ def fn_rmsnorm_quant(x_parts: Sequence[int], num_parts: int, residual: Optional[
     arr = (ctypes.c_void_p * max(1, len(x_parts)))(*x_parts)
     return _lib.fn_rmsnorm_quant(arr, num_parts, residual, weight, eps, mode, M, H, out_q,
                                  out_scale, out_residual, out_y, stream)
+
+
+def _ptr_array(ptrs: Optional[Sequence[int]]):
+    return None if ptrs is None else (ctypes.c_void_p * max(1, len(ptrs)))(*ptrs)
+
+
+def fn_ar_rmsnorm_quant(x_parts: Sequence[int], num_ranks: int, rank: int,
+                        residual: Optional[int], weight: int, eps: float, mode: int, M: int,
+                        H: int, out_q: Sequence[int], out_scale: Sequence[int],
+                        out_residual: Optional[Sequence[int]], out_y: Optional[Sequence[int]],
+                        stream: Optional[int]) -> int:
+    return _lib.fn_ar_rmsnorm_quant(_ptr_array(x_parts), num_ranks, rank, residual, weight, eps,
+                                    mode, M, H, _ptr_array(out_q), _ptr_array(out_scale),
+                                    _ptr_array(out_residual), _ptr_array(out_y), stream)
 
 
 def fn_quant(y: int, mode: int, M: int, H: int, out_q: int, out_scale: int,

@@ -27,7 +27,8 @@ def declared_symbols():
 
 
 def test_header_declares_the_abi():
-    assert declared_symbols() == sorted(["fn_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate",
+    assert declared_symbols() == sorted(["fn_rmsnorm_quant", "fn_ar_rmsnorm_quant", "fn_quant",
+                                         "fn_qk_norm_gate",
                                          "fn_qk_norm_gate_fp8",
                                          "fn_status_string", "fn_last_variant",
                                          "fn_last_launch", "fn_prefer_variant",
@@ -51,7 +52,8 @@ def test_header_constants_match_binding(fnb):
     for name in ("FN_FP8_PER_TOKEN", "FN_FP8_PER_GROUP128", "FN_MXFP4", "FN_ERR_INVALID",
                  "FN_ERR_ALIGN", "FN_ERR_UNSUPPORTED", "FN_ERR_CUDA", "FN_VARIANT_ROW_CTA",
                  "FN_VARIANT_ROW_CLUSTER", "FN_VARIANT_QUANT_ONLY", "FN_VARIANT_QK_WARP",
-                 "FN_VARIANT_ROW_TMA", "FN_VARIANT_QK_WARP_FP8", "FN_ERR_TIMEOUT"):
+                 "FN_VARIANT_ROW_TMA", "FN_VARIANT_QK_WARP_FP8", "FN_VARIANT_ROW_ALLREDUCE",
+                 "FN_ERR_TIMEOUT"):
         m = re.search(rf"\b{name}\s*=\s*(-?\d+)", src)
         assert m and int(m.group(1)) == getattr(fnb, name), name
     for name in ("FN_MAX_PARTS", "FN_MAX_H", "FN_MAX_HEAD_DIM"):
@@ -220,3 +222,47 @@ def test_programmatic_launch_is_thread_local_and_returns_previous(fnb):
     with fnb.programmatic_launch(False):
         assert fnb.fn_programmatic_launch(0) == 0
     assert fnb.fn_programmatic_launch(0) == 1
+
+
+def ar(fnb, n=2, rank=0, **kw):
+    """fn_ar_rmsnorm_quant on fake, disjoint addresses (rank d's buffers at
+    BASE + d << 40); a rejected call never touches them."""
+    a = dict(x_parts=[BASE + (d << 40) for d in range(n)], num_ranks=n, rank=rank,
+             residual=BASE + (1 << 32), weight=BASE + (2 << 32), eps=1e-6, mode=2, M=4, H=256,
+             out_q=[BASE + (d << 40) + (3 << 32) for d in range(n)],
+             out_scale=[BASE + (d << 40) + (4 << 32) for d in range(n)],
+             out_residual=[BASE + (d << 40) + (5 << 32) for d in range(n)], out_y=None,
+             stream=None)
+    a.update(kw)
+    return fnb.fn_ar_rmsnorm_quant(a["x_parts"], a["num_ranks"], a["rank"], a["residual"],
+                                   a["weight"], a["eps"], a["mode"], a["M"], a["H"], a["out_q"],
+                                   a["out_scale"], a["out_residual"], a["out_y"], a["stream"])
+
+
+def test_allreduce_rejects_bad_arguments(fnb):
+    E, A, U = fnb.FN_ERR_INVALID, fnb.FN_ERR_ALIGN, fnb.FN_ERR_UNSUPPORTED
+    for kw, want in [
+        (dict(n=1), E), (dict(n=9), E), (dict(rank=2), E), (dict(rank=-1), E),
+        (dict(mode=3), E), (dict(H=12), E), (dict(mode=1, H=192), E), (dict(eps=-1.0), E),
+        (dict(mode=2 | fnb.FN_IO_FP16), U), (dict(weight=None), E),
+        (dict(out_residual=None), E),  # a residual needs residual_out on every rank
+        (dict(x_parts=[BASE, None]), E), (dict(x_parts=[BASE, BASE + 8]), A),
+        (dict(out_q=[BASE + (3 << 32), BASE + (3 << 32)]), E),  # two ranks' codes overlap
+        (dict(out_q=[BASE + (3 << 32) + 2, BASE + (1 << 40) + (3 << 32)]), A),
+        # another rank's residual_out on this rank's residual: only the own entry may alias
+        (dict(out_residual=[BASE + (5 << 32), BASE + (1 << 32)]), E),
+        (dict(out_q=[BASE, BASE + (1 << 40) + (3 << 32)]), E),  # codes over a partial
+    ]:
+        n = kw.pop("n", 2)
+        assert ar(fnb, n=n, **kw) == want, (kw, n)
+    assert fnb.fn_last_variant() == fnb.FN_VARIANT_NONE
+
+
+def test_allreduce_empty_shard_and_in_place(fnb):
+    # M=1 over 2 ranks: rank 0's shard is empty, nothing is launched
+    assert ar(fnb, rank=0, M=1) == fnb.FN_OK
+    assert ar(fnb, M=0) == fnb.FN_OK
+    # in place on the own replica passes every check and reaches the launch,
+    # which fails here for want of a device
+    assert ar(fnb, out_residual=[BASE + (1 << 32), BASE + (1 << 40) + (5 << 32)]) == \
+        fnb.FN_ERR_CUDA
