@@ -8,28 +8,49 @@ namespace fn {
 // FP8 scale of a group (or row) and the reciprocal pair the codes use.
 struct Fp8Scale {
   float s;         // RN(amax / 448), 1 for an all-zero group
-  float r, r_lo;   // RN(1/s), RN(RN(1 - s r) r)
+  float r, r_lo;   // 1/s within one ulp of RN(1/s); RN(RN(1 - s r) r)
   bool exact_div;  // the fast quotient is not proven here: use the IEEE division
 };
 
-// The formulas themselves (IEEE division and reciprocal).
+// RN(amax / 448) without a division: the product with c = RN(1/448),
+// corrected by its exact FMA remainder (Markstein's method).  Equal to the
+// IEEE quotient for every bf16 and every binary16 amax, subnormals included
+// (checked exhaustively by tests/quotient_proof.c).
+__device__ __forceinline__ float scale_div448(float amax) {
+  constexpr float c = 1.0f / 448.0f;
+  const float q0 = __fmul_rn(amax, c);
+  const float rem = fmaf(-448.0f, q0, amax);
+  return fmaf(rem, c, q0);
+}
+
+// 1/s within one ulp of RN(1/s): the hardware approximation (at most one ulp
+// from 1/s) refined by one Newton-Raphson step y + y (1 - s y), which leaves a
+// relative error below 2^-46 before the final rounding.  The quotient below
+// is proven for every r within one ulp of RN(1/s).
+__device__ __forceinline__ float recip_near(float s) {
+  float y;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(y) : "f"(s));
+  return fmaf(fmaf(-s, y, 1.0f), y, y);
+}
+
+// The group's scale and the reciprocal pair of the codes.
 __device__ __forceinline__ Fp8Scale fp8_scale_direct(float amax) {
   Fp8Scale c;
-  c.s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+  c.s = amax == 0.f ? 1.f : scale_div448(amax);
   c.exact_div = !(c.s >= 0x1p-120f);
-  c.r = c.exact_div ? 1.f : __frcp_rn(c.s);
-  c.r_lo = fmaf(-c.s, c.r, 1.f) * c.r;
+  c.r = c.exact_div ? 1.f : recip_near(c.s);
+  c.r_lo = __fmul_rn(fmaf(-c.s, c.r, 1.f), c.r);
   return c;
 }
 
 // Eight E4M3 codes of fl32(y / s), the IEEE quotient.
 //
-// Fast path: with r = RN(1/s) and r_lo = RN(RN(1 - s r) r) (r + r_lo carries
-// 1/s to about 2^-46), q = RN(|y| r + RN(|y| r_lo)) has the same E4M3 code as
-// RN(|y| / s) for every bf16 y with |y| <= amax and every bf16 amax with
-// s = RN(amax / 448) >= 2^-120, and likewise for every binary16 pair (whose
-// scales are all above 2^-120): checked exhaustively over all such (amax, y)
-// pairs by tests/quotient_proof.c.  The code is computed from |y| and y's
+// Fast path: with r within one ulp of RN(1/s) and r_lo = RN(RN(1 - s r) r)
+// (r + r_lo carries 1/s to about 2^-46), q = RN(|y| r + RN(|y| r_lo)) has the
+// same E4M3 code as RN(|y| / s) for every bf16 y with |y| <= amax and every
+// bf16 amax with s = RN(amax / 448) >= 2^-120, and likewise for every
+// binary16 pair (whose scales are all above 2^-120): checked exhaustively over
+// all such (amax, y) pairs and all three such r by tests/quotient_proof.c.  The code is computed from |y| and y's
 // sign bit is copied onto it, which also gives -0 the code 0x80.  If any lane
 // of the warp needs the IEEE division the whole warp takes it (warp-uniform
 // branch).  All 32 lanes must call.

@@ -61,33 +61,62 @@ static int e4m3_code(float v)
     return ((ex + 7) << 3) | (int)((r / ldexp(1.0, ex) - 1.0) * 8.0);
 }
 
+/* The kernels' scale: RN(amax / 448) without a division, by the FMA
+ * correction of a product with the rounded reciprocal (Markstein's method):
+ * q0 = RN(amax c) with c = RN(1/448), rem = amax - 448 q0 (exact in one FMA),
+ * s = RN(q0 + rem c). */
+static float scale_fma(float amax)
+{
+    const float c = 1.0f / 448.0f;
+    const float q0 = amax * c;
+    const float rem = fmaf(-448.0f, q0, amax);
+    return fmaf(rem, c, q0);
+}
+
 int main(int argc, char** argv)
 {
     uint32_t stride = argc > 1 ? (uint32_t)strtoul(argv[1], NULL, 10) : 1u;
     if (stride == 0)
         stride = 1;
     const int fp16 = argc > 2 && strcmp(argv[2], "fp16") == 0;
+    /* "near": every r within one ulp of RN(1/s), not only RN(1/s) itself */
+    const int near = argc > 3 && strcmp(argv[3], "near") == 0;
     float (*from_bits)(uint32_t) = fp16 ? from_fp16 : from_bf16;
     const uint32_t end = fp16 ? 0x7C00u : 0x7F80u; /* first non-finite pattern */
-    long pairs = 0, bad = 0;
+    long pairs = 0, bad = 0, scales = 0, bad_scales = 0;
+    for (uint32_t ab = 1; ab < end; ++ab) { /* the scale formula, every amax */
+        const float amax = from_bits(ab);
+        if (scale_fma(amax) != amax / 448.0f) {
+            if (bad_scales < 10)
+                printf("scale mismatch: amax=%a fma=%a div=%a\n", amax, scale_fma(amax),
+                       amax / 448.0f);
+            ++bad_scales;
+        }
+        ++scales;
+    }
     for (uint32_t ab = 1; ab < end; ab += stride) {
         const float amax = from_bits(ab);
         const float s = amax / 448.0f;
         if (!(s >= 0x1p-120f))
             continue;
-        const float r = 1.0f / s;
-        const float r_lo = fmaf(-s, r, 1.0f) * r;
-        for (uint32_t yb = 0; yb <= ab; ++yb) {
-            const float y = from_bits(yb);
-            const float q = fmaf(y, r, y * r_lo);
-            if (e4m3_code(q) != e4m3_code(y / s)) {
-                if (bad < 10)
-                    printf("mismatch: amax=%a y=%a q=%a y/s=%a\n", amax, y, q, y / s);
-                ++bad;
+        const float r_rn = 1.0f / s;
+        const float cand[3] = {nextafterf(r_rn, 0.0f), r_rn, nextafterf(r_rn, INFINITY)};
+        for (int c = near ? 0 : 1; c < (near ? 3 : 2); ++c) {
+            const float r = cand[c];
+            const float r_lo = fmaf(-s, r, 1.0f) * r;
+            for (uint32_t yb = 0; yb <= ab; ++yb) {
+                const float y = from_bits(yb);
+                const float q = fmaf(y, r, y * r_lo);
+                if (e4m3_code(q) != e4m3_code(y / s)) {
+                    if (bad < 10)
+                        printf("mismatch: amax=%a y=%a r=%a q=%a y/s=%a\n", amax, y, r, q, y / s);
+                    ++bad;
+                }
+                ++pairs;
             }
-            ++pairs;
         }
     }
+    printf("scales %ld scale mismatches %ld\n", scales, bad_scales);
     printf("pairs %ld mismatches %ld\n", pairs, bad);
-    return bad != 0;
+    return bad != 0 || bad_scales != 0;
 }

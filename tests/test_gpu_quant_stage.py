@@ -1,6 +1,8 @@
 """fn_quant (the quantization stage alone) against the oracle, bit for bit,
 over every finite bf16 value and the rounding corner cases of E4M3 / E2M1 /
 E8M0.  The fused kernel runs the same device code for its quantization stage."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -93,3 +95,20 @@ def test_quant_stage_random_scales(fnb, mode):
     q, s = fnb.quant(yb.cuda(), mode)
     torch.cuda.synchronize()
     parity.compare_quant_stage(gpu_util.bits(yb), gpu_util.u8(q), gpu_util.scale_np(s, mode), mode)
+
+
+def test_scale_and_reciprocal_arithmetic_exhaustive(tmp_path):
+    """The kernels' FP8 scale (division-free) equals CUDA's IEEE quotient and
+    their reciprocal is within one ulp of CUDA's IEEE reciprocal, for every
+    positive finite bf16 and binary16 amax (tests/recip_check.cu)."""
+    import subprocess
+    here = os.path.dirname(os.path.abspath(__file__))
+    csrc = os.path.join(os.path.dirname(here), "mxfp4_quantization_b200", "csrc")
+    exe = os.path.join(tmp_path, "recip_check")
+    nvcc = "/usr/local/cuda/bin/nvcc" if os.path.exists("/usr/local/cuda/bin/nvcc") else "nvcc"
+    subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17",
+                    "-ftz=false", "-prec-div=true", "-prec-sqrt=true", "-I", csrc, "-o", exe,
+                    os.path.join(here, "recip_check.cu")], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.count("scale mismatches 0") == 2 and r.stdout.count("beyond one ulp 0") == 2

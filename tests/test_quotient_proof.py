@@ -12,9 +12,10 @@ def test_quotient_matches_ieee_division_in_e4m3(tmp_path):
     exe = os.path.join(tmp_path, "quotient_proof")
     subprocess.run(["gcc", "-O2", "-ffp-contract=off", "-o", exe,
                     os.path.join(HERE, "quotient_proof.c"), "-lm"], check=True)
-    r = subprocess.run([exe, "97"], capture_output=True, text=True, timeout=300)
+    r = subprocess.run([exe, "97", "bf16", "near"], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout
-    assert "mismatches 0" in r.stdout
+    assert "scale mismatches 0" in r.stdout and "pairs" in r.stdout
+    assert r.stdout.strip().endswith("mismatches 0")
 
 
 def test_quotient_matches_ieee_division_in_e4m3_fp16(tmp_path):
@@ -22,6 +23,7 @@ def test_quotient_matches_ieee_division_in_e4m3_fp16(tmp_path):
     exe = os.path.join(tmp_path, "quotient_proof")
     subprocess.run(["gcc", "-O2", "-ffp-contract=off", "-o", exe,
                     os.path.join(HERE, "quotient_proof.c"), "-lm"], check=True)
-    r = subprocess.run([exe, "89", "fp16"], capture_output=True, text=True, timeout=300)
+    r = subprocess.run([exe, "89", "fp16", "near"], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout
-    assert "mismatches 0" in r.stdout
+    assert "scale mismatches 0" in r.stdout and "pairs" in r.stdout
+    assert r.stdout.strip().endswith("mismatches 0")
