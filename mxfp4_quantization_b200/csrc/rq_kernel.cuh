@@ -211,23 +211,36 @@ __device__ __forceinline__ void cluster_wait() {
 }
 
 // Sum of `s` and max of `m` over the block and, with CL, over the cluster.
-// The combination order is fixed (warps in index order, cluster ranks in rank
-// order), so every block of a cluster gets the same bits.  With CL the caller
-// must call cluster_wait() once before exiting: the last arrive here tells the
-// peers this block is done reading their shared memory, and the wait keeps
-// this block's own slot alive until every peer has read it.
+// The warps' results are combined in a fixed order, so every thread and every
+// block of a cluster (ranks in rank order) gets the same bits: in index order
+// by every thread (the shortest chain: decode-sized launches), or, with
+// `butterfly` (uniform over the launch), lane i of every warp takes warp i's
+// result and an xor butterfly combines them — both operands of every step are
+// the same in all lanes and addition commutes, so all lanes agree — which
+// takes fewer instructions for wide blocks (large-M launches).  With CL the
+// caller must call cluster_wait() once before exiting: the last arrive here
+// tells the peers this block is done reading their shared memory, and the
+// wait keeps this block's own slot alive until every peer has read it.
 template <bool CL, bool WANT_MAX>
-__device__ __forceinline__ float2 row_reduce(float s, float m, float2* red, float2* cl_slot) {
+__device__ __forceinline__ float2 row_reduce(float s, float m, float2* red, float2* cl_slot,
+                                             bool butterfly = false) {
   s = warp_sum(s);
   if (WANT_MAX) m = warp_max(m);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   if (lane == 0) red[warp] = make_float2(s, m);
   __syncthreads();
-  float2 t = red[0];
-  for (int i = 1; i < nw; ++i) {
-    const float2 o = red[i];
-    t.x += o.x;
-    if (WANT_MAX) t.y = fmaxf(t.y, o.y);
+  float2 t;
+  if (butterfly) {
+    t = lane < nw ? red[lane] : make_float2(0.f, 0.f);
+    t.x = warp_sum(t.x);
+    if (WANT_MAX) t.y = warp_max(t.y);
+  } else {
+    t = red[0];
+    for (int i = 1; i < nw; ++i) {
+      const float2 o = red[i];
+      t.x += o.x;
+      if (WANT_MAX) t.y = fmaxf(t.y, o.y);
+    }
   }
   if constexpr (CL) {
     cg::cluster_group cl = cg::this_cluster();
@@ -339,7 +352,12 @@ __global__ void __launch_bounds__((CL || TB > 256) ? 512 : 256)
         st_stream(prm.out_residual + rowv + v, hv[k]);
     }
     // ---- 3. rstd (and the per-token amax) ---------------------------------------------
-    const float2 tot = row_reduce<CL, MODE == MODE_TOKEN>(ss.x + ss.y, pmax, red, &cl_slot);
+    // exact-cover instances in large-M launches take the butterfly (measured
+    // on B200 at sustained clocks: MXFP4 H=7168 P=4 115.6 -> 114.0 us,
+    // group-128 H=8192 294.0 -> 292.0 us; decode calls keep the in-order sum,
+    // 0.3 us faster there)
+    const float2 tot = row_reduce<CL, MODE == MODE_TOKEN>(ss.x + ss.y, pmax, red, &cl_slot,
+                                                         TB > 0 && prm.prefetch_rows > 0);
     const float rstd = row_rstd(tot.x, prm.inv_h, prm.eps);
     if (MODE == MODE_TOKEN) scale_tok = fp8_scale_direct(row_amax_from_pmax<IO>(tot.y, rstd));
     // ---- 4. y = bf16(fl(h * w) * rstd) ----------------------------------------------

@@ -26,7 +26,8 @@ struct RQParams {
   float inv_h;             // 1 / H (fp32), for the mean of squares
   int* status;             // library status word: set to 1 if a bounded wait gave up
   uint32_t debug_extra_tx; // test hook: extra bytes each TMA stage expects (0 normally)
-  int prefetch_rows;       // L2 prefetch distance in rows of this block (0: none)
+  int prefetch_rows;       // L2 prefetch distance in rows of this block (0: none); a
+                           // positive distance also marks a large-M launch (row_reduce)
   int scale_layout;        // SCALE_*
   int64_t scale_ld;        // swizzled: column tiles per row tile; MN-major: row stride
 };

@@ -53,6 +53,34 @@ def test_layout_matches_oracle(fnb, mode, M, H, variant):
         assert np.array_equal(got.view(np.uint32), want.astype(np.float32).view(np.uint32))
 
 
+@pytest.mark.parametrize("variant", [0, 1])
+@pytest.mark.parametrize("mode,M,H", [(MX, 300, 7168), (MX, 5, 2048), (G128, 301, 8192),
+                                      (G128, 7, 1024)])
+def test_layout_with_fp16_rows(fnb, mode, M, H, variant):
+    """The layout flags combined with float16 rows (FN_IO_FP16)."""
+    flag = fnb.FN_SCALE_SWIZZLE_32_4_4 if mode == MX else fnb.FN_SCALE_MN_MAJOR
+    wl = synth.RowWorkload("layout16", M=M, H=H, P=2, mode=mode, eps=1e-6, seed=M + H + 1,
+                           dtype=torch.float16)
+    inp = wl.inputs(device="cpu")
+    q, s = fnb.alloc_outputs(mode | flag, M, H, "cuda")
+    with fnb.prefer_variant(variant):
+        out = fnb.rmsnorm_quant([p.cuda() for p in inp["parts"]], inp["weight"].cuda(), wl.eps,
+                                mode | flag, residual=inp["residual"].cuda(), emit_y=True,
+                                out_q=q, out_scale=s)
+    torch.cuda.synchronize()
+    assert out.y.dtype == torch.float16 and out.residual_out.dtype == torch.float16
+    y = gpu_util.bits(out.y)
+    rq, rs = oracle.quant_rows(y, mode, io=oracle.IO_FP16)
+    assert np.array_equal(gpu_util.u8(out.q).reshape(rq.shape), rq)
+    want = oracle.place_scales(rs.reshape(M, -1), oracle.SCALE_SWIZZLE_32_4_4 if mode == MX
+                               else oracle.SCALE_MN_MAJOR, fill=0)
+    got = gpu_util.scale_np(s, mode).reshape(-1)
+    if mode == MX:
+        assert np.array_equal(got, want)
+    else:
+        assert np.array_equal(got.view(np.uint32), want.astype(np.float32).view(np.uint32))
+
+
 def _dequant_mx(codes_u8, scales_rowmajor_u8):
     """Dequantized MXFP4 values (float64) from packed codes and E8M0 scales."""
     table = np.array([oracle.e2m1_decode([c])[0] for c in range(16)])
