@@ -414,3 +414,34 @@ def test_programmatic_launch_chain(fnb, M, H, P, mode, graph):
     for (q0, s0), (q1, s1) in zip(o0, o1):
         assert torch.equal(q0.view(torch.uint8), q1.view(torch.uint8))
         assert torch.equal(s0.view(torch.uint8), s1.view(torch.uint8))
+
+
+@pytest.mark.parametrize("mode,M,H,P", [(MX, 1200, 7168, 4), (G128, 700, 8192, 1), (TOKEN, 16, 7168, 1)])
+def test_graph_replays_are_bit_identical(fnb, mode, M, H, P):
+    """Two hundred replays of one captured call (the bench's launch shape, not
+    in place): every replay's codes, scales and residual_out equal the first
+    replay's, bit for bit (SHA-256 of the host copies)."""
+    import hashlib
+    wl = synth.RowWorkload("replay", M=M, H=H, P=P, mode=mode, eps=1e-6, seed=M + P,
+                           channel_decades=1.0 if P > 1 else 0.0)
+    inp = wl.inputs(device="cuda")
+    q, s = fnb.alloc_outputs(mode, M, H, "cuda")
+    r_out = torch.empty_like(inp["residual"])
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            fnb.rmsnorm_quant(inp["parts"], inp["weight"], wl.eps, mode, residual=inp["residual"],
+                              out_residual=r_out, out_q=q, out_scale=s)
+    digests = set()
+    for _ in range(200):
+        for t in (q, s, r_out):
+            t.view(torch.uint8).zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        h = hashlib.sha256()
+        for t in (q, s, r_out):
+            h.update(t.view(torch.uint8).cpu().numpy().tobytes())
+        digests.add(h.hexdigest())
+    assert len(digests) == 1

@@ -1,0 +1,103 @@
+"""Negative controls for the parity harness (tests/parity.py), on the CPU.
+
+The GPU parity tests are only as good as the comparison they run.  Here the
+oracle's own outputs stand in for a kernel's: unchanged they must pass, and
+each planted fault — one flipped code bit, a wrong scale, y off by two ulps,
+a residual off by one ulp, a code two steps away, a code that moved where y
+did not — must make the comparison fail."""
+import numpy as np
+import pytest
+
+import oracle
+from mxfp4_quantization_b200 import synth
+from tests import parity
+
+
+def _case(mode, seed=5, M=12, H=1024, P=2, io=oracle.IO_BF16):
+    import torch
+    wl = synth.RowWorkload("ctl", M=M, H=H, P=P, mode=mode, eps=1e-6, seed=seed,
+                           outlier_frac=0.01,
+                           dtype=torch.float16 if io == oracle.IO_FP16 else torch.bfloat16)
+    inp = wl.inputs(device="cpu")
+    parts = [synth.to_bits(p) for p in inp["parts"]]
+    res, w = synth.to_bits(inp["residual"]), synth.to_bits(inp["weight"])
+    orc = oracle.rmsnorm_quant(parts, res, w, wl.eps, mode, io=io)
+    gpu = {"q": orc["q"].copy(), "scale": orc["scale"].copy(),
+           "residual_out": orc["residual_out"].copy(), "y": orc["y"].copy()}
+    return wl, parts, res, w, gpu
+
+
+def _check(wl, parts, res, w, gpu, io=oracle.IO_BF16):
+    return parity.check_rmsnorm(wl.mode, wl.eps, parts, res, w, gpu, io)
+
+
+MODES = [oracle.FP8_PER_TOKEN, oracle.FP8_PER_GROUP128, oracle.MXFP4]
+
+
+@pytest.mark.parametrize("io", [oracle.IO_BF16, oracle.IO_FP16])
+@pytest.mark.parametrize("mode", MODES)
+def test_exact_outputs_pass(mode, io):
+    wl, parts, res, w, gpu = _case(mode, io=io)
+    stats = _check(wl, parts, res, w, gpu, io)
+    assert stats["codes_diff"] == 0 and stats["scale_diff"] == 0
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_flipped_code_bit_fails(mode):
+    wl, parts, res, w, gpu = _case(mode)
+    gpu["q"][3, 17] ^= 0x01
+    with pytest.raises(AssertionError):
+        _check(wl, parts, res, w, gpu)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_wrong_scale_fails(mode):
+    wl, parts, res, w, gpu = _case(mode)
+    s = gpu["scale"].reshape(wl.M, -1)
+    if mode == oracle.MXFP4:
+        s[2, 1] = s[2, 1] + 1
+    else:
+        s[2, 0] = np.float32(s[2, 0]) * np.float32(1.0 + 2 ** -20)
+    with pytest.raises(AssertionError):
+        _check(wl, parts, res, w, gpu)
+
+
+def test_y_two_ulps_off_fails():
+    wl, parts, res, w, gpu = _case(oracle.MXFP4)
+    y = gpu["y"]
+    i = int(np.argmax((y & 0x7FFF) > 0x3000))  # a normal, nonzero element of row 0
+    y[0, i] = y[0, i] + 2
+    with pytest.raises(AssertionError):
+        _check(wl, parts, res, w, gpu)
+
+
+def test_residual_one_ulp_off_fails():
+    wl, parts, res, w, gpu = _case(oracle.FP8_PER_TOKEN)
+    gpu["residual_out"][5, 9] += 1
+    with pytest.raises(AssertionError):
+        _check(wl, parts, res, w, gpu)
+
+
+def test_code_two_steps_away_fails_end_to_end():
+    """A kernel whose y moved by one ulp but whose code moved by two steps."""
+    wl, parts, res, w, gpu = _case(oracle.FP8_PER_GROUP128)
+    orc = oracle.rmsnorm_quant(parts, res, w, wl.eps, wl.mode)
+    q, y = gpu["q"], gpu["y"]
+    j = 40
+    y[1, j] += 1
+    q[1, j] = (q[1, j] & 0x80) | ((q[1, j] & 0x7F) + 2)
+    with pytest.raises(AssertionError):
+        parity.compare_end_to_end(wl.mode, wl.H, y, q, gpu["scale"], orc["y"], orc["q"],
+                                  orc["scale"])
+
+
+def test_code_moved_where_y_did_not_fails_end_to_end():
+    wl, parts, res, w, gpu = _case(oracle.MXFP4)
+    orc = oracle.rmsnorm_quant(parts, res, w, wl.eps, wl.mode)
+    q = gpu["q"]
+    lo = q[4, 3] & 0x0F
+    q[4, 3] = (q[4, 3] & 0xF0) | ((lo & 0x8) | min((lo & 0x7) + 1, 7) if (lo & 0x7) < 7
+                                  else (lo & 0x8) | 6)
+    with pytest.raises(AssertionError):
+        parity.compare_end_to_end(wl.mode, wl.H, gpu["y"], q, gpu["scale"], orc["y"], orc["q"],
+                                  orc["scale"])
