@@ -445,3 +445,32 @@ def test_graph_replays_are_bit_identical(fnb, mode, M, H, P):
             h.update(t.view(torch.uint8).cpu().numpy().tobytes())
         digests.add(h.hexdigest())
     assert len(digests) == 1
+
+
+def _random_cases(n, seed=2024):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        mode = int(rng.integers(0, 3))
+        unit = {TOKEN: 8, G128: 128, MX: 32}[mode]
+        H = int(unit * rng.integers(1, max(2, 4096 // unit) + 1))
+        M = int(rng.choice([1, 2, 5, 16, 17, 63, 150, 151, 300, 333]))
+        P = int(rng.integers(1, 9))
+        out.append((i, mode, M, H, P, bool(rng.integers(0, 4) > 0), bool(rng.integers(0, 3) == 0),
+                    int(rng.choice([0, 1, 2, 5]))))
+    return out
+
+
+@pytest.mark.parametrize("i,mode,M,H,P,has_res,fp16,variant", _random_cases(48),
+                         ids=[f"r{c[0]}" for c in _random_cases(48)])
+def test_random_shapes(fnb, i, mode, M, H, P, has_res, fp16, variant):
+    """Seeded random shapes, partial counts, formats and kernels (any H the
+    mode allows up to 4096, M across the dispatch switches) against the
+    oracle, with guard bytes around every output."""
+    wl = synth.RowWorkload("rand", M=M, H=H, P=P, mode=mode, eps=1e-6 if i % 2 else 1e-5,
+                           seed=1000 + i, residual=has_res, outlier_frac=0.01,
+                           channel_decades=1.0 if P > 1 else 0.0,
+                           dtype=torch.float16 if fp16 else torch.bfloat16)
+    inp, gpu, got, launch = run(fnb, wl, variant=variant)
+    assert got in (fnb.FN_VARIANT_ROW_CTA, fnb.FN_VARIANT_ROW_CLUSTER, fnb.FN_VARIANT_ROW_TMA)
+    check(wl, inp, gpu)
