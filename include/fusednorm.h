@@ -76,7 +76,7 @@ typedef enum {
 typedef enum {
     FN_VARIANT_NONE = 0,        /* nothing launched (M == 0 or an error)          */
     FN_VARIANT_ROW_CTA = 1,     /* one thread block per row                        */
-    FN_VARIANT_ROW_CLUSTER = 2, /* a cluster of 2..8 blocks per row (small M)      */
+    FN_VARIANT_ROW_CLUSTER = 2, /* a cluster of 2..8 blocks per row (small M, long rows) */
     FN_VARIANT_QUANT_ONLY = 3,  /* fn_quant                                        */
     FN_VARIANT_QK_WARP = 4,     /* fn_qk_norm_gate: one warp per (token, head)     */
     FN_VARIANT_ROW_TMA = 5,     /* persistent blocks, rows staged by bulk copies  */
@@ -271,8 +271,11 @@ FN_API void fn_last_launch(int32_t out[4]);
  * FN_VARIANT_ROW_CLUSTER or FN_VARIANT_ROW_TMA asks for that kernel where the
  * shape allows it (the cluster kernel needs a row that splits into 2..8
  * group-aligned segments with M * blocks <= SMs, the TMA kernel at least two
- * row stages in shared memory).  Every kernel computes the same bits.
- * Returns the previous preference. */
+ * row stages in shared memory).  Every kernel meets the same accuracy
+ * contract; kernels that reduce a row in another order (block size, cluster
+ * split, row groups) may differ from one another by the one-ulp rounding of
+ * y it allows, while any one kernel and launch shape always gives the same
+ * bits.  Returns the previous preference. */
 FN_API int fn_prefer_variant(int variant);
 
 /* Reads and clears the library's device status word on the current device

@@ -9,8 +9,9 @@
 // HBM-bound, no tensor cores.  Three kernels share the per-vector stages below:
 //  * rq_kernel, CL = false: one thread block per row.  Every load of the row
 //    is issued before the first arithmetic; the row then lives in registers.
-//  * rq_kernel, CL = true (small M): a cluster of 2..8 blocks per row; the
-//    blocks exchange their partial sums through distributed shared memory.
+//  * rq_kernel, CL = true (small M with rows too long for one wide block, or on
+//    request): a cluster of 2..8 blocks per row; the blocks exchange their
+//    partial sums through distributed shared memory.
 //  * rq_tma_kernel (large M): one persistent block per SM; a ring of shared
 //    memory stages is filled by bulk asynchronous copies (cp.async.bulk, the
 //    TMA engine, no multicast) several rows ahead of the row being computed.
