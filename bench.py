@@ -23,6 +23,7 @@ import dataclasses
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -200,13 +201,21 @@ def time_steps(fn_step, steps: int, warmup: int, device, stream, clocks=None):
     return e0.elapsed_time(e1) / steps
 
 
+def _code_only(src: str) -> str:
+    """Kernel source with comments and layout removed: the hash below changes
+    with the code, not with its comments."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mxfp4_quantization_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
         if f.endswith((".cu", ".cuh", ".h")):
             h.update(f.encode())
-            h.update(open(os.path.join(csrc, f), "rb").read())
+            h.update(_code_only(open(os.path.join(csrc, f)).read()).encode())
     return h.hexdigest()[:16]
 
 
