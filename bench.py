@@ -516,6 +516,30 @@ def secondary_workloads(fn, device, peak):
         torch.cuda.empty_cache()
     res["fp16_rows"] = f16
 
+    # the quantization step alone (fn_quant) on the two large shapes' rows
+    qo = {}
+    for base in (synth.PREFILL_MXFP4, synth.PREFILL_GROUP128):
+        wl = dataclasses.replace(base, P=1, residual=False)
+        y = synth.normal_bf16((wl.M, wl.H), wl.seed, "y", device=device)
+        q, s = fn.alloc_outputs(wl.mode, wl.M, wl.H, device)
+        stream = torch.cuda.current_stream(device)
+
+        def qstep(y=y, q=q, s=s, wl=wl, sp=stream.cuda_stream):
+            st = fn.fn_quant(y.data_ptr(), wl.mode, wl.M, wl.H, q.data_ptr(), s.data_ptr(), sp)
+            if st != fn.FN_OK:
+                raise fn.FusedNormError("fn_quant", st)
+
+        ms = time_steps(qstep, 100, 5, device, stream)
+        b = wl.M * (2 * wl.H + (wl.H // 2 + wl.H // 32 if wl.mode == synth.MXFP4
+                                else wl.H + 4 * (wl.H // 128)))
+        qo[base.name] = {"M": wl.M, "H": wl.H, "us_per_call": ms * 1e3,
+                         "GB_s": b / (ms * 1e-3) / 1e9, "frac_of_peak": b / (ms * 1e-3) / 1e9 / peak,
+                         "bytes_per_call": b, "variant": fn.fn_last_variant(),
+                         "launch": list(fn.fn_last_launch())}
+        del y, q, s
+        torch.cuda.empty_cache()
+    res["quant_only"] = qo
+
     def small(wl, per_call_bytes, make):
         n_sets = max(64, int(2 * L2_BYTES / per_call_bytes) + 1)
         n_sets = min(n_sets, 8192)

@@ -99,12 +99,12 @@ RQKernel pick_kernel(int mode, int P, int V, bool cluster, bool norm, bool f16) 
 }
 
 // The exact-cover instance for a row of T * V vectors, or nullptr.
-RQKernel pick_exact_kernel(int mode, int P, int T, int V, bool f16) {
+RQKernel pick_exact_kernel(int mode, int P, int T, int V, bool f16, bool norm = true) {
   const int maxp = P == 1 ? 1 : P == 2 ? 2 : P <= 4 ? 4 : 8;
 #define FN_CASE(MODE, MAXP)                                                              \
   if (mode == MODE && maxp == MAXP)                                                      \
-    return f16 ? fn::rq_exact_pick_##MODE##_##MAXP##_1(T, V)                             \
-               : fn::rq_exact_pick_##MODE##_##MAXP##_0(T, V);
+    return f16 ? fn::rq_exact_pick_##MODE##_##MAXP##_1(T, V, norm)                       \
+               : fn::rq_exact_pick_##MODE##_##MAXP##_0(T, V, norm);
   FN_CASE(0, 1) FN_CASE(0, 2) FN_CASE(0, 4) FN_CASE(0, 8)
   FN_CASE(1, 1) FN_CASE(1, 2) FN_CASE(1, 4) FN_CASE(1, 8)
   FN_CASE(2, 1) FN_CASE(2, 2) FN_CASE(2, 4) FN_CASE(2, 8)
@@ -398,7 +398,7 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, bo
     p.prefetch_rows = M > (int64_t)kRowPrefetchSms * sms ? kRowPrefetchSms * sms : 0;
     int threads = wide_k ? wide_T : round32((nvec + V - 1) / V);
     RQKernel k = wide_k;
-    if (!k && norm && threads * V == nvec) k = pick_exact_kernel(mode, P, threads, V, f16);
+    if (!k && threads * V == nvec) k = pick_exact_kernel(mode, P, threads, V, f16, norm);
     if (k && !wide_k && V >= 4) {
       // Many partials held in registers leave room for few blocks per SM:
       // below kMinRowWarps resident warps, split the row twice as finely.

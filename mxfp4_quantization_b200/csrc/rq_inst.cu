@@ -54,9 +54,21 @@ RQKernel FN_CAT(rq_pick, FN_INST_MODE, FN_INST_MAXP)(int V, bool cluster, bool n
 // T = 224 serves H = 3584, 7168, 14336; T = 256 serves H = 4096, 8192, 16384;
 // T = 448 and 512 are the same rows split more finely (more warps per SM when
 // the partials leave room for few blocks; the widest block for decode-sized M).
-RQKernel FN_CAT(rq_exact_pick, FN_INST_MODE, FN_INST_MAXP)(int T, int V) {
+RQKernel FN_CAT(rq_exact_pick, FN_INST_MODE, FN_INST_MAXP)(int T, int V, bool norm) {
   constexpr int MODE = FN_INST_MODE, MAXP = FN_INST_MAXP;
   using IO = std::conditional_t<FN_INST_IO == 1, F16, Bf16>;
+  if (!norm) {  // the quantization step alone (fn_quant): one input, MAXP = 1
+    if constexpr (MAXP != 1) {
+      return nullptr;
+    } else {
+      if (T == 224 && V == 4) return rq_kernel<MODE, 1, 4, false, false, 224, IO>;
+      if (T == 256 && V == 4) return rq_kernel<MODE, 1, 4, false, false, 256, IO>;
+      if (T == 256 && V == 2) return rq_kernel<MODE, 1, 2, false, false, 256, IO>;
+      if (T == 224 && V == 8) return rq_kernel<MODE, 1, 8, false, false, 224, IO>;
+      if (T == 256 && V == 8) return rq_kernel<MODE, 1, 8, false, false, 256, IO>;
+      return nullptr;
+    }
+  }
 #define FN_EXACT(TT, VV) \
   if (T == TT && V == VV) return rq_kernel<MODE, MAXP, VV, true, false, TT, IO>;
   FN_EXACT(224, 2) FN_EXACT(224, 4) FN_EXACT(224, 8)

@@ -289,7 +289,7 @@ __device__ __forceinline__ float row_amax_from_pmax(float pmax, float rstd) {
 template <int MODE, int MAXP, int V, bool NORM, bool CL, int TB = 0, class IO = Bf16>
 __global__ void __launch_bounds__((CL || TB > 256) ? 512 : 256)
     rq_kernel(const __grid_constant__ RQParams prm) {
-  static_assert(TB == 0 || (!CL && NORM), "exact-cover instances are one block per row");
+  static_assert(TB == 0 || !CL, "exact-cover instances are one block per row");
   __shared__ float2 red[32];
   __shared__ float2 cl_slot;
   pdl_enter();

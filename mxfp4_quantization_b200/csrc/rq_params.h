@@ -46,7 +46,7 @@ using RQTmaKernel = void (*)(const RQParams, int, int);
 // IO: 0 = bf16 rows, 1 = binary16 rows.
 #define FN_RQ_DECL(MODE, MAXP, IO)                                          \
   RQKernel rq_pick_##MODE##_##MAXP##_##IO(int V, bool cluster, bool norm); \
-  RQKernel rq_exact_pick_##MODE##_##MAXP##_##IO(int T, int V);             \
+  RQKernel rq_exact_pick_##MODE##_##MAXP##_##IO(int T, int V, bool norm);  \
   RQTmaKernel rq_tma_pick_##MODE##_##MAXP##_##IO(int V);
 #define FN_RQ_DECL_IO(MODE, MAXP) FN_RQ_DECL(MODE, MAXP, 0) FN_RQ_DECL(MODE, MAXP, 1)
 FN_RQ_DECL_IO(0, 1)
