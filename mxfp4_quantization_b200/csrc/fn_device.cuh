@@ -85,10 +85,12 @@ __device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b) {
   return d;
 }
 
-// Packed max of |a| and |b| (exact: max only selects).
+// Packed max of |a| and |b| per half (exact: max only selects).  The sign
+// bit of each result half is the xor of the operands' signs: only the
+// magnitude is meaningful, and further absmax calls may take it as is.
 __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a & 0x7FFF7FFFu), "r"(b & 0x7FFF7FFFu));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
 
@@ -187,7 +189,7 @@ __device__ __forceinline__ uint32_t add_f16x2(uint32_t a, uint32_t b) {
 
 __device__ __forceinline__ uint32_t absmax_f16x2(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("max.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a & 0x7FFF7FFFu), "r"(b & 0x7FFF7FFFu));
+  asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
 
@@ -270,7 +272,7 @@ struct F16 {
 template <class IO = Bf16>
 __device__ __forceinline__ float vec_absmax(const uint4& y) {
   const uint32_t m = IO::absmax2(IO::absmax2(y.x, y.y), IO::absmax2(y.z, y.w));
-  return fmaxf(IO::lo(m), IO::hi(m));
+  return fmaxf(fabsf(IO::lo(m)), fabsf(IO::hi(m)));
 }
 
 // ---- FP8 E4M3 -----------------------------------------------------------------
