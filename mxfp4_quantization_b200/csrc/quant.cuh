@@ -8,7 +8,7 @@ namespace fn {
 // FP8 scale of a group (or row) and the reciprocal pair the codes use.
 struct Fp8Scale {
   float s;         // RN(amax / 448), 1 for an all-zero group
-  float r, r_lo;   // 1/s within one ulp of RN(1/s); RN(RN(1 - s r) r)
+  float r, r_lo;   // the float at or just below 1/s (RD or RD - 1 ulp); RN(RN(1 - s r) r) >= 0
   bool exact_div;  // the fast quotient is not proven here: use the IEEE division
 };
 
@@ -33,12 +33,25 @@ __device__ __forceinline__ float recip_near(float s) {
   return fmaf(fmaf(-s, y, 1.0f), y, y);
 }
 
+// A reciprocal not above 1/s: recip_near stepped down (at most twice, since it
+// is within one ulp of RN(1/s)) while the exact residual 1 - s r is negative.
+// The result is RD(1/s) or, when recip_near was already below, RD(1/s) - 1 ulp:
+// within one ulp of RN(1/s) either way.  For s >= 2^-120 r is a normal float,
+// so one step down is one less in its bit pattern.
+__device__ __forceinline__ float recip_down(float s) {
+  float r = recip_near(s);
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    if (fmaf(-s, r, 1.0f) < 0.f) r = __int_as_float(__float_as_int(r) - 1);
+  return r;
+}
+
 // The group's scale and the reciprocal pair of the codes.
 __device__ __forceinline__ Fp8Scale fp8_scale_direct(float amax) {
   Fp8Scale c;
   c.s = amax == 0.f ? 1.f : scale_div448(amax);
   c.exact_div = !(c.s >= 0x1p-120f);
-  c.r = c.exact_div ? 1.f : recip_near(c.s);
+  c.r = c.exact_div ? 1.f : recip_down(c.s);
   c.r_lo = __fmul_rn(fmaf(-c.s, c.r, 1.f), c.r);
   return c;
 }
@@ -50,34 +63,31 @@ __device__ __forceinline__ Fp8Scale fp8_scale_direct(float amax) {
 // same E4M3 code as RN(|y| / s) for every bf16 y with |y| <= amax and every
 // bf16 amax with s = RN(amax / 448) >= 2^-120, and likewise for every
 // binary16 pair (whose scales are all above 2^-120): checked exhaustively over
-// all such (amax, y) pairs and all three such r by tests/quotient_proof.c.  The code is computed from |y| and y's
-// sign bit is copied onto it, which also gives -0 the code 0x80.  If any lane
-// of the warp needs the IEEE division the whole warp takes it (warp-uniform
-// branch).  All 32 lanes must call.
+// all such (amax, y) pairs and all three such r by tests/quotient_proof.c.
+// The codes are computed from the signed y: every step rounds to nearest
+// even, which is odd-symmetric, so a negative y gets minus the quotient of
+// |y| and the conversion writes the sign.  Zeros keep their sign because
+// r_lo >= 0 (r is not above 1/s): -0 r_lo = -0 and -0 + -0 = -0 (code 0x80).
+// If any lane of the warp needs the IEEE division the whole warp takes it
+// (warp-uniform branch; the signed quotient keeps signs there too).  All 32
+// lanes must call.
 template <class IO = Bf16>
 __device__ __forceinline__ uint2 e4m3_codes(const uint4& y, const Fp8Scale& c) {
   uint32_t q8[4];
   if (!__any_sync(0xffffffffu, c.exact_div)) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t a = word(y, i) & 0x7FFF7FFFu;
-      const float2 ya = make_float2(IO::lo(a), IO::hi(a));
-      const float2 t = mul_f32x2(ya, make_float2(c.r_lo, c.r_lo));
-      const float2 q = fma_f32x2(ya, make_float2(c.r, c.r), t);
+      const float2 yf = make_float2(IO::lo(word(y, i)), IO::hi(word(y, i)));
+      const float2 t = mul_f32x2(yf, make_float2(c.r_lo, c.r_lo));
+      const float2 q = fma_f32x2(yf, make_float2(c.r, c.r), t);
       q8[i] = cvt_e4m3x2(q.x, q.y);
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t a = word(y, i) & 0x7FFF7FFFu;
-      q8[i] = cvt_e4m3x2(__fdiv_rn(IO::lo(a), c.s), __fdiv_rn(IO::hi(a), c.s));
-    }
+    for (int i = 0; i < 4; ++i)
+      q8[i] = cvt_e4m3x2(__fdiv_rn(IO::lo(word(y, i)), c.s), __fdiv_rn(IO::hi(word(y, i)), c.s));
   }
-  // byte k of code word j takes the sign of element 4j + k: the sign bits sit
-  // at bits 15 and 31 of each y word (both formats), i.e. in bytes 1 and 3
-  const uint32_t s0 = __byte_perm(y.x, y.y, 0x7531) & 0x80808080u;
-  const uint32_t s1 = __byte_perm(y.z, y.w, 0x7531) & 0x80808080u;
-  return make_uint2((q8[0] | (q8[1] << 16)) | s0, (q8[2] | (q8[3] << 16)) | s1);
+  return make_uint2(q8[0] | (q8[1] << 16), q8[2] | (q8[3] << 16));
 }
 
 }  // namespace fn

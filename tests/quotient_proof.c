@@ -7,7 +7,8 @@
  *     r    = RN(1 / s)
  *     r_lo = RN(RN(1 - s r) * r)          (1 - s r by one fused multiply-add)
  *     q    = RN(|y| r + RN(|y| r_lo))      (one multiply, one fused multiply-add)
- * and copy y's sign onto the code.  This program runs every positive finite
+ * (a negative y gives minus the same quotient: every step rounds to nearest
+ * even, which is odd-symmetric).  This program runs every positive finite
  * bf16 amax with s >= 2^-120 against every bf16 |y| <= amax (about 5.3e8
  * pairs) and counts the pairs whose E4M3 codes differ.  It exits 0 iff there
  * are none.  argv[1] (optional) strides the amax loop for a quicker run;

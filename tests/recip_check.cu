@@ -2,7 +2,8 @@
 // (csrc/quant.cuh) against CUDA's IEEE operations, for every positive finite
 // bf16 and binary16 amax:
 //   scale_div448(amax) == __fdiv_rn(amax, 448)          (bit for bit)
-//   |recip_near(s) - __frcp_rn(s)| <= 1 ulp for s >= 2^-120
+//   recip_down(s) is RN(1/s) or one ulp below it, and s * recip_down(s) <= 1
+//   (exact residual not negative) for s >= 2^-120
 // (the E4M3 quotient is proven on the CPU for every r within one ulp of
 // RN(1/s), tests/quotient_proof.c).  Prints the counts; exits 0 iff clean.
 #include <cstdio>
@@ -21,10 +22,10 @@ __global__ void check(int fp16, unsigned long long* bad_scale, unsigned long lon
   const float s = scale_div448(amax);
   if (__float_as_uint(s) != __float_as_uint(s_ref)) atomicAdd(bad_scale, 1ull);
   if (s_ref >= 0x1p-120f) {
-    const float r_ref = __frcp_rn(s_ref), r = recip_near(s_ref);
-    const int d = abs((int)__float_as_uint(r) - (int)__float_as_uint(r_ref));
-    atomicMax(max_ulp, d);
-    if (d > 1) atomicAdd(bad_recip, 1ull);
+    const float r_ref = __frcp_rn(s_ref), r = recip_down(s_ref);
+    const int d = (int)__float_as_uint(r_ref) - (int)__float_as_uint(r);
+    atomicMax(max_ulp, abs(d));
+    if (d < 0 || d > 1 || fmaf(-s_ref, r, 1.0f) < 0.f) atomicAdd(bad_recip, 1ull);
     atomicAdd(checked, 1ull);
   }
 }
@@ -45,7 +46,7 @@ int main() {
     if (cudaMemcpy(h, c, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess ||
         cudaMemcpy(&hm, m, sizeof hm, cudaMemcpyDeviceToHost) != cudaSuccess)
       return 2;
-    printf("%s: scale mismatches %llu, reciprocals checked %llu, beyond one ulp %llu, max ulp %d\n",
+    printf("%s: scale mismatches %llu, reciprocals checked %llu, bad reciprocals %llu, max ulp %d\n",
            fp16 ? "fp16" : "bf16", h[0], h[2], h[1], hm);
     if (h[0] || h[1] || h[2] == 0) rc = 1;
   }
