@@ -319,6 +319,18 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// Max of a non-negative value over each 16-lane half of the warp, by two
+// hardware warp reductions on the bit patterns (non-negative floats order as
+// unsigned integers).  All 32 lanes must call.
+__device__ __forceinline__ float half_warp_max(float v) {
+  const uint32_t u = __float_as_uint(v);
+  const bool lo = (threadIdx.x & 16) == 0;
+  uint32_t a, b;
+  asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(a) : "r"(lo ? u : 0u));
+  asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(b) : "r"(lo ? 0u : u));
+  return __uint_as_float(lo ? a : b);
+}
+
 // Max over aligned groups of `G` lanes (G a power of two, <= 32).
 template <int G>
 __device__ __forceinline__ float group_max(float v) {

@@ -160,7 +160,7 @@ __device__ __forceinline__ QuantVec quant_vec(const uint4& y, const Fp8Scale& to
   QuantVec r;
   if constexpr (MODE == MODE_TOKEN || MODE == MODE_G128) {
     Fp8Scale c = tok;
-    if constexpr (MODE == MODE_G128) c = fp8_scale_direct(group_max<16>(vec_absmax<IO>(y)));
+    if constexpr (MODE == MODE_G128) c = fp8_scale_direct(half_warp_max(vec_absmax<IO>(y)));
     r.s = c.s;
     r.q8 = e4m3_codes<IO>(y, c);
   } else {
