@@ -607,6 +607,23 @@ def oracle_rows_per_s(rows: int, min_seconds: float, max_seconds: float, workloa
     return done / el, done, el
 
 
+def _oracle_worker(job):
+    rows, seconds, workload = job
+    rate, done, el = oracle_rows_per_s(rows, seconds, 3 * seconds, workload)
+    return done, el
+
+
+def oracle_rows_per_s_all_cores(rows: int, seconds: float, workload: str):
+    """The same oracle run row-parallel: one process per host core (spawned,
+    so no process inherits a CUDA context), each on its own `rows` rows for
+    about `seconds`.  Returns (rows/s over all processes, processes)."""
+    import multiprocessing as mp
+    n = os.cpu_count() or 1
+    with mp.get_context("spawn").Pool(n) as pool:
+        res = pool.map(_oracle_worker, [(rows, seconds, workload)] * n)
+    return sum(d for d, _ in res) / max(el for _, el in res), n
+
+
 def reference_arm(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -691,7 +708,7 @@ def main_arm(args):
     e2e_ms_max = dist_max(e2e_ms, device)
 
     extra = None
-    cpu = None
+    cpu = cpu_all = None
     if world == 1 and not args.no_extras and args.workload == "prefill_mxfp4":
         extra = secondary_workloads(fn, device, peak)
     if world == 1 and not args.no_cpu_baseline:
@@ -701,6 +718,12 @@ def main_arm(args):
                "sample": f"{rows} rows (256 rows of the {wl.name} recipe, H={wl.H}, P={wl.P}, "
                          f"repeated) in {el:.1f} s, single-threaded; "
                          f"host has {os.cpu_count()} cores"}
+        rate_all, procs = oracle_rows_per_s_all_cores(64, max(1.0, args.cpu_seconds / 2),
+                                                      args.workload)
+        cpu_all = {"value": rate_all, "unit": "rows/s", "cores": procs,
+                   "kind": "oracle, row-parallel processes (context beside cpu_baseline)",
+                   "sample": f"64 rows of the {wl.name} recipe per process, repeated for "
+                             f"about {max(1.0, args.cpu_seconds / 2):.0f} s, {procs} processes"}
 
     if rank == 0:
         line = {
@@ -727,6 +750,7 @@ def main_arm(args):
             "gpu_launches": args.steps,
             "clocks": clk,
             "cpu_baseline": cpu,
+            "cpu_baseline_all_cores": cpu_all,
             "workloads": extra,
         }
         print(json.dumps(line), flush=True)
