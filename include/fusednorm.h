@@ -22,15 +22,19 @@
  *    32-element block, X = 2^(floor(log2 amax) - 2).
  *
  * The cross-GPU all-reduce in front of the norm is replaced by an in-kernel
- * sum of up to 8 partial buffers that live on the same device.
+ * sum of up to 8 partial buffers that live on the same device
+ * (fn_rmsnorm_quant), or done by the kernel itself over peer memory across
+ * the ranks of a tensor-parallel group (fn_ar_rmsnorm_quant).
  *
  * Conventions for every entry point:
  *  - bf16 tensors are IEEE bfloat16 bit patterns, row-major, contiguous rows
  *    (row stride H elements unless a stride argument says otherwise).
  *  - Every data pointer is a DEVICE pointer owned by the caller.  The library
- *    allocates nothing, keeps no state besides a thread-local record of the
- *    last dispatch, and never synchronizes: work is queued on `stream`
- *    (a cudaStream_t passed as void*; NULL means the legacy default stream).
+ *    allocates nothing and never synchronizes (fn_device_status excepted):
+ *    work is queued on `stream` (a cudaStream_t passed as void*; NULL means
+ *    the legacy default stream).  Its only state: thread-local settings and
+ *    a record of the last dispatch, a per-device cache of device facts, and
+ *    one static device status word.
  *  - All argument checks run on the host before anything is launched; on any
  *    error nothing is launched and no output is touched.  M == 0 returns
  *    FN_OK and launches nothing once the sizes and the mode are valid; the
