@@ -69,3 +69,25 @@ def test_two_gloo_ranks_agree_on_the_plan():
         assert len(stages) == 1  # every rank takes the same form
         rows = sorted(x for r in range(world) for x in range(*every[r][i][2]))
         assert rows == list(range(M))
+
+
+def test_object_rejects_what_it_does_not_offer():
+    """Checks that run before any device buffer or collective: M-major scales
+    (their stride depends on M), float16 rows, an unknown sync mode, and a
+    group of one rank."""
+    import pytest
+    import torch.distributed as dist
+    from mxfp4_quantization_b200 import fusednorm as fn
+    for mode in (fn.FN_FP8_PER_GROUP128 | fn.FN_SCALE_MN_MAJOR, fn.FN_MXFP4 | fn.FN_IO_FP16):
+        with pytest.raises(ValueError):
+            tp.FusedAllReduceRMSNormQuant(64, 2048, mode)
+    with pytest.raises(ValueError):
+        tp.FusedAllReduceRMSNormQuant(64, 2048, fn.FN_MXFP4, sync="spin")
+    port = _free_port()
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=30))
+    try:
+        with pytest.raises(ValueError):
+            tp.FusedAllReduceRMSNormQuant(64, 2048, fn.FN_MXFP4)
+    finally:
+        dist.destroy_process_group()
