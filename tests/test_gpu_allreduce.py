@@ -72,6 +72,48 @@ def test_virtual_ranks(fnb, world, mode, M, H):
                          gpu_util.bits(w), gpu)
 
 
+def _random_ar_cases(n, seed=77):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        mode = int(rng.integers(0, 3))
+        unit = {TOKEN: 8, G128: 128, MX: 32}[mode]
+        H = int(unit * rng.integers(1, max(2, 8192 // unit) + 1))
+        out.append((i, mode, int(rng.integers(2, 9)), int(rng.choice([1, 2, 7, 16, 63, 200])), H,
+                    bool(rng.integers(0, 4) > 0)))
+    return out
+
+
+@pytest.mark.parametrize("i,mode,world,M,H,has_res", _random_ar_cases(24),
+                         ids=[f"r{c[0]}" for c in _random_ar_cases(24)])
+def test_virtual_ranks_random(fnb, i, mode, world, M, H, has_res):
+    """Seeded random groups (2..8 ranks, shards from empty to many rows, any
+    H the mode allows up to 8192, with or without a residual)."""
+    wl = synth.RowWorkload("ar_rand", M=M, H=H, P=world, mode=mode, eps=1e-6, seed=500 + i,
+                           residual=has_res, channel_decades=1.0)
+    inp = wl.inputs(device="cuda")
+    parts, res0, w = inp["parts"], inp["residual"], inp["weight"]
+    bufs = _rank_buffers(fnb, mode, M, H, world)
+    for b in bufs:
+        b["residual"] = res0.clone() if has_res else torch.empty((M, H), dtype=torch.bfloat16,
+                                                                 device="cuda")
+    ptr = lambda key: [b[key].data_ptr() for b in bufs]  # noqa: E731
+    for r in range(world):
+        st = fnb.fn_ar_rmsnorm_quant([p.data_ptr() for p in parts], world, r,
+                                     bufs[r]["residual"].data_ptr() if has_res else None,
+                                     w.data_ptr(), wl.eps, mode, M, H, ptr("q"), ptr("scale"),
+                                     ptr("residual"), ptr("y"), None)
+        assert st == fnb.FN_OK, fnb.fn_status_string(st)
+    torch.cuda.synchronize()
+    for b in bufs[1:]:
+        for key in ("q", "scale", "residual", "y"):
+            assert torch.equal(b[key].view(torch.uint8), bufs[0][key].view(torch.uint8)), key
+    gpu = {"q": gpu_util.u8(bufs[0]["q"]), "scale": gpu_util.scale_np(bufs[0]["scale"], mode),
+           "residual_out": gpu_util.bits(bufs[0]["residual"]), "y": gpu_util.bits(bufs[0]["y"])}
+    parity.check_rmsnorm(mode, wl.eps, [gpu_util.bits(p) for p in parts],
+                         gpu_util.bits(res0) if has_res else None, gpu_util.bits(w), gpu)
+
+
 def test_virtual_ranks_swizzled_scales_no_residual(fnb):
     M, H, world = 130, 7168, 4
     SW = fnb.FN_SCALE_SWIZZLE_32_4_4

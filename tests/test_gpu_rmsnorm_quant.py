@@ -453,7 +453,7 @@ def _random_cases(n, seed=2024):
     for i in range(n):
         mode = int(rng.integers(0, 3))
         unit = {TOKEN: 8, G128: 128, MX: 32}[mode]
-        H = int(unit * rng.integers(1, max(2, 4096 // unit) + 1))
+        H = int(unit * rng.integers(1, max(2, (8192 if i % 4 == 0 else 4096) // unit) + 1))
         M = int(rng.choice([1, 2, 5, 16, 17, 63, 150, 151, 300, 333]))
         P = int(rng.integers(1, 9))
         out.append((i, mode, M, H, P, bool(rng.integers(0, 4) > 0), bool(rng.integers(0, 3) == 0),
@@ -461,8 +461,8 @@ def _random_cases(n, seed=2024):
     return out
 
 
-@pytest.mark.parametrize("i,mode,M,H,P,has_res,fp16,variant", _random_cases(48),
-                         ids=[f"r{c[0]}" for c in _random_cases(48)])
+@pytest.mark.parametrize("i,mode,M,H,P,has_res,fp16,variant", _random_cases(120),
+                         ids=[f"r{c[0]}" for c in _random_cases(120)])
 def test_random_shapes(fnb, i, mode, M, H, P, has_res, fp16, variant):
     """Seeded random shapes, partial counts, formats and kernels (any H the
     mode allows up to 4096, M across the dispatch switches) against the
