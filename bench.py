@@ -2,17 +2,21 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-A step is one fused call over the prefill MXFP4 workload (M=8192 rows of
-H=7168, P=4 same-device partial buffers summed in the kernel, residual add,
-RMSNorm, MXFP4 quantization): every step of the hot path on one batch.
-`value` is rows/s over all ranks (weak scaling: each rank owns its own 8192
-rows, no collective on the data path).  Inputs are larger than L2 (587 MB),
-so no flush is needed between steps.
+The workload is the largest one-GPU configuration, the large prefill
+per-group-128 FP8 pass: M=32768 rows of H=8192, x = 2 N(0,1), residual
+N(0,1) updated in place, RMSNorm, per-group-128 E4M3 quantization.  A step is
+192 back-to-back fused calls, alternating between two independently drawn
+input slabs (each call reads 1.07 GB, far more than L2, so no flush is
+needed); every call runs every step of the hot path on its rows.  A step
+lasts about 55 ms, so even 20 steps time about a second.  `value` is rows/s
+over all ranks (weak scaling: each rank owns its own rows, no collective on
+the data path); `us_per_call` and the roofline figures are per launch.
 
-Rank 0 prints one JSON line.  It also carries, for N=1, the secondary
-workloads (large prefill group-128 in place, per-token decode at M=16, the
-decode sweep per mode, the QK prologue), each timed with CUDA events, and the
-CPU oracle timed on a bounded sample of the same workload.
+Rank 0 prints one JSON line.  For N=1 it also carries the secondary workloads
+(prefill MXFP4 with four partials, float16 rows, the quantization step alone,
+per-token decode at M=16, the decode sweep per mode, the QK prologue), each
+timed with CUDA events, and the CPU oracle timed on a bounded sample of the
+same workload.
 
 `--impl reference` times the CPU oracle instead (the method's plain
 definition; there is no runnable GPU reference for this path) on the same
@@ -36,6 +40,7 @@ if ROOT not in sys.path:
 
 METRIC = "rows/s and achieved HBM GB/s (% of B200 peak); µs/call at M≤16"
 L2_BYTES = 126 * 1024 * 1024
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (context beside the measured copy peak)
 
 
 # ---------------------------------------------------------------------------
@@ -249,38 +254,62 @@ def hbm_peak():
 MODE_NAMES = {0: "fp8_per_token", 1: "fp8_per_group128", 2: "mxfp4"}
 
 
-def workload_config(wl, world: int) -> dict:
+# One benchmark step: this many back-to-back fused calls, alternating between
+# two input slabs of the workload, so that even the driver's short runs
+# (20 steps) time about a second of work and the clock sampler (one sample
+# per 50 ms) sees the timed region.
+CALLS_PER_STEP = 192
+SLABS = 2
+
+
+def workload_config(wl, world: int, calls_per_step: int = 1) -> dict:
     """The `config` object of the JSON line (both arms)."""
+    in_mb = wl.M * wl.H * 2 * (wl.P + (1 if wl.residual else 0)) / 1e6
     return {"workload": wl.name, "M": wl.M, "H": wl.H, "P": wl.P, "mode": MODE_NAMES[wl.mode],
-            "eps": wl.eps, "rows_per_gpu": wl.M, "in_place": wl.in_place,
+            "eps": wl.eps, "calls_per_step": calls_per_step,
+            "rows_per_step_per_gpu": wl.M * calls_per_step, "in_place": wl.in_place,
             "io": "bf16 in; codes + scales + bf16 residual out",
-            "l2": f"inputs larger than L2 ({wl.M * wl.H * 2 * (wl.P + 1) / 1e6:.0f} MB read per"
-                  " step), no flush",
+            "l2": f"each call reads {in_mb:.0f} MB of inputs (L2 is 126 MB) and calls alternate "
+                  f"between {SLABS} input slabs: no flush needed",
             "parallelism": f"dp{world} (independent rows, no collective)"}
 
 
-def make_row_call(fn, wl, device, seed):
+def make_row_step(fn, wl, device, seed, calls: int = 1, slabs: int = 1):
+    """A step of `calls` fused calls through the C ABI, alternating between
+    `slabs` independently drawn input sets of the workload (each with its own
+    outputs; with an in-place workload each slab's residual is updated in
+    place by every call on it)."""
     import torch
     from mxfp4_quantization_b200 import synth
-    wl = synth.RowWorkload(**{**wl.__dict__, "seed": seed})
-    inp = wl.inputs(device=device)
-    parts, res, w = inp["parts"], inp["residual"], inp["weight"]
     mode = wl.mode | (fn.FN_IO_FP16 if wl.dtype == torch.float16 else 0)
-    q, s = fn.alloc_outputs(mode, wl.M, wl.H, device)
-    r_out = res if wl.in_place else torch.empty_like(res)
-    ptrs = [p.data_ptr() for p in parts]
+    sets = []
+    for i in range(slabs):
+        wli = synth.RowWorkload(**{**wl.__dict__, "seed": seed + 7919 * i})
+        inp = wli.inputs(device=device)
+        parts, res, w = inp["parts"], inp["residual"], inp["weight"]
+        q, s = fn.alloc_outputs(mode, wl.M, wl.H, device)
+        r_out = res if wl.in_place else torch.empty_like(res)
+        sets.append({"parts": parts, "ptrs": [p.data_ptr() for p in parts], "residual": res,
+                     "weight": w, "q": q, "scale": s, "r_out": r_out})
     stream = torch.cuda.current_stream(device)
     sp = stream.cuda_stream
+    args = [(st["ptrs"], len(st["ptrs"]), st["residual"].data_ptr(), st["weight"].data_ptr(),
+             wl.eps, mode, wl.M, wl.H, st["q"].data_ptr(), st["scale"].data_ptr(),
+             st["r_out"].data_ptr(), None, sp) for st in sets]
 
     def step():
-        st = fn.fn_rmsnorm_quant(ptrs, len(ptrs), res.data_ptr(), w.data_ptr(), wl.eps, mode,
-                                 wl.M, wl.H, q.data_ptr(), s.data_ptr(), r_out.data_ptr(), None,
-                                 sp)
-        if st != fn.FN_OK:
-            raise fn.FusedNormError("fn_rmsnorm_quant", st)
+        for i in range(calls):
+            st = fn.fn_rmsnorm_quant(*args[i % slabs])
+            if st != fn.FN_OK:
+                raise fn.FusedNormError("fn_rmsnorm_quant", st)
 
-    return step, stream, {"parts": parts, "residual": res, "weight": w, "q": q, "scale": s,
-                          "r_out": r_out}
+    return step, stream, sets
+
+
+def make_row_call(fn, wl, device, seed):
+    """One fused call per step on one input set."""
+    step, stream, sets = make_row_step(fn, wl, device, seed, 1, 1)
+    return step, stream, sets[0]
 
 
 def e2e_row(fn, wl, device, steps, warmup, seed):
@@ -471,35 +500,19 @@ def secondary_workloads(fn, device, peak):
     import torch
     from mxfp4_quantization_b200 import synth
     res = {}
-    # large prefill, per-group-128, residual in place (inputs 1.07 GB > L2)
-    wl = synth.PREFILL_GROUP128
-    step, stream, keep = make_row_call(fn, wl, device, wl.seed)
-    ms = time_steps(step, 200, 5, device, stream)
+    # prefill MXFP4 with four partials summed in the kernel (inputs 587 MB > L2)
+    wl = synth.PREFILL_MXFP4
+    step, stream, keep = make_row_step(fn, wl, device, wl.seed, 64, SLABS)
+    ms = time_steps(step, 10, 3, device, stream) / 64
     b = wl.bytes_per_call()
-    res["prefill_group128"] = {"M": wl.M, "H": wl.H, "us_per_call": ms * 1e3,
-                               "rows_per_s": wl.M / (ms * 1e-3), "GB_s": b / (ms * 1e-3) / 1e9,
-                               "frac_of_peak": b / (ms * 1e-3) / 1e9 / peak,
-                               "bytes_per_call": b, "variant": fn.fn_last_variant()}
+    res["prefill_mxfp4"] = {"M": wl.M, "H": wl.H, "P": wl.P, "us_per_call": ms * 1e3,
+                            "rows_per_s": wl.M / (ms * 1e-3), "GB_s": b / (ms * 1e-3) / 1e9,
+                            "frac_of_peak": b / (ms * 1e-3) / 1e9 / peak,
+                            "bytes_per_call": b, "variant": fn.fn_last_variant(),
+                            "launch": list(fn.fn_last_launch()),
+                            "traffic": measured_traffic(wl.name)}
     del keep
     torch.cuda.empty_cache()
-
-    # the large-M kernels side by side (the library picks one by shape)
-    cmp = {}
-    for wl in (synth.PREFILL_MXFP4, synth.PREFILL_GROUP128):
-        step, stream, keep = make_row_call(fn, wl, device, wl.seed)
-        b = wl.bytes_per_call()
-        row = {}
-        for name, v in (("row_cta", fn.FN_VARIANT_ROW_CTA), ("row_tma", fn.FN_VARIANT_ROW_TMA)):
-            with fn.prefer_variant(v):
-                ms = time_steps(step, 100, 5, device, stream)
-                got = fn.fn_last_variant()
-            row[name] = {"us_per_call": ms * 1e3, "GB_s": b / (ms * 1e-3) / 1e9,
-                         "frac_of_peak": b / (ms * 1e-3) / 1e9 / peak, "variant": got,
-                         "launch": list(fn.fn_last_launch())}
-        cmp[wl.name] = row
-        del keep
-        torch.cuda.empty_cache()
-    res["large_m_kernels"] = cmp
 
     # the two large-M shapes with float16 rows (FN_IO_FP16: the producer's dtype
     # carried through the tuple; same bytes per call)
@@ -651,7 +664,8 @@ def reference_arm(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {**workload_config(wl, world), "rows_per_step": rows_per_step},
+            "config": workload_config(wl, world, args.calls_per_step),
+            "rows_per_step": rows_per_step,
             "cpu_baseline": {"value": value, "unit": "rows/s", "cores": 1, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0,
@@ -683,7 +697,8 @@ def main_arm(args):
 
     wl = pick_workload(args.workload)
     seed = rank_seed(wl.seed, rank)
-    step, stream, keep = make_row_call(fn, wl, device, seed)
+    calls = args.calls_per_step
+    step, stream, keep = make_row_step(fn, wl, device, seed, calls, SLABS)
     clocks = ClockSampler(local)
     # the sampler needs a moment to start; it runs over the warm-up and the
     # timed steps, and only samples taken while steps run are kept
@@ -696,10 +711,12 @@ def main_arm(args):
     clk = clocks.stop()
     variant, launch = fn.fn_last_variant(), fn.fn_last_launch()
     ms_max = dist_max(ms, device)
-    value = aggregate(wl.M, world, ms_max)
+    value = aggregate(wl.M * calls, world, ms_max)
     bytes_call = wl.bytes_per_call()
     peak, peak_kind = hbm_peak()
-    achieved = bytes_call / (ms * 1e-3) / 1e9
+    us_call = ms * 1e3 / calls  # every launch of the step is the same kernel
+    achieved = bytes_call / (us_call * 1e-6) / 1e9
+    traffic = measured_traffic(wl.name)
     del keep
     torch.cuda.empty_cache()
 
@@ -709,7 +726,7 @@ def main_arm(args):
 
     extra = None
     cpu = cpu_all = None
-    if world == 1 and not args.no_extras and args.workload == "prefill_mxfp4":
+    if world == 1 and not args.no_extras and args.workload == "prefill_group128":
         extra = secondary_workloads(fn, device, peak)
     if world == 1 and not args.no_cpu_baseline:
         rate, rows, el = oracle_rows_per_s(256, args.cpu_seconds, 3 * args.cpu_seconds,
@@ -731,23 +748,29 @@ def main_arm(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": workload_config(wl, world),
+            "config": workload_config(wl, world, calls),
+            "us_per_call": us_call,
             "hbm_GB_s": achieved, "frac_of_peak": achieved / peak,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
-                         "traffic": measured_traffic(wl.name),
+                         "achieved_is": "algorithmic bytes per launch / CUDA-event time per "
+                                        "launch (timed region / launches)",
+                         "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
+                         "traffic": traffic,
+                         "traffic_is": "ncu dram__bytes_read.sum + dram__bytes_write.sum per "
+                                       "launch (profiles/), null if the kernel changed since",
                          "algorithmic_bytes_per_launch": bytes_call,
-                         "kernel": {fn.FN_VARIANT_ROW_TMA: "rq_tma_kernel (TMA-staged, persistent)",
-                                    fn.FN_VARIANT_ROW_CTA: "rq_kernel (one block per row)",
+                         "kernel": {fn.FN_VARIANT_ROW_CTA: "rq_kernel (one block per row)",
                                     fn.FN_VARIANT_ROW_CLUSTER: "rq_kernel (cluster per row)"}.get(
                                         variant, str(variant)),
                          "launch": list(launch), "variant": variant},
             "e2e": {"value": aggregate(wl.M, world, e2e_ms_max), "unit": "rows/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps,
-                    "method": "public tensor API; pinned host buffers; copies in, kernel and "
-                              "copies out on three streams, two buffer sets (steps pipelined)"},
-            "gpu_launches": args.steps,
+                    "method": "public tensor API, one call per e2e step; pinned host buffers; "
+                              "copies in, kernel and copies out on three streams, two buffer "
+                              "sets (steps pipelined)"},
+            "gpu_launches": args.steps * calls,
             "clocks": clk,
             "cpu_baseline": cpu,
             "cpu_baseline_all_cores": cpu_all,
@@ -764,11 +787,13 @@ def main_arm(args):
 def parse(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=12000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", choices=["prefill_mxfp4", "prefill_group128"],
-                    default="prefill_mxfp4", help="the workload a step runs")
+                    default="prefill_group128", help="the workload a step runs")
+    ap.add_argument("--calls-per-step", type=int, default=CALLS_PER_STEP,
+                    help="fused calls per step (alternating between input slabs)")
     ap.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -30,20 +30,19 @@
  *  - bf16 tensors are IEEE bfloat16 bit patterns, row-major, contiguous rows
  *    (row stride H elements unless a stride argument says otherwise).
  *  - Every data pointer is a DEVICE pointer owned by the caller.  The library
- *    allocates nothing and never synchronizes (fn_device_status excepted):
- *    work is queued on `stream` (a cudaStream_t passed as void*; NULL means
- *    the legacy default stream).  Its only state: thread-local settings and
- *    a record of the last dispatch, a per-device cache of device facts, and
- *    one static device status word.
+ *    allocates nothing and never synchronizes: work is queued on `stream` (a
+ *    cudaStream_t passed as void*; NULL means the legacy default stream).
+ *    Its only state: thread-local settings, a record of the last dispatch,
+ *    and a cache of occupancy queries.
  *  - All argument checks run on the host before anything is launched; on any
  *    error nothing is launched and no output is touched.  M == 0 returns
  *    FN_OK and launches nothing once the sizes and the mode are valid; the
  *    data pointers are not examined then and may be NULL (an empty torch
  *    tensor has a NULL data pointer).
  *  - A launch that the CUDA runtime rejects returns FN_ERR_CUDA.
- *  - Calls are thread-safe.  No kernel waits on another thread block.  The
- *    TMA-staged kernel waits on its own bulk copies with a bounded poll
- *    (see fn_device_status).
+ *  - Calls are thread-safe.  No kernel waits on another thread block or on
+ *    another kernel (beyond the launch ordering of the stream), so no kernel
+ *    of the library has a device-side wait that could fail to end.
  */
 #ifndef FUSEDNORM_H
 #define FUSEDNORM_H
@@ -72,8 +71,7 @@ typedef enum {
     FN_ERR_INVALID = -1,     /* null pointer, bad size, bad mode, forbidden overlap */
     FN_ERR_ALIGN = -2,       /* a pointer or stride breaks the alignment rule      */
     FN_ERR_UNSUPPORTED = -3, /* valid request outside the built shapes (e.g. H)    */
-    FN_ERR_CUDA = -4,        /* the CUDA runtime rejected the launch               */
-    FN_ERR_TIMEOUT = -5      /* a bounded device wait gave up (fn_device_status)   */
+    FN_ERR_CUDA = -4         /* the CUDA runtime rejected the launch               */
 } fn_status;
 
 /* Which kernel the calling thread's last successful call launched. */
@@ -83,7 +81,7 @@ typedef enum {
     FN_VARIANT_ROW_CLUSTER = 2, /* a cluster of 2..8 blocks per row (small M, long rows) */
     FN_VARIANT_QUANT_ONLY = 3,  /* fn_quant                                        */
     FN_VARIANT_QK_WARP = 4,     /* fn_qk_norm_gate: one warp per (token, head)     */
-    FN_VARIANT_ROW_TMA = 5,     /* persistent blocks, rows staged by bulk copies  */
+    /* 5 is not used */
     FN_VARIANT_QK_WARP_FP8 = 6, /* fn_qk_norm_gate_fp8                             */
     FN_VARIANT_ROW_ALLREDUCE = 7 /* fn_ar_rmsnorm_quant: one block per row of the shard */
 } fn_variant;
@@ -265,38 +263,25 @@ FN_API int fn_programmatic_launch(int on);
 FN_API int fn_last_variant(void);
 
 /* Launch shape of the calling thread's last launch: out[0] grid blocks,
- * out[1] threads per block, out[2] blocks per cluster (FN_VARIANT_ROW_TMA:
- * 10 * shared-memory stages + row groups), out[3] 16-byte vectors per
- * thread per tensor. */
+ * out[1] threads per block, out[2] blocks per cluster for
+ * FN_VARIANT_ROW_CLUSTER, or, for one block per row (FN_VARIANT_ROW_CTA,
+ * FN_VARIANT_QUANT_ONLY), the L2 prefetch distance in rows (0: no prefetch;
+ * large-M launches start the rows about one wave ahead towards L2, and only
+ * when every partial and the residual is device memory of the current
+ * device: memory of another GPU or of the host is read with plain loads
+ * alone), out[3] 16-byte vectors per thread per tensor. */
 FN_API void fn_last_launch(int32_t out[4]);
 
 /* Thread-local kernel preference for fn_rmsnorm_quant: FN_VARIANT_NONE (the
- * default) lets the library choose by M, H and P; FN_VARIANT_ROW_CTA,
- * FN_VARIANT_ROW_CLUSTER or FN_VARIANT_ROW_TMA asks for that kernel where the
- * shape allows it (the cluster kernel needs a row that splits into 2..8
- * group-aligned segments with M * blocks <= SMs, the TMA kernel at least two
- * row stages in shared memory).  Every kernel meets the same accuracy
- * contract; kernels that reduce a row in another order (block size, cluster
- * split, row groups) may differ from one another by the one-ulp rounding of
- * y it allows, while any one kernel and launch shape always gives the same
- * bits.  Returns the previous preference. */
+ * default) lets the library choose by M, H and P; FN_VARIANT_ROW_CTA or
+ * FN_VARIANT_ROW_CLUSTER asks for that kernel where the shape allows it (the
+ * cluster kernel needs a row that splits into 2..8 group-aligned segments
+ * with M * blocks <= SMs).  Every kernel meets the same accuracy contract;
+ * kernels that reduce a row in another order (block size, cluster split) may
+ * differ from one another by the one-ulp rounding of y it allows, while any
+ * one kernel and launch shape always gives the same bits.  Returns the
+ * previous preference. */
 FN_API int fn_prefer_variant(int variant);
-
-/* Reads and clears the library's device status word on the current device
- * (synchronizes `stream`).  FN_ERR_TIMEOUT means a kernel's bounded wait for
- * its own bulk copies gave up since the last call, so that call's outputs are
- * not valid; FN_OK otherwise.  The word is a static device variable of the
- * library, not an allocation. */
-FN_API int fn_device_status(void* stream);
-
-/* Test hook for the failure path (thread-local, off by default).  While on,
- * FN_VARIANT_ROW_TMA launches make every stage's mbarrier expect 16 bytes more
- * than its copies bring, so the kernel's bounded waits run out: each thread
- * gives up after one second, stops waiting and issuing, and the block
- * finishes; nothing faults or hangs.  Outputs of such a call are not valid and
- * the next fn_device_status returns FN_ERR_TIMEOUT.  No page describes this:
- * it exists to test the timeout path.  Returns the previous setting. */
-FN_API int fn_debug_stall_copies(int on);
 
 /* Library ABI version (major * 100 + minor). */
 FN_API int fn_version(void);

@@ -20,42 +20,7 @@ namespace {
 thread_local int tl_variant = FN_VARIANT_NONE;
 thread_local int32_t tl_launch[4] = {0, 0, 0, 0};
 thread_local int tl_prefer = FN_VARIANT_NONE;
-thread_local int tl_stall_copies = 0;
 thread_local int tl_pdl = 0;  // launch as a programmatic dependent (fn_programmatic_launch)
-
-}  // namespace
-
-// Library status word, one per device that loads the library: a kernel whose
-// bounded wait gives up sets it (it is never part of a computation).
-__device__ int fn_status_word;
-
-namespace {
-
-constexpr int kMaxDevices = 64;
-std::mutex g_dev_mu;
-int* g_status_ptr[kMaxDevices];
-int g_smem_optin[kMaxDevices];
-
-// Per-device facts fetched once with the device current: the device address
-// of the status word and the opt-in shared memory per block.
-bool device_facts(int* dev_out, int** status, int* smem_optin) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
-  std::lock_guard<std::mutex> lk(g_dev_mu);
-  if (!g_status_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, fn_status_word) != cudaSuccess) return false;
-    int optin = 0;
-    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-      return false;
-    g_smem_optin[dev] = optin;
-    g_status_ptr[dev] = static_cast<int*>(p);
-  }
-  *dev_out = dev;
-  *status = g_status_ptr[dev];
-  *smem_optin = g_smem_optin[dev];
-  return true;
-}
 
 struct Range {
   uintptr_t lo, hi;  // [lo, hi)
@@ -112,20 +77,6 @@ RQKernel pick_exact_kernel(int mode, int P, int T, int V, bool f16, bool norm = 
   return nullptr;
 }
 
-using fn::RQTmaKernel;
-
-RQTmaKernel pick_tma_kernel(int mode, int P, int V, bool f16) {
-  const int maxp = P == 1 ? 1 : P == 2 ? 2 : P <= 4 ? 4 : 8;
-#define FN_CASE(MODE, MAXP)                                                                \
-  if (mode == MODE && maxp == MAXP)                                                        \
-    return f16 ? fn::rq_tma_pick_##MODE##_##MAXP##_1(V) : fn::rq_tma_pick_##MODE##_##MAXP##_0(V);
-  FN_CASE(0, 1) FN_CASE(0, 2) FN_CASE(0, 4) FN_CASE(0, 8)
-  FN_CASE(1, 1) FN_CASE(1, 2) FN_CASE(1, 4) FN_CASE(1, 8)
-  FN_CASE(2, 1) FN_CASE(2, 2) FN_CASE(2, 4) FN_CASE(2, 8)
-#undef FN_CASE
-  return nullptr;
-}
-
 // Smallest power-of-two V in {1..vmax} with ceil(nvec / V) <= max_threads.
 int vectors_per_thread(int nvec, int max_threads, int vmax) {
   int V = 1;
@@ -135,15 +86,33 @@ int vectors_per_thread(int nvec, int max_threads, int vmax) {
 
 int row_vectors_per_thread(int nvec) { return vectors_per_thread(nvec, 256, 16); }
 
-constexpr int kTmaMaxStages = 8;
 // L2 prefetch distance, in rows, of the one-block-per-row kernel, in units of
 // SMs: a block starts the row 2 * #SMs blocks later towards L2, about one
 // wave ahead.  Measured on B200 (prefill MXFP4 H=7168 P=4 / group-128
 // H=8192 P=1): 0 -> 121.8 / 315 us, 2 SMs' worth -> 114.6 / 281-305 us;
-// 4 SMs' worth and more is slower again.  The TMA ring gains nothing from it
-// (120 -> 128 us with any distance), so it does not prefetch.
+// 4 SMs' worth and more is slower again.
 constexpr int kRowPrefetchSms = 2;
-constexpr int kTmaStaticSmem = 2 * 2 * 16 * 8 + 8 * 4;  // reduction slots and stage tags
+
+// True when `p` is device memory of device `dev`.  The L2 bulk prefetch is
+// issued only on such memory: a partial that lives on a peer GPU (the
+// one-stage form of the fused all-reduce passes the peers' partials here) or
+// in host memory is read with plain loads alone, so no bulk operation ever
+// takes another device's memory as its source.
+bool on_device(const void* p, int dev) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice && a.device == dev;
+}
+
+// Every row input of a call (the partials and the residual) is on `dev`.
+bool rows_on_device(const fn::RQParams& p, int dev) {
+  for (int i = 0; i < p.P; ++i)
+    if (!on_device(p.parts[i], dev)) return false;
+  return p.residual == nullptr || on_device(p.residual, dev);
+}
 
 // Launch `k(args...)` on `st`: with a cluster dimension when `cluster` > 1,
 // and, when the calling thread asked for it (fn_programmatic_launch), as a
@@ -236,18 +205,6 @@ RQKernel wide_row_block(int mode, int P, int nvec, bool f16, int* T, int* V) {
   return nullptr;
 }
 
-// Stages of the TMA ring that fit in shared memory (0 when fewer than 2 fit).
-int tma_stages(int64_t stage_bytes, int smem_optin) {
-  const int64_t avail = (int64_t)smem_optin - kTmaStaticSmem - 1024;
-  int n = (int)std::min<int64_t>(kTmaMaxStages, avail / (stage_bytes + 8));
-  return n >= 2 ? n : 0;
-}
-
-// The TMA ring is taken only on request (fn_prefer_variant): with the L2
-// prefetch above, one block per row keeps enough bytes in flight and is the
-// faster large-M kernel on B200 for every shape measured (MXFP4 H=7168 P=4:
-// 114.6 us vs 120.1 us; group-128 H=8192 P=1: 281-305 us vs 395 us).
-
 // Cluster size for a small-M launch: the largest C in 2..8 that splits the
 // row into equal segments aligned to the quantization group, each at most 512
 // vectors, with M * C blocks fitting on the GPU at once.  0 when none fits.
@@ -334,53 +291,16 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, bo
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   fn::RQParams p = prm;
 
-  int dev = 0, smem_optin = 0;
-  if (!device_facts(&dev, &p.status, &smem_optin)) return FN_ERR_CUDA;
-
   const int pref = tl_prefer;
   // Decode-sized M: one wide block per row when one fits (see wide_row_block).
   int wide_T = 0, wide_V = 0;
   RQKernel wide_k = nullptr;
-  if (norm && M <= sms && pref != FN_VARIANT_ROW_CLUSTER && pref != FN_VARIANT_ROW_TMA)
+  if (norm && M <= sms && pref != FN_VARIANT_ROW_CLUSTER)
     wide_k = wide_row_block(mode, P, nvec, f16, &wide_T, &wide_V);
   int C = norm && !wide_k ? pick_cluster(M, nvec, mode, sms) : 0;
-  if (pref == FN_VARIANT_ROW_CTA || pref == FN_VARIANT_ROW_TMA) C = 0;
+  if (pref == FN_VARIANT_ROW_CTA) C = 0;
 
-  const int ntensor = P + (prm.residual ? 1 : 0);
-  const int64_t stage_bytes = (int64_t)ntensor * nvec * 16;
-  const int nst = tma_stages(stage_bytes, smem_optin);
-  const bool tma = norm && nst > 0 && pref != FN_VARIANT_ROW_CTA &&
-                   pref != FN_VARIANT_ROW_CLUSTER &&
-                   pref == FN_VARIANT_ROW_TMA;
-
-  if (tma) {
-    // Two row groups of up to 256 threads each, so one group's per-row latency
-    // (reduction, rstd, scales) overlaps the other's arithmetic.
-    const int V = vectors_per_thread(nvec, 256, 8);
-    const int group_threads = round32((nvec + V - 1) / V);
-    const int groups = (int)std::min<int64_t>(2, (M + sms - 1) / sms);
-    const int threads = group_threads * groups;
-    if (group_threads > 256) return FN_ERR_UNSUPPORTED;
-    RQTmaKernel k = pick_tma_kernel(mode, P, V, f16);
-    if (!k) return FN_ERR_UNSUPPORTED;
-    const size_t smem = (size_t)nst * (size_t)(stage_bytes + 8);
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess) {
-      (void)cudaGetLastError();
-      return FN_ERR_CUDA;
-    }
-    const int64_t grid = std::min<int64_t>(M, sms);
-    p.seg = nvec;
-    p.debug_extra_tx = tl_stall_copies ? 16u : 0u;
-    p.prefetch_rows = 0;
-    if (launch_kernel(k, (unsigned)grid, (unsigned)threads, smem, st, 1, p, nst, groups) != FN_OK)
-      return FN_ERR_CUDA;
-    tl_variant = FN_VARIANT_ROW_TMA;
-    tl_launch[0] = (int32_t)grid;
-    tl_launch[1] = threads;
-    tl_launch[2] = nst * 10 + groups;
-    tl_launch[3] = V;
-  } else if (C >= 2) {
+  if (C >= 2) {
     p.seg = nvec / C;
     const int threads = round32(p.seg);
     RQKernel k = pick_kernel(mode, P, 1, true, true, f16);
@@ -396,6 +316,11 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, bo
     int V = wide_k ? wide_V : row_vectors_per_thread(nvec);
     p.seg = nvec;
     p.prefetch_rows = M > (int64_t)kRowPrefetchSms * sms ? kRowPrefetchSms * sms : 0;
+    if (p.prefetch_rows > 0) {
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess) return FN_ERR_CUDA;
+      if (!rows_on_device(p, dev)) p.prefetch_rows = 0;
+    }
     int threads = wide_k ? wide_T : round32((nvec + V - 1) / V);
     RQKernel k = wide_k;
     if (!k && threads * V == nvec) k = pick_exact_kernel(mode, P, threads, V, f16, norm);
@@ -419,7 +344,7 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, bo
     tl_variant = norm ? variant_if_norm : FN_VARIANT_QUANT_ONLY;
     tl_launch[0] = (int32_t)M;
     tl_launch[1] = threads;
-    tl_launch[2] = 1;
+    tl_launch[2] = p.prefetch_rows;
     tl_launch[3] = V;
   }
   return FN_OK;
@@ -539,28 +464,10 @@ int fn_prefer_variant(int variant) {
   return old;
 }
 
-int fn_debug_stall_copies(int on) {
-  const int old = tl_stall_copies;
-  tl_stall_copies = on ? 1 : 0;
-  return old;
-}
-
 int fn_programmatic_launch(int on) {
   const int old = tl_pdl;
   tl_pdl = on ? 1 : 0;
   return old;
-}
-
-int fn_device_status(void* stream) {
-  int dev = 0, optin = 0;
-  int* p = nullptr;
-  if (!device_facts(&dev, &p, &optin)) return FN_ERR_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int h = 0;
-  if (cudaMemcpyAsync(&h, p, sizeof h, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-      cudaMemsetAsync(p, 0, sizeof h, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
-    return FN_ERR_CUDA;
-  return h ? FN_ERR_TIMEOUT : FN_OK;
 }
 
 void fn_last_launch(int32_t out[4]) {
@@ -574,7 +481,6 @@ const char* fn_status_string(int status) {
     case FN_ERR_ALIGN: return "misaligned pointer or stride";
     case FN_ERR_UNSUPPORTED: return "shape outside the built kernels";
     case FN_ERR_CUDA: return "CUDA launch failed";
-    case FN_ERR_TIMEOUT: return "timed out";
     default: return "unknown status";
   }
 }
@@ -704,10 +610,8 @@ int fn_ar_rmsnorm_quant(const void* const* x_parts, int num_ranks, int rank, con
 
   const int sms = sm_count();
   if (sms <= 0) return FN_ERR_CUDA;
-  int dev = 0, smem_optin = 0;
   fn::ARParams ap;
   std::memset(&ap, 0, sizeof ap);
-  if (!device_facts(&dev, &ap.rq.status, &smem_optin)) return FN_ERR_CUDA;
   fn::RQParams& prm = ap.rq;
   for (int d = 0; d < n; ++d) prm.parts[d] = static_cast<const uint4*>(x_parts[d]);
   prm.residual = static_cast<const uint4*>(residual);

@@ -79,15 +79,4 @@ RQKernel FN_CAT(rq_exact_pick, FN_INST_MODE, FN_INST_MAXP)(int T, int V, bool no
   return nullptr;
 }
 
-RQTmaKernel FN_CAT(rq_tma_pick, FN_INST_MODE, FN_INST_MAXP)(int V) {
-  constexpr int MODE = FN_INST_MODE, MAXP = FN_INST_MAXP;
-  using IO = std::conditional_t<FN_INST_IO == 1, F16, Bf16>;
-  switch (V) {
-    case 1: return rq_tma_kernel<MODE, MAXP, 1, IO>;
-    case 2: return rq_tma_kernel<MODE, MAXP, 2, IO>;
-    case 4: return rq_tma_kernel<MODE, MAXP, 4, IO>;
-    default: return rq_tma_kernel<MODE, MAXP, 8, IO>;
-  }
-}
-
 }  // namespace fn

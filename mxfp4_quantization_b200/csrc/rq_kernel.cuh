@@ -6,15 +6,15 @@
 // the quantization of the bf16 normed row that sgl-amd-mono PR #26's monokernel
 // notes call bit-exact against stand-alone quantization.
 //
-// HBM-bound, no tensor cores.  Three kernels share the per-vector stages below:
+// HBM-bound, no tensor cores.  Two forms of one kernel share the per-vector
+// stages below:
 //  * rq_kernel, CL = false: one thread block per row.  Every load of the row
 //    is issued before the first arithmetic; the row then lives in registers.
+//    Large-M launches also start rows about one wave ahead towards L2 with a
+//    bulk prefetch (cp.async.bulk.prefetch.L2, nothing waits on it).
 //  * rq_kernel, CL = true (small M with rows too long for one wide block, or on
 //    request): a cluster of 2..8 blocks per row; the blocks exchange their
 //    partial sums through distributed shared memory.
-//  * rq_tma_kernel (large M): one persistent block per SM; a ring of shared
-//    memory stages is filled by bulk asynchronous copies (cp.async.bulk, the
-//    TMA engine, no multicast) several rows ahead of the row being computed.
 // A thread owns 16-byte vectors (8 bf16) with index seg_base + threadIdx.x +
 // k * blockDim.x, so a warp touches 512 contiguous bytes per tensor per k.
 // MX blocks (32 elements) are 4 adjacent lanes and FP8 groups (128) 16
@@ -393,242 +393,6 @@ __global__ void __launch_bounds__((CL || TB > 256) ? 512 : 256)
     // No block may leave while a peer can still read its shared-memory slot.
     cluster_wait();
   }
-}
-
-// ---------------------------------------------------------------------------
-// TMA-staged persistent kernel (large M)
-// ---------------------------------------------------------------------------
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Wait for the phase with the given parity to complete.  Bounded in time:
-// gives up and returns false once `deadline` (globaltimer ns) has passed.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t deadline) {
-  const uint32_t a = smem_addr(bar);
-  while (true) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(a), "r"(parity), "r"(20000u)
-        : "memory");
-    if (done) return true;
-    if (global_ns() > deadline) return false;
-  }
-}
-
-// Bulk asynchronous copy global -> this block's shared memory (no multicast);
-// completion is counted in bytes on `bar`.  16-byte aligned, size % 16 == 0.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
-
-// A wait on the block's own bulk copies gives up after this long (one second;
-// a healthy copy lands in microseconds).
-constexpr uint64_t kWaitNs = 1000000000ull;
-
-// Row index published per stage (release) and read before the parity wait
-// (acquire): see rq_tma_kernel.
-__device__ __forceinline__ void tag_store(int* p, int v) {
-  asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(p)), "r"(v) : "memory");
-}
-__device__ __forceinline__ int tag_load(const int* p) {
-  int v;
-  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)) : "memory");
-  return v;
-}
-
-// Wait (bounded in time, see mbar_wait) until `tag` holds `want`.
-__device__ __forceinline__ bool tag_wait(const int* tag, int want, uint64_t deadline) {
-  while (true) {
-    if (tag_load(tag) == want) return true;
-    if (global_ns() > deadline) return false;
-    __nanosleep(64);
-  }
-}
-
-// Named barrier over the `count` threads of one row group (id 1 + group).
-__device__ __forceinline__ void group_barrier(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-// Sum of `s` and max of `m` over one row group of `tg` threads (whole warps),
-// combined in a fixed order (warps in index order).
-template <bool WANT_MAX>
-__device__ __forceinline__ float2 group_reduce(float s, float m, float2* red, int g, int tg,
-                                               int t) {
-  s = warp_sum(s);
-  if (WANT_MAX) m = warp_max(m);
-  const int lane = t & 31, warp = t >> 5, nw = tg >> 5;
-  if (lane == 0) red[warp] = make_float2(s, m);
-  group_barrier(1 + g, tg);
-  float2 r = red[0];
-  for (int i = 1; i < nw; ++i) {
-    const float2 o = red[i];
-    r.x += o.x;
-    if (WANT_MAX) r.y = fmaxf(r.y, o.y);
-  }
-  return r;
-}
-
-// Shared memory: nstages stages of (P + has_res) row segments of H bf16, then
-// one mbarrier per stage.  Block b handles rows b, b + gridDim.x, ...; its
-// threads form `groups` row groups of blockDim.x / groups threads (whole
-// warps) that take the block's rows in turn, each group synchronising on its
-// own named barrier, so one group's reduction and scale latency overlaps the
-// other's arithmetic.  The copies of the next rows are in flight while rows
-// are computed: a stage is refilled, by the group that read it, as soon as
-// that group has it in registers (after the sum-of-squares barrier), before
-// rstd, y and the codes.
-//
-// A stage is consumed by the groups in turn (row i by group i % groups), so a
-// group skips phases of a stage's mbarrier, and a parity wait alone could be
-// satisfied by an older completed phase of the same parity.  Each stage
-// therefore carries the index of the row last issued into it; a group first
-// waits (bounded) for its row's index there, which also proves that the
-// stage's previous row has been consumed, and only then waits on the parity.
-template <int MODE, int MAXP, int V, class IO = Bf16>
-__global__ void __launch_bounds__(512, 1)
-    rq_tma_kernel(const __grid_constant__ RQParams prm, int nstages, int groups) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float2 red[2][2][16];  // [group][buffer][warp]
-  __shared__ int issued[8];         // row index last issued into each stage
-  pdl_enter();
-
-  const int tg = blockDim.x / groups;
-  const int g = threadIdx.x / tg, t = threadIdx.x - g * tg, lane = threadIdx.x & 31;
-  const int nvec = prm.nvec, H = nvec * 8;
-  const bool has_res = prm.residual != nullptr;
-  const int ntensor = prm.P + (has_res ? 1 : 0);
-  const uint32_t seg_bytes = (uint32_t)H * 2u;
-  const uint32_t stage_bytes = seg_bytes * (uint32_t)ntensor;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)nstages * stage_bytes);
-  const int64_t M = prm.M;
-  const int64_t first = blockIdx.x, step = gridDim.x;
-  const int64_t nrows = first < M ? (M - first + step - 1) / step : 0;
-
-  // The weight stays in registers for every row this group handles.
-  uint4 wv[V];
-#pragma unroll
-  for (int k = 0; k < V; ++k) {
-    const int v = t + k * tg;
-    wv[k] = v < nvec ? ld_keep(prm.weight + v) : make_uint4(0u, 0u, 0u, 0u);
-  }
-
-  auto issue = [&](int64_t i) {
-    const int s = (int)(i % nstages);
-    const int64_t row = first + i * step;
-    uint8_t* dst = smem + (size_t)s * stage_bytes;
-    mbar_expect_tx(&full[s], stage_bytes + prm.debug_extra_tx);
-    for (int p = 0; p < prm.P; ++p)
-      bulk_load(dst + (size_t)p * seg_bytes, prm.parts[p] + row * nvec, seg_bytes, &full[s]);
-    if (has_res)
-      bulk_load(dst + (size_t)prm.P * seg_bytes, prm.residual + row * nvec, seg_bytes, &full[s]);
-    tag_store(&issued[s], (int)i);
-    // start the row prefetch_rows further on towards L2, so that its copy
-    // into shared memory finds it there
-    const int64_t ip = i + prm.prefetch_rows;
-    if (prm.prefetch_rows > 0 && ip < nrows) {
-      const int64_t prow = first + ip * step;
-      for (int p = 0; p < prm.P; ++p) bulk_prefetch_l2(prm.parts[p] + prow * nvec, seg_bytes);
-      if (has_res) bulk_prefetch_l2(prm.residual + prow * nvec, seg_bytes);
-    }
-  };
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < nstages; ++s) {
-      mbar_init(&full[s], 1);
-      issued[s] = -1;
-    }
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    for (int64_t i = 0; i < nrows && i < nstages; ++i) issue(i);
-  }
-  __syncthreads();
-
-  // After a wait gives up, the thread stops waiting and its group stops
-  // issuing copies (the stage's mbarrier would be left with an open phase);
-  // it still takes part in every barrier, so the block finishes, and the
-  // status word records the failure.  No copy is left in flight: every copy
-  // issued was for a row whose wait either completed or gave up on its phase
-  // having already received all its bytes.
-  bool timed_out = false;
-  int buf = 0;
-  for (int64_t i = g; i < nrows; i += groups, buf ^= 1) {
-    const int s = (int)(i % nstages);
-    const int64_t row = first + i * step;
-    const int64_t rowv = row * nvec;
-    if (!timed_out) {
-      const uint64_t deadline = global_ns() + kWaitNs;
-      if (!tag_wait(&issued[s], (int)i, deadline) ||
-          !mbar_wait(&full[s], (uint32_t)((i / nstages) & 1), deadline))
-        timed_out = true;
-    }
-    const uint4* st = reinterpret_cast<const uint4*>(smem + (size_t)s * stage_bytes);
-
-    uint4 hv[V];
-    float2 ss = make_float2(0.f, 0.f);
-    float pmax = 0.f;
-#pragma unroll
-    for (int k = 0; k < V; ++k) {
-      const int v = t + k * tg;
-      const bool ok = v < nvec;
-      uint4 x[MAXP];
-#pragma unroll
-      for (int p = 0; p < MAXP; ++p)
-        x[p] = (ok && p < prm.P) ? st[p * nvec + v] : make_uint4(0u, 0u, 0u, 0u);
-      const uint4 r = (ok && has_res) ? st[prm.P * nvec + v] : make_uint4(0u, 0u, 0u, 0u);
-      hv[k] = sum_vec<MAXP, IO>(x, r, prm.P, has_res);
-      stats_vec<MODE == MODE_TOKEN, IO>(hv[k], wv[k], ss, pmax);
-      if (ok && prm.out_residual != nullptr) st_stream(prm.out_residual + rowv + v, hv[k]);
-    }
-    const float2 tot =
-        group_reduce<MODE == MODE_TOKEN>(ss.x + ss.y, pmax, red[g][buf], g, tg, t);
-    // the whole group has read stage s: refill it with the row nstages ahead
-    if (t == 0 && !timed_out && i + nstages < nrows) issue(i + nstages);
-
-    const float rstd = row_rstd(tot.x, prm.inv_h, prm.eps);
-    Fp8Scale scale_tok = {1.f, 1.f, 0.f, false};
-    if (MODE == MODE_TOKEN) {
-      scale_tok = fp8_scale_direct(row_amax_from_pmax<IO>(tot.y, rstd));
-      if (t == 0) static_cast<float*>(prm.out_scale)[row] = scale_tok.s;
-    }
-#pragma unroll
-    for (int k = 0; k < V; ++k) {
-      const int v = t + k * tg;
-      const bool ok = v < nvec;
-      const uint4 y = norm_vec<IO>(hv[k], wv[k], rstd);
-      if (ok && prm.out_y != nullptr) st_stream(prm.out_y + rowv + v, y);
-      quant_store<MODE, IO>(y, ok, lane, row, v, H, scale_tok, prm.out_q, prm.out_scale,
-                            prm.scale_layout, prm.scale_ld);
-    }
-  }
-  if (timed_out && prm.status != nullptr) atomicExch(prm.status, 1);
 }
 
 }  // namespace fn

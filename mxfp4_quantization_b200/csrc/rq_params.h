@@ -24,8 +24,6 @@ struct RQParams {
   int P;                   // partial count, <= MAXP
   float eps;
   float inv_h;             // 1 / H (fp32), for the mean of squares
-  int* status;             // library status word: set to 1 if a bounded wait gave up
-  uint32_t debug_extra_tx; // test hook: extra bytes each TMA stage expects (0 normally)
   int prefetch_rows;       // L2 prefetch distance in rows of this block (0: none); a
                            // positive distance also marks a large-M launch (row_reduce)
   int scale_layout;        // SCALE_*
@@ -39,15 +37,11 @@ using RQKernel = void (*)(const RQParams);
 // Per-(mode, partial bound) instantiation units, each compiled separately
 // (rq_inst.cu) so the library builds in parallel.  `V` is ignored for
 // cluster launches (always one vector per thread there).
-// The TMA-staged persistent kernel takes the stage count and the number of row
-// groups per block as further arguments.
-using RQTmaKernel = void (*)(const RQParams, int, int);
 
 // IO: 0 = bf16 rows, 1 = binary16 rows.
 #define FN_RQ_DECL(MODE, MAXP, IO)                                          \
   RQKernel rq_pick_##MODE##_##MAXP##_##IO(int V, bool cluster, bool norm); \
-  RQKernel rq_exact_pick_##MODE##_##MAXP##_##IO(int T, int V, bool norm);  \
-  RQTmaKernel rq_tma_pick_##MODE##_##MAXP##_##IO(int V);
+  RQKernel rq_exact_pick_##MODE##_##MAXP##_##IO(int T, int V, bool norm);
 #define FN_RQ_DECL_IO(MODE, MAXP) FN_RQ_DECL(MODE, MAXP, 0) FN_RQ_DECL(MODE, MAXP, 1)
 FN_RQ_DECL_IO(0, 1)
 FN_RQ_DECL_IO(0, 2)

@@ -30,14 +30,12 @@ FN_ERR_INVALID = -1
 FN_ERR_ALIGN = -2
 FN_ERR_UNSUPPORTED = -3
 FN_ERR_CUDA = -4
-FN_ERR_TIMEOUT = -5
 
 FN_VARIANT_NONE = 0
 FN_VARIANT_ROW_CTA = 1
 FN_VARIANT_ROW_CLUSTER = 2
 FN_VARIANT_QUANT_ONLY = 3
 FN_VARIANT_QK_WARP = 4
-FN_VARIANT_ROW_TMA = 5
 FN_VARIANT_QK_WARP_FP8 = 6
 FN_VARIANT_ROW_ALLREDUCE = 7
 
@@ -57,8 +55,8 @@ MODES = {"fp8_per_token": FN_FP8_PER_TOKEN, "fp8_per_group128": FN_FP8_PER_GROUP
 ABI_SYMBOLS = ("fn_rmsnorm_quant", "fn_ar_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate",
                "fn_qk_norm_gate_fp8",
                "fn_status_string",
-               "fn_last_variant", "fn_last_launch", "fn_prefer_variant", "fn_device_status",
-               "fn_debug_stall_copies", "fn_programmatic_launch", "fn_version")
+               "fn_last_variant", "fn_last_launch", "fn_prefer_variant",
+               "fn_programmatic_launch", "fn_version")
 
 
 class FusedNormError(RuntimeError):
@@ -96,10 +94,6 @@ def _load():
     lib.fn_last_launch.restype = None
     lib.fn_prefer_variant.argtypes = [i32]
     lib.fn_prefer_variant.restype = i32
-    lib.fn_device_status.argtypes = [vp]
-    lib.fn_device_status.restype = i32
-    lib.fn_debug_stall_copies.argtypes = [i32]
-    lib.fn_debug_stall_copies.restype = i32
     lib.fn_programmatic_launch.argtypes = [i32]
     lib.fn_programmatic_launch.restype = i32
     lib.fn_version.argtypes = []
@@ -178,14 +172,6 @@ def fn_prefer_variant(variant: int) -> int:
     return _lib.fn_prefer_variant(variant)
 
 
-def fn_device_status(stream: Optional[int]) -> int:
-    return _lib.fn_device_status(stream)
-
-
-def fn_debug_stall_copies(on: int) -> int:
-    return _lib.fn_debug_stall_copies(on)
-
-
 def fn_programmatic_launch(on: int) -> int:
     return _lib.fn_programmatic_launch(on)
 
@@ -223,11 +209,6 @@ class prefer_variant:
     def __exit__(self, *exc):
         fn_prefer_variant(self.old)
         return False
-
-
-def device_status() -> int:
-    """fn_device_status on the current stream."""
-    return fn_device_status(torch.cuda.current_stream().cuda_stream)
 
 
 # ---- tensor API ----------------------------------------------------------------------

@@ -12,6 +12,23 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU")
 
 
+# Lines that tests add to the end-of-run summary (the parity statistics of the
+# full-size workloads), printed even in quiet mode.
+_SUMMARY = []
+
+
+@pytest.fixture(scope="session")
+def summary_lines():
+    return _SUMMARY
+
+
+def pytest_terminal_summary(terminalreporter):
+    if _SUMMARY:
+        terminalreporter.write_sep("-", "parity statistics")
+        for line in _SUMMARY:
+            terminalreporter.write_line(line)
+
+
 @pytest.fixture(scope="session")
 def orc():
     """The C oracle, built if needed."""

@@ -111,3 +111,53 @@ def check_rmsnorm(mode, eps, parts_bits, res_bits, w_bits, gpu, io=oracle.IO_BF1
     compare_quant_stage(gpu["y"], gpu["q"], gpu["scale"], mode, io)
     return compare_end_to_end(mode, H, gpu["y"], gpu["q"], gpu["scale"], orc["y"], orc["q"],
                               orc["scale"])
+
+
+# ---- every row of a full-size workload, row-parallel ---------------------------------
+
+def _check_rows_job(job):
+    """Worker (spawned process): the oracle and the criteria above on rows
+    [r0, r1) of arrays saved by check_rmsnorm_all_rows."""
+    d, names, n_parts, mode, eps, io, r0, r1 = job
+    a = {n: np.load(f"{d}/{n}.npy", mmap_mode="r") for n in names}
+    parts = [np.ascontiguousarray(a[f"part{p}"][r0:r1]) for p in range(n_parts)]
+    res = np.ascontiguousarray(a["residual"][r0:r1]) if "residual" in a else None
+    gpu = {"q": np.ascontiguousarray(a["q"][r0:r1]),
+           "scale": np.ascontiguousarray(a["scale"][r0:r1]),
+           "residual_out": (np.ascontiguousarray(a["residual_out"][r0:r1])
+                            if "residual_out" in a else None),
+           "y": np.ascontiguousarray(a["y"][r0:r1])}
+    return check_rmsnorm(mode, eps, parts, res, np.asarray(a["weight"]), gpu, io)
+
+
+def check_rmsnorm_all_rows(mode, eps, parts_bits, res_bits, w_bits, gpu, io=oracle.IO_BF16,
+                           chunk=512, procs=None):
+    """check_rmsnorm over every row, the oracle run row-parallel: one spawned
+    process per host core (spawned, so none inherits the caller's CUDA
+    context), each on chunks of `chunk` rows read from memory-mapped copies.
+    Returns the summed statistics plus the number of rows compared."""
+    import multiprocessing as mp
+    import os
+    import tempfile
+    M = parts_bits[0].shape[0]
+    base = "/dev/shm" if os.path.isdir("/dev/shm") else None
+    with tempfile.TemporaryDirectory(dir=base) as d:
+        arrays = {f"part{p}": x for p, x in enumerate(parts_bits)}
+        arrays["weight"] = w_bits
+        if res_bits is not None:
+            arrays["residual"] = res_bits
+        for k in ("q", "scale", "residual_out", "y"):
+            if gpu.get(k) is not None:
+                arrays[k] = gpu[k]
+        for n, x in arrays.items():
+            np.save(f"{d}/{n}.npy", np.asarray(x))
+        jobs = [(d, tuple(arrays), len(parts_bits), mode, eps, io, r0, min(M, r0 + chunk))
+                for r0 in range(0, M, chunk)]
+        n = procs or os.cpu_count() or 1
+        with mp.get_context("spawn").Pool(min(n, len(jobs))) as pool:
+            results = pool.map(_check_rows_job, jobs)
+    out = {"rows": M}
+    for r in results:
+        for k, v in r.items():
+            out[k] = max(out.get(k, 0), v) if k == "max_step" else out.get(k, 0) + v
+    return out

@@ -41,7 +41,6 @@ def run(fnb, wl, M=None, in_place=False, guarded=True, emit_y=True, device_input
                                 out_scale=gs.t, out_y=None if gy is None else gy.t)
     variant, launch = fnb.fn_last_variant(), fnb.fn_last_launch()
     torch.cuda.synchronize()
-    assert fnb.device_status() == fnb.FN_OK
     for g in (gq, gs, gy, gr):
         assert g is None or g.intact(), "write outside an output"
     gpu = {"q": gpu_util.u8(gq.t), "scale": gpu_util.scale_np(gs.t, wl.mode),
@@ -69,19 +68,15 @@ SHAPES = [
     (64, 4096, 3, False), (33, 1024, 8, True), (7, 32768, 1, True), (200, 2176, 5, True),
     (3, 128, 1, True), (75, 1152, 6, False), (40, 16384, 2, True), (300, 256, 7, True),
     (45, 3584, 8, True), (9, 14336, 3, False), (21, 6144, 2, True),
-    # many rows per block: the persistent kernels wrap their stage ring many times
+    # more rows than two waves of blocks: the L2 prefetch of large-M launches
     (1500, 7168, 4, True), (2400, 1024, 3, True),
 ]
 
 
-VARIANTS = {"auto": 0, "cta": 1, "cluster": 2, "tma": 5}
+VARIANTS = {"auto": 0, "cta": 1, "cluster": 2}
 
 
-def tma_fits(H, P, has_res):
-    return (P + (1 if has_res else 0)) * H * 2 * 2 <= 220 * 1024
-
-
-@pytest.mark.parametrize("variant", ["auto", "cta", "tma"])
+@pytest.mark.parametrize("variant", ["auto", "cta"])
 @pytest.mark.parametrize("mode", [TOKEN, G128, MX], ids=["token", "g128", "mxfp4"])
 @pytest.mark.parametrize("M,H,P,has_res", SHAPES, ids=[f"M{s[0]}_H{s[1]}_P{s[2]}_{'r' if s[3] else 'nr'}" for s in SHAPES])
 def test_parity(fnb, mode, M, H, P, has_res, variant):
@@ -89,11 +84,9 @@ def test_parity(fnb, mode, M, H, P, has_res, variant):
                            seed=M * 31 + H + P, residual=has_res, outlier_frac=0.01,
                            channel_decades=1.0 if P > 1 else 0.0)
     inp, gpu, got, launch = run(fnb, wl, variant=VARIANTS[variant])
-    assert got in (fnb.FN_VARIANT_ROW_CTA, fnb.FN_VARIANT_ROW_CLUSTER, fnb.FN_VARIANT_ROW_TMA)
+    assert got in (fnb.FN_VARIANT_ROW_CTA, fnb.FN_VARIANT_ROW_CLUSTER)
     if variant == "cta":
         assert got == fnb.FN_VARIANT_ROW_CTA
-    if variant == "tma" and tma_fits(H, P, has_res):
-        assert got == fnb.FN_VARIANT_ROW_TMA, launch
     check(wl, inp, gpu)
 
 
@@ -104,7 +97,7 @@ def test_smallest_rows(fnb, mode, H):
     check(wl, inp, gpu)
 
 
-@pytest.mark.parametrize("variant", ["auto", "cta", "tma", "cluster"])
+@pytest.mark.parametrize("variant", ["auto", "cta", "cluster"])
 @pytest.mark.parametrize("mode", [TOKEN, G128, MX])
 def test_in_place_residual(fnb, mode, variant):
     wl = synth.RowWorkload("inplace", M=48, H=8192, P=1, mode=mode, eps=1e-5, seed=5, x_std=2.0)
@@ -171,9 +164,9 @@ def test_empty_and_rejected_calls_touch_nothing(fnb):
                           out_scale=gs.t.view(torch.uint8))
 
 
-@pytest.mark.parametrize("variant", ["cta", "tma"])
-def test_replays_are_bit_identical(fnb, variant):
-    wl = synth.RowWorkload("det", M=300, H=7168, P=4, mode=MX, eps=1e-6, seed=9,
+@pytest.mark.parametrize("variant,M", [("cta", 300), ("cluster", 16)])
+def test_replays_are_bit_identical(fnb, variant, M):
+    wl = synth.RowWorkload("det", M=M, H=7168, P=4, mode=MX, eps=1e-6, seed=9,
                            channel_decades=1.0)
     inp = wl.inputs(device="cuda")
     outs = []
@@ -207,9 +200,11 @@ def test_graph_capture(fnb):
         assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
 
 
-def _sampled_full_size(fnb, wl, n_rows=48):
+def _full_size_all_rows(fnb, wl, summary_lines):
     """Full-size workload on the device in the launch shape the benchmark times
-    (no y side output), then with y for the oracle's sampled rows."""
+    (no y side output), then again from the original residual with y; the two
+    runs agree bit for bit, and every row of the second is compared with the
+    oracle (run row-parallel on the host cores)."""
     inp = wl.inputs(device="cuda")
     parts, w = inp["parts"], inp["weight"]
     res = inp["residual"]
@@ -218,7 +213,6 @@ def _sampled_full_size(fnb, wl, n_rows=48):
     launch_bench = fnb.fn_last_launch()
     q1, s1 = o1.q.clone(), o1.scale.clone()
     r1 = o1.residual_out.clone()
-    # second run from the original residual, with the y side output
     res2 = res0.clone()
     o2 = fnb.rmsnorm_quant(parts, w, wl.eps, wl.mode, residual=res2, in_place=wl.in_place,
                            emit_y=True)
@@ -227,36 +221,29 @@ def _sampled_full_size(fnb, wl, n_rows=48):
     assert torch.equal(q1.view(torch.uint8), o2.q.view(torch.uint8))
     assert torch.equal(s1.view(torch.uint8), o2.scale.view(torch.uint8))
     assert torch.equal(r1, o2.residual_out)
-    # properties at full size: every non-zero group's amax element encodes +-448 (FP8)
-    # and every E8M0 code is finite
-    if wl.mode == MX:
-        assert int(o2.scale.max()) <= 252
-    else:
-        G = wl.H if wl.mode == TOKEN else 128
-        y = o2.y.float().view(wl.M, -1, G).abs()
-        idx = y.argmax(dim=-1, keepdim=True)
-        codes = o2.q.view(torch.uint8).view(wl.M, -1, G).gather(-1, idx)
-        nz = y.amax(dim=-1, keepdim=True) > 0
-        assert bool(((codes & 0x7F) == 0x7E)[nz].all())
-    g = torch.Generator().manual_seed(1)
-    rows = torch.cat([torch.tensor([0, wl.M - 1]), torch.randint(1, wl.M - 1, (n_rows - 2,),
-                                                                  generator=g)]).tolist()
-    sel = torch.tensor(rows, device="cuda")
-    gpu = {"q": gpu_util.u8(o2.q.index_select(0, sel)),
-           "scale": gpu_util.scale_np(o2.scale.index_select(0, sel), wl.mode),
-           "residual_out": gpu_util.bits(o2.residual_out.index_select(0, sel)),
-           "y": gpu_util.bits(o2.y.index_select(0, sel))}
-    parts_b = [gpu_util.bits(p.index_select(0, sel)) for p in parts]
-    return parity.check_rmsnorm(wl.mode, wl.eps, parts_b, gpu_util.bits(res0.index_select(0, sel)),
-                                gpu_util.bits(w), gpu)
+    del q1, s1, r1
+    gpu = {"q": gpu_util.u8(o2.q), "scale": gpu_util.scale_np(o2.scale, wl.mode),
+           "residual_out": gpu_util.bits(o2.residual_out), "y": gpu_util.bits(o2.y)}
+    parts_b = [gpu_util.bits(p) for p in parts]
+    res_b, w_b = gpu_util.bits(res0), gpu_util.bits(w)
+    del inp, parts, res, res0, res2, o1, o2
+    torch.cuda.empty_cache()
+    st = parity.check_rmsnorm_all_rows(wl.mode, wl.eps, parts_b, res_b, w_b, gpu)
+    assert st["rows"] == wl.M
+    summary_lines.append(
+        f"{wl.name} (M={wl.M}, H={wl.H}, P={wl.P}, launch {list(launch_bench)}): all {st['rows']} "
+        f"rows compared with the oracle; codes {st['codes']}, codes_diff {st['codes_diff']}, "
+        f"max_step {st['max_step']}, groups {st['groups']}, scale_diff {st['scale_diff']}, "
+        f"y_flips {st['y_flips']}")
+    return st
 
 
-def test_prefill_mxfp4_full_size(fnb):
-    _sampled_full_size(fnb, synth.PREFILL_MXFP4)
+def test_prefill_mxfp4_full_size(fnb, summary_lines):
+    _full_size_all_rows(fnb, synth.PREFILL_MXFP4, summary_lines)
 
 
-def test_prefill_group128_full_size(fnb):
-    _sampled_full_size(fnb, synth.PREFILL_GROUP128)
+def test_prefill_group128_full_size(fnb, summary_lines):
+    _full_size_all_rows(fnb, synth.PREFILL_GROUP128, summary_lines)
 
 
 def test_per_token_small_config(fnb):
@@ -278,30 +265,6 @@ def test_decode_sweep_config(fnb, M, mode, variant):
     check(wl, inp, gpu)
 
 
-def test_bounded_wait_reports_timeout_and_context_survives(fnb):
-    """Failure path of the TMA kernel without a fault: the test hook makes its
-    stage barriers expect more bytes than arrive, the bounded waits give up
-    after about a second, the call completes, and the status word says so.
-    The next ordinary call works and the status is clean again."""
-    wl = synth.RowWorkload("stall", M=300, H=1024, P=3, mode=MX, eps=1e-6, seed=13)
-    inp = wl.inputs(device="cuda")
-    assert fnb.device_status() == fnb.FN_OK
-    old = fnb.fn_debug_stall_copies(1)
-    try:
-        with fnb.prefer_variant(fnb.FN_VARIANT_ROW_TMA):
-            fnb.rmsnorm_quant(inp["parts"], inp["weight"], wl.eps, MX, residual=inp["residual"])
-            assert fnb.fn_last_variant() == fnb.FN_VARIANT_ROW_TMA
-    finally:
-        fnb.fn_debug_stall_copies(old)
-    torch.cuda.synchronize()
-    assert fnb.device_status() == fnb.FN_ERR_TIMEOUT
-    assert fnb.device_status() == fnb.FN_OK  # read-and-clear
-    # the context is still usable and the kernel correct
-    inp2, gpu, variant, _ = run(fnb, wl, variant=fnb.FN_VARIANT_ROW_TMA)
-    assert variant == fnb.FN_VARIANT_ROW_TMA
-    check(wl, inp2, gpu)
-
-
 # ---- binary16 rows (FN_IO_FP16) ---------------------------------------------------
 
 F16_SHAPES = [
@@ -311,7 +274,7 @@ F16_SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("variant", ["auto", "cta", "tma"])
+@pytest.mark.parametrize("variant", ["auto", "cta"])
 @pytest.mark.parametrize("mode", [TOKEN, G128, MX], ids=["token", "g128", "mxfp4"])
 @pytest.mark.parametrize("M,H,P,has_res", F16_SHAPES,
                          ids=[f"M{s[0]}_H{s[1]}_P{s[2]}" for s in F16_SHAPES])
@@ -325,8 +288,6 @@ def test_fp16_parity(fnb, mode, M, H, P, has_res, variant):
     inp, gpu, got, launch = run(fnb, wl, variant=VARIANTS[variant])
     if variant == "cta":
         assert got == fnb.FN_VARIANT_ROW_CTA
-    if variant == "tma" and tma_fits(H, P, has_res):
-        assert got == fnb.FN_VARIANT_ROW_TMA, launch
     check(wl, inp, gpu)
 
 
@@ -457,7 +418,9 @@ def _random_cases(n, seed=2024):
         M = int(rng.choice([1, 2, 5, 16, 17, 63, 150, 151, 300, 333]))
         P = int(rng.integers(1, 9))
         out.append((i, mode, M, H, P, bool(rng.integers(0, 4) > 0), bool(rng.integers(0, 3) == 0),
-                    int(rng.choice([0, 1, 2, 5]))))
+                    # (the fourth draw once named a kernel that no longer exists; it
+                    # keeps the random stream of the other cases and asks for auto)
+                    int(rng.choice([0, 1, 2, 0]))))
     return out
 
 
@@ -472,5 +435,47 @@ def test_random_shapes(fnb, i, mode, M, H, P, has_res, fp16, variant):
                            channel_decades=1.0 if P > 1 else 0.0,
                            dtype=torch.float16 if fp16 else torch.bfloat16)
     inp, gpu, got, launch = run(fnb, wl, variant=variant)
-    assert got in (fnb.FN_VARIANT_ROW_CTA, fnb.FN_VARIANT_ROW_CLUSTER, fnb.FN_VARIANT_ROW_TMA)
+    assert got in (fnb.FN_VARIANT_ROW_CTA, fnb.FN_VARIANT_ROW_CLUSTER)
+    check(wl, inp, gpu)
+
+
+@pytest.mark.parametrize("host_tensor", ["parts", "residual"])
+def test_l2_prefetch_only_on_this_devices_memory(fnb, host_tensor):
+    """The large-M launch starts rows towards L2 with a bulk prefetch only when
+    every row input is device memory of the current device.  Rows given in
+    another place (here pinned host memory, read over the bus with plain
+    loads, as a peer GPU's partials would be read over NVLink) run without
+    it, and the results still match the oracle; the same rows on the device
+    get the prefetch."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    M = 2 * sms + 40
+    wl = synth.RowWorkload("place", M=M, H=1024, P=2, mode=MX, eps=1e-6, seed=77,
+                           outlier_frac=0.01)
+    inp = wl.inputs(device="cpu")
+    w = inp["weight"].cuda()
+    q, s = fnb.alloc_outputs(MX, M, wl.H, "cuda")
+    r_out = torch.empty((M, wl.H), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((M, wl.H), dtype=torch.bfloat16, device="cuda")
+
+    def call(parts, res):
+        st = fnb.fn_rmsnorm_quant([p.data_ptr() for p in parts], len(parts), res.data_ptr(),
+                                  w.data_ptr(), wl.eps, MX, M, wl.H, q.data_ptr(), s.data_ptr(),
+                                  r_out.data_ptr(), y.data_ptr(),
+                                  torch.cuda.current_stream().cuda_stream)
+        assert st == fnb.FN_OK, fnb.fn_status_string(st)
+        launch = fnb.fn_last_launch()
+        torch.cuda.synchronize()
+        return launch
+
+    dev_parts = [p.cuda() for p in inp["parts"]]
+    dev_res = inp["residual"].cuda()
+    assert call(dev_parts, dev_res)[2] == 2 * sms  # device rows: prefetch one wave ahead
+    if host_tensor == "parts":
+        parts, res = [p.pin_memory() for p in inp["parts"]], dev_res
+    else:
+        parts, res = dev_parts, inp["residual"].pin_memory()
+    launch = call(parts, res)
+    assert fnb.fn_last_variant() == fnb.FN_VARIANT_ROW_CTA and launch[2] == 0, launch
+    gpu = {"q": gpu_util.u8(q), "scale": gpu_util.scale_np(s, MX),
+           "residual_out": gpu_util.bits(r_out), "y": gpu_util.bits(y)}
     check(wl, inp, gpu)

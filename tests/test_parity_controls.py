@@ -101,3 +101,16 @@ def test_code_moved_where_y_did_not_fails_end_to_end():
     with pytest.raises(AssertionError):
         parity.compare_end_to_end(wl.mode, wl.H, gpu["y"], q, gpu["scale"], orc["y"], orc["q"],
                                   orc["scale"])
+
+
+def test_all_rows_runner_passes_exact_and_catches_a_fault_in_a_late_chunk():
+    """The row-parallel runner of the full-size tests (spawned processes over
+    chunks of rows) sums the statistics of every chunk, and a fault planted in
+    the last chunk only still fails the comparison."""
+    wl, parts, res, w, gpu = _case(oracle.FP8_PER_GROUP128, M=70, H=1024)
+    st = parity.check_rmsnorm_all_rows(wl.mode, wl.eps, parts, res, w, gpu, chunk=16, procs=3)
+    assert st["rows"] == 70 and st["codes"] == 70 * 1024 and st["codes_diff"] == 0
+    assert st["groups"] == 70 * 8
+    gpu["q"][69, 5] ^= 0x01
+    with pytest.raises(AssertionError):
+        parity.check_rmsnorm_all_rows(wl.mode, wl.eps, parts, res, w, gpu, chunk=16, procs=3)
