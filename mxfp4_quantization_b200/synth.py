@@ -23,6 +23,11 @@ interleaved gate heads from the fused QK-norm + gate PR):
                     partials; residual ~ N(0,1); w = 1 + 0.1 N(0,1)
   prefill_group128  M=32768, H=8192, P=1; x = 2 N(0,1); residual ~ N(0,1);
                     w = 1 + 0.1 N(0,1); residual updated in place
+  hc_mix            M in {1,2,4,8,16} rows of the hyper-state, hc = 4 streams of
+                    C = 2560 (the hc_mix PR's [M, 4*2560]), rank r = 64;
+                    x ~ N(0,1); W_down [r, hc*C] ~ N(0,1) / sqrt(hc*C);
+                    W_up [hc*C, r] ~ N(0,1) / sqrt(r) (unit-variance gate
+                    logits, so the gates spread over (0, 1))
 """
 import zlib
 from dataclasses import dataclass, field
@@ -156,6 +161,45 @@ class QKWorkload:
         M = self.M if M is None else M
         per_tok = 2 * self.D * (2 * self.Hq + self.Hk) * 2
         return M * per_tok + 2 * 2 * self.D
+
+
+@dataclass
+class HCWorkload:
+    """Inputs of the low-rank gate over the hyper-state (hc_mix)."""
+    name: str
+    M: int
+    hc: int = 4
+    C: int = 2560
+    r: int = 64
+    seed: int = 0
+
+    @property
+    def K(self) -> int:
+        return self.hc * self.C
+
+    def inputs(self, device="cpu", M: Optional[int] = None):
+        M = self.M if M is None else M
+        s, K, r = self.seed, self.K, self.r
+        x = normal_bf16((M, K), s, "x", device=device)
+        w_down = normal_bf16((r, K), s, "w_down", std=K ** -0.5, device=device)
+        w_up = normal_bf16((K, r), s, "w_up", std=r ** -0.5, device=device)
+        return {"x": x, "w_down": w_down, "w_up": w_up}
+
+    def weight_bytes(self) -> int:
+        return 2 * (2 * self.K * self.r)
+
+    def bytes_per_call(self, M: Optional[int] = None) -> int:
+        """Algorithmic HBM bytes: both weight factors, the hyper-state rows
+        and the mixed output (bf16 each)."""
+        M = self.M if M is None else M
+        return self.weight_bytes() + M * self.K * 2 + M * self.C * 2
+
+
+HC_M = (1, 2, 4, 8, 16)
+
+
+def hc_mix(M: int) -> HCWorkload:
+    return HCWorkload(f"hc_mix_m{M}", M=M, seed=5)
 
 
 PER_TOKEN_SMALL = RowWorkload("per_token_small", M=16, H=2048, P=1, mode=FP8_PER_TOKEN,

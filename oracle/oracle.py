@@ -69,6 +69,10 @@ def load(path: str = LIB):
                                          ctypes.c_float, _u8p, _f32p, _u8p, _f32p, _u16p,
                                          _u16p, _u16p]
     lib.orc_qk_norm_gate_fp8.restype = ctypes.c_int
+    lib.orc_hc_mix.argtypes = [_u16p, _u16p, _u16p, ctypes.c_int64, ctypes.c_int,
+                               ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_double),
+                               _u16p]
+    lib.orc_hc_mix.restype = ctypes.c_int
     if path == LIB:
         _lib = lib
     return lib
@@ -235,6 +239,25 @@ def qk_norm_gate_fp8(qkv, row_stride: int, Hq: int, Hk: int, D: int, q_weight, k
     if rc != 0:
         raise OracleError("orc_qk_norm_gate_fp8 rejected the shape")
     return out
+
+
+def hc_mix(x, w_down, w_up, hc: int, C: int, r: int, lib=None):
+    """Low-rank gate over the hyper-state (reading A19 of orc.c).
+
+    x: uint16 bf16 [M, hc*C]; w_down: uint16 bf16 [r, hc*C]; w_up: uint16 bf16
+    [hc*C, r].  Returns (u fp64 [M, C], u_bf16 uint16 [M, C])."""
+    lib = lib or load()
+    xx, wd, wu = _u16(x), _u16(w_down), _u16(w_up)
+    M = xx.shape[0]
+    if xx.shape[1] != hc * C or wd.shape != (r, hc * C) or wu.shape != (hc * C, r):
+        raise OracleError("hc_mix: shapes do not match hc, C, r")
+    u = np.zeros((M, C), dtype=np.float64)
+    ub = np.zeros((M, C), dtype=np.uint16)
+    rc = lib.orc_hc_mix(_p16(xx), _p16(wd), _p16(wu), M, hc, C, r,
+                        u.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), _p16(ub))
+    if rc != 0:
+        raise OracleError("orc_hc_mix rejected the shape")
+    return u, ub
 
 
 # ---- scale layouts ------------------------------------------------------------

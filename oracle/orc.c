@@ -26,6 +26,12 @@
  *  [OCP]  OCP Microscaling (MX) v1.0: shared scale X = 2^(floor(log2 amax) -
  *         emax_elem), emax_elem = 2 for E2M1; E8M0 scale; E4M3 "fn" element
  *         format (max 448, no infinities).
+ *  [HC]   sglang PR #41880, "AITER FlyDSL hc_mix for Qwen3.8 hyper-connections
+ *         on gfx950": "Motivation" (the input mix of GatedResidual is a
+ *         low-rank gate over the [M, 4*2560] hyper-state; decode-sized M <= 16,
+ *         bound by reading the weights), "Modifications" (BF16, contiguous,
+ *         1 <= M <= 16, hc = 4), "Accuracy Tests" (float64 reference,
+ *         atol 4e-3, rtol 1e-2).
  *
  * Readings where the pages are silent (each one is listed in the design
  * notes under the same tag):
@@ -49,6 +55,15 @@
  *      instead of bf16, and every "bf16(...)" rounding above is a binary16
  *      rounding (nearest even, subnormals kept, overflow to infinity).
  *      Codes and scales are unchanged.
+ *  A19 [HC] prints no formula.  Reading: the hyper-state row x holds hc
+ *      streams of C values (stream s at [s*C, (s+1)*C)); the gate has the
+ *      hyper-state's shape, its logits a rank-r linear map of the whole row,
+ *      z = W_up (W_down x) with W_down [r, hc*C] and W_up [hc*C, r] (the two
+ *      low-rank factors, each in the row layout of a linear layer's weight),
+ *      g = logistic sigmoid(z) = 1 / (1 + exp(-z)), and the input mix is the
+ *      gated sum of the streams, u[c] = sum_s g[s*C + c] * x[s*C + c], one
+ *      value per channel: the sublayer's input [M, C].  No bias, no norm
+ *      (the norm is a separate step before the mix).  Evaluated in fp64.
  *
  * Build: plain C99, -O2 -ffp-contract=off, no fast-math, x86-64 SSE float
  * arithmetic (FLT_EVAL_METHOD == 0), so `float` operations are IEEE binary32
@@ -509,5 +524,60 @@ int orc_qk_norm_gate_fp8(const uint16_t* qkv, int64_t M, int64_t row_stride, int
         }
     }
     free(y);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* hc_mix: low-rank gate over the hyper-state ([HC], reading A19)       */
+/* ------------------------------------------------------------------ */
+
+/*
+ * For each row m of x [M, hc*C] (bf16):
+ *     t[j]  = sum_k x[k] * w_down[j, k]            j < r, k < hc*C
+ *     z[e]  = sum_j t[j] * w_up[e, j]              e < hc*C
+ *     g[e]  = 1 / (1 + exp(-z[e]))
+ *     u[c]  = sum_s g[s*C + c] * x[s*C + c]        c < C
+ * every sum in fp64, in index order.  out_u (fp64 [M, C]) receives u and
+ * out_bf16 (bf16 [M, C]), if not NULL, bf16_rn(u).  w_down is bf16 [r, hc*C]
+ * and w_up bf16 [hc*C, r], both row-major.
+ */
+int orc_hc_mix(const uint16_t* x, const uint16_t* w_down, const uint16_t* w_up, int64_t M,
+               int hc, int64_t C, int r, double* out_u, uint16_t* out_bf16)
+{
+    if (M < 0 || hc < 1 || C < 1 || r < 1 || !x || !w_down || !w_up || !out_u)
+        return ORC_BAD;
+    const int64_t K = (int64_t)hc * C;
+    double* t = (double*)malloc((size_t)r * sizeof(double));
+    double* g = (double*)malloc((size_t)K * sizeof(double));
+    if (!t || !g) {
+        free(t);
+        free(g);
+        return ORC_BAD;
+    }
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t* xr = x + m * K;
+        for (int j = 0; j < r; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += orc_bf16_to_double(xr[k]) * orc_bf16_to_double(w_down[(int64_t)j * K + k]);
+            t[j] = acc;
+        }
+        for (int64_t e = 0; e < K; ++e) {
+            double z = 0.0;
+            for (int j = 0; j < r; ++j)
+                z += t[j] * orc_bf16_to_double(w_up[e * r + j]);
+            g[e] = 1.0 / (1.0 + exp(-z));
+        }
+        for (int64_t c = 0; c < C; ++c) {
+            double u = 0.0;
+            for (int s = 0; s < hc; ++s)
+                u += g[(int64_t)s * C + c] * orc_bf16_to_double(xr[(int64_t)s * C + c]);
+            out_u[m * C + c] = u;
+            if (out_bf16)
+                out_bf16[m * C + c] = orc_bf16_from_double(u);
+        }
+    }
+    free(t);
+    free(g);
     return ORC_OK;
 }

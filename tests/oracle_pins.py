@@ -669,3 +669,98 @@ def pin_fp16_path(lib):
 
 
 ALL_PINS += [pin_fp16_format, pin_fp16_path]
+
+
+# ----------------------------------------------------------------------------
+# hc_mix: the low-rank gate over the hyper-state (reading A19)
+# ----------------------------------------------------------------------------
+
+
+def _bf16_bits_f64(a):
+    """float64 values that are exact in bf16 -> their bit patterns."""
+    return f32_to_bf16_bits_torch(np.asarray(a, dtype=np.float32))
+
+
+def _hc_case(seed, M, hc, C, r, wd_std=None, wu_std=None):
+    rng = np.random.default_rng(seed)
+    K = hc * C
+    x = f32_to_bf16_bits_torch(rng.standard_normal((M, K)).astype(np.float32))
+    wd = f32_to_bf16_bits_torch((rng.standard_normal((r, K)) * (wd_std or K ** -0.5)).astype(np.float32))
+    wu = f32_to_bf16_bits_torch((rng.standard_normal((K, r)) * (wu_std or r ** -0.5)).astype(np.float32))
+    return x, wd, wu
+
+
+def pin_hc_mix_worked(lib):
+    """The hand-worked row of tests/golden/hc_mix_worked.json."""
+    d = json.load(open(os.path.join(GOLDEN, "hc_mix_worked.json")))
+    x = _bf16_bits_f64([d["x"]])
+    wd, wu = _bf16_bits_f64(d["w_down"]), _bf16_bits_f64(d["w_up"])
+    u, ub = oracle.hc_mix(x, wd, wu, d["hc"], d["C"], d["r"], lib)
+    assert np.allclose(u[0], d["u"], rtol=0, atol=1e-15), f"hc_mix worked u {u[0]}"
+    assert list(bf16_bits_to_f64(ub[0])) == d["u_bf16"], f"hc_mix worked bf16 {ub[0]}"
+
+
+def pin_hc_mix_closed_forms(lib):
+    """Closed forms and invariants of the gated mix on random rows:
+    zero up-factor -> every gate 1/2 and u = (sum of the streams) / 2, exactly;
+    negated up-factor -> gates 1 - g, so u + u' = sum of the streams;
+    logits of +-40 built through both factors select stream 0 alone;
+    a permutation of the streams (applied to x, to W_down's column blocks and
+    to W_up's row blocks) leaves u unchanged; a permutation of the channels
+    permutes u."""
+    hc, C, r, M = 4, 24, 8, 3
+    K = hc * C
+    x, wd, wu = _hc_case(11, M, hc, C, r)
+    xv = bf16_bits_to_f64(x).reshape(M, hc, C)
+    streams = xv.sum(axis=1)
+    u0, _ = oracle.hc_mix(x, wd, np.zeros_like(wu), hc, C, r, lib)
+    assert np.array_equal(u0, 0.5 * streams), "zero up-factor: u = sum/2"
+    u, _ = oracle.hc_mix(x, wd, wu, hc, C, r, lib)
+    un, _ = oracle.hc_mix(x, wd, wu ^ np.uint16(0x8000), hc, C, r, lib)
+    assert np.allclose(u + un, streams, rtol=0, atol=1e-12), "negated up-factor"
+    # selection: t0 = x[0] = 1 through a one-hot down row; z = +-40 per stream
+    xs = x.copy()
+    xs[:, 0] = 0x3F80  # 1.0
+    wds = np.zeros_like(wd)
+    wds[0, 0] = 0x3F80
+    wus = np.zeros_like(wu)
+    wus[:, 0] = 0xC220  # -40
+    wus[:C, 0] = 0x4220  # +40 on stream 0
+    us, _ = oracle.hc_mix(xs, wds, wus, hc, C, r, lib)
+    xsv = bf16_bits_to_f64(xs).reshape(M, hc, C)
+    assert np.allclose(us, xsv[:, 0, :], rtol=0, atol=1e-15), "selection of stream 0"
+    # stream permutation
+    perm = [2, 0, 3, 1]
+    cols = np.concatenate([np.arange(s * C, (s + 1) * C) for s in perm])
+    up, _ = oracle.hc_mix(x[:, cols], wd[:, cols], wu[cols, :], hc, C, r, lib)
+    assert np.allclose(up, u, rtol=0, atol=1e-12), "stream permutation"
+    # channel permutation
+    cp = np.random.default_rng(5).permutation(C)
+    ccols = np.concatenate([s * C + cp for s in range(hc)])
+    uc, _ = oracle.hc_mix(x[:, ccols], wd[:, ccols], wu[ccols, :], hc, C, r, lib)
+    assert np.allclose(uc, u[:, cp], rtol=0, atol=1e-12), "channel permutation"
+    assert K == x.shape[1]
+
+
+def pin_hc_mix_library(lib):
+    """The whole mix recomputed with library routines on tiny random cases:
+    numpy fp64 matrix products for the two factors, scipy's logistic function
+    for the gate, a sum over the reshaped streams, and the bf16 output by the
+    60-digit nearest search."""
+    from scipy.special import expit
+    for seed, (M, hc, C, r) in enumerate([(1, 4, 8, 8), (5, 4, 16, 4), (3, 2, 40, 16),
+                                          (2, 4, 64, 64)]):
+        x, wd, wu = _hc_case(100 + seed, M, hc, C, r, wd_std=2.0 / (hc * C) ** 0.5,
+                             wu_std=2.0 / r ** 0.5)
+        xv, wdv, wuv = bf16_bits_to_f64(x), bf16_bits_to_f64(wd), bf16_bits_to_f64(wu)
+        g = expit((xv @ wdv.T) @ wuv.T)
+        want = (g * xv).reshape(M, hc, C).sum(axis=1)
+        u, ub = oracle.hc_mix(x, wd, wu, hc, C, r, lib)
+        assert np.allclose(u, want, rtol=1e-12, atol=1e-12), f"hc_mix library case {seed}"
+        getcontext().prec = 60
+        wb = np.array([[nearest_bf16_decimal(Decimal(float(v))) for v in row] for row in u],
+                      dtype=np.uint16)
+        assert np.array_equal(ub, wb), f"hc_mix bf16 output case {seed}"
+
+
+ALL_PINS += [pin_hc_mix_worked, pin_hc_mix_closed_forms, pin_hc_mix_library]

@@ -53,6 +53,19 @@ MUTANTS = [
      "float t = elem_to_float(ORC_IO_BF16, y[j]) / scale;"),
     ("fp16_h_rounded_as_bf16", "hbuf[j] = elem_from_double(io, (double)s);",
      "hbuf[j] = orc_bf16_from_double((double)s);"),
+    # hc_mix (reading A19)
+    ("hc_gate_sign", "g[e] = 1.0 / (1.0 + exp(-z));", "g[e] = 1.0 / (1.0 + exp(z));"),
+    ("hc_gate_tanh", "g[e] = 1.0 / (1.0 + exp(-z));", "g[e] = 0.5 * (1.0 + tanh(z));"),
+    ("hc_streams_interleaved", "u += g[(int64_t)s * C + c] * orc_bf16_to_double(xr[(int64_t)s * C + c]);",
+     "u += g[(int64_t)c * hc + s] * orc_bf16_to_double(xr[(int64_t)c * hc + s]);"),
+    ("hc_gate_applied_to_stream0", "orc_bf16_to_double(xr[(int64_t)s * C + c]);",
+     "orc_bf16_to_double(xr[c]);"),
+    ("hc_w_down_transposed", "orc_bf16_to_double(w_down[(int64_t)j * K + k]);",
+     "orc_bf16_to_double(w_down[k * r + j]);"),
+    ("hc_w_up_transposed", "z += t[j] * orc_bf16_to_double(w_up[e * r + j]);",
+     "z += t[j] * orc_bf16_to_double(w_up[(int64_t)j * K + e]);"),
+    ("hc_last_stream_dropped", "for (int s = 0; s < hc; ++s)", "for (int s = 0; s < hc - 1; ++s)"),
+    ("hc_t_rounded_to_bf16", "t[j] = acc;", "t[j] = orc_bf16_to_double(orc_bf16_from_double(acc));"),
 ]
 
 
