@@ -495,6 +495,33 @@ def qk_calls(fn, wl, device, fp8=False):
     return make
 
 
+def hc_calls(fn, wl, device):
+    """Factory of rotating-weight hc_mix calls: every call of a graph reads its
+    own copy of both weight factors (and of x), enough copies that they exceed
+    L2, so every call reads its weights cold from HBM (the hc_mix page's
+    method: CUDA-graph replay with rotating weights)."""
+    import torch
+
+    def make(n):
+        inp = wl.inputs(device=device)
+        calls = []
+        for i in range(n):
+            x = inp["x"].roll(i, 1).clone()
+            wd = inp["w_down"].roll(i, 1).clone()
+            wu = inp["w_up"].roll(i, 0).clone()
+            out = torch.empty((wl.M, wl.C), dtype=torch.bfloat16, device=device)
+            ws = torch.empty((wl.M * wl.r,), dtype=torch.float32, device=device)
+
+            def call(x=x, wd=wd, wu=wu, out=out, ws=ws):
+                st = fn.fn_hc_mix(x.data_ptr(), wd.data_ptr(), wu.data_ptr(), wl.M, wl.hc, wl.C,
+                                  wl.r, out.data_ptr(), ws.data_ptr(),
+                                  torch.cuda.current_stream(device).cuda_stream)
+                assert st == fn.FN_OK
+            calls.append(call)
+        return calls
+    return make
+
+
 def secondary_workloads(fn, device, peak):
     """Every other workload, each on its own timed region (N=1 only)."""
     import torch
@@ -588,6 +615,21 @@ def secondary_workloads(fn, device, peak):
         b8 = wl.bytes_per_call() - M * (wl.Hq + wl.Hk) * (wl.D - 4)
         qk[f"m{M}_fp8"] = small(wl, b8, qk_calls(fn, wl, device, fp8=True))
     res["qk_prologue"] = qk
+    hc = {}
+    for M in synth.HC_M:
+        wl = synth.hc_mix(M)
+        r = small(wl, wl.bytes_per_call(), hc_calls(fn, wl, device))
+        wb = wl.weight_bytes()
+        r.update({"hc": wl.hc, "C": wl.C, "r": wl.r, "bytes_per_call": wl.bytes_per_call(),
+                  "weight_bytes_per_call": wb,
+                  "weight_GB_s": wb / (r["us_per_call_graph"] * 1e-6) / 1e9,
+                  "weight_GB_s_programmatic": wb / (r["us_per_call_graph_programmatic"] * 1e-6) / 1e9,
+                  "frac_of_peak_programmatic": wl.bytes_per_call()
+                  / (r["us_per_call_graph_programmatic"] * 1e-6) / 1e9 / peak,
+                  "variant": fn.fn_last_variant()})
+        hc[f"m{M}"] = r
+        torch.cuda.empty_cache()
+    res["hc_mix"] = hc
     return res
 
 

@@ -83,7 +83,8 @@ typedef enum {
     FN_VARIANT_QK_WARP = 4,     /* fn_qk_norm_gate: one warp per (token, head)     */
     /* 5 is not used */
     FN_VARIANT_QK_WARP_FP8 = 6, /* fn_qk_norm_gate_fp8                             */
-    FN_VARIANT_ROW_ALLREDUCE = 7 /* fn_ar_rmsnorm_quant: one block per row of the shard */
+    FN_VARIANT_ROW_ALLREDUCE = 7, /* fn_ar_rmsnorm_quant: one block per row of the shard */
+    FN_VARIANT_HC_MIX = 8        /* fn_hc_mix: column-split product, then gate and mix */
 } fn_variant;
 
 /* Scale-layout flags, OR-ed into `mode` (fn_rmsnorm_quant, fn_quant).  No
@@ -244,6 +245,46 @@ FN_API int fn_qk_norm_gate_fp8(const void* qkv, int64_t M, int64_t row_stride, i
                                int D, const void* q_weight, const void* k_weight, float eps,
                                void* out_q8, void* out_q_scale, void* out_k8, void* out_k_scale,
                                void* out_gate, void* out_q, void* out_k, void* stream);
+
+/*
+ * hc_mix: the low-rank gate over the hyper-state (sglang PR #41880,
+ * "Motivation": the input mix of GatedResidual, a low-rank gate over the
+ * [M, 4*2560] hyper-state, decode-sized M <= 16, bound by reading the
+ * weights; "Modifications": BF16, contiguous, 1 <= M <= 16, hc = 4).  The
+ * page prints no formula; per row x of hc streams of C values (stream s at
+ * columns [s*C, (s+1)*C)) this computes
+ *     t    = W_down x                     (fp32, rank r)
+ *     z    = W_up t
+ *     u[c] = sum_s sigmoid(z[s*C + c]) * x[s*C + c],   sigmoid(z) = 1/(1+e^-z)
+ *     out  = bf16_rn(u)                   [M, C]
+ * in fp32 with one rounding to bf16; accuracy against the float64 definition:
+ * |out - u| <= 4e-3 + 1e-2 |u| (the page's "Accuracy Tests").  Two kernels
+ * run, the second launched as a programmatic dependent of the first.
+ *
+ * x          bf16 [M, hc*C], row-major, 16-byte aligned.
+ * w_down     bf16 [r, hc*C] (a linear layer's weight layout: row j is the
+ *            j-th down vector), 16-byte aligned.
+ * w_up       bf16 [hc*C, r], 16-byte aligned.
+ * M          0..16 (above: FN_ERR_UNSUPPORTED); M == 0 launches nothing.
+ * hc         4 (other values: FN_ERR_UNSUPPORTED).
+ * C          multiple of 16, hc*C <= 16384 (else FN_ERR_UNSUPPORTED).
+ * r          multiple of 8, 8..128 (else FN_ERR_UNSUPPORTED).
+ * out        bf16 [M, C], 16-byte aligned.
+ * workspace  device memory of at least fn_hc_mix_workspace_bytes(M, r) bytes,
+ *            16-byte aligned, owned by the caller; it receives t (fp32 [M, r])
+ *            and may be reused as soon as the call's work on `stream` is done.
+ * Overlap    out and workspace must not overlap each other or any input
+ *            (FN_ERR_INVALID).
+ * fn_last_launch: out[0] blocks and out[1] threads of the first kernel
+ * (clusters of 8 blocks), out[2] blocks of the second, out[3] weight rows per
+ * cluster.
+ */
+FN_API int fn_hc_mix(const void* x, const void* w_down, const void* w_up, int64_t M, int hc,
+                     int64_t C, int r, void* out, void* workspace, void* stream);
+
+/* Bytes of workspace fn_hc_mix needs for M rows at rank r (M * r * 4), or -1
+ * for a negative M or a non-positive r. */
+FN_API int64_t fn_hc_mix_workspace_bytes(int64_t M, int r);
 
 /* Static, NUL-terminated description of a status code. */
 FN_API const char* fn_status_string(int status);

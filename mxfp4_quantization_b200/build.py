@@ -29,7 +29,8 @@ UNITS = [("fusednorm", "fusednorm.cu", [])] + [
     (f"rq_{mode}_{maxp}_{io}", "rq_inst.cu",
      [f"-DFN_INST_MODE={mode}", f"-DFN_INST_MAXP={maxp}", f"-DFN_INST_IO={io}"])
     for mode in (0, 1, 2) for maxp in (1, 2, 4, 8) for io in (0, 1)
-] + [(f"ar_{mode}", "ar_inst.cu", [f"-DFN_INST_MODE={mode}"]) for mode in (0, 1, 2)]
+] + [(f"ar_{mode}", "ar_inst.cu", [f"-DFN_INST_MODE={mode}"]) for mode in (0, 1, 2)] + [
+    ("hc", "hc_inst.cu", [])]
 
 
 def deps():

@@ -12,6 +12,7 @@
 
 #include "fusednorm.h"
 #include "ar_kernel.cuh"
+#include "hc_params.h"
 #include "qk_kernel.cuh"
 #include "rq_params.h"
 
@@ -120,8 +121,8 @@ bool rows_on_device(const fn::RQParams& p, int dev) {
 // starts by waiting for the grids it depends on (griddepcontrol.wait), so the
 // dependent launch only lets its blocks be scheduled early.
 template <typename... KArgs, typename... Args>
-int launch_kernel(void (*k)(KArgs...), unsigned grid, unsigned threads, size_t smem,
-                  cudaStream_t st, int cluster, Args... args) {
+int launch_kernel_pdl(void (*k)(KArgs...), unsigned grid, unsigned threads, size_t smem,
+                      cudaStream_t st, int cluster, bool pdl, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(threads);
@@ -136,7 +137,7 @@ int launch_kernel(void (*k)(KArgs...), unsigned grid, unsigned threads, size_t s
     attr[n].val.clusterDim.z = 1;
     ++n;
   }
-  if (tl_pdl) {
+  if (pdl) {
     attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[n].val.programmaticStreamSerializationAllowed = 1;
     ++n;
@@ -148,6 +149,12 @@ int launch_kernel(void (*k)(KArgs...), unsigned grid, unsigned threads, size_t s
     return FN_ERR_CUDA;
   }
   return FN_OK;
+}
+
+template <typename... KArgs, typename... Args>
+int launch_kernel(void (*k)(KArgs...), unsigned grid, unsigned threads, size_t smem,
+                  cudaStream_t st, int cluster, Args... args) {
+  return launch_kernel_pdl(k, grid, threads, smem, st, cluster, tl_pdl != 0, args...);
 }
 
 // Fewest resident warps per SM the one-block-per-row kernel should run with
@@ -450,6 +457,64 @@ int qk_impl(const void* qkv, int64_t M, int64_t row_stride, int Hq, int Hk, int 
   return rc;
 }
 
+// ---- hc_mix -------------------------------------------------------------------
+
+// Weight rows of W_down per cluster: 4, or fewer for small ranks, so that the
+// (r / CW) clusters of 8 blocks still spread the weight over about 128 SMs.
+int hc_rows_per_cluster(int r) { return r >= 64 ? 4 : r >= 32 ? 2 : 1; }
+
+int hc_rows_bound(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
+
+int hc_check(const void* x, const void* w_down, const void* w_up, int64_t M, int hc, int64_t C,
+             int r, const void* out) {
+  if (M < 0 || hc < 1 || C <= 0 || r <= 0) return FN_ERR_INVALID;
+  if (hc != fn::kHcStreams || M > fn::kHcMaxRows || C % fn::kHcChannels ||
+      (int64_t)hc * C > (int64_t)fn::kHcDownThreads * 64 || r % 8 || r > fn::kHcMaxRank)
+    return FN_ERR_UNSUPPORTED;
+  if (M == 0) return FN_OK;
+  if (!x || !w_down || !w_up || !out) return FN_ERR_INVALID;
+  if (!aligned(x, 16) || !aligned(w_down, 16) || !aligned(w_up, 16) || !aligned(out, 16))
+    return FN_ERR_ALIGN;
+  return FN_OK;
+}
+
+// Launches the two hc_mix kernels with t in `ws` (fp32 [M, r], checked by the
+// caller): the column-split product t = W_down x, then the gate and mix as its
+// programmatic dependent.
+int hc_launch(const void* x, const void* w_down, const void* w_up, int64_t M, int64_t C, int r,
+              void* out, float* ws, void* stream) {
+  fn::HCParams p;
+  std::memset(&p, 0, sizeof p);
+  p.x = static_cast<const uint4*>(x);
+  p.w_down = static_cast<const uint4*>(w_down);
+  p.w_up = static_cast<const uint4*>(w_up);
+  p.t = ws;
+  p.out = static_cast<uint16_t*>(out);
+  p.M = (int)M;
+  p.C = (int)C;
+  p.K = (int)(fn::kHcStreams * C);
+  p.r = r;
+  const int cw = hc_rows_per_cluster(r);
+  fn::HCKernel k1 = fn::hc_down_pick(hc_rows_bound(M), cw);
+  if (!k1) return FN_ERR_UNSUPPORTED;
+  const int cvec = p.K / 8 / fn::kHcCluster;
+  // at least one thread per partial sum of the block (rows bound x weight rows)
+  const int t1 = std::max(round32(cvec), round32(hc_rows_bound(M) * cw));
+  const unsigned g1 = (unsigned)(r / cw * fn::kHcCluster);
+  const unsigned g2 = (unsigned)(C / fn::kHcChannels);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (launch_kernel(k1, g1, (unsigned)t1, 0, st, fn::kHcCluster, p) != FN_OK) return FN_ERR_CUDA;
+  if (launch_kernel_pdl(fn::hc_gate_mix_pick(), g2, (unsigned)fn::kHcMixThreads, 0, st, 1, true,
+                        p) != FN_OK)
+    return FN_ERR_CUDA;
+  tl_variant = FN_VARIANT_HC_MIX;
+  tl_launch[0] = (int32_t)g1;
+  tl_launch[1] = t1;
+  tl_launch[2] = (int32_t)g2;
+  tl_launch[3] = cw;
+  return FN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -649,6 +714,28 @@ int fn_ar_rmsnorm_quant(const void* const* x_parts, int num_ranks, int rank, con
   tl_launch[2] = 1;
   tl_launch[3] = V;
   return FN_OK;
+}
+
+int64_t fn_hc_mix_workspace_bytes(int64_t M, int r) {
+  if (M < 0 || r <= 0) return -1;
+  return M * r * (int64_t)sizeof(float);
+}
+
+int fn_hc_mix(const void* x, const void* w_down, const void* w_up, int64_t M, int hc, int64_t C,
+              int r, void* out, void* workspace, void* stream) {
+  tl_variant = FN_VARIANT_NONE;
+  int rc = hc_check(x, w_down, w_up, M, hc, C, r, out);
+  if (rc != FN_OK || M == 0) return rc;
+  if (!workspace) return FN_ERR_INVALID;
+  if (!aligned(workspace, 16)) return FN_ERR_ALIGN;
+  const int64_t K = (int64_t)hc * C;
+  const Range ins[3] = {range_of(x, M * K * 2), range_of(w_down, (int64_t)r * K * 2),
+                        range_of(w_up, K * r * 2)};
+  const Range o = range_of(out, M * C * 2), ws = range_of(workspace, M * r * 4);
+  if (overlap(o, ws)) return FN_ERR_INVALID;
+  for (const Range& in : ins)
+    if (overlap(o, in) || overlap(ws, in)) return FN_ERR_INVALID;
+  return hc_launch(x, w_down, w_up, M, C, r, out, static_cast<float*>(workspace), stream);
 }
 
 int fn_quant(const void* y, int mode, int64_t M, int64_t H, void* out_q, void* out_scale,

@@ -1,0 +1,22 @@
+// Instances of the hc_mix column-split kernel (rows bound x weight rows per
+// cluster); the gate-and-mix kernel has one instance, taken by the host code.
+#include "hc_kernel.cuh"
+
+namespace fn {
+
+HCKernel hc_down_pick(int mm, int cw) {
+#define FN_HC(MM)                                   \
+  if (mm == MM) {                                   \
+    if (cw == 1) return hc_down_kernel<MM, 1>;      \
+    if (cw == 2) return hc_down_kernel<MM, 2>;      \
+    if (cw == 4) return hc_down_kernel<MM, 4>;      \
+    return nullptr;                                 \
+  }
+  FN_HC(1) FN_HC(2) FN_HC(4) FN_HC(8) FN_HC(16)
+#undef FN_HC
+  return nullptr;
+}
+
+HCKernel hc_gate_mix_pick() { return hc_gate_mix_kernel; }
+
+}  // namespace fn

@@ -1,0 +1,32 @@
+// Parameter block and instance table of the hc_mix kernels (hc_kernel.cuh),
+// shared by the host dispatch and the instantiation unit.
+#pragma once
+#include <cstdint>
+#include <vector_types.h>
+
+namespace fn {
+
+struct HCParams {
+  const uint4* x;       // bf16 [M, hc*C] (16-byte vectors)
+  const uint4* w_down;  // bf16 [r, hc*C]
+  const uint4* w_up;    // bf16 [hc*C, r]
+  float* t;             // workspace: fp32 [M, r]
+  uint16_t* out;        // bf16 [M, C]
+  int M, C, K, r;       // K = hc * C
+};
+
+constexpr int kHcStreams = 4;     // hc: the streams of the hyper-state
+constexpr int kHcCluster = 8;     // blocks per cluster of hc_down_kernel (column split)
+constexpr int kHcChannels = 16;   // channels per block of hc_gate_mix_kernel
+constexpr int kHcMaxRows = 16;    // M <= 16 (decode-sized)
+constexpr int kHcMaxRank = 128;   // r <= 128
+constexpr int kHcMixThreads = kHcMaxRows * kHcChannels;
+constexpr int kHcDownThreads = 256;  // one 16-byte vector per thread: hc*C <= 16384
+
+// Instances (hc_inst.cu): hc_down_kernel for rows bound MM in {1, 2, 4, 8, 16}
+// and weight rows per cluster CW in {1, 2, 4}; the one hc_gate_mix_kernel.
+using HCKernel = void (*)(const HCParams);
+HCKernel hc_down_pick(int mm, int cw);
+HCKernel hc_gate_mix_pick();
+
+}  // namespace fn

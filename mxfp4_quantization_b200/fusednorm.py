@@ -38,11 +38,15 @@ FN_VARIANT_QUANT_ONLY = 3
 FN_VARIANT_QK_WARP = 4
 FN_VARIANT_QK_WARP_FP8 = 6
 FN_VARIANT_ROW_ALLREDUCE = 7
+FN_VARIANT_HC_MIX = 8
 
 FN_MODE_MASK = 0xFF
 FN_SCALE_SWIZZLE_32_4_4 = 0x100
 FN_SCALE_MN_MAJOR = 0x200
 FN_IO_FP16 = 0x1000
+
+HC_STREAMS = 4
+HC_MAX_ROWS = 16
 
 FN_MAX_PARTS = 8
 FN_MAX_H = 32768
@@ -53,7 +57,7 @@ MODES = {"fp8_per_token": FN_FP8_PER_TOKEN, "fp8_per_group128": FN_FP8_PER_GROUP
 
 # The exported symbols of include/fusednorm.h.
 ABI_SYMBOLS = ("fn_rmsnorm_quant", "fn_ar_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate",
-               "fn_qk_norm_gate_fp8",
+               "fn_qk_norm_gate_fp8", "fn_hc_mix", "fn_hc_mix_workspace_bytes",
                "fn_status_string",
                "fn_last_variant", "fn_last_launch", "fn_prefer_variant",
                "fn_programmatic_launch", "fn_version")
@@ -86,6 +90,10 @@ def _load():
     lib.fn_qk_norm_gate_fp8.argtypes = [vp, i64, i64, i32, i32, i32, vp, vp, ctypes.c_float, vp,
                                         vp, vp, vp, vp, vp, vp, vp]
     lib.fn_qk_norm_gate_fp8.restype = i32
+    lib.fn_hc_mix.argtypes = [vp, vp, vp, i64, i32, i64, i32, vp, vp, vp]
+    lib.fn_hc_mix.restype = i32
+    lib.fn_hc_mix_workspace_bytes.argtypes = [i64, i32]
+    lib.fn_hc_mix_workspace_bytes.restype = i64
     lib.fn_status_string.argtypes = [i32]
     lib.fn_status_string.restype = ctypes.c_char_p
     lib.fn_last_variant.argtypes = []
@@ -152,6 +160,15 @@ def fn_qk_norm_gate_fp8(qkv: int, M: int, row_stride: int, Hq: int, Hk: int, D: 
     return _lib.fn_qk_norm_gate_fp8(qkv, M, row_stride, Hq, Hk, D, q_weight, k_weight, eps,
                                     out_q8, out_q_scale, out_k8, out_k_scale, out_gate, out_q,
                                     out_k, stream)
+
+
+def fn_hc_mix(x: int, w_down: int, w_up: int, M: int, hc: int, C: int, r: int,
+              out: int, workspace: int, stream: Optional[int]) -> int:
+    return _lib.fn_hc_mix(x, w_down, w_up, M, hc, C, r, out, workspace, stream)
+
+
+def fn_hc_mix_workspace_bytes(M: int, r: int) -> int:
+    return _lib.fn_hc_mix_workspace_bytes(M, r)
 
 
 def fn_status_string(status: int) -> str:
@@ -416,4 +433,30 @@ def qk_norm_gate_fp8(qkv: torch.Tensor, Hq: int, Hk: int, D: int, q_weight: torc
                              _ptr(out.q), _ptr(out.k), _stream(dev))
     if st != FN_OK:
         raise FusedNormError("fn_qk_norm_gate_fp8", st)
+    return out
+
+
+def hc_mix(x: torch.Tensor, w_down: torch.Tensor, w_up: torch.Tensor, *, hc: int = HC_STREAMS,
+           out: Optional[torch.Tensor] = None,
+           workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Low-rank gate over the hyper-state: x bf16 [M, hc*C] (M <= 16),
+    w_down bf16 [r, hc*C], w_up bf16 [hc*C, r]; returns the gated mix of the
+    hc streams, bf16 [M, C] (see fn_hc_mix).  The workspace (fp32 [M, r]) is
+    allocated with torch unless given."""
+    for t, n in ((x, "x"), (w_down, "w_down"), (w_up, "w_up")):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 2 or not t.is_contiguous():
+            raise TypeError(f"{n} must be a contiguous 2-D bf16 CUDA tensor")
+    M, K = x.shape
+    r = w_down.shape[0]
+    if K % hc or w_down.shape[1] != K or tuple(w_up.shape) != (K, r):
+        raise ValueError("shapes must be x [M, hc*C], w_down [r, hc*C], w_up [hc*C, r]")
+    C = K // hc
+    if out is None:
+        out = torch.empty((M, C), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((max(1, M * r),), dtype=torch.float32, device=x.device)
+    st = fn_hc_mix(x.data_ptr(), w_down.data_ptr(), w_up.data_ptr(), M, hc, C, r,
+                   out.data_ptr(), workspace.data_ptr(), _stream(x.device))
+    if st != FN_OK:
+        raise FusedNormError("fn_hc_mix", st)
     return out

@@ -29,7 +29,8 @@ def declared_symbols():
 def test_header_declares_the_abi():
     assert declared_symbols() == sorted(["fn_rmsnorm_quant", "fn_ar_rmsnorm_quant", "fn_quant",
                                          "fn_qk_norm_gate",
-                                         "fn_qk_norm_gate_fp8",
+                                         "fn_qk_norm_gate_fp8", "fn_hc_mix",
+                                         "fn_hc_mix_workspace_bytes",
                                          "fn_status_string", "fn_last_variant",
                                          "fn_last_launch", "fn_prefer_variant",
                                          "fn_programmatic_launch", "fn_version"])
@@ -51,7 +52,7 @@ def test_header_constants_match_binding(fnb):
     for name in ("FN_FP8_PER_TOKEN", "FN_FP8_PER_GROUP128", "FN_MXFP4", "FN_ERR_INVALID",
                  "FN_ERR_ALIGN", "FN_ERR_UNSUPPORTED", "FN_ERR_CUDA", "FN_VARIANT_ROW_CTA",
                  "FN_VARIANT_ROW_CLUSTER", "FN_VARIANT_QUANT_ONLY", "FN_VARIANT_QK_WARP",
-                 "FN_VARIANT_QK_WARP_FP8", "FN_VARIANT_ROW_ALLREDUCE"):
+                 "FN_VARIANT_QK_WARP_FP8", "FN_VARIANT_ROW_ALLREDUCE", "FN_VARIANT_HC_MIX"):
         m = re.search(rf"\b{name}\s*=\s*(-?\d+)", src)
         assert m and int(m.group(1)) == getattr(fnb, name), name
     for name in ("FN_MAX_PARTS", "FN_MAX_H", "FN_MAX_HEAD_DIM"):
@@ -265,3 +266,37 @@ def test_allreduce_empty_shard_and_in_place(fnb):
     # which fails here for want of a device
     assert ar(fnb, out_residual=[BASE + (1 << 32), BASE + (1 << 40) + (5 << 32)]) == \
         fnb.FN_ERR_CUDA
+
+
+def hc(fnb, **kw):
+    a = dict(x=BASE, w_down=BASE + (1 << 32), w_up=BASE + (2 << 32), M=4, hc=4, C=2560, r=64,
+             out=BASE + (3 << 32), workspace=BASE + (4 << 32), stream=None)
+    a.update(kw)
+    return fnb.fn_hc_mix(a["x"], a["w_down"], a["w_up"], a["M"], a["hc"], a["C"], a["r"],
+                         a["out"], a["workspace"], a["stream"])
+
+
+def test_hc_mix_rejects_bad_arguments(fnb):
+    """Every rule of fn_hc_mix's contract is checked on the host before any
+    launch (the pointers here are never dereferenced)."""
+    E, A, U = fnb.FN_ERR_INVALID, fnb.FN_ERR_ALIGN, fnb.FN_ERR_UNSUPPORTED
+    cases = [
+        (dict(M=-1), E), (dict(C=0), E), (dict(r=0), E), (dict(hc=0), E),
+        (dict(M=17), U), (dict(hc=2), U), (dict(C=2568), U), (dict(C=4112), U),
+        (dict(r=12), U), (dict(r=136), U),
+        (dict(x=None), E), (dict(w_down=None), E), (dict(w_up=None), E), (dict(out=None), E),
+        (dict(workspace=None), E),
+        (dict(x=BASE + 8), A), (dict(w_up=BASE + (2 << 32) + 2), A),
+        (dict(out=BASE + (3 << 32) + 4), A), (dict(workspace=BASE + (4 << 32) + 8), A),
+        # outputs overlapping the inputs or each other
+        (dict(out=BASE + 4096), E), (dict(workspace=BASE + (1 << 32) + 64), E),
+        (dict(workspace=BASE + (3 << 32) + 32), E),
+    ]
+    for kw, want in cases:
+        assert hc(fnb, **kw) == want, kw
+        assert fnb.fn_last_variant() == fnb.FN_VARIANT_NONE
+    assert hc(fnb, M=0) == fnb.FN_OK
+    assert hc(fnb, M=0, x=None, out=None, workspace=None) == fnb.FN_OK
+    assert fnb.fn_hc_mix_workspace_bytes(16, 64) == 16 * 64 * 4
+    assert fnb.fn_hc_mix_workspace_bytes(0, 64) == 0
+    assert fnb.fn_hc_mix_workspace_bytes(-1, 64) == -1 and fnb.fn_hc_mix_workspace_bytes(4, 0) == -1
