@@ -468,7 +468,7 @@ int hc_rows_bound(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <
 int hc_check(const void* x, const void* w_down, const void* w_up, int64_t M, int hc, int64_t C,
              int r, const void* out) {
   if (M < 0 || hc < 1 || C <= 0 || r <= 0) return FN_ERR_INVALID;
-  if (hc != fn::kHcStreams || M > fn::kHcMaxRows || C % fn::kHcChannels ||
+  if (hc != fn::kHcStreams || M > fn::kHcMaxRows || C % 16 ||
       (int64_t)hc * C > (int64_t)fn::kHcDownThreads * 64 || r % 8 || r > fn::kHcMaxRank)
     return FN_ERR_UNSUPPORTED;
   if (M == 0) return FN_OK;
@@ -476,6 +476,16 @@ int hc_check(const void* x, const void* w_down, const void* w_up, int64_t M, int
   if (!aligned(x, 16) || !aligned(w_down, 16) || !aligned(w_up, 16) || !aligned(out, 16))
     return FN_ERR_ALIGN;
   return FN_OK;
+}
+
+// Channels per block of the gate-and-mix kernel: the fewest, in steps of 4,
+// that divide C and need no more blocks than SMs (C = 2560 on 148 SMs: 20,
+// 128 blocks), else 16 (C % 16 == 0), with more blocks than SMs.
+int hc_mix_channels(int64_t C, int sms) {
+  for (int64_t cpb = std::max<int64_t>(4, (C + sms - 1) / sms + 3) / 4 * 4;
+       cpb <= fn::kHcMaxMixChannels; cpb += 4)
+    if (C % cpb == 0) return (int)cpb;
+  return 16;
 }
 
 // Launches the two hc_mix kernels with t in `ws` (fp32 [M, r], checked by the
@@ -501,17 +511,22 @@ int hc_launch(const void* x, const void* w_down, const void* w_up, int64_t M, in
   // at least one thread per partial sum of the block (rows bound x weight rows)
   const int t1 = std::max(round32(cvec), round32(hc_rows_bound(M) * cw));
   const unsigned g1 = (unsigned)(r / cw * fn::kHcCluster);
-  const unsigned g2 = (unsigned)(C / fn::kHcChannels);
+  const int sms = sm_count();
+  if (sms <= 0) return FN_ERR_CUDA;
+  p.cpb = hc_mix_channels(C, sms);
+  if (p.cpb == 0) return FN_ERR_UNSUPPORTED;
+  const unsigned g2 = (unsigned)(C / p.cpb);
+  const int t2 = fn::kHcStreams * p.cpb * (int)((M + 3) / 4);
+  fn::HCKernel k2 = fn::hc_gate_mix_pick(r / 8);
+  if (!k2) return FN_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (launch_kernel(k1, g1, (unsigned)t1, 0, st, fn::kHcCluster, p) != FN_OK) return FN_ERR_CUDA;
-  if (launch_kernel_pdl(fn::hc_gate_mix_pick(), g2, (unsigned)fn::kHcMixThreads, 0, st, 1, true,
-                        p) != FN_OK)
-    return FN_ERR_CUDA;
+  if (launch_kernel_pdl(k2, g2, (unsigned)t2, 0, st, 1, true, p) != FN_OK) return FN_ERR_CUDA;
   tl_variant = FN_VARIANT_HC_MIX;
   tl_launch[0] = (int32_t)g1;
   tl_launch[1] = t1;
   tl_launch[2] = (int32_t)g2;
-  tl_launch[3] = cw;
+  tl_launch[3] = t2;
   return FN_OK;
 }
 

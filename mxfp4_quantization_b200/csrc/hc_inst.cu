@@ -17,6 +17,13 @@ HCKernel hc_down_pick(int mm, int cw) {
   return nullptr;
 }
 
-HCKernel hc_gate_mix_pick() { return hc_gate_mix_kernel; }
+HCKernel hc_gate_mix_pick(int rv) {
+  if (rv <= 1) return hc_gate_mix_kernel<1>;
+  if (rv <= 2) return hc_gate_mix_kernel<2>;
+  if (rv <= 4) return hc_gate_mix_kernel<4>;
+  if (rv <= 8) return hc_gate_mix_kernel<8>;
+  if (rv <= 16) return hc_gate_mix_kernel<16>;
+  return nullptr;
+}
 
 }  // namespace fn

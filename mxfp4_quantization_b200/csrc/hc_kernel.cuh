@@ -17,14 +17,13 @@
 //    read exactly once over the grid) and the matching columns of every x row.
 //    A thread owns one 16-byte vector of the piece; the block reduces its
 //    threads' M * CW partial sums with a warp reduce-scatter and shared
-//    memory, and the cluster's 8 partials meet in distributed shared memory,
-//    summed by rank 0 in rank order.  t (fp32 [M, r]) goes to the caller's
-//    workspace.
-//  * hc_gate_mix_kernel: one block per 16 channels.  Before it waits for the
-//    first kernel it stages its 4 * 16 rows of W_up (converted to fp32,
-//    laid out [j][c][s]) and its slice of every x row in shared memory; once
-//    t is visible it forms the 64 gate logits of each row, the sigmoids and
-//    the mix.
+//    memory, every block stores its partials into rank 0's shared memory
+//    (distributed shared memory), and after one cluster barrier rank 0 sums
+//    them in rank order.  t (fp32 [M, r]) goes to the caller's workspace.
+//  * hc_gate_mix_kernel: one block per cpb channels (no more blocks than
+//    SMs).  Before it waits for the first kernel every thread loads its row
+//    of W_up into registers and its x values; once t is visible it forms the
+//    gate logits, the sigmoids and the mix.
 // Every sum has a fixed order, so a launch shape always gives the same bits.
 #pragma once
 #include <cooperative_groups.h>
@@ -71,7 +70,7 @@ __global__ void __launch_bounds__(kHcDownThreads) hc_down_kernel(const __grid_co
   namespace cg = cooperative_groups;
   constexpr int V = MM * CW;
   __shared__ float red[kHcDownThreads / 32][V];
-  __shared__ float part[V];
+  __shared__ float slots[kHcCluster][V];  // rank 0's: every block's partials
   pdl_enter();
 
   cg::cluster_group cl = cg::this_cluster();
@@ -119,82 +118,117 @@ __global__ void __launch_bounds__(kHcDownThreads) hc_down_kernel(const __grid_co
   if (o < V) {
     float s = red[0][o];
     for (int w = 1; w < nw; ++w) s += red[w][o];
-    part[o] = s;
+    *cl.map_shared_rank(&slots[rank][o], 0) = s;
   }
-  // the cluster's sums, read by rank 0 from every block's shared memory
+  // the stores into rank 0's shared memory are complete and visible to it
+  // after the barrier; only rank 0 reads them, so the others may leave
   cl.sync();
   if (rank == 0 && o < V) {
-    float s = *cl.map_shared_rank(&part[o], 0);
+    float s = slots[0][o];
 #pragma unroll
-    for (int c = 1; c < kHcCluster; ++c) s += *cl.map_shared_rank(&part[o], c);
+    for (int c = 1; c < kHcCluster; ++c) s += slots[c][o];
     const int m = o / CW, j = o % CW;
     if (m < p.M) p.t[(int64_t)m * p.r + g * CW + j] = s;
   }
-  // no block leaves while rank 0 may still read its shared memory
-  cl.sync();
 }
 
-// u[m, c] for the kHcChannels channels of this block: gate logits of the 4
-// streams from t and W_up, logistic sigmoid, gated sum of the streams.
-// Launched as a programmatic dependent of hc_down_kernel: everything that
-// does not depend on t is staged before the wait.  blockDim.x = 256.
+// u[m, c] for the channels [c0, c0 + cpb) of this block: gate logits of the
+// 4 streams from t and W_up, logistic sigmoid, gated sum of the streams.
+// Thread (mg, s, c) keeps W_up row s*C + c0 + c (r values, RV 16-byte vectors
+// at most) in registers and forms the logits of rows 4mg .. 4mg+3 from t,
+// read from shared memory transposed ([j][m], so one 16-byte read gives four
+// rows, the same address for a whole m-group: a broadcast); the gates meet
+// in shared memory, and thread (m, c) forms the gated sum of the streams in
+// stream order.  Launched as a programmatic dependent of hc_down_kernel:
+// every load that does not depend on t is issued before the wait.
+// blockDim.x = 4 * cpb * ceil(M / 4).
+template <int RV>
 __global__ void __launch_bounds__(kHcMixThreads) hc_gate_mix_kernel(
     const __grid_constant__ HCParams p) {
-  __shared__ __align__(16) float wu[kHcMaxRank * kHcChannels * kHcStreams];  // [j][c][s]
-  __shared__ __align__(16) float tt[kHcMaxRows * kHcMaxRank];                // [m][j]
-  __shared__ __align__(16) uint16_t xs[kHcMaxRows][kHcStreams][kHcChannels];
+  __shared__ __align__(16) float tt[RV * 8][kHcMaxRows];                    // [j][m]
+  __shared__ float gs[kHcMaxRows][kHcStreams][kHcMaxMixChannels];         // gates
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  const int c0 = blockIdx.x * kHcChannels;
-  const int rv = p.r / 8;  // 16-byte vectors per W_up row
-  // W_up rows s*C + c0 + c, in fp32 at [j][c][s]; consecutive threads take
-  // consecutive channels (c fastest) so the shared stores spread over banks
-  for (int i = threadIdx.x; i < kHcStreams * rv * kHcChannels; i += blockDim.x) {
-    const int c = i % kHcChannels, q = (i / kHcChannels) % rv, s = i / (kHcChannels * rv);
-    const uint4 wv = ld_stream_nc(p.w_up + ((int64_t)s * p.C + c0 + c) * rv + q);
+  const int cpb = p.cpb, c0 = blockIdx.x * cpb, tid = threadIdx.x;
+  const int rv = p.r / 8;
+  const int mg = tid / (kHcStreams * cpb), rem = tid % (kHcStreams * cpb);
+  const int s = rem / cpb, c = rem % cpb;
+  // every global load first: this thread's W_up row ...
+  uint4 w[RV];
+  const uint4* wrow = p.w_up + ((int64_t)s * p.C + c0 + c) * rv;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int j = 8 * q + 2 * k;
-      wu[(j * kHcChannels + c) * kHcStreams + s] = bf_lo(word(wv, k));
-      wu[((j + 1) * kHcChannels + c) * kHcStreams + s] = bf_hi(word(wv, k));
-    }
-  }
-  // this block's 16 channels of every stream of every row (two vectors each)
-  for (int i = threadIdx.x; i < p.M * kHcStreams * 2; i += blockDim.x) {
-    const int h = i & 1, s = (i >> 1) % kHcStreams, m = i / (2 * kHcStreams);
-    const uint4 xv = ld_stream_nc(p.x + ((int64_t)m * p.K + (int64_t)s * p.C + c0) / 8 + h);
-    *reinterpret_cast<uint4*>(&xs[m][s][8 * h]) = xv;
-  }
+  for (int q = 0; q < RV; ++q) w[q] = q < rv ? ld_keep(wrow + q) : make_uint4(0u, 0u, 0u, 0u);
+  // ... and, as thread (xm, xc) of the mix, the four streams of x[xm, c0 + xc]
+  const int xm = tid / cpb, xc = tid % cpb;
+  const bool mixer = xm < p.M;
+  float xv[kHcStreams];
+  const uint16_t* xr = reinterpret_cast<const uint16_t*>(p.x) + (int64_t)xm * p.K + c0 + xc;
+#pragma unroll
+  for (int k = 0; k < kHcStreams; ++k)
+    xv[k] = mixer ? __uint_as_float((uint32_t)__ldg(xr + (int64_t)k * p.C) << 16) : 0.f;
 
-  // t is written by the kernel this one depends on
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  for (int i = threadIdx.x; i < p.M * p.r / 4; i += blockDim.x)
-    reinterpret_cast<float4*>(tt)[i] = __ldcg(reinterpret_cast<const float4*>(p.t) + i);
+  // entries of t beyond M rows or r columns read as zero (they add nothing)
+  for (int i = tid; i < RV * 8 * kHcMaxRows; i += blockDim.x) (&tt[0][0])[i] = 0.f;
   __syncthreads();
 
-  const int m = threadIdx.x / kHcChannels, c = threadIdx.x % kHcChannels;
-  if (m >= p.M) return;
-  float2 z01 = make_float2(0.f, 0.f), z23 = make_float2(0.f, 0.f);
-  const float* tm = tt + m * p.r;
-  for (int j = 0; j < p.r; j += 4) {
-    const float4 t4 = *reinterpret_cast<const float4*>(tm + j);
-    const float tj[4] = {t4.x, t4.y, t4.z, t4.w};
+  // t is written by the kernel this one depends on: 16-byte loads, two per
+  // thread in flight (M * r / 4 vectors: one pass for every C >= 1024), stored
+  // transposed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int nt = p.M * p.r / 4;
+  for (int i0 = 0; i0 < nt; i0 += 2 * blockDim.x) {
+    float4 tq[2];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float4 w = *reinterpret_cast<const float4*>(&wu[((j + k) * kHcChannels + c) * kHcStreams]);
-      const float2 tk = make_float2(tj[k], tj[k]);
-      z01 = fma_f32x2(tk, make_float2(w.x, w.y), z01);
-      z23 = fma_f32x2(tk, make_float2(w.z, w.w), z23);
+    for (int k = 0; k < 2; ++k) {
+      const int i = i0 + tid + k * blockDim.x;
+      tq[k] = i < nt ? __ldcg(reinterpret_cast<const float4*>(p.t) + i)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int i = i0 + tid + k * blockDim.x;
+      if (i < nt) {
+        const int m = (4 * i) / p.r, j = (4 * i) % p.r;
+        tt[j][m] = tq[k].x;
+        tt[j + 1][m] = tq[k].y;
+        tt[j + 2][m] = tq[k].z;
+        tt[j + 3][m] = tq[k].w;
+      }
     }
   }
-  const float z[kHcStreams] = {z01.x, z01.y, z23.x, z23.y};
+  __syncthreads();
+
+  // logits of rows 4mg .. 4mg+3; two accumulator pairs per row pair (even
+  // and odd j) halve the dependent chains
+  float2 za[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float2 zb[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int q = 0; q < RV; ++q) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 8 * q + 2 * e;
+      const float wl = bf_lo(word(w[q], e)), wh = bf_hi(word(w[q], e));
+      const float4 t0 = *reinterpret_cast<const float4*>(&tt[j][4 * mg]);
+      const float4 t1 = *reinterpret_cast<const float4*>(&tt[j + 1][4 * mg]);
+      za[0] = fma_f32x2(make_float2(t0.x, t0.y), make_float2(wl, wl), za[0]);
+      za[1] = fma_f32x2(make_float2(t0.z, t0.w), make_float2(wl, wl), za[1]);
+      zb[0] = fma_f32x2(make_float2(t1.x, t1.y), make_float2(wh, wh), zb[0]);
+      zb[1] = fma_f32x2(make_float2(t1.z, t1.w), make_float2(wh, wh), zb[1]);
+    }
+  }
+  const float z[4] = {za[0].x + zb[0].x, za[0].y + zb[0].y, za[1].x + zb[1].x,
+                      za[1].y + zb[1].y};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = 4 * mg + i;
+    if (m < p.M) gs[m][s][c] = 1.f / (1.f + __expf(-z[i]));
+  }
+  __syncthreads();
+  if (!mixer) return;
   float u = 0.f;
 #pragma unroll
-  for (int s = 0; s < kHcStreams; ++s) {
-    const float gate = 1.f / (1.f + __expf(-z[s]));
-    u = fmaf(gate, __uint_as_float((uint32_t)xs[m][s][c] << 16), u);
-  }
-  p.out[(int64_t)m * p.C + c0 + c] = (uint16_t)(pack_bf16x2(u, 0.f) & 0xFFFFu);
+  for (int k = 0; k < kHcStreams; ++k) u = fmaf(gs[xm][k][xc], xv[k], u);
+  p.out[(int64_t)xm * p.C + c0 + xc] = (uint16_t)(pack_bf16x2(u, 0.f) & 0xFFFFu);
 }
 
 }  // namespace fn

@@ -13,20 +13,22 @@ struct HCParams {
   float* t;             // workspace: fp32 [M, r]
   uint16_t* out;        // bf16 [M, C]
   int M, C, K, r;       // K = hc * C
+  int cpb;              // channels per block of hc_gate_mix_kernel
 };
 
 constexpr int kHcStreams = 4;     // hc: the streams of the hyper-state
 constexpr int kHcCluster = 8;     // blocks per cluster of hc_down_kernel (column split)
-constexpr int kHcChannels = 16;   // channels per block of hc_gate_mix_kernel
-constexpr int kHcMaxRows = 16;    // M <= 16 (decode-sized)
-constexpr int kHcMaxRank = 128;   // r <= 128
-constexpr int kHcMixThreads = kHcMaxRows * kHcChannels;
-constexpr int kHcDownThreads = 256;  // one 16-byte vector per thread: hc*C <= 16384
+constexpr int kHcMaxRows = 16;         // M <= 16 (decode-sized)
+constexpr int kHcMaxRank = 128;        // r <= 128
+constexpr int kHcMaxMixChannels = 32;  // channels per block of hc_gate_mix_kernel, at most
+constexpr int kHcMixThreads = 512;     // 4 streams x channels x row groups of 4, at most
+constexpr int kHcDownThreads = 256;    // one 16-byte vector per thread: hc*C <= 16384
 
 // Instances (hc_inst.cu): hc_down_kernel for rows bound MM in {1, 2, 4, 8, 16}
-// and weight rows per cluster CW in {1, 2, 4}; the one hc_gate_mix_kernel.
+// and weight rows per cluster CW in {1, 2, 4}; hc_gate_mix_kernel for W_up
+// row vectors RV in {1, 2, 4, 8, 16} (rows of r <= 8 * RV values).
 using HCKernel = void (*)(const HCParams);
 HCKernel hc_down_pick(int mm, int cw);
-HCKernel hc_gate_mix_pick();
+HCKernel hc_gate_mix_pick(int rv);
 
 }  // namespace fn

@@ -68,14 +68,16 @@ def test_workload_every_decode_m(fnb, M):
     wl = synth.hc_mix(M)
     inp, got, launch = run(fnb, wl)
     st = check(wl, inp, got)
-    # 16 clusters of 8 blocks (4 weight rows each), 160 gate-and-mix blocks
-    assert list(launch) == [128, 160, 160, 4], launch
+    # 16 clusters of 8 blocks (4 weight rows of W_down each, 160 threads), then
+    # 128 gate-and-mix blocks of 20 channels (4 streams x 20 x ceil(M/4) threads)
+    assert list(launch) == [128, 160, 128, 80 * ((M + 3) // 4)], launch
     assert st["bf16_equal_frac"] > 0.99, st
 
 
 SHAPES = [  # (M, C, r): ranks 8..128, C from one block of channels to the largest
     (1, 16, 8), (3, 32, 16), (5, 64, 24), (16, 16, 128), (2, 1024, 32), (7, 4096, 64),
     (16, 4096, 128), (9, 2560, 40), (4, 48, 56), (12, 512, 8), (16, 2560, 128),
+    (3, 2384, 64),  # 2384 = 16 * 149: no divisor of C in steps of 4 keeps blocks <= SMs
 ]
 
 
