@@ -286,6 +286,34 @@ FN_API int fn_hc_mix(const void* x, const void* w_down, const void* w_up, int64_
  * for a negative M or a non-positive r. */
 FN_API int64_t fn_hc_mix_workspace_bytes(int64_t M, int r);
 
+/*
+ * fn_hc_mix for callers that cannot allocate device memory: the same
+ * computation, kernels and results as fn_hc_mix, with the intermediate t kept
+ * in a fixed scratch array inside the library instead of a caller-provided
+ * workspace.  Some callers cannot call cudaMalloc or any allocator at the
+ * point where they run this step: code inside a section that must not
+ * allocate (a real-time or inference loop that has reserved all its memory up
+ * front, a host callback, a plugin whose framework owns every allocation).
+ * The paper has no counterpart; it describes no memory management.
+ *
+ * Arguments, checks and errors as fn_hc_mix, without `workspace`.
+ * Scratch    a file-scope device array of the library holding t for at most
+ *            16 rows at rank 128 (fp32 [M, r], M * r <= 2048: 8 KB); a larger
+ *            M * r returns FN_ERR_UNSUPPORTED.  Every device that loads the
+ *            library holds the array from load until the process exits; no
+ *            call allocates or frees anything.
+ * First call the first call on a device, with that device current, looks up
+ *            the array's device address (cudaGetSymbolAddress) and caches it;
+ *            make that first call before any stream capture.
+ * Sharing    every call on a device uses the same array and finds there what
+ *            the previous call left; each call writes all of t before reading
+ *            it, so nothing needs clearing, but calls that overlap on the GPU
+ *            (different streams, concurrent graphs) race on the array: order
+ *            them on one stream.
+ */
+FN_API int fn_hc_mix_noalloc(const void* x, const void* w_down, const void* w_up, int64_t M,
+                             int hc, int64_t C, int r, void* out, void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 FN_API const char* fn_status_string(int status);
 

@@ -753,6 +753,66 @@ int fn_hc_mix(const void* x, const void* w_down, const void* w_up, int64_t M, in
   return hc_launch(x, w_down, w_up, M, C, r, out, static_cast<float*>(workspace), stream);
 }
 
+}  // extern "C"
+
+// ---- hc_mix without a caller-provided workspace ------------------------------------
+
+// The intermediate t of fn_hc_mix_noalloc: fp32 [M, r] for at most 16 rows at
+// rank 128, 8 KB.  A file-scope device array, so it exists on every device
+// that loads the library, from load until exit, and no call allocates it.  In
+// host code this name is only a stand-in for the array: its device address
+// comes from cudaGetSymbolAddress, once per device (hc_noalloc_scratch).
+static __device__ __align__(256) float g_hc_noalloc_t[fn::kHcMaxRows * fn::kHcMaxRank];
+
+namespace {
+
+constexpr int64_t kHcNoallocFloats = (int64_t)fn::kHcMaxRows * fn::kHcMaxRank;
+
+std::mutex g_hc_noalloc_mu;
+float* g_hc_noalloc_ptr[64];  // device address of g_hc_noalloc_t, per device ordinal
+
+// The device address of the scratch array on the current device, looked up on
+// the first call with that device current and cached; nullptr if the runtime
+// cannot tell (the call then returns FN_ERR_CUDA).
+float* hc_noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_hc_noalloc_mu);
+  if (!g_hc_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_hc_noalloc_t) != cudaSuccess || ptr == nullptr) {
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    g_hc_noalloc_ptr[dev] = static_cast<float*>(ptr);
+  }
+  return g_hc_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int fn_hc_mix_noalloc(const void* x, const void* w_down, const void* w_up, int64_t M, int hc,
+                      int64_t C, int r, void* out, void* stream) {
+  tl_variant = FN_VARIANT_NONE;
+  int rc = hc_check(x, w_down, w_up, M, hc, C, r, out);
+  if (rc != FN_OK || M == 0) return rc;
+  if (M * (int64_t)r > kHcNoallocFloats) return FN_ERR_UNSUPPORTED;  // beyond the static scratch
+  const int64_t K = (int64_t)hc * C;
+  const Range ins[3] = {range_of(x, M * K * 2), range_of(w_down, (int64_t)r * K * 2),
+                        range_of(w_up, K * r * 2)};
+  const Range o = range_of(out, M * C * 2);
+  for (const Range& in : ins)
+    if (overlap(o, in)) return FN_ERR_INVALID;
+  float* scratch = hc_noalloc_scratch();
+  if (!scratch) return FN_ERR_CUDA;
+  return hc_launch(x, w_down, w_up, M, C, r, out, scratch, stream);
+}
+
 int fn_quant(const void* y, int mode, int64_t M, int64_t H, void* out_q, void* out_scale,
              void* stream) {
   tl_variant = FN_VARIANT_NONE;

@@ -58,6 +58,7 @@ MODES = {"fp8_per_token": FN_FP8_PER_TOKEN, "fp8_per_group128": FN_FP8_PER_GROUP
 # The exported symbols of include/fusednorm.h.
 ABI_SYMBOLS = ("fn_rmsnorm_quant", "fn_ar_rmsnorm_quant", "fn_quant", "fn_qk_norm_gate",
                "fn_qk_norm_gate_fp8", "fn_hc_mix", "fn_hc_mix_workspace_bytes",
+               "fn_hc_mix_noalloc",
                "fn_status_string",
                "fn_last_variant", "fn_last_launch", "fn_prefer_variant",
                "fn_programmatic_launch", "fn_version")
@@ -94,6 +95,8 @@ def _load():
     lib.fn_hc_mix.restype = i32
     lib.fn_hc_mix_workspace_bytes.argtypes = [i64, i32]
     lib.fn_hc_mix_workspace_bytes.restype = i64
+    lib.fn_hc_mix_noalloc.argtypes = [vp, vp, vp, i64, i32, i64, i32, vp, vp]
+    lib.fn_hc_mix_noalloc.restype = i32
     lib.fn_status_string.argtypes = [i32]
     lib.fn_status_string.restype = ctypes.c_char_p
     lib.fn_last_variant.argtypes = []
@@ -169,6 +172,11 @@ def fn_hc_mix(x: int, w_down: int, w_up: int, M: int, hc: int, C: int, r: int,
 
 def fn_hc_mix_workspace_bytes(M: int, r: int) -> int:
     return _lib.fn_hc_mix_workspace_bytes(M, r)
+
+
+def fn_hc_mix_noalloc(x: int, w_down: int, w_up: int, M: int, hc: int, C: int, r: int,
+                      out: int, stream: Optional[int]) -> int:
+    return _lib.fn_hc_mix_noalloc(x, w_down, w_up, M, hc, C, r, out, stream)
 
 
 def fn_status_string(status: int) -> str:

@@ -30,7 +30,7 @@ def test_header_declares_the_abi():
     assert declared_symbols() == sorted(["fn_rmsnorm_quant", "fn_ar_rmsnorm_quant", "fn_quant",
                                          "fn_qk_norm_gate",
                                          "fn_qk_norm_gate_fp8", "fn_hc_mix",
-                                         "fn_hc_mix_workspace_bytes",
+                                         "fn_hc_mix_workspace_bytes", "fn_hc_mix_noalloc",
                                          "fn_status_string", "fn_last_variant",
                                          "fn_last_launch", "fn_prefer_variant",
                                          "fn_programmatic_launch", "fn_version"])
