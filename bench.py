@@ -214,19 +214,24 @@ def _code_only(src: str) -> str:
     return " ".join(src.split())
 
 
-def source_hash() -> str:
+# The sources of the row kernels (rmsnorm_quant): the traffic record below
+# stays valid while these are unchanged and the launch shape is the recorded one.
+ROW_KERNEL_SOURCES = ("fn_device.cuh", "quant.cuh", "rq_kernel.cuh", "rq_params.h", "rq_inst.cu")
+
+
+def source_hash(files=ROW_KERNEL_SOURCES) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mxfp4_quantization_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(f.encode())
-            h.update(_code_only(open(os.path.join(csrc, f)).read()).encode())
+    for f in sorted(files):
+        h.update(f.encode())
+        h.update(_code_only(open(os.path.join(csrc, f)).read()).encode())
     return h.hexdigest()[:16]
 
 
-def measured_traffic(kernel_key: str):
+def measured_traffic(kernel_key: str, launch=None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources; None otherwise."""
+    on the current row-kernel sources and (when given) the same launch shape;
+    None otherwise."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         d = json.load(open(p))
@@ -234,6 +239,8 @@ def measured_traffic(kernel_key: str):
         return None
     e = d.get(kernel_key)
     if not e or e.get("source_hash") != source_hash():
+        return None
+    if launch is not None and e.get("launch") is not None and list(e["launch"]) != list(launch):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -537,7 +544,7 @@ def secondary_workloads(fn, device, peak):
                             "frac_of_peak": b / (ms * 1e-3) / 1e9 / peak,
                             "bytes_per_call": b, "variant": fn.fn_last_variant(),
                             "launch": list(fn.fn_last_launch()),
-                            "traffic": measured_traffic(wl.name)}
+                            "traffic": measured_traffic(wl.name, fn.fn_last_launch())}
     del keep
     torch.cuda.empty_cache()
 
@@ -758,7 +765,7 @@ def main_arm(args):
     peak, peak_kind = hbm_peak()
     us_call = ms * 1e3 / calls  # every launch of the step is the same kernel
     achieved = bytes_call / (us_call * 1e-6) / 1e9
-    traffic = measured_traffic(wl.name)
+    traffic = measured_traffic(wl.name, launch)
     del keep
     torch.cuda.empty_cache()
 

@@ -69,12 +69,12 @@ __device__ __forceinline__ Fp8Scale fp8_scale_direct(float amax) {
 // |y| and the conversion writes the sign.  Zeros keep their sign because
 // r_lo >= 0 (r is not above 1/s): -0 r_lo = -0 and -0 + -0 = -0 (code 0x80).
 // If any lane of the warp needs the IEEE division the whole warp takes it
-// (warp-uniform branch; the signed quotient keeps signs there too).  All 32
-// lanes must call.
+// (warp-uniform branch; the signed quotient keeps signs there too): `exact`
+// must be the same in every lane and true if any lane's scale needs it.
 template <class IO = Bf16>
-__device__ __forceinline__ uint2 e4m3_codes(const uint4& y, const Fp8Scale& c) {
+__device__ __forceinline__ uint2 e4m3_codes_uniform(const uint4& y, const Fp8Scale& c, bool exact) {
   uint32_t q8[4];
-  if (!__any_sync(0xffffffffu, c.exact_div)) {
+  if (!exact) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float2 yf = make_float2(IO::lo(word(y, i)), IO::hi(word(y, i)));
@@ -88,6 +88,12 @@ __device__ __forceinline__ uint2 e4m3_codes(const uint4& y, const Fp8Scale& c) {
       q8[i] = cvt_e4m3x2(__fdiv_rn(IO::lo(word(y, i)), c.s), __fdiv_rn(IO::hi(word(y, i)), c.s));
   }
   return make_uint2(q8[0] | (q8[1] << 16), q8[2] | (q8[3] << 16));
+}
+
+// e4m3_codes_uniform with the path voted by the warp.  All 32 lanes must call.
+template <class IO = Bf16>
+__device__ __forceinline__ uint2 e4m3_codes(const uint4& y, const Fp8Scale& c) {
+  return e4m3_codes_uniform<IO>(y, c, __any_sync(0xffffffffu, c.exact_div));
 }
 
 }  // namespace fn

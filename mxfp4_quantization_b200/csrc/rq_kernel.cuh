@@ -199,6 +199,71 @@ __device__ __forceinline__ void quant_store(const uint4& y, bool ok, int lane, i
                     ld);
 }
 
+// Per-group-128 codes and scales of the V vectors yv[k] = vector vbase + k*T
+// of a row that one thread holds (V a power of two, 2..16; T a multiple of 16,
+// so each 16-lane half-warp shares one group per k), with one scale
+// computation per lane instead of one per vector: the V group maxima travel
+// together as bf16 pairs through four xor-shuffle steps (the amax of bf16 or
+// binary16 values is one of them, so the packing is exact), lane l computes
+// the scale and reciprocal pair of group k = l % V, every lane fetches the
+// pairs of its V groups with two shuffles each, and lane k of each half-warp
+// (which computed group k) stores that group's scale.  Same bits as V calls
+// of quant_store<MODE_G128>.  All 32 lanes must call; `ok` is false in whole
+// half-warps past the row end.
+template <int V, class IO = Bf16>
+__device__ __forceinline__ void quant_store_g128_rows(const uint4 (&yv)[V], const bool (&ok)[V],
+                                                      int lane, int64_t row, int vbase, int T,
+                                                      int H, uint8_t* out_q, float* out_scale,
+                                                      int layout, int64_t ld) {
+  static_assert(V >= 2 && V <= 16 && (V & (V - 1)) == 0, "V: a power of two in 2..16");
+  // group maxima, two groups per 32-bit word
+  uint32_t pm[V / 2];
+#pragma unroll
+  for (int i = 0; i < V / 2; ++i) {
+    uint32_t m[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint4& y = yv[2 * i + h];
+      const uint32_t a = IO::absmax2(IO::absmax2(y.x, y.y), IO::absmax2(y.z, y.w));
+      m[h] = IO::absmax2(a, __byte_perm(a, 0u, 0x1032));  // both halves: the vector's |max|
+    }
+    pm[i] = __byte_perm(m[0], m[1], 0x5410) & 0x7FFF7FFFu;  // (group 2i, group 2i+1)
+  }
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) {
+#pragma unroll
+    for (int i = 0; i < V / 2; ++i) pm[i] = IO::absmax2(pm[i], __shfl_xor_sync(0xffffffffu, pm[i], o));
+  }
+  // this lane's group: k = lane % V
+  const int ks = lane & (V - 1);
+  uint32_t sel = pm[0];
+#pragma unroll
+  for (int i = 1; i < V / 2; ++i)
+    if ((ks >> 1) == i) sel = pm[i];
+  const Fp8Scale own = fp8_scale_direct((ks & 1) ? IO::hi(sel) : IO::lo(sel));
+  const bool exact = __any_sync(0xffffffffu, own.exact_div);
+  const int src = lane & ~(V - 1);
+#pragma unroll
+  for (int k = 0; k < V; ++k) {
+    Fp8Scale c;
+    c.r = __shfl_sync(0xffffffffu, own.r, src + k);
+    c.r_lo = __shfl_sync(0xffffffffu, own.r_lo, src + k);
+    c.s = exact ? __shfl_sync(0xffffffffu, own.s, src + k) : 1.f;
+    c.exact_div = exact;
+    if (ok[k])
+      st_stream(reinterpret_cast<uint2*>(out_q + row * (int64_t)H) + vbase + k * T,
+                e4m3_codes_uniform<IO>(yv[k], c, exact));
+  }
+  if ((lane & 15) < V) {
+    const int vk = vbase + ks * T;  // this lane's vector in group ks of its half-warp
+    bool ok_sel = ok[0];
+#pragma unroll
+    for (int k = 1; k < V; ++k)
+      if (ks == k) ok_sel = ok[k];
+    if (ok_sel) out_scale[scale_index(layout, ld, row, vk / 16, H / 128)] = own.s;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // reductions
 // ---------------------------------------------------------------------------
@@ -382,11 +447,20 @@ __global__ void __launch_bounds__((CL || TB > 256) ? 512 : 256)
     static_cast<float*>(prm.out_scale)[row] = scale_tok.s;
 
   // ---- 5. quantize y ----------------------------------------------------------------
+  if constexpr (MODE == MODE_G128 && V >= 2) {
+    bool ok[V];
 #pragma unroll
-  for (int k = 0; k < V; ++k) {
-    const int v = seg_base + t + k * T;
-    quant_store<MODE, IO>(yv[k], TB || v < seg_end, lane, row, v, H, scale_tok, prm.out_q,
-                          prm.out_scale, prm.scale_layout, prm.scale_ld);
+    for (int k = 0; k < V; ++k) ok[k] = TB || seg_base + t + k * T < seg_end;
+    quant_store_g128_rows<V, IO>(yv, ok, lane, row, seg_base + t, T, H, prm.out_q,
+                                 static_cast<float*>(prm.out_scale), prm.scale_layout,
+                                 prm.scale_ld);
+  } else {
+#pragma unroll
+    for (int k = 0; k < V; ++k) {
+      const int v = seg_base + t + k * T;
+      quant_store<MODE, IO>(yv[k], TB || v < seg_end, lane, row, v, H, scale_tok, prm.out_q,
+                            prm.out_scale, prm.scale_layout, prm.scale_ld);
+    }
   }
 
   if constexpr (CL) {
