@@ -641,6 +641,109 @@ def secondary_workloads(fn, device, peak):
 
 
 # ---------------------------------------------------------------------------
+# fused all-reduce across the ranks (opt-in: --tp-leg, N > 1)
+# ---------------------------------------------------------------------------
+
+TP_M = (56, 57, 80, 81, 4096)
+
+
+def tp_leg(fn, device, rank: int, world: int, sync: str = "stream", Ms=TP_M, steps: int = 20,
+           H: int = 7168, sample_rows: int = 8):
+    """The fused all-reduce + RMSNorm + MXFP4 step across the ranks of the job
+    (tp.FusedAllReduceRMSNormQuant: peer loads and stores over NVLink, no
+    multicast), both forms at each M: per-call time (two group barriers and
+    the kernel) and kernel-only time, both the max over ranks, the NVLink
+    bytes each rank moves, a check of sampled rows against the one-GPU kernel
+    on the same partials (rank 0) and of all ranks holding the same bits.  Every
+    rank takes the same collective steps.  Returns the record (rank 0's is
+    complete)."""
+    import hashlib
+    import torch
+    import torch.distributed as dist
+    from mxfp4_quantization_b200 import synth, tp
+    mode = synth.MXFP4
+    M_max = max(Ms)
+    wl = synth.RowWorkload("tp_leg", M=M_max, H=H, P=world, mode=mode, eps=1e-6, seed=23,
+                           channel_decades=1.0)
+    inp = wl.inputs(device=device)  # every rank draws every partial; each keeps its own
+    ar = tp.FusedAllReduceRMSNormQuant(M_max, H, mode, device=device, sync=sync)
+    ar.partial.copy_(inp["parts"][rank])
+    w = inp["weight"]
+    codes_scales = H // 2 + H // 32
+    out = {"H": H, "mode": "mxfp4", "world": world, "sync": sync, "steps": steps, "rows": {}}
+    try:
+        for M in Ms:
+            row = {}
+            for form, limits in (("one_stage", (M_max, M_max)), ("two_stage", (0, 0))):
+                ar.max_tokens, ar.max_tokens_h7168 = limits
+                # parity: one call from the drawn residual
+                ar.residual.copy_(inp["residual"])
+                o = ar(w, wl.eps, M)
+                torch.cuda.synchronize(device)
+                h = hashlib.sha256()
+                for t in o[:3]:
+                    h.update(t.contiguous().view(torch.uint8).cpu().numpy().tobytes())
+                digests = [None] * world
+                dist.all_gather_object(digests, h.hexdigest())
+                check = None
+                if rank == 0:
+                    # against the one-GPU kernel on local copies of every
+                    # rank's partial rows (the tests check that kernel against
+                    # the oracle): residual bit-exact, codes equal except where
+                    # the one-ulp freedom of y moves one
+                    g = torch.Generator().manual_seed(M)
+                    rows = sorted(set([0, M - 1] + torch.randint(0, M, (sample_rows,),
+                                                                 generator=g).tolist()))
+                    sel = torch.tensor(rows, device=device)
+                    pick = lambda t: t.index_select(0, sel).contiguous()  # noqa: E731
+                    ref = fn.rmsnorm_quant([pick(p) for p in inp["parts"]], w, wl.eps, mode,
+                                           residual=pick(inp["residual"]))
+                    torch.cuda.synchronize(device)
+                    q, qr = pick(o[0]), ref.q
+                    check = {"rows": len(rows),
+                             "residual_equal": bool(torch.equal(pick(o[2]), ref.residual_out)),
+                             "code_bytes_equal_frac": float((q == qr).float().mean()),
+                             "scales_equal_frac": float((pick(o[1]) == ref.scale).float().mean())}
+                # timing
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                ek = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(steps)]
+                for _ in range(3):
+                    ar(w, wl.eps, M)
+                torch.cuda.synchronize(device)
+                e[0].record()
+                for i in range(steps):
+                    ar(w, wl.eps, M, events=ek[i])
+                e[1].record()
+                torch.cuda.synchronize(device)
+                us_call = dist_max(e[0].elapsed_time(e[1]) * 1e3 / steps, device)
+                us_kernel = dist_max(statistics.median(a.elapsed_time(b) * 1e3 for a, b in ek),
+                                     device)
+                if form == "one_stage":
+                    nvl_read, nvl_write = (world - 1) * M * 2 * H, 0
+                else:
+                    shard = M // world + (1 if M % world else 0)
+                    nvl_read = (world - 1) * shard * 2 * H
+                    nvl_write = (world - 1) * shard * (2 * H + codes_scales)
+                row[form] = {"us_per_call": us_call, "us_kernel": us_kernel,
+                             "nvlink_bytes_read_per_rank": nvl_read,
+                             "nvlink_bytes_written_per_rank": nvl_write,
+                             "nvlink_GB_s_per_rank": (nvl_read + nvl_write) / (us_kernel * 1e-6)
+                             / 1e9 if us_kernel > 0 else None,
+                             "ranks_identical": len(set(digests)) == 1,
+                             "vs_one_gpu_kernel": check}
+            row["faster_kernel"] = min(("one_stage", "two_stage"),
+                                       key=lambda f: row[f]["us_kernel"])
+            out["rows"][str(M)] = row
+    finally:
+        ar.close()
+        dist.barrier()
+        del ar
+        torch.cuda.empty_cache()
+    return out
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle timing (reported baseline; the reference arm)
 # ---------------------------------------------------------------------------
 
@@ -773,6 +876,10 @@ def main_arm(args):
     e2e_ms, h2d, d2h = e2e_row(fn, wl, device, e2e_steps, 2, seed)
     e2e_ms_max = dist_max(e2e_ms, device)
 
+    tp_record = None
+    if world > 1 and args.tp_leg:
+        tp_record = tp_leg(fn, device, rank, world)
+
     extra = None
     cpu = cpu_all = None
     if world == 1 and not args.no_extras and args.workload == "prefill_group128":
@@ -824,6 +931,7 @@ def main_arm(args):
             "cpu_baseline": cpu,
             "cpu_baseline_all_cores": cpu_all,
             "workloads": extra,
+            "tensor_parallel": tp_record,
         }
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
@@ -844,6 +952,8 @@ def parse(argv=None):
     ap.add_argument("--calls-per-step", type=int, default=CALLS_PER_STEP,
                     help="fused calls per step (alternating between input slabs)")
     ap.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--tp-leg", action="store_true",
+                    help="with N > 1: also time the fused all-reduce across the ranks")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     a = ap.parse_args(argv)

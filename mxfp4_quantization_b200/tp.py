@@ -6,9 +6,11 @@ RMSNorm and the activation quantization that precede the next linear (sglang
 PR #29723, "Motivation"): one kernel instead of AllReduce -> RMSNorm ->
 quantize.  Here every rank owns a partial buffer (where its row-parallel GEMM
 writes), a residual replica and the output buffers of the quantized tuple;
-the buffers are mapped into every other rank's address space once (CUDA IPC
-through torch's tensor sharing, exchanged over torch.distributed), and each
-step runs one of two forms of the fused kernel between two group barriers:
+the buffers are mapped into every other rank's address space once (CUDA IPC:
+each rank opens its peers' memory handles, exchanged over torch.distributed,
+with its own device current and peer access enabled, so its kernels reach
+the peers' memory over NVLink with plain loads and stores), and each step
+runs one of two forms of the fused kernel between two group barriers:
 
   one-stage  every rank computes every row from all ranks' partials and
              writes only its own outputs (fn_rmsnorm_quant with the peer
@@ -29,11 +31,10 @@ deterministic preflight checks, before any collective; once the first
 barrier is entered every error raises, on every rank alike.
 """
 import datetime
-from typing import List, Optional, Sequence, Tuple
+from typing import Optional, Sequence, Tuple
 
 import torch
 import torch.distributed as dist
-from torch.multiprocessing.reductions import reduce_tensor
 
 from . import fusednorm as fn
 
@@ -56,21 +57,55 @@ def one_stage(M: int, H: int, max_tokens: int = ONE_STAGE_MAX_TOKENS,
     return M <= max_tokens_h7168 if H == 7168 else True
 
 
-def share(tensors: Sequence[Optional[torch.Tensor]], group=None) -> List[List[Optional[torch.Tensor]]]:
-    """Map every rank's `tensors` into this process: entry [d][i] is rank d's
-    i-th tensor (this rank's own tensors at d == rank, peers' through CUDA
-    IPC).  Collective over `group`; the owners must keep their tensors alive."""
+def _ipc_handle(t: torch.Tensor):
+    """(CUDA IPC handle of the allocation holding t, byte offset of t in it)."""
+    info = t.untyped_storage()._share_cuda_()
+    handle, storage_offset = info[1], info[3]
+    return bytes(handle), int(storage_offset) + t.storage_offset() * t.element_size()
+
+
+def share(tensors: Sequence[Optional[torch.Tensor]], group=None):
+    """Map every rank's `tensors` into this process: returns (addresses,
+    opened), where addresses[d][i] is the device address (int) of rank d's
+    i-th tensor, valid for kernels on this rank's device (this rank's own
+    tensors at d == rank; peers' through their CUDA IPC handles, opened with
+    this rank's device current and peer access enabled), and `opened` lists
+    the mappings to close with unshare().  Collective over `group`; the
+    owners must keep their tensors alive until every rank has unshared."""
+    from cuda.bindings import runtime as cudart
     rank, world = dist.get_rank(group), dist.get_world_size(group)
-    mine = [None if t is None else reduce_tensor(t) for t in tensors]
+    mine = [None if t is None else _ipc_handle(t) for t in tensors]
     everyone = [None] * world
     dist.all_gather_object(everyone, mine, group=group)
-    out = []
+    addresses, opened = [], []
     for d in range(world):
         if d == rank:
-            out.append(list(tensors))
-        else:
-            out.append([None if h is None else h[0](*h[1]) for h in everyone[d]])
-    return out
+            addresses.append([None if t is None else t.data_ptr() for t in tensors])
+            continue
+        row = []
+        for h in everyone[d]:
+            if h is None:
+                row.append(None)
+                continue
+            handle = cudart.cudaIpcMemHandle_t()
+            handle.reserved = h[0]
+            err, base = cudart.cudaIpcOpenMemHandle(handle,
+                                                    cudart.cudaIpcMemLazyEnablePeerAccess)
+            if err != cudart.cudaError_t.cudaSuccess:
+                unshare(opened)
+                raise RuntimeError(f"cudaIpcOpenMemHandle of rank {d}'s buffer: {err}")
+            opened.append(int(base))
+            row.append(int(base) + h[1])
+        addresses.append(row)
+    return addresses, opened
+
+
+def unshare(opened: Sequence[int]) -> None:
+    """Close the peer mappings that share() opened (this rank's device must be
+    current, and no work may still use them)."""
+    from cuda.bindings import runtime as cudart
+    for base in opened:
+        cudart.cudaIpcCloseMemHandle(base)
 
 
 class FusedAllReduceRMSNormQuant:
@@ -107,8 +142,16 @@ class FusedAllReduceRMSNormQuant:
         # the residual is updated in place on every rank (its replica)
         self._flag = torch.zeros(1, dtype=torch.float32, device=dev)
         torch.cuda.synchronize(dev)
-        self.peers = share([self.partial, self.residual, self.q, self.scale, self.y], group)
+        self.peers, self._opened = share([self.partial, self.residual, self.q, self.scale, self.y],
+                                         group)
         self.device = dev
+
+    def close(self) -> None:
+        """Close this rank's mappings of its peers' buffers.  Every rank calls
+        it after its last step, before any rank frees its buffers."""
+        torch.cuda.synchronize(self.device)
+        unshare(self._opened)
+        self._opened = []
 
     # -- ordering ---------------------------------------------------------------------
     def _barrier(self):
@@ -124,16 +167,20 @@ class FusedAllReduceRMSNormQuant:
         return (0 < M <= self.M_max and weight.dtype == torch.bfloat16 and weight.is_cuda and
                 weight.numel() == self.H and weight.is_contiguous() and eps >= 0.0)
 
-    def __call__(self, weight: torch.Tensor, eps: float, M: int):
+    def __call__(self, weight: torch.Tensor, eps: float, M: int, events=None):
         """One fused step over rows [0, M).  Returns (q, scale, residual_out, y)
         views of this rank's buffers, or None if the preflight declined (no
-        collective entered)."""
+        collective entered).  `events`: an optional pair of CUDA events
+        recorded on the current stream just before and just after the kernel
+        (the time between the two barriers)."""
         if not self.preflight(weight, eps, M):
             return None
         self._barrier()  # every rank's partial and residual are complete
+        if events is not None:
+            events[0].record()
         stream = torch.cuda.current_stream(self.device).cuda_stream
         H, mode = self.H, self.mode
-        parts = [p[0].data_ptr() for p in self.peers]
+        parts = [p[0] for p in self.peers]
         res = None if self.residual is None else self.residual.data_ptr()
         if one_stage(M, H, self.max_tokens, self.max_tokens_h7168):
             st = fn.fn_rmsnorm_quant(parts, self.world, res, weight.data_ptr(), float(eps), mode,
@@ -141,7 +188,7 @@ class FusedAllReduceRMSNormQuant:
                                      None if self.y is None else self.y.data_ptr(), stream)
             name = "fn_rmsnorm_quant"
         else:
-            col = lambda i: [p[i].data_ptr() for p in self.peers]  # noqa: E731
+            col = lambda i: [p[i] for p in self.peers]  # noqa: E731
             st = fn.fn_ar_rmsnorm_quant(parts, self.world, self.rank, res, weight.data_ptr(),
                                         float(eps), mode, M, H, col(2), col(3),
                                         None if res is None else col(1),
@@ -149,6 +196,8 @@ class FusedAllReduceRMSNormQuant:
             name = "fn_ar_rmsnorm_quant"
         if st != fn.FN_OK:
             raise fn.FusedNormError(name, st)
+        if events is not None:
+            events[1].record()
         self._barrier()  # every rank's outputs are complete
         scale = self.scale[:M] if self.scale.dim() == 2 else self.scale  # swizzled: padded, flat
         return (self.q[:M], scale, None if self.residual is None else self.residual[:M],

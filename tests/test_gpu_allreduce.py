@@ -179,6 +179,8 @@ def _rank_main(rank, world, port, mode, H, M_list, out):
                       for k in ("q", "scale", "residual_out", "y")]
             results.append((M, tp.one_stage(M, H), digest))
         assert ar(inp["weight"], wl.eps, M_max + 1) is None  # preflight: no collective
+        ar.close()
+        dist.barrier()
         out[rank] = results
     except Exception as e:  # reported to the parent
         out[rank] = f"error: {type(e).__name__}: {e}"
@@ -205,3 +207,49 @@ def test_two_processes_share_one_gpu(mode):
     assert codes == [0, 0], (codes, res)
     assert res[0] == res[1], "ranks disagree"
     assert [(m, s) for m, s, _ in res[0]] == [(40, True), (150, False)]
+
+
+def _leg_main(rank, world, port, out):
+    import torch.distributed as dist
+
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=90))
+    try:
+        torch.cuda.set_device(0)
+        fnb = gpu_util.lib()
+        out[rank] = bench.tp_leg(fnb, torch.device("cuda", 0), rank, world, sync="host",
+                                 Ms=(40, 150), steps=3, H=2048)
+    except Exception as e:  # reported to the parent
+        out[rank] = f"error: {type(e).__name__}: {e}"
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_tensor_parallel_leg_runs_on_two_processes():
+    """The bench's fused all-reduce leg (both forms, timing, the check against
+    the one-GPU kernel, ranks holding the same bits), run by two processes
+    sharing one GPU through CUDA IPC with host barriers."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        procs = [ctx.Process(target=_leg_main, args=(r, world, port, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=240)
+        codes = [p.exitcode for p in procs]
+        res = dict(out)
+    assert codes == [0, 0], (codes, res)
+    rec = res[0]
+    for M in ("40", "150"):
+        for form in ("one_stage", "two_stage"):
+            r = rec["rows"][M][form]
+            assert r["ranks_identical"], (M, form)
+            c = r["vs_one_gpu_kernel"]
+            assert c["residual_equal"] and c["code_bytes_equal_frac"] > 0.99, (M, form, c)
+            assert r["us_kernel"] > 0 and r["us_per_call"] >= r["us_kernel"]
