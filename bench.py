@@ -529,6 +529,22 @@ def hc_calls(fn, wl, device):
     return make
 
 
+def small_graph_leg(fn, device, wl, per_call_bytes, make):
+    """µs per call of a small-M workload: a CUDA graph of calls over rotating
+    buffers whose total exceeds L2 (cold inputs), plain and as a chain of
+    programmatic launches."""
+    n_sets = max(64, int(2 * L2_BYTES / per_call_bytes) + 1)
+    n_sets = min(n_sets, 8192)
+    us, eager = time_graph_calls(make, n_sets, 7, device)
+    launch = list(fn.fn_last_launch())
+    # the same graph with every call a programmatic dependent of the one before
+    with fn.programmatic_launch(True):
+        us_pdl, _ = time_graph_calls(make, n_sets, 7, device)
+    return {"us_per_call_graph": us, "us_per_call_graph_programmatic": us_pdl,
+            "us_single_call_host_to_device": eager, "calls_per_graph": n_sets,
+            "GB_s": per_call_bytes / (us * 1e-6) / 1e9, "launch": launch}
+
+
 def secondary_workloads(fn, device, peak):
     """Every other workload, each on its own timed region (N=1 only)."""
     import torch
@@ -588,16 +604,7 @@ def secondary_workloads(fn, device, peak):
     res["quant_only"] = qo
 
     def small(wl, per_call_bytes, make):
-        n_sets = max(64, int(2 * L2_BYTES / per_call_bytes) + 1)
-        n_sets = min(n_sets, 8192)
-        us, eager = time_graph_calls(make, n_sets, 7, device)
-        launch = list(fn.fn_last_launch())
-        # the same graph with every call a programmatic dependent of the one before
-        with fn.programmatic_launch(True):
-            us_pdl, _ = time_graph_calls(make, n_sets, 7, device)
-        return {"us_per_call_graph": us, "us_per_call_graph_programmatic": us_pdl,
-                "us_single_call_host_to_device": eager, "calls_per_graph": n_sets,
-                "GB_s": per_call_bytes / (us * 1e-6) / 1e9, "launch": launch}
+        return small_graph_leg(fn, device, wl, per_call_bytes, make)
 
     wl = synth.PER_TOKEN_SMALL
     r = small(wl, wl.bytes_per_call(), decode_calls(fn, wl, device))
@@ -622,8 +629,16 @@ def secondary_workloads(fn, device, peak):
         b8 = wl.bytes_per_call() - M * (wl.Hq + wl.Hk) * (wl.D - 4)
         qk[f"m{M}_fp8"] = small(wl, b8, qk_calls(fn, wl, device, fp8=True))
     res["qk_prologue"] = qk
+    res["hc_mix"] = hc_mix_leg(fn, device, peak, small)
+    return res
+
+
+def hc_mix_leg(fn, device, peak, small, Ms=None):
+    """hc_mix at each M: graph replays over rotating cold weight sets."""
+    import torch
+    from mxfp4_quantization_b200 import synth
     hc = {}
-    for M in synth.HC_M:
+    for M in (Ms or synth.HC_M):
         wl = synth.hc_mix(M)
         r = small(wl, wl.bytes_per_call(), hc_calls(fn, wl, device))
         wb = wl.weight_bytes()
@@ -636,8 +651,7 @@ def secondary_workloads(fn, device, peak):
                   "variant": fn.fn_last_variant()})
         hc[f"m{M}"] = r
         torch.cuda.empty_cache()
-    res["hc_mix"] = hc
-    return res
+    return hc
 
 
 # ---------------------------------------------------------------------------
@@ -952,6 +966,10 @@ def parse(argv=None):
     ap.add_argument("--calls-per-step", type=int, default=CALLS_PER_STEP,
                     help="fused calls per step (alternating between input slabs)")
     ap.add_argument("--no-extras", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--leg", choices=["hc_mix"], default=None,
+                    help="run only this secondary workload and print its record")
+    ap.add_argument("--hc-m", type=int, nargs="*", default=None,
+                    help="with --leg hc_mix: the row counts (default 1 2 4 8 16)")
     ap.add_argument("--tp-leg", action="store_true",
                     help="with N > 1: also time the fused all-reduce across the ranks")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -961,6 +979,23 @@ def parse(argv=None):
     return a
 
 
+def leg_arm(args):
+    """One secondary workload alone (one GPU), its record as one JSON line."""
+    import torch
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    from mxfp4_quantization_b200.build import build_library
+    build_library()
+    from mxfp4_quantization_b200 import fusednorm as fn
+    peak, _ = hbm_peak()
+    small = lambda wl, b, make: small_graph_leg(fn, device, wl, b, make)  # noqa: E731
+    rec = hc_mix_leg(fn, device, peak, small, args.hc_m)
+    print(json.dumps({"leg": args.leg, "record": rec}), flush=True)
+    return 0
+
+
 if __name__ == "__main__":
     args = parse()
-    sys.exit(reference_arm(args) if args.impl == "reference" else main_arm(args))
+    if args.impl == "reference":
+        sys.exit(reference_arm(args))
+    sys.exit(leg_arm(args) if args.leg else main_arm(args))

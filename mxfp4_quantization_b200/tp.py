@@ -58,10 +58,21 @@ def one_stage(M: int, H: int, max_tokens: int = ONE_STAGE_MAX_TOKENS,
 
 
 def _ipc_handle(t: torch.Tensor):
-    """(CUDA IPC handle of the allocation holding t, byte offset of t in it)."""
+    """(CUDA IPC handle of the cudaMalloc allocation holding t, byte offset of
+    t in it), from torch's storage sharing.  torch's handle string is a
+    version byte, a kind byte ('c': a plain cudaMalloc segment) and the 64
+    bytes of the cudaIpcMemHandle_t; the offset is the storage's offset in
+    that segment."""
     info = t.untyped_storage()._share_cuda_()
-    handle, storage_offset = info[1], info[3]
-    return bytes(handle), int(storage_offset) + t.storage_offset() * t.element_size()
+    raw, storage_offset = bytes(info[1]), int(info[3])
+    if len(raw) == 66 and raw[1:2] == b"c":
+        handle = raw[2:]
+    elif len(raw) == 64:
+        handle = raw
+    else:
+        raise RuntimeError("this CUDA allocation cannot be shared through a CUDA IPC handle "
+                           "(expandable segments?)")
+    return handle, storage_offset + t.storage_offset() * t.element_size()
 
 
 def share(tensors: Sequence[Optional[torch.Tensor]], group=None):
