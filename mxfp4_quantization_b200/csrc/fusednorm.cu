@@ -469,7 +469,7 @@ int hc_check(const void* x, const void* w_down, const void* w_up, int64_t M, int
              int r, const void* out) {
   if (M < 0 || hc < 1 || C <= 0 || r <= 0) return FN_ERR_INVALID;
   if (hc != fn::kHcStreams || M > fn::kHcMaxRows || C % 16 ||
-      (int64_t)hc * C > (int64_t)fn::kHcDownThreads * 64 || r % 8 || r > fn::kHcMaxRank)
+      (int64_t)hc * C > fn::kHcMaxK || r % 8 || r > fn::kHcMaxRank)
     return FN_ERR_UNSUPPORTED;
   if (M == 0) return FN_OK;
   if (!x || !w_down || !w_up || !out) return FN_ERR_INVALID;
@@ -486,6 +486,40 @@ int hc_mix_channels(int64_t C, int sms) {
        cpb <= fn::kHcMaxMixChannels; cpb += 4)
     if (C % cpb == 0) return (int)cpb;
   return 16;
+}
+
+// Shared memory a launch of the gate-and-mix kernel `k` asks for so that no SM
+// holds two of its blocks (more than half of an SM's shared memory), with the
+// shared-memory carveout of both hc_mix kernels at its maximum so that a gate
+// block still fits beside a block of the first kernel; cached per kernel, -1
+// if the runtime refuses.  Launched early as a programmatic dependent, the
+// small gate blocks were otherwise packed up to five to an SM onto the SMs the
+// first kernel left free (measured on B200 with per-block SM ids: 128 blocks
+// on 28 SMs at M = 4 and 8), multiplying their logit time.
+int hc_spread_blocks(fn::HCKernel k, fn::HCKernel first) {
+  static std::mutex mu;
+  static std::map<const void*, int> cache;
+  const void* key = reinterpret_cast<const void*>(k);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int dev = 0, per_sm = 0, bytes = -1;
+  cudaFuncAttributes fa;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) ==
+          cudaSuccess &&
+      cudaFuncGetAttributes(&fa, k) == cudaSuccess) {
+    const int want = per_sm / 2 + 1 - (int)fa.sharedSizeBytes;
+    if (cudaFuncSetAttribute(first, cudaFuncAttributePreferredSharedMemoryCarveout, 100) ==
+            cudaSuccess &&
+        cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100) ==
+            cudaSuccess &&
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, want) == cudaSuccess)
+      bytes = want;
+  }
+  if (bytes < 0) (void)cudaGetLastError();
+  cache[key] = bytes;
+  return bytes;
 }
 
 // Launches the two hc_mix kernels with t in `ws` (fp32 [M, r], checked by the
@@ -508,8 +542,8 @@ int hc_launch(const void* x, const void* w_down, const void* w_up, int64_t M, in
   fn::HCKernel k1 = fn::hc_down_pick(hc_rows_bound(M), cw);
   if (!k1) return FN_ERR_UNSUPPORTED;
   const int cvec = p.K / 8 / fn::kHcCluster;
-  // at least one thread per partial sum of the block (rows bound x weight rows)
-  const int t1 = std::max(round32(cvec), round32(hc_rows_bound(M) * cw));
+  // row groups of 4 rows: one warp-aligned set of threads per row group
+  const int t1 = round32(cvec) * std::max(1, hc_rows_bound(M) / 4);
   const unsigned g1 = (unsigned)(r / cw * fn::kHcCluster);
   const int sms = sm_count();
   if (sms <= 0) return FN_ERR_CUDA;
@@ -519,9 +553,13 @@ int hc_launch(const void* x, const void* w_down, const void* w_up, int64_t M, in
   const int t2 = fn::kHcStreams * p.cpb * (int)((M + 3) / 4);
   fn::HCKernel k2 = fn::hc_gate_mix_pick(r / 8);
   if (!k2) return FN_ERR_UNSUPPORTED;
+  // one gate block per SM while the blocks fit the GPU at once
+  const int smem2 = (int)g2 <= sms ? hc_spread_blocks(k2, k1) : 0;
+  if (smem2 < 0) return FN_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (launch_kernel(k1, g1, (unsigned)t1, 0, st, fn::kHcCluster, p) != FN_OK) return FN_ERR_CUDA;
-  if (launch_kernel_pdl(k2, g2, (unsigned)t2, 0, st, 1, true, p) != FN_OK) return FN_ERR_CUDA;
+  if (launch_kernel_pdl(k2, g2, (unsigned)t2, (size_t)smem2, st, 1, true, p) != FN_OK)
+    return FN_ERR_CUDA;
   tl_variant = FN_VARIANT_HC_MIX;
   tl_launch[0] = (int32_t)g1;
   tl_launch[1] = t1;

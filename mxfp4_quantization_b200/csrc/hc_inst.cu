@@ -5,14 +5,14 @@
 namespace fn {
 
 HCKernel hc_down_pick(int mm, int cw) {
-#define FN_HC(MM)                                   \
-  if (mm == MM) {                                   \
-    if (cw == 1) return hc_down_kernel<MM, 1>;      \
-    if (cw == 2) return hc_down_kernel<MM, 2>;      \
-    if (cw == 4) return hc_down_kernel<MM, 4>;      \
-    return nullptr;                                 \
+#define FN_HC(MM, MR, NG)                             \
+  if (mm == MM) {                                     \
+    if (cw == 1) return hc_down_kernel<MR, NG, 1>;    \
+    if (cw == 2) return hc_down_kernel<MR, NG, 2>;    \
+    if (cw == 4) return hc_down_kernel<MR, NG, 4>;    \
+    return nullptr;                                   \
   }
-  FN_HC(1) FN_HC(2) FN_HC(4) FN_HC(8) FN_HC(16)
+  FN_HC(1, 1, 1) FN_HC(2, 2, 1) FN_HC(4, 4, 1) FN_HC(8, 4, 2) FN_HC(16, 4, 4)
 #undef FN_HC
   return nullptr;
 }

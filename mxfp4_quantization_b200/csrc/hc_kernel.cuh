@@ -14,10 +14,11 @@
 //  * hc_down_kernel: t = W_down x.  Clusters of 8 blocks; cluster g owns CW
 //    rows of W_down and its 8 blocks split the hc*C columns, so every block
 //    reads one contiguous piece of each of its CW weight rows (the weight is
-//    read exactly once over the grid) and the matching columns of every x row.
-//    A thread owns one 16-byte vector of the piece; the block reduces its
-//    threads' M * CW partial sums with a warp reduce-scatter and shared
-//    memory, every block stores its partials into rank 0's shared memory
+//    read exactly once from HBM over the grid) and the matching columns of
+//    every x row.  A thread owns one 16-byte vector of the piece for up to 4
+//    rows (more rows: more row groups of threads); the block reduces its
+//    threads' partial sums with a warp reduce-scatter and shared memory,
+//    every block stores its partials into rank 0's shared memory
 //    (distributed shared memory), and after one cluster barrier rank 0 sums
 //    them in rank order.  t (fp32 [M, r]) goes to the caller's workspace.
 //  * hc_gate_mix_kernel: one block per cpb channels (no more blocks than
@@ -63,49 +64,58 @@ __device__ __forceinline__ void warp_reduce_scatter(float (&a)[V]) {
 }
 
 // t[m, g*CW + j] = sum_k x[m, k] * w_down[g*CW + j, k] for m < M, j < CW.
-// Grid: (r / CW) clusters of kHcCluster blocks; blockDim.x = the larger of
-// round32(K / 64) and M * CW, at most kHcDownThreads.
-template <int MM, int CW>
+// Grid: (r / CW) clusters of kHcCluster blocks.  The rows are split over NG
+// row groups of threads, MR rows each (MM = NG * MR rows at most): thread
+// (rg, o) owns vector o of the block's piece for rows rg*MR .. rg*MR+MR-1, so
+// each thread holds MR * CW partial sums (16 at most) whatever M is, and a
+// block has NG times as many warps to cover its loads' latency.
+// blockDim.x = NG * nv, nv = round32(K / 64) threads per row group.
+template <int MR, int NG, int CW>
 __global__ void __launch_bounds__(kHcDownThreads) hc_down_kernel(const __grid_constant__ HCParams p) {
   namespace cg = cooperative_groups;
-  constexpr int V = MM * CW;
+  constexpr int V = MR * CW;         // partial sums per thread
+  constexpr int VB = NG * V;         // per block: every row times CW
   __shared__ float red[kHcDownThreads / 32][V];
-  __shared__ float slots[kHcCluster][V];  // rank 0's: every block's partials
+  __shared__ float slots[kHcCluster][VB];  // rank 0's: every block's partials
   pdl_enter();
 
   cg::cluster_group cl = cg::this_cluster();
   const int rank = (int)cl.block_rank();
   const int g = blockIdx.x / kHcCluster;
   const int kvec = p.K / 8, cvec = kvec / kHcCluster;
-  const int o = threadIdx.x, lane = o & 31, warp = o >> 5;
+  const int nv = blockDim.x / NG;    // threads per row group (whole warps)
+  const int tid = threadIdx.x, rg = tid / nv, o = tid % nv;
+  const int lane = tid & 31, warp = tid >> 5;
   const int64_t v = (int64_t)rank * cvec + o;
 
   float acc[V];
 #pragma unroll
   for (int i = 0; i < V; ++i) acc[i] = 0.f;
   if (o < cvec) {
-    uint4 w[CW], xv[MM];
+    uint4 w[CW], xv[MR];
 #pragma unroll
-    for (int j = 0; j < CW; ++j) w[j] = ld_stream_nc(p.w_down + (int64_t)(g * CW + j) * kvec + v);
+    for (int j = 0; j < CW; ++j) w[j] = ld_keep(p.w_down + (int64_t)(g * CW + j) * kvec + v);
 #pragma unroll
-    for (int m = 0; m < MM; ++m)
-      xv[m] = m < p.M ? ld_stream_nc(p.x + (int64_t)m * kvec + v) : make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < MR; ++i) {
+      const int m = rg * MR + i;
+      xv[i] = m < p.M ? ld_stream_nc(p.x + (int64_t)m * kvec + v) : make_uint4(0u, 0u, 0u, 0u);
+    }
 #pragma unroll
-    for (int m = 0; m < MM; ++m) {
+    for (int i = 0; i < MR; ++i) {
 #pragma unroll
       for (int j = 0; j < CW; ++j) {
         float s = 0.f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          s = fma_bf16<false>(word(xv[m], i), word(w[j], i), s);
-          s = fma_bf16<true>(word(xv[m], i), word(w[j], i), s);
+        for (int e = 0; e < 4; ++e) {
+          s = fma_bf16<false>(word(xv[i], e), word(w[j], e), s);
+          s = fma_bf16<true>(word(xv[i], e), word(w[j], e), s);
         }
-        acc[m * CW + j] = s;
+        acc[i * CW + j] = s;
       }
     }
   }
 
-  // the block's sums: warps first, then the warps' results in warp order
+  // the block's sums: warps first, then each row group's warps in warp order
   warp_reduce_scatter<V>(acc);
   if constexpr (V >= 32) {
 #pragma unroll
@@ -114,20 +124,22 @@ __global__ void __launch_bounds__(kHcDownThreads) hc_down_kernel(const __grid_co
     if (lane % (32 / V) == 0) red[warp][lane / (32 / V)] = acc[0];
   }
   __syncthreads();
-  const int nw = blockDim.x >> 5;
-  if (o < V) {
-    float s = red[0][o];
-    for (int w = 1; w < nw; ++w) s += red[w][o];
-    *cl.map_shared_rank(&slots[rank][o], 0) = s;
+  const int nwg = nv >> 5;  // warps per row group
+  if (tid < VB) {
+    const int grp = tid / V, idx = tid % V;
+    float s = red[grp * nwg][idx];
+    for (int w = 1; w < nwg; ++w) s += red[grp * nwg + w][idx];
+    *cl.map_shared_rank(&slots[rank][tid], 0) = s;
   }
   // the stores into rank 0's shared memory are complete and visible to it
   // after the barrier; only rank 0 reads them, so the others may leave
   cl.sync();
-  if (rank == 0 && o < V) {
-    float s = slots[0][o];
+  if (rank == 0 && tid < VB) {
+    float s = slots[0][tid];
 #pragma unroll
-    for (int c = 1; c < kHcCluster; ++c) s += slots[c][o];
-    const int m = o / CW, j = o % CW;
+    for (int c = 1; c < kHcCluster; ++c) s += slots[c][tid];
+    const int grp = tid / V, idx = tid % V;
+    const int m = grp * MR + idx / CW, j = idx % CW;
     if (m < p.M) p.t[(int64_t)m * p.r + g * CW + j] = s;
   }
 }

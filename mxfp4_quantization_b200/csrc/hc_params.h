@@ -22,10 +22,12 @@ constexpr int kHcMaxRows = 16;         // M <= 16 (decode-sized)
 constexpr int kHcMaxRank = 128;        // r <= 128
 constexpr int kHcMaxMixChannels = 32;  // channels per block of hc_gate_mix_kernel, at most
 constexpr int kHcMixThreads = 512;     // 4 streams x channels x row groups of 4, at most
-constexpr int kHcDownThreads = 256;    // one 16-byte vector per thread: hc*C <= 16384
+constexpr int kHcDownThreads = 1024;   // row groups x (one 16-byte vector per thread)
+constexpr int kHcMaxK = 16384;         // hc*C: K / 64 <= 256 vectors per block and row group
 
 // Instances (hc_inst.cu): hc_down_kernel for rows bound MM in {1, 2, 4, 8, 16}
-// and weight rows per cluster CW in {1, 2, 4}; hc_gate_mix_kernel for W_up
+// (rows per thread MR = min(MM, 4), row groups MM / MR) and weight rows per
+// cluster CW in {1, 2, 4}; hc_gate_mix_kernel for W_up
 // row vectors RV in {1, 2, 4, 8, 16} (rows of r <= 8 * RV values).
 using HCKernel = void (*)(const HCParams);
 HCKernel hc_down_pick(int mm, int cw);
