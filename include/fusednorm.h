@@ -275,9 +275,8 @@ FN_API int fn_qk_norm_gate_fp8(const void* qkv, int64_t M, int64_t row_stride, i
  *            and may be reused as soon as the call's work on `stream` is done.
  * Overlap    out and workspace must not overlap each other or any input
  *            (FN_ERR_INVALID).
- * fn_last_launch: out[0] blocks and out[1] threads of the first kernel
- * (clusters of 8 blocks), out[2] blocks of the second, out[3] weight rows per
- * cluster.
+ * fn_last_launch: out[0] blocks (clusters of 8) and out[1] threads of the
+ * first kernel, out[2] blocks and out[3] threads of the second.
  */
 FN_API int fn_hc_mix(const void* x, const void* w_down, const void* w_up, int64_t M, int hc,
                      int64_t C, int r, void* out, void* workspace, void* stream);
@@ -294,7 +293,7 @@ FN_API int64_t fn_hc_mix_workspace_bytes(int64_t M, int r);
  * point where they run this step: code inside a section that must not
  * allocate (a real-time or inference loop that has reserved all its memory up
  * front, a host callback, a plugin whose framework owns every allocation).
- * The paper has no counterpart; it describes no memory management.
+ * The pages have no counterpart; they describe no memory management.
  *
  * Arguments, checks and errors as fn_hc_mix, without `workspace`.
  * Scratch    a file-scope device array of the library holding t for at most

@@ -1,5 +1,5 @@
-// Instances of the hc_mix column-split kernel (rows bound x weight rows per
-// cluster); the gate-and-mix kernel has one instance, taken by the host code.
+// Instances of the hc_mix kernels: the column-split kernel per rows bound and
+// weight rows per block, the gate-and-mix kernel per W_up row length.
 #include "hc_kernel.cuh"
 
 namespace fn {

@@ -449,8 +449,9 @@ def hc_mix(x: torch.Tensor, w_down: torch.Tensor, w_up: torch.Tensor, *, hc: int
            workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Low-rank gate over the hyper-state: x bf16 [M, hc*C] (M <= 16),
     w_down bf16 [r, hc*C], w_up bf16 [hc*C, r]; returns the gated mix of the
-    hc streams, bf16 [M, C] (see fn_hc_mix).  The workspace (fp32 [M, r]) is
-    allocated with torch unless given."""
+    hc streams, bf16 [M, C] (see fn_hc_mix).  The workspace (t, fp32 [M, r]:
+    fn_hc_mix_workspace_bytes(M, r) bytes) is allocated with torch unless
+    given."""
     for t, n in ((x, "x"), (w_down, "w_down"), (w_up, "w_up")):
         if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 2 or not t.is_contiguous():
             raise TypeError(f"{n} must be a contiguous 2-D bf16 CUDA tensor")
@@ -461,8 +462,11 @@ def hc_mix(x: torch.Tensor, w_down: torch.Tensor, w_up: torch.Tensor, *, hc: int
     C = K // hc
     if out is None:
         out = torch.empty((M, C), dtype=torch.bfloat16, device=x.device)
+    need = fn_hc_mix_workspace_bytes(M, r)
     if workspace is None:
-        workspace = torch.empty((max(1, M * r),), dtype=torch.float32, device=x.device)
+        workspace = torch.empty((max(1, need // 4),), dtype=torch.float32, device=x.device)
+    elif workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace holds fewer than the {need} bytes fn_hc_mix needs")
     st = fn_hc_mix(x.data_ptr(), w_down.data_ptr(), w_up.data_ptr(), M, hc, C, r,
                    out.data_ptr(), workspace.data_ptr(), _stream(x.device))
     if st != FN_OK:

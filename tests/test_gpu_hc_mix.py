@@ -177,5 +177,8 @@ def test_rejected_calls_touch_nothing(fnb):
     assert st == fnb.FN_ERR_ALIGN
     st = fnb.fn_hc_mix(*args, 4, 4, wl.C, wl.r, go.t.data_ptr(), go.t.data_ptr() + 64, None)
     assert st == fnb.FN_ERR_INVALID
+    # the tensor API refuses a workspace smaller than fn_hc_mix_workspace_bytes
+    with pytest.raises(ValueError):
+        fnb.hc_mix(inp["x"], inp["w_down"], inp["w_up"], out=go.t, workspace=gw.t[:-1])
     torch.cuda.synchronize()
     assert go.untouched() and gw.untouched()
