@@ -550,7 +550,8 @@ int hc_launch(const void* x, const void* w_down, const void* w_up, int64_t M, in
   p.cpb = hc_mix_channels(C, sms);
   if (p.cpb == 0) return FN_ERR_UNSUPPORTED;
   const unsigned g2 = (unsigned)(C / p.cpb);
-  const int t2 = fn::kHcStreams * p.cpb * (int)((M + 3) / 4);
+  // one warp per 8 of the block's 4 * cpb W_up rows
+  const int t2 = 32 * (fn::kHcStreams * p.cpb / 8);
   fn::HCKernel k2 = fn::hc_gate_mix_pick(r / 8);
   if (!k2) return FN_ERR_UNSUPPORTED;
   // one gate block per SM while the blocks fit the GPU at once

@@ -22,9 +22,10 @@
 //    (distributed shared memory), and after one cluster barrier rank 0 sums
 //    them in rank order.  t (fp32 [M, r]) goes to the caller's workspace.
 //  * hc_gate_mix_kernel: one block per cpb channels (no more blocks than
-//    SMs).  Before it waits for the first kernel every thread loads its row
-//    of W_up into registers and its x values; once t is visible it forms the
-//    gate logits, the sigmoids and the mix.
+//    SMs).  Before it waits for the first kernel every warp loads its W_up
+//    rows into tensor-core fragments and every thread its x values; once t
+//    is visible the warps form the gate logits (mma tiles), the sigmoids and
+//    the mix.
 // Every sum has a fixed order, so a launch shape always gives the same bits.
 #pragma once
 #include <cooperative_groups.h>
@@ -144,32 +145,86 @@ __global__ void __launch_bounds__(kHcDownThreads) hc_down_kernel(const __grid_co
   }
 }
 
+// D += A B for one m16n8k16 tile: A bf16 16 x 16 (row-major fragment a0..a3),
+// B bf16 16 x 8 (column fragment b0, b1), D fp32 16 x 8 (d0..d3).  Lane (g,
+// q) = (lane / 4, lane % 4) holds A rows g and g+8 at k = 2q, 2q+1 (a0, a1)
+// and k = 2q+8, 2q+9 (a2, a3), B column g at those k (b0, b1), and D rows g
+// and g+8 at columns 2q, 2q+1.
+__device__ __forceinline__ void mma_bf16_16x8x16(float (&d)[4], const uint32_t (&a)[4],
+                                                 uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two fp32 values as three bf16 pairs whose sum is the pair to within 2^-24
+// relative: hi = bf16(v), mid = bf16(v - hi), lo = bf16(v - hi - mid).  Each
+// difference is exact in fp32 (v and its bf16 rounding share their leading
+// bits), so only the last rounding is lost.
+struct Bf16Split3 {
+  uint32_t hi, mid, lo;
+};
+__device__ __forceinline__ Bf16Split3 split3_bf16x2(float v0, float v1) {
+  Bf16Split3 r;
+  r.hi = pack_bf16x2(v0, v1);
+  const float e0 = v0 - bf_lo(r.hi), e1 = v1 - bf_hi(r.hi);
+  r.mid = pack_bf16x2(e0, e1);
+  r.lo = pack_bf16x2(e0 - bf_lo(r.mid), e1 - bf_hi(r.mid));
+  return r;
+}
+
 // u[m, c] for the channels [c0, c0 + cpb) of this block: gate logits of the
 // 4 streams from t and W_up, logistic sigmoid, gated sum of the streams.
-// Thread (mg, s, c) keeps W_up row s*C + c0 + c (r values, RV 16-byte vectors
-// at most) in registers and forms the logits of rows 4mg .. 4mg+3 from t,
-// read from shared memory transposed ([j][m], so one 16-byte read gives four
-// rows, the same address for a whole m-group: a broadcast); the gates meet
-// in shared memory, and thread (m, c) forms the gated sum of the streams in
-// stream order.  Launched as a programmatic dependent of hc_down_kernel:
-// every load that does not depend on t is issued before the wait.
-// blockDim.x = 4 * cpb * ceil(M / 4).
+// The logits of the block are one small product z = t W_up^T of 16 rows
+// (M <= 16; rows beyond M are zero) by 4 * cpb W_up rows (n = s * cpb + c
+// is W_up row s*C + c0 + c) over the rank, on the tensor cores: warp w owns
+// the 8 W_up rows 8w .. 8w+7 (one n-tile) and runs m16n8k16 tiles over the
+// rank padded to 16 * KS.  t (fp32) enters as three bf16 parts (hi + mid +
+// lo, exact to 2^-24 relative): every product of a part with a bf16 weight
+// is exact in fp32, so the logits carry fp32 accuracy.  The thread that
+// reads a vector of t splits it and stores the parts in shared memory, once
+// per block; the warps read their A fragments from there and accumulate
+// each part's products separately, adding them from the smallest.  The
+// W_up fragments come straight from global memory.  The gates meet in
+// shared memory, and thread (m, c) forms the gated sum of the streams in
+// stream order.  Launched as a programmatic dependent of hc_down_kernel: the
+// W_up fragments and the x values, which do not depend on t, are loaded
+// before the wait.  blockDim.x = 32 * (4 * cpb / 8); the padded rank 16 * KS
+// covers r (RV = r / 8 rounded up to a power of two).
 template <int RV>
 __global__ void __launch_bounds__(kHcMixThreads) hc_gate_mix_kernel(
     const __grid_constant__ HCParams p) {
-  __shared__ __align__(16) float tt[RV * 8][kHcMaxRows];                    // [j][m]
-  __shared__ float gs[kHcMaxRows][kHcStreams][kHcMaxMixChannels];         // gates
+  constexpr int KS = RV >= 2 ? RV / 2 : 1;  // k-steps of 16
+  // the parts of t in shared memory: per row, per 4 columns, 8 words {hi01,
+  // hi23, mid01, mid23, lo01, lo23, -, -} (bf16 pairs of columns 0-1 and
+  // 2-3); row stride 32 KS + 4 words, so the two rows a quarter-warp reads
+  // fall in disjoint banks
+  constexpr int RS = 32 * KS + 4;
+  __shared__ __align__(16) uint32_t tp[kHcMaxRows][RS];
+  __shared__ float gs[kHcMaxRows][kHcStreams][kHcMaxMixChannels];  // gates
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int cpb = p.cpb, c0 = blockIdx.x * cpb, tid = threadIdx.x;
-  const int rv = p.r / 8;
-  const int mg = tid / (kHcStreams * cpb), rem = tid % (kHcStreams * cpb);
-  const int s = rem / cpb, c = rem % cpb;
-  // every global load first: this thread's W_up row ...
-  uint4 w[RV];
-  const uint4* wrow = p.w_up + ((int64_t)s * p.C + c0 + c) * rv;
+  const int lane = tid & 31, warp = tid >> 5, g = lane >> 2, q = lane & 3;
+  // Lane quarter q takes columns 16k + 4q .. 16k + 4q + 3 of k-step k (the
+  // order of the rank inside a tile is free: the tile sums over it).  B
+  // fragments: W_up row of n = 8 * warp + g at those columns; columns at or
+  // beyond r (whole 4-column chunks, since r % 8 == 0) are zero.
+  uint32_t b[KS][2];
+  {
+    const int n = 8 * warp + g;
+    const uint16_t* wrow =
+        reinterpret_cast<const uint16_t*>(p.w_up) + ((int64_t)(n / cpb) * p.C + c0 + n % cpb) * p.r;
 #pragma unroll
-  for (int q = 0; q < RV; ++q) w[q] = q < rv ? ld_keep(wrow + q) : make_uint4(0u, 0u, 0u, 0u);
+    for (int k = 0; k < KS; ++k) {
+      const int col = 16 * k + 4 * q;
+      const uint2 w = col < p.r ? __ldg(reinterpret_cast<const uint2*>(wrow + col)) : make_uint2(0u, 0u);
+      b[k][0] = w.x;
+      b[k][1] = w.y;
+    }
+  }
   // ... and, as thread (xm, xc) of the mix, the four streams of x[xm, c0 + xc]
   const int xm = tid / cpb, xc = tid % cpb;
   const bool mixer = xm < p.M;
@@ -179,13 +234,15 @@ __global__ void __launch_bounds__(kHcMixThreads) hc_gate_mix_kernel(
   for (int k = 0; k < kHcStreams; ++k)
     xv[k] = mixer ? __uint_as_float((uint32_t)__ldg(xr + (int64_t)k * p.C) << 16) : 0.f;
 
-  // entries of t beyond M rows or r columns read as zero (they add nothing)
-  for (int i = tid; i < RV * 8 * kHcMaxRows; i += blockDim.x) (&tt[0][0])[i] = 0.f;
+  // entries of t beyond M rows or r columns read as zero (they add nothing);
+  // cleared before the wait, where the barrier costs nothing
+  for (int i = tid; i < kHcMaxRows * RS / 4; i += blockDim.x)
+    reinterpret_cast<uint4*>(&tp[0][0])[i] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
 
   // t is written by the kernel this one depends on: 16-byte loads, two per
-  // thread in flight (M * r / 4 vectors: one pass for every C >= 1024), stored
-  // transposed
+  // thread in flight (M * r / 4 vectors: one pass for every C >= 256), each
+  // split into its parts
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int nt = p.M * p.r / 4;
   for (int i0 = 0; i0 < nt; i0 += 2 * blockDim.x) {
@@ -199,41 +256,40 @@ __global__ void __launch_bounds__(kHcMixThreads) hc_gate_mix_kernel(
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int i = i0 + tid + k * blockDim.x;
-      if (i < nt) {
-        const int m = (4 * i) / p.r, j = (4 * i) % p.r;
-        tt[j][m] = tq[k].x;
-        tt[j + 1][m] = tq[k].y;
-        tt[j + 2][m] = tq[k].z;
-        tt[j + 3][m] = tq[k].w;
-      }
+      if (i >= nt) continue;
+      const Bf16Split3 v01 = split3_bf16x2(tq[k].x, tq[k].y), v23 = split3_bf16x2(tq[k].z, tq[k].w);
+      uint32_t* dst = &tp[(4 * i) / p.r][2 * ((4 * i) % p.r)];
+      *reinterpret_cast<uint4*>(dst) = make_uint4(v01.hi, v23.hi, v01.mid, v23.mid);
+      *reinterpret_cast<uint2*>(dst + 4) = make_uint2(v01.lo, v23.lo);
     }
   }
   __syncthreads();
 
-  // logits of rows 4mg .. 4mg+3; two accumulator pairs per row pair (even
-  // and odd j) halve the dependent chains
-  float2 za[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-  float2 zb[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  // one chain of tiles per part; rows g+8 only where M has them (warp-uniform)
+  float dh[4] = {0.f, 0.f, 0.f, 0.f}, dm[4] = {0.f, 0.f, 0.f, 0.f}, dl[4] = {0.f, 0.f, 0.f, 0.f};
+  const bool upper = p.M > 8;
 #pragma unroll
-  for (int q = 0; q < RV; ++q) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = 8 * q + 2 * e;
-      const float wl = bf_lo(word(w[q], e)), wh = bf_hi(word(w[q], e));
-      const float4 t0 = *reinterpret_cast<const float4*>(&tt[j][4 * mg]);
-      const float4 t1 = *reinterpret_cast<const float4*>(&tt[j + 1][4 * mg]);
-      za[0] = fma_f32x2(make_float2(t0.x, t0.y), make_float2(wl, wl), za[0]);
-      za[1] = fma_f32x2(make_float2(t0.z, t0.w), make_float2(wl, wl), za[1]);
-      zb[0] = fma_f32x2(make_float2(t1.x, t1.y), make_float2(wh, wh), zb[0]);
-      zb[1] = fma_f32x2(make_float2(t1.z, t1.w), make_float2(wh, wh), zb[1]);
-    }
+  for (int k = 0; k < KS; ++k) {
+    const uint32_t* ra = &tp[g][8 * (4 * k + q)];
+    const uint32_t* rb = &tp[g + 8][8 * (4 * k + q)];
+    const uint4 a4 = *reinterpret_cast<const uint4*>(ra);
+    const uint2 a2 = *reinterpret_cast<const uint2*>(ra + 4);
+    const uint4 b4 = upper ? *reinterpret_cast<const uint4*>(rb) : make_uint4(0u, 0u, 0u, 0u);
+    const uint2 b2 = upper ? *reinterpret_cast<const uint2*>(rb + 4) : make_uint2(0u, 0u);
+    const uint32_t hi[4] = {a4.x, b4.x, a4.y, b4.y};
+    const uint32_t mid[4] = {a4.z, b4.z, a4.w, b4.w};
+    const uint32_t lo[4] = {a2.x, b2.x, a2.y, b2.y};
+    mma_bf16_16x8x16(dl, lo, b[k][0], b[k][1]);
+    mma_bf16_16x8x16(dm, mid, b[k][0], b[k][1]);
+    mma_bf16_16x8x16(dh, hi, b[k][0], b[k][1]);
   }
-  const float z[4] = {za[0].x + zb[0].x, za[0].y + zb[0].y, za[1].x + zb[1].x,
-                      za[1].y + zb[1].y};
+  // z at rows g, g+8 and W_up rows n = 8 * warp + 2q, 2q+1: the same stream
+  // (n is even and cpb a multiple of 4), channels cc and cc + 1
+  const int n0 = 8 * warp + 2 * q, sn = n0 / cpb, cc = n0 % cpb;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int m = 4 * mg + i;
-    if (m < p.M) gs[m][s][c] = 1.f / (1.f + __expf(-z[i]));
+    const int m = g + 8 * (i >> 1);
+    if (m < p.M) gs[m][sn][cc + (i & 1)] = 1.f / (1.f + __expf(-((dl[i] + dm[i]) + dh[i])));
   }
   __syncthreads();
   if (!mixer) return;

@@ -21,7 +21,7 @@ constexpr int kHcCluster = 8;     // blocks per cluster of hc_down_kernel (colum
 constexpr int kHcMaxRows = 16;         // M <= 16 (decode-sized)
 constexpr int kHcMaxRank = 128;        // r <= 128
 constexpr int kHcMaxMixChannels = 32;  // channels per block of hc_gate_mix_kernel, at most
-constexpr int kHcMixThreads = 512;     // 4 streams x channels x row groups of 4, at most
+constexpr int kHcMixThreads = 512;     // a warp per 8 of the 4 x channels W_up rows, at most
 constexpr int kHcDownThreads = 1024;   // row groups x (one 16-byte vector per thread)
 constexpr int kHcMaxK = 16384;         // hc*C: K / 64 <= 256 vectors per block and row group
 

@@ -70,9 +70,9 @@ def test_workload_every_decode_m(fnb, M):
     st = check(wl, inp, got)
     # 16 clusters of 8 blocks (4 weight rows of W_down each; 160 threads per
     # row group of at most 4 rows, for M padded to 1, 2, 4, 8 or 16), then 128
-    # gate-and-mix blocks of 20 channels (4 streams x 20 x ceil(M/4) threads)
+    # gate-and-mix blocks of 20 channels (a warp per 8 of their 80 W_up rows)
     mm = next(b for b in (1, 2, 4, 8, 16) if b >= M)
-    assert list(launch) == [128, 160 * max(1, mm // 4), 128, 80 * ((M + 3) // 4)], launch
+    assert list(launch) == [128, 160 * max(1, mm // 4), 128, 320], launch
     assert st["bf16_equal_frac"] > 0.99, st
 
 
