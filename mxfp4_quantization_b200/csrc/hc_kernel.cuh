@@ -18,9 +18,10 @@
 //    every x row.  A thread owns one 16-byte vector of the piece for up to 4
 //    rows (more rows: more row groups of threads); the block reduces its
 //    threads' partial sums with a warp reduce-scatter and shared memory,
-//    every block stores its partials into rank 0's shared memory
-//    (distributed shared memory), and after one cluster barrier rank 0 sums
-//    them in rank order.  t (fp32 [M, r]) goes to the caller's workspace.
+//    the other blocks store their partials into rank 0's shared memory
+//    (distributed shared memory, st.async counted on rank 0's mbarrier) and
+//    exit, and rank 0, once they have landed, sums them in rank order.  t
+//    (fp32 [M, r]) goes to the caller's workspace.
 //  * hc_gate_mix_kernel: one block per cpb channels (no more blocks than
 //    SMs).  Before it waits for the first kernel every warp loads its W_up
 //    rows into tensor-core fragments and every thread its x values; once t
@@ -64,6 +65,40 @@ __device__ __forceinline__ void warp_reduce_scatter(float (&a)[V]) {
   }
 }
 
+// ---- the partial-sum handoff of hc_down_kernel ----------------------------------
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+// The shared::cluster address of the same variable in block `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+// One 4-byte store into another block's shared memory that counts its bytes
+// on that block's mbarrier (the transaction count) when it lands.
+__device__ __forceinline__ void st_async_b32(uint32_t raddr, float v, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+               :: "r"(raddr), "r"(__float_as_uint(v)), "r"(rbar) : "memory");
+}
+// Whether the mbarrier's phase 0 has completed (waits a hardware-chosen
+// while before answering no); acquire at cluster scope, so the stores that
+// completed the phase are visible after a yes.
+__device__ __forceinline__ bool mbar_phase0_done(uint32_t bar) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(done) : "r"(bar) : "memory");
+  return done != 0;
+}
+// Attempts of mbar_phase0_done before rank 0 of hc_down_kernel gives up (far
+// beyond any wait that can end: the other ranks' stores land within
+// microseconds of its own).
+constexpr int kHcHandoffTries = 1 << 20;
+
 // t[m, g*CW + j] = sum_k x[m, k] * w_down[g*CW + j, k] for m < M, j < CW.
 // Grid: (r / CW) clusters of kHcCluster blocks.  The rows are split over NG
 // row groups of threads, MR rows each (MM = NG * MR rows at most): thread
@@ -71,17 +106,34 @@ __device__ __forceinline__ void warp_reduce_scatter(float (&a)[V]) {
 // each thread holds MR * CW partial sums (16 at most) whatever M is, and a
 // block has NG times as many warps to cover its loads' latency.
 // blockDim.x = NG * nv, nv = round32(K / 64) threads per row group.
+// The handoff to rank 0 is one-way: the other ranks store their partials
+// into rank 0's shared memory with st.async, each store counting its bytes on
+// rank 0's mbarrier, and exit; only rank 0 waits, for the byte count of all
+// seven.  Rank 0 initialises the mbarrier and announces its byte count before
+// an early cluster arrive, which the others wait on (long since complete by
+// then) before their first store.  If the count never completes (a wait of
+// kHcHandoffTries attempts) rank 0 writes NaN into its columns of t, so the
+// call's outputs show the failure.
 template <int MR, int NG, int CW>
 __global__ void __launch_bounds__(kHcDownThreads) hc_down_kernel(const __grid_constant__ HCParams p) {
   namespace cg = cooperative_groups;
   constexpr int V = MR * CW;         // partial sums per thread
   constexpr int VB = NG * V;         // per block: every row times CW
   __shared__ float red[kHcDownThreads / 32][V];
-  __shared__ float slots[kHcCluster][VB];  // rank 0's: every block's partials
+  __shared__ float slots[kHcCluster][VB];  // rank 0's: the other blocks' partials (row 0 unused)
+  __shared__ __align__(8) uint64_t handoff;  // rank 0's: the others' partials landed
   pdl_enter();
 
   cg::cluster_group cl = cg::this_cluster();
   const int rank = (int)cl.block_rank();
+  const uint32_t bar = smem_addr(&handoff);
+  if (rank == 0 && threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(bar) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 :: "r"(bar), "r"((kHcCluster - 1) * VB * 4) : "memory");
+  }
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
   const int g = blockIdx.x / kHcCluster;
   const int kvec = p.K / 8, cvec = kvec / kHcCluster;
   const int nv = blockDim.x / NG;    // threads per row group (whole warps)
@@ -126,23 +178,26 @@ __global__ void __launch_bounds__(kHcDownThreads) hc_down_kernel(const __grid_co
   }
   __syncthreads();
   const int nwg = nv >> 5;  // warps per row group
-  if (tid < VB) {
-    const int grp = tid / V, idx = tid % V;
-    float s = red[grp * nwg][idx];
-    for (int w = 1; w < nwg; ++w) s += red[grp * nwg + w][idx];
-    *cl.map_shared_rank(&slots[rank][tid], 0) = s;
+  // rank 0's mbarrier is initialised (its early arrive is long past)
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+  if (tid >= VB) return;
+  const int grp = tid / V, idx = tid % V;
+  float s = red[grp * nwg][idx];
+  for (int w = 1; w < nwg; ++w) s += red[grp * nwg + w][idx];
+  if (rank != 0) {
+    st_async_b32(cluster_map(smem_addr(&slots[rank][tid]), 0), s, cluster_map(bar, 0));
+    return;
   }
-  // the stores into rank 0's shared memory are complete and visible to it
-  // after the barrier; only rank 0 reads them, so the others may leave
-  cl.sync();
-  if (rank == 0 && tid < VB) {
-    float s = slots[0][tid];
+  bool landed = false;
+  for (int i = 0; i < kHcHandoffTries && !landed; ++i) landed = mbar_phase0_done(bar);
+  if (landed) {
 #pragma unroll
     for (int c = 1; c < kHcCluster; ++c) s += slots[c][tid];
-    const int grp = tid / V, idx = tid % V;
-    const int m = grp * MR + idx / CW, j = idx % CW;
-    if (m < p.M) p.t[(int64_t)m * p.r + g * CW + j] = s;
+  } else {
+    s = __int_as_float(0x7fc00000);
   }
+  const int m = grp * MR + idx / CW, j = idx % CW;
+  if (m < p.M) p.t[(int64_t)m * p.r + g * CW + j] = s;
 }
 
 // D += A B for one m16n8k16 tile: A bf16 16 x 16 (row-major fragment a0..a3),
