@@ -13,6 +13,12 @@ Criteria (the tolerances of the fused path):
                  of positions; a group whose scale differs must have a 1-ulp
                  difference of its amax element, and the count is reported
                  separately.
+  hc_mix         against the oracle's float64 u, per element: the page's
+                 |gpu - u| <= 4e-3 + 1e-2 |u| (sglang PR #41880, "Accuracy
+                 Tests") and the derived |gpu - u| <= 2^-8 |u| + 2e-5 * scale
+                 (one bf16 rounding, at most half an ulp of 8 significant
+                 bits, plus the fp32 path; `scale` grows the fp32 term with
+                 the size of the logits).
 """
 import numpy as np
 
@@ -161,3 +167,23 @@ def check_rmsnorm_all_rows(mode, eps, parts_bits, res_bits, w_bits, gpu, io=orac
         for k, v in r.items():
             out[k] = max(out.get(k, 0), v) if k == "max_step" else out.get(k, 0) + v
     return out
+
+
+HC_ATOL, HC_RTOL = 4e-3, 1e-2
+
+
+def bf16_bits_to_f64(bits):
+    return (np.asarray(bits, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def check_hc_mix(u, ub, got_bits, logit_scale=1.0):
+    """hc_mix output bits (bf16 [M, C]) against the oracle's float64 u and its
+    bf16 rounding ub; raises AssertionError on a failed criterion, returns
+    the statistics."""
+    g = bf16_bits_to_f64(got_bits)
+    err = np.abs(g - u)
+    assert np.all(err <= HC_ATOL + HC_RTOL * np.abs(u)), f"page tolerance: max err {err.max()}"
+    bad = err > 2.0 ** -8 * np.abs(u) + 2e-5 * logit_scale
+    assert not bad.any(), f"derived bound at {np.argwhere(bad)[:5].tolist()}, err {err[bad][:5]}"
+    return {"max_abs_err": float(err.max()),
+            "bf16_equal_frac": float(np.mean(np.asarray(got_bits) == np.asarray(ub)))}

@@ -114,3 +114,61 @@ def test_all_rows_runner_passes_exact_and_catches_a_fault_in_a_late_chunk():
     gpu["q"][69, 5] ^= 0x01
     with pytest.raises(AssertionError):
         parity.check_rmsnorm_all_rows(wl.mode, wl.eps, parts, res, w, gpu, chunk=16, procs=3)
+
+
+# ---- hc_mix ------------------------------------------------------------------------
+#
+# The criterion of the hc_mix GPU tests (parity.check_hc_mix) must pass the
+# oracle's own bf16 result and fail a kernel that made any of the plausible
+# mistakes below.  A mistaken kernel is stood in for by a copy of the oracle
+# with the mistake planted (built on the CPU, as the oracle's own negative
+# controls do), run on the same inputs at the workload's shape.
+
+HC_FAULTS = [
+    ("gate_sign", "g[e] = 1.0 / (1.0 + exp(-z));", "g[e] = 1.0 / (1.0 + exp(z));"),
+    ("last_stream_dropped", "for (int s = 0; s < hc; ++s)", "for (int s = 0; s < hc - 1; ++s)"),
+    ("w_up_transposed", "z += t[j] * orc_bf16_to_double(w_up[e * r + j]);",
+     "z += t[j] * orc_bf16_to_double(w_up[(int64_t)j * K + e]);"),
+    # the rounding that the gate kernel's three-part split of t avoids
+    ("t_rounded_to_bf16", "t[j] = acc;", "t[j] = orc_bf16_to_double(orc_bf16_from_double(acc));"),
+]
+
+
+def _hc_case(M=4, C=512, r=64, seed=21):
+    wl = synth.HCWorkload("ctl", M=M, C=C, r=r, seed=seed)
+    inp = wl.inputs(device="cpu")
+    bits = {k: synth.to_bits(inp[k]) for k in ("x", "w_down", "w_up")}
+    u, ub = oracle.hc_mix(bits["x"], bits["w_down"], bits["w_up"], wl.hc, wl.C, wl.r)
+    return wl, bits, u, ub
+
+
+def test_hc_exact_outputs_pass():
+    _, _, u, ub = _hc_case()
+    st = parity.check_hc_mix(u, ub, ub)
+    assert st["bf16_equal_frac"] == 1.0
+
+
+def test_hc_two_ulps_off_fails():
+    _, _, u, ub = _hc_case()
+    bad = ub.copy()
+    i = np.unravel_index(np.argmax(np.abs(u)), u.shape)
+    bad[i] = np.uint16(int(bad[i]) + 2)
+    with pytest.raises(AssertionError):
+        parity.check_hc_mix(u, ub, bad)
+
+
+@pytest.mark.parametrize("name,old,new", HC_FAULTS, ids=[f[0] for f in HC_FAULTS])
+def test_hc_planted_mistake_fails(tmp_path, name, old, new):
+    import os
+    from oracle.build import SRC, build_oracle
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation site for {name} missing"
+    mut = os.path.join(tmp_path, "orc_fault.c")
+    with open(mut, "w") as fh:
+        fh.write(src.replace(old, new))
+    lib = oracle.load(build_oracle(src=mut, out=os.path.join(tmp_path, "liborc_fault.so"),
+                                   extra_flags=("-Wno-error",), force=True))
+    wl, bits, u, ub = _hc_case()
+    _, wrong = oracle.hc_mix(bits["x"], bits["w_down"], bits["w_up"], wl.hc, wl.C, wl.r, lib=lib)
+    with pytest.raises(AssertionError):
+        parity.check_hc_mix(u, ub, wrong)
