@@ -275,6 +275,10 @@ FN_API int fn_qk_norm_gate_fp8(const void* qkv, int64_t M, int64_t row_stride, i
  *            and may be reused as soon as the call's work on `stream` is done.
  * Overlap    out and workspace must not overlap each other or any input
  *            (FN_ERR_INVALID).
+ * Device     the first kernel's blocks hand their partial sums to one block
+ *            of their cluster, which waits for them with a bounded wait; if
+ *            that wait ever ran out (not seen on working hardware) the
+ *            affected entries of t, and so the outputs, are NaN.
  * fn_last_launch: out[0] blocks (clusters of 8) and out[1] threads of the
  * first kernel, out[2] blocks and out[3] threads of the second.
  */
