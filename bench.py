@@ -786,6 +786,68 @@ def oracle_rows_per_s(rows: int, min_seconds: float, max_seconds: float, workloa
     return done / el, done, el
 
 
+def _time_calls(fn, min_seconds: float, max_calls: int):
+    """Calls of `fn` until `min_seconds` have passed (at least one, at most
+    max_calls); returns (seconds per call, calls)."""
+    done, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or done >= max_calls:
+            return el / done, done
+
+
+def oracle_per_config(seconds: float = 1.0):
+    """The oracle, as it stands, single-threaded, on every other configuration
+    of the run: each call of a decode-sized configuration whole (µs per call,
+    the GPU figures' unit), the MXFP4 prefill on a 64-row sample (rows/s);
+    about `seconds` of repeated calls each."""
+    import oracle
+    from mxfp4_quantization_b200 import synth
+    out = {}
+
+    def rows_cfg(wl, M=None):
+        inp = wl.inputs(device="cpu", M=M)
+        parts = [synth.to_bits(p) for p in inp["parts"]]
+        res = synth.to_bits(inp["residual"]) if inp.get("residual") is not None else None
+        w = synth.to_bits(inp["weight"])
+        return lambda: oracle.rmsnorm_quant(parts, res, w, wl.eps, wl.mode)
+
+    wl = synth.PREFILL_MXFP4
+    sec, n = _time_calls(rows_cfg(wl, 64), seconds, 1000)
+    out["prefill_mxfp4"] = {"value": 64 / sec, "unit": "rows/s", "cores": 1,
+                            "sample": f"64 rows of the recipe (H={wl.H}, P={wl.P}), {n} calls"}
+    wl = synth.PER_TOKEN_SMALL
+    sec, n = _time_calls(rows_cfg(wl), seconds, 10000)
+    out["per_token_small"] = {"value": sec * 1e6, "unit": "us/call", "cores": 1,
+                              "sample": f"whole call (M={wl.M}, H={wl.H}), {n} calls"}
+    for mode, mname in ((synth.FP8_PER_TOKEN, "fp8_per_token"),
+                        (synth.FP8_PER_GROUP128, "fp8_per_group128"), (synth.MXFP4, "mxfp4")):
+        wl = synth.decode(16, mode)
+        sec, n = _time_calls(rows_cfg(wl), seconds / 3, 10000)
+        out[f"decode_{mname}_m16"] = {"value": sec * 1e6, "unit": "us/call", "cores": 1,
+                                      "sample": f"whole call (M=16, H={wl.H}), {n} calls"}
+    for M in synth.QK_M:
+        wl = synth.qk_prologue(M)
+        inp = wl.inputs(device="cpu")
+        qkv, qw, kw = (synth.to_bits(inp[k]) for k in ("qkv", "q_weight", "k_weight"))
+        sec, n = _time_calls(lambda: oracle.qk_norm_gate(qkv, wl.row_stride, wl.Hq, wl.Hk, wl.D,
+                                                         qw, kw, wl.eps),
+                             seconds / 2, 10000)
+        out[f"qk_prologue_m{M}"] = {"value": sec * 1e6, "unit": "us/call", "cores": 1,
+                                    "sample": f"whole call (M={M}), {n} calls"}
+    for M in (1, 16):
+        wl = synth.hc_mix(M)
+        inp = wl.inputs(device="cpu")
+        x, wd, wu = (synth.to_bits(inp[k]) for k in ("x", "w_down", "w_up"))
+        sec, n = _time_calls(lambda: oracle.hc_mix(x, wd, wu, wl.hc, wl.C, wl.r), seconds / 2,
+                             10000)
+        out[f"hc_mix_m{M}"] = {"value": sec * 1e6, "unit": "us/call", "cores": 1,
+                               "sample": f"whole call (M={M}, C={wl.C}, r={wl.r}), {n} calls"}
+    return out
+
+
 def _oracle_worker(job):
     rows, seconds, workload = job
     rate, done, el = oracle_rows_per_s(rows, seconds, 3 * seconds, workload)
@@ -895,7 +957,7 @@ def main_arm(args):
         tp_record = tp_leg(fn, device, rank, world)
 
     extra = None
-    cpu = cpu_all = None
+    cpu = cpu_all = cpu_configs = None
     if world == 1 and not args.no_extras and args.workload == "prefill_group128":
         extra = secondary_workloads(fn, device, peak)
     if world == 1 and not args.no_cpu_baseline:
@@ -911,6 +973,8 @@ def main_arm(args):
                    "kind": "oracle, row-parallel processes (context beside cpu_baseline)",
                    "sample": f"64 rows of the {wl.name} recipe per process, repeated for "
                              f"about {max(1.0, args.cpu_seconds / 2):.0f} s, {procs} processes"}
+        if extra is not None:
+            cpu_configs = oracle_per_config()
 
     if rank == 0:
         line = {
@@ -944,6 +1008,7 @@ def main_arm(args):
             "clocks": clk,
             "cpu_baseline": cpu,
             "cpu_baseline_all_cores": cpu_all,
+            "cpu_baseline_per_config": cpu_configs,
             "workloads": extra,
             "tensor_parallel": tp_record,
         }
