@@ -489,14 +489,15 @@ int hc_mix_channels(int64_t C, int sms) {
 }
 
 // Shared memory a launch of the gate-and-mix kernel `k` asks for so that no SM
-// holds two of its blocks (more than half of an SM's shared memory), with the
-// shared-memory carveout of both hc_mix kernels at its maximum so that a gate
-// block still fits beside a block of the first kernel; cached per kernel, -1
-// if the runtime refuses.  Launched early as a programmatic dependent, the
-// small gate blocks were otherwise packed up to five to an SM onto the SMs the
-// first kernel left free (measured on B200 with per-block SM ids: 128 blocks
-// on 28 SMs at M = 4 and 8), multiplying their logit time.
-int hc_spread_blocks(fn::HCKernel k, fn::HCKernel first) {
+// holds two of its blocks (more than half of an SM's shared memory, with the
+// kernel's shared-memory carveout at its maximum); cached per kernel, -1 if
+// the runtime refuses.  Launched early as a programmatic dependent, the small
+// gate blocks were otherwise packed up to five to an SM onto the SMs the first
+// kernel left free (measured on B200 with per-block SM ids: 128 blocks on 28
+// SMs at M = 4 and 8), multiplying their logit time.  The first kernel keeps
+// the default carveout: setting it to the maximum there too was measured
+// slightly slower at M >= 4 (5.07 -> 5.15 us at M = 4, 6.09 -> 6.16 at 16).
+int hc_spread_blocks(fn::HCKernel k) {
   static std::mutex mu;
   static std::map<const void*, int> cache;
   const void* key = reinterpret_cast<const void*>(k);
@@ -510,9 +511,7 @@ int hc_spread_blocks(fn::HCKernel k, fn::HCKernel first) {
           cudaSuccess &&
       cudaFuncGetAttributes(&fa, k) == cudaSuccess) {
     const int want = per_sm / 2 + 1 - (int)fa.sharedSizeBytes;
-    if (cudaFuncSetAttribute(first, cudaFuncAttributePreferredSharedMemoryCarveout, 100) ==
-            cudaSuccess &&
-        cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100) ==
+    if (cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100) ==
             cudaSuccess &&
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, want) == cudaSuccess)
       bytes = want;
@@ -555,7 +554,7 @@ int hc_launch(const void* x, const void* w_down, const void* w_up, int64_t M, in
   fn::HCKernel k2 = fn::hc_gate_mix_pick(r / 8);
   if (!k2) return FN_ERR_UNSUPPORTED;
   // one gate block per SM while the blocks fit the GPU at once
-  const int smem2 = (int)g2 <= sms ? hc_spread_blocks(k2, k1) : 0;
+  const int smem2 = (int)g2 <= sms ? hc_spread_blocks(k2) : 0;
   if (smem2 < 0) return FN_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (launch_kernel(k1, g1, (unsigned)t1, 0, st, fn::kHcCluster, p) != FN_OK) return FN_ERR_CUDA;
