@@ -490,8 +490,9 @@ int hc_mix_channels(int64_t C, int sms) {
 
 // Shared memory a launch of the gate-and-mix kernel `k` asks for so that no SM
 // holds two of its blocks (more than half of an SM's shared memory, with the
-// kernel's shared-memory carveout at its maximum); cached per kernel, -1 if
-// the runtime refuses.  Launched early as a programmatic dependent, the small
+// kernel's shared-memory carveout at its maximum); the attributes are set
+// once per kernel and device (function attributes belong to a device's
+// context) and cached, -1 if the runtime refuses.  Launched early as a programmatic dependent, the small
 // gate blocks were otherwise packed up to five to an SM onto the SMs the first
 // kernel left free (measured on B200 with per-block SM ids: 128 blocks on 28
 // SMs at M = 4 and 8), multiplying their logit time.  The first kernel keeps
@@ -499,15 +500,19 @@ int hc_mix_channels(int64_t C, int sms) {
 // slightly slower at M >= 4 (5.07 -> 5.15 us at M = 4, 6.09 -> 6.16 at 16).
 int hc_spread_blocks(fn::HCKernel k) {
   static std::mutex mu;
-  static std::map<const void*, int> cache;
-  const void* key = reinterpret_cast<const void*>(k);
+  static std::map<std::pair<const void*, int>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return -1;
+  }
+  const auto key = std::make_pair(reinterpret_cast<const void*>(k), dev);
   std::lock_guard<std::mutex> lock(mu);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
-  int dev = 0, per_sm = 0, bytes = -1;
+  int per_sm = 0, bytes = -1;
   cudaFuncAttributes fa;
-  if (cudaGetDevice(&dev) == cudaSuccess &&
-      cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) ==
+  if (cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) ==
           cudaSuccess &&
       cudaFuncGetAttributes(&fa, k) == cudaSuccess) {
     const int want = per_sm / 2 + 1 - (int)fa.sharedSizeBytes;
