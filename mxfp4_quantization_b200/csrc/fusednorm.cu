@@ -542,6 +542,13 @@ int hc_launch(const void* x, const void* w_down, const void* w_up, int64_t M, in
   p.C = (int)C;
   p.K = (int)(fn::kHcStreams * C);
   p.r = r;
+  // the first kernel's prologue prefetch (only as a programmatic dependent,
+  // and never from another device's memory)
+  if (tl_pdl) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FN_ERR_CUDA;
+    p.prefetch = on_device(x, dev) && on_device(w_down, dev) ? 1 : 0;
+  }
   const int cw = hc_rows_per_cluster(r);
   fn::HCKernel k1 = fn::hc_down_pick(hc_rows_bound(M), cw);
   if (!k1) return FN_ERR_UNSUPPORTED;

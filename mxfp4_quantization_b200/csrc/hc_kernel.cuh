@@ -122,6 +122,19 @@ __global__ void __launch_bounds__(kHcDownThreads) hc_down_kernel(const __grid_co
   __shared__ float red[kHcDownThreads / 32][V];
   __shared__ float slots[kHcCluster][VB];  // rank 0's: the other blocks' partials (row 0 unused)
   __shared__ __align__(8) uint64_t handoff;  // rank 0's: the others' partials landed
+  if (p.prefetch) {
+    // Launched as a programmatic dependent, the block may start while the
+    // previous kernel still runs: start its pieces of W_down and x towards
+    // L2 before the wait (a hint with no result: data that the previous
+    // kernel writes meanwhile lands in L2 over the prefetched lines, so the
+    // loads after the wait see it).
+    const int gq = blockIdx.x / kHcCluster, rq = blockIdx.x % kHcCluster;
+    const int kv = p.K / 8, cv = kv / kHcCluster, i = threadIdx.x;
+    if (i < CW)
+      bulk_prefetch_l2(p.w_down + (int64_t)(gq * CW + i) * kv + rq * cv, (uint32_t)cv * 16u);
+    else if (i < CW + p.M)
+      bulk_prefetch_l2(p.x + (int64_t)(i - CW) * kv + rq * cv, (uint32_t)cv * 16u);
+  }
   pdl_enter();
 
   cg::cluster_group cl = cg::this_cluster();

@@ -14,6 +14,7 @@ struct HCParams {
   uint16_t* out;        // bf16 [M, C]
   int M, C, K, r;       // K = hc * C
   int cpb;              // channels per block of hc_gate_mix_kernel
+  int prefetch;         // hc_down_kernel: L2-prefetch its pieces before its wait
 };
 
 constexpr int kHcStreams = 4;     // hc: the streams of the hyper-state
