@@ -328,6 +328,15 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, bo
       if (cudaGetDevice(&dev) != cudaSuccess) return FN_ERR_CUDA;
       if (!rows_on_device(p, dev)) p.prefetch_rows = 0;
     }
+    // as a programmatic dependent, each block prefetches its own row before
+    // its wait (never from another device's memory)
+    p.prefetch_self = 0;
+    if (tl_pdl && p.prefetch_rows == 0) {
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess) return FN_ERR_CUDA;
+      p.prefetch_self =
+          rows_on_device(p, dev) && (!norm || on_device(p.weight, dev)) ? 1 : 0;
+    }
     int threads = wide_k ? wide_T : round32((nvec + V - 1) / V);
     RQKernel k = wide_k;
     if (!k && threads * V == nvec) k = pick_exact_kernel(mode, P, threads, V, f16, norm);

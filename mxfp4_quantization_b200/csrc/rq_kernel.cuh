@@ -357,6 +357,23 @@ __global__ void __launch_bounds__((CL || TB > 256) ? 512 : 256)
   static_assert(TB == 0 || !CL, "exact-cover instances are one block per row");
   __shared__ float2 red[32];
   __shared__ float2 cl_slot;
+  if (!CL && prm.prefetch_self) {
+    // Launched as a programmatic dependent, the block may start while the
+    // previous kernel still runs: start this row's inputs towards L2 before
+    // the wait (a hint with no result: data that the previous kernel writes
+    // meanwhile, an in-place residual included, lands in L2 over the
+    // prefetched lines, so the loads after the wait see it).
+    const int nv = TB ? TB * V : prm.nvec;
+    const int64_t rv = (int64_t)blockIdx.x * nv;
+    const uint32_t bytes = (uint32_t)nv * 16u;
+    const int i = threadIdx.x;
+    if (i < prm.P)
+      bulk_prefetch_l2(prm.parts[i] + rv, bytes);
+    else if (i == prm.P && NORM && prm.residual != nullptr)
+      bulk_prefetch_l2(prm.residual + rv, bytes);
+    else if (i == prm.P + 1 && NORM)
+      bulk_prefetch_l2(prm.weight, bytes);
+  }
   pdl_enter();
 
   const int T = TB ? TB : (int)blockDim.x, t = threadIdx.x, lane = t & 31;

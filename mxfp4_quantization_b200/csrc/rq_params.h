@@ -26,6 +26,8 @@ struct RQParams {
   float inv_h;             // 1 / H (fp32), for the mean of squares
   int prefetch_rows;       // L2 prefetch distance in rows of this block (0: none); a
                            // positive distance also marks a large-M launch (row_reduce)
+  int prefetch_self;       // one block per row: L2-prefetch the block's own row inputs
+                           // before the programmatic-launch wait
   int scale_layout;        // SCALE_*
   int64_t scale_ld;        // swizzled: column tiles per row tile; MN-major: row stride
 };
