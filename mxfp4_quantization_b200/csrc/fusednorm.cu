@@ -449,6 +449,16 @@ int qk_impl(const void* qkv, int64_t M, int64_t row_stride, int Hq, int Hk, int 
   p.out_qs = static_cast<float*>(out_qs);
   p.out_k8 = static_cast<uint8_t*>(out_k8);
   p.out_ks = static_cast<float*>(out_ks);
+  // as a programmatic dependent, each warp prefetches its head before its
+  // wait (never from another device's memory)
+  if (tl_pdl) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FN_ERR_CUDA;
+    p.prefetch_self = on_device(qkv, dev) && (!q_weight || on_device(q_weight, dev)) &&
+                              (!k_weight || on_device(k_weight, dev))
+                          ? 1
+                          : 0;
+  }
   const int64_t items = M * (Hq + Hk);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int rc;

@@ -29,6 +29,7 @@ struct QKParams {
   float* out_qs;
   uint8_t* out_k8;  // E4M3 codes [M, Hk, D] and fp32 scales [M, Hk]
   float* out_ks;
+  int prefetch_self;  // L2-prefetch each warp's head before the programmatic-launch wait
 };
 
 // FP8: also quantize each normed q and k head to E4M3 with one fp32 scale per
@@ -36,10 +37,27 @@ struct QKParams {
 // applied to each head vector, for an FP8 attention consumer.
 template <int VPL, bool FP8>
 __global__ void __launch_bounds__(256) qk_kernel(const __grid_constant__ QKParams p) {
-  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int heads = p.Hq + p.Hk;
+  if (p.prefetch_self) {
+    // Launched as a programmatic dependent, the block may start while the
+    // previous kernel still runs: start this warp's head (q with its gate, or
+    // k) and the norm weights towards L2 before the wait (a hint with no
+    // result: data written meanwhile lands in L2 over the prefetched lines).
+    if (lane == 0 && item < p.M * heads) {
+      const int64_t m = item / heads;
+      const int j = (int)(item - m * heads);
+      const uint4* row = p.qkv + m * p.row_vec;
+      if (j < p.Hq)
+        bulk_prefetch_l2(row + (int64_t)(2 * j) * p.dv, (uint32_t)p.dv * 32u);
+      else
+        bulk_prefetch_l2(row + (int64_t)(2 * p.Hq + (j - p.Hq)) * p.dv, (uint32_t)p.dv * 16u);
+    }
+    if (threadIdx.x == 1 && p.qw != nullptr) bulk_prefetch_l2(p.qw, (uint32_t)p.dv * 16u);
+    if (threadIdx.x == 2 && p.kw != nullptr) bulk_prefetch_l2(p.kw, (uint32_t)p.dv * 16u);
+  }
+  pdl_enter();
   if (item >= p.M * heads) return;  // warp-uniform
   const int64_t m = item / heads;
   const int j = (int)(item - m * heads);
