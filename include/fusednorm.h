@@ -337,11 +337,13 @@ FN_API int fn_last_variant(void);
 /* Launch shape of the calling thread's last launch: out[0] grid blocks,
  * out[1] threads per block, out[2] blocks per cluster for
  * FN_VARIANT_ROW_CLUSTER, or, for one block per row (FN_VARIANT_ROW_CTA,
- * FN_VARIANT_QUANT_ONLY), the L2 prefetch distance in rows (0: no prefetch;
- * large-M launches start the rows about one wave ahead towards L2, and only
- * when every partial and the residual is device memory of the current
- * device: memory of another GPU or of the host is read with plain loads
- * alone), out[3] 16-byte vectors per thread per tensor. */
+ * FN_VARIANT_QUANT_ONLY), the L2 prefetch: the distance in rows (large-M
+ * launches start the rows about one wave ahead towards L2), -1 (launched as
+ * programmatic dependents, every block starts its own row towards L2 before
+ * it waits for the previous kernel) or 0 (none); either prefetch is taken
+ * only when every row input (and, for -1, the weight) is device memory of
+ * the current device: memory of another GPU or of the host is read with
+ * plain loads alone.  out[3] 16-byte vectors per thread per tensor. */
 FN_API void fn_last_launch(int32_t out[4]);
 
 /* Thread-local kernel preference for fn_rmsnorm_quant: FN_VARIANT_NONE (the

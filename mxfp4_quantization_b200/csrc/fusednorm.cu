@@ -360,7 +360,7 @@ int launch_rq(const fn::RQParams& prm, int mode, int P, int64_t M, bool norm, bo
     tl_variant = norm ? variant_if_norm : FN_VARIANT_QUANT_ONLY;
     tl_launch[0] = (int32_t)M;
     tl_launch[1] = threads;
-    tl_launch[2] = p.prefetch_rows;
+    tl_launch[2] = p.prefetch_self ? -1 : p.prefetch_rows;
     tl_launch[3] = V;
   }
   return FN_OK;

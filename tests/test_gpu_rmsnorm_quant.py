@@ -439,6 +439,48 @@ def test_random_shapes(fnb, i, mode, M, H, P, has_res, fp16, variant):
     check(wl, inp, gpu)
 
 
+@pytest.mark.parametrize("host_tensor", [None, "parts", "residual", "weight"])
+def test_own_row_prefetch_only_as_programmatic_dependent_on_this_devices_memory(fnb,
+                                                                               host_tensor):
+    """Launched as programmatic dependents, decode-sized blocks start their own
+    row towards L2 before they wait (launch record -1): only when every row
+    input and the weight are device memory of the current device (host rows
+    here stand in for any memory that is not), and never without programmatic
+    launch.  The results stay those of the oracle either way."""
+    wl = synth.decode(16, MX)
+    inp = wl.inputs(device="cpu")
+    M = wl.M
+    q, s = fnb.alloc_outputs(MX, M, wl.H, "cuda")
+    r_out = torch.empty((M, wl.H), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((M, wl.H), dtype=torch.bfloat16, device="cuda")
+    dev = {"parts": [p.cuda() for p in inp["parts"]], "residual": inp["residual"].cuda(),
+           "weight": inp["weight"].cuda()}
+    use = dict(dev)
+    if host_tensor == "parts":
+        use["parts"] = [p.pin_memory() for p in inp["parts"]]
+    elif host_tensor is not None:
+        use[host_tensor] = inp[host_tensor].pin_memory()
+
+    def call(pdl):
+        with fnb.programmatic_launch(pdl):
+            st = fnb.fn_rmsnorm_quant([p.data_ptr() for p in use["parts"]], len(use["parts"]),
+                                      use["residual"].data_ptr(), use["weight"].data_ptr(),
+                                      wl.eps, MX, M, wl.H, q.data_ptr(), s.data_ptr(),
+                                      r_out.data_ptr(), y.data_ptr(),
+                                      torch.cuda.current_stream().cuda_stream)
+            assert st == fnb.FN_OK, fnb.fn_status_string(st)
+            launch = fnb.fn_last_launch()
+        torch.cuda.synchronize()
+        return launch
+
+    assert call(False)[2] == 0
+    launch = call(True)
+    assert launch[2] == (-1 if host_tensor is None else 0), launch
+    gpu = {"q": gpu_util.u8(q), "scale": gpu_util.scale_np(s, MX),
+           "residual_out": gpu_util.bits(r_out), "y": gpu_util.bits(y)}
+    check(wl, inp, gpu)
+
+
 @pytest.mark.parametrize("host_tensor", ["parts", "residual"])
 def test_l2_prefetch_only_on_this_devices_memory(fnb, host_tensor):
     """The large-M launch starts rows towards L2 with a bulk prefetch only when
