@@ -945,6 +945,12 @@ def main_arm(args):
     us_call = ms * 1e3 / calls  # every launch of the step is the same kernel
     achieved = bytes_call / (us_call * 1e-6) / 1e9
     traffic = measured_traffic(wl.name, launch)
+    # the same step with every call a programmatic dependent of the one before
+    # (reported beside the line's value, which keeps plain launches)
+    with fn.programmatic_launch(True):
+        step()
+        ms_pdl = time_steps(step, max(3, min(args.steps, 5)), 0, device, stream)
+    us_call_pdl = dist_max(ms_pdl, device) * 1e3 / calls
     del keep
     torch.cuda.empty_cache()
 
@@ -984,6 +990,7 @@ def main_arm(args):
             "dtype": "f32", "data": "synthetic",
             "config": workload_config(wl, world, calls),
             "us_per_call": us_call,
+            "us_per_call_programmatic": us_call_pdl,
             "hbm_GB_s": achieved, "frac_of_peak": achieved / peak,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
