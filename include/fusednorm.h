@@ -326,9 +326,13 @@ FN_API const char* fn_status_string(int status);
  * and later), so its blocks may be scheduled while the previous kernel
  * drains; every kernel of this library first waits, on the device, until the
  * grids it depends on have completed and their writes are visible, so results
- * are those of ordinary stream order.  Works inside CUDA graph capture.
- * Default 0.  Returns the previous setting.  (A launch-latency measure for
- * decode-sized calls; the pages describe no counterpart.) */
+ * are those of ordinary stream order.  Before that wait, decode-sized row
+ * calls, the QK prologue and hc_mix's first kernel start their inputs
+ * towards L2 (cp.async.bulk.prefetch.L2: a hint with no result, and only
+ * for the current device's memory), so their loads after the wait find L2.
+ * Works inside CUDA graph capture.  Default 0.  Returns the previous
+ * setting.  (A launch-latency measure for decode-sized calls; the pages
+ * describe no counterpart.) */
 FN_API int fn_programmatic_launch(int on);
 
 /* fn_variant of the calling thread's last call (FN_VARIANT_NONE after an error). */
