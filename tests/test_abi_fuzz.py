@@ -1,4 +1,5 @@
-"""Property test of fn_rmsnorm_quant's argument checks (no GPU).
+"""Property tests of the argument checks of fn_rmsnorm_quant, fn_hc_mix and
+fn_hc_mix_noalloc (no GPU).
 
 Random calls over fake, far-apart device addresses, with sizes, modes, flags,
 alignments and overlaps drawn to hit every rule of include/fusednorm.h.  The
@@ -149,5 +150,96 @@ def test_status_follows_the_documented_rules(fnb, a):
                                a["M"], a["H"], ptr["out_q"], ptr["out_scale"], ptr["out_residual"],
                                ptr["out_y"], None)
     want = expected(fnb, a)
+    assert got in want, (got, want, a)
+    assert fnb.fn_last_variant() == fnb.FN_VARIANT_NONE
+
+
+# ---- fn_hc_mix and fn_hc_mix_noalloc -------------------------------------------------
+
+
+def expected_hc(fnb, a, noalloc=False):
+    """The statuses include/fusednorm.h allows for hc_mix call `a`
+    ({FN_ERR_CUDA} when no rule is broken: the call reaches the launch)."""
+    E, A, U, OK = fnb.FN_ERR_INVALID, fnb.FN_ERR_ALIGN, fnb.FN_ERR_UNSUPPORTED, fnb.FN_OK
+    M, hc, C, r = a["M"], a["hc"], a["C"], a["r"]
+    if M < 0 or hc < 1 or C <= 0 or r <= 0:
+        return {E}
+    if hc != 4 or M > 16 or C % 16 or hc * C > 16384 or r % 8 or r > 128:
+        return {U}
+    if M == 0:
+        return {OK}
+    ptr = a["ptr"]
+    names = ("x", "w_down", "w_up", "out") + (() if noalloc else ("workspace",))
+    bad = set()
+    for k in names:
+        if ptr[k] is None:
+            bad.add(E)
+        elif ptr[k] % 16:
+            bad.add(A)
+    if bad:
+        return bad
+    if noalloc and M * r > 16 * 128:
+        return {U}
+    K = hc * C
+    ins = [(ptr["x"], M * K * 2), (ptr["w_down"], r * K * 2), (ptr["w_up"], K * r * 2)]
+    outs = [(ptr["out"], M * C * 2)] + ([] if noalloc else [(ptr["workspace"], M * r * 4)])
+    hit = lambda a0, n0, a1, n1: a0 < a1 + n1 and a1 < a0 + n0  # noqa: E731
+    for i, (p, n) in enumerate(outs):
+        for p2, n2 in outs[i + 1:]:
+            if hit(p, n, p2, n2):
+                bad.add(E)
+        for p2, n2 in ins:
+            if hit(p, n, p2, n2):
+                bad.add(E)
+    return bad or {fnb.FN_ERR_CUDA}
+
+
+@st.composite
+def hc_calls(draw):
+    rare = lambda: draw(st.integers(0, 9)) == 0  # noqa: E731
+    M = draw(st.sampled_from([-1, 0, 17, 40])) if rare() else draw(st.sampled_from([1, 3, 8, 16]))
+    hc = draw(st.sampled_from([0, 2, 8])) if rare() else 4
+    C = draw(st.sampled_from([0, 24, 4112, 8192])) if rare() else \
+        draw(st.sampled_from([16, 512, 2560, 4096]))
+    r = draw(st.sampled_from([0, 12, 136])) if rare() else draw(st.sampled_from([8, 64, 128]))
+    slot = iter(range(1, 16))
+
+    def addr():
+        if draw(st.integers(0, 39)) == 0:
+            return None
+        base = next(slot) * SPACE
+        if draw(st.integers(0, 14)) == 0:
+            return base + draw(st.sampled_from([4, 8, 2]))
+        return base + draw(st.sampled_from([0, 16, 256]))
+
+    ptr = {k: addr() for k in ("x", "w_down", "w_up", "out", "workspace")}
+    kind = draw(st.integers(0, 5))
+    if kind == 1 and ptr["x"] is not None:
+        ptr[draw(st.sampled_from(["out", "workspace"]))] = ptr["x"] + 64
+    elif kind == 2 and ptr["out"] is not None:
+        ptr["workspace"] = ptr["out"] + 32
+    elif kind == 3 and ptr["w_up"] is not None:
+        ptr["out"] = ptr["w_up"] + 16
+    return {"M": M, "hc": hc, "C": C, "r": r, "ptr": ptr}
+
+
+@settings(max_examples=400, deadline=None, suppress_health_check=list(HealthCheck))
+@given(a=hc_calls())
+def test_hc_mix_status_follows_the_documented_rules(fnb, a):
+    p = a["ptr"]
+    got = fnb.fn_hc_mix(p["x"], p["w_down"], p["w_up"], a["M"], a["hc"], a["C"], a["r"], p["out"],
+                        p["workspace"], None)
+    want = expected_hc(fnb, a)
+    assert got in want, (got, want, a)
+    assert fnb.fn_last_variant() == fnb.FN_VARIANT_NONE
+
+
+@settings(max_examples=300, deadline=None, suppress_health_check=list(HealthCheck))
+@given(a=hc_calls())
+def test_hc_mix_noalloc_status_follows_the_documented_rules(fnb, a):
+    p = a["ptr"]
+    got = fnb.fn_hc_mix_noalloc(p["x"], p["w_down"], p["w_up"], a["M"], a["hc"], a["C"], a["r"],
+                                p["out"], None)
+    want = expected_hc(fnb, a, noalloc=True)
     assert got in want, (got, want, a)
     assert fnb.fn_last_variant() == fnb.FN_VARIANT_NONE
