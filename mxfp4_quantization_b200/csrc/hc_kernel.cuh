@@ -21,7 +21,9 @@
 //    the other blocks store their partials into rank 0's shared memory
 //    (distributed shared memory, st.async counted on rank 0's mbarrier) and
 //    exit, and rank 0, once they have landed, sums them in rank order.  t
-//    (fp32 [M, r]) goes to the caller's workspace.
+//    (fp32 [M, r]) goes to the caller's workspace.  Launched as a
+//    programmatic dependent of the previous call, each block first starts
+//    its pieces of W_down and x towards L2, then waits.
 //  * hc_gate_mix_kernel: one block per cpb channels (no more blocks than
 //    SMs).  Before it waits for the first kernel every warp loads its W_up
 //    rows into tensor-core fragments and every thread its x values; once t
